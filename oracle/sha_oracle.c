@@ -1,0 +1,254 @@
+/*
+ * sha_oracle.c -- float64 CPU oracle for Selective Head Attention (SHA) decode.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the slow, obviously correct
+ * reference that the CUDA path is checked against.  Only the test suite, the
+ * smoke check and the benchmark's CPU-baseline / reference arm may load it.
+ * It shares no code, header, table or helper with the CUDA library, and the
+ * CUDA library never calls it.
+ *
+ * What it computes (sources: the pages about "Polar Sparsity: High Throughput
+ * Batched LLM Inferencing with Scalable Contextual Sparsity"):
+ *
+ *  - attention of one query row against one head's cache, as the equation
+ *    under "Attention Head 稀疏性" (papernotes.org summary) defines it:
+ *        O = softmax(scale * q K^T) V,   scale = 1/sqrt(d_h) by default;
+ *  - the same quantity by the tiled online-softmax recurrence of Algorithm 1,
+ *    "Selective Head Flash Attention (Decode)" (ri.k117.org reproducibility
+ *    record, "Pseudocode" row), which renormalises the accumulator after
+ *    every tile of Bc keys;
+ *  - the routing of Algorithm 1 and of the "Selective Head Attention (SHA)
+ *    Kernel" section (papernotes.org): for every batch row b and slot k the
+ *    head id h = batch_head_index[b,k] is looked up, only that head's K/V are
+ *    read and only its output rows are written; all other output rows keep
+ *    whatever the caller put there.  For GQA the unit of selection is a KV
+ *    group (same section: "group sparsity"); query head h*G + j, j < G, reads
+ *    KV head h.
+ *
+ * Inputs are the raw 16-bit patterns of IEEE binary16 (fp16) or bfloat16
+ * values.  Each is widened to double exactly; every sum, product and exp is
+ * then done in double, in the plain order of the definition.
+ *
+ * Function pins (tests/test_oracle_pins.py): all 65536 patterns of each
+ * format against numpy's widening; hand-derived exact results
+ * (tests/golden/); torch's scaled_dot_product_attention in float64 when every
+ * head is active; closed forms (one key, equal keys, zero scale); the
+ * online recurrence against the two-pass definition; permutation and shift
+ * invariance; convexity; untouched inactive rows.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { ORACLE_FP16 = 0, ORACLE_BF16 = 1 };
+
+/* IEEE 754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits. */
+static double fp16_to_double(uint16_t bits)
+{
+    int sign = (bits >> 15) & 1;
+    int exponent = (bits >> 10) & 0x1f;
+    int fraction = bits & 0x3ff;
+    double magnitude;
+    if (exponent == 0)          /* zero or subnormal: fraction * 2^-24 */
+        magnitude = ldexp((double)fraction, -24);
+    else if (exponent == 31)    /* infinity or NaN */
+        magnitude = fraction ? NAN : INFINITY;
+    else                        /* normal: (1 + fraction/1024) * 2^(exponent-15) */
+        magnitude = ldexp((double)(1024 + fraction), exponent - 25);
+    return sign ? -magnitude : magnitude;
+}
+
+/* bfloat16 is the upper half of an IEEE binary32 pattern. */
+static double bf16_to_double(uint16_t bits)
+{
+    uint32_t word = (uint32_t)bits << 16;
+    float value;
+    memcpy(&value, &word, sizeof value);
+    return (double)value;
+}
+
+static double widen(uint16_t bits, int dtype)
+{
+    return dtype == ORACLE_BF16 ? bf16_to_double(bits) : fp16_to_double(bits);
+}
+
+double sha_oracle_widen(uint16_t bits, int dtype) { return widen(bits, dtype); }
+
+/* scale * <q, K[n]> for one key row n. */
+static double score(const uint16_t *q, const uint16_t *key_row, int d,
+                    double scale, int dtype)
+{
+    double dot = 0.0;
+    for (int c = 0; c < d; ++c)
+        dot += widen(q[c], dtype) * widen(key_row[c], dtype);
+    return scale * dot;
+}
+
+/*
+ * Definition: O = softmax(scale * q K^T) V over all n_kv keys.
+ * Pass 1 forms the scores and their maximum M; pass 2 forms
+ * p[n] = exp(s[n] - M), L = sum p[n] and O[c] = sum_n p[n] V[n,c] / L.
+ * Subtracting M leaves the quotient unchanged; it only keeps exp finite.
+ * s is caller scratch of n_kv doubles.
+ */
+static void attention_definition(const uint16_t *q, const uint16_t *K,
+                                 const uint16_t *V, int n_kv, int d,
+                                 double scale, int dtype, double *s, double *o)
+{
+    double M = -INFINITY;
+    for (int n = 0; n < n_kv; ++n) {
+        s[n] = score(q, K + (size_t)n * d, d, scale, dtype);
+        if (s[n] > M) M = s[n];
+    }
+    double L = 0.0;
+    for (int c = 0; c < d; ++c) o[c] = 0.0;
+    for (int n = 0; n < n_kv; ++n) {
+        double p = exp(s[n] - M);
+        L += p;
+        const uint16_t *v_row = V + (size_t)n * d;
+        for (int c = 0; c < d; ++c) o[c] += p * widen(v_row[c], dtype);
+    }
+    for (int c = 0; c < d; ++c) o[c] /= L;
+}
+
+/*
+ * Algorithm 1's recurrence, taken as the pages give it: state
+ * (O_acc, l_acc, m_acc) starts at (0, 0, -inf); the keys are visited in
+ * Tc = ceil(n_kv / Bc) tiles [kstart, kend), kend = min(j*Bc, n_kv).  Per tile:
+ *   S_j = scale * q K_j^T,  m_j = max S_j,  P_j = exp(S_j - m_j),  l_j = sum P_j
+ *   m_new = max(m_acc, m_j),  alpha = exp(m_acc - m_new),  beta = exp(m_j - m_new)
+ *   l_new = alpha*l_acc + beta*l_j
+ *   O_acc = (alpha*l_acc*O_acc + beta*(P_j V_j)) / l_new
+ * so O_acc is a normalised average after every tile.
+ * s and pv are caller scratch of Bc and d doubles.
+ */
+static void attention_online(const uint16_t *q, const uint16_t *K,
+                             const uint16_t *V, int n_kv, int d, double scale,
+                             int dtype, int Bc, double *s, double *pv,
+                             double *o)
+{
+    double m_acc = -INFINITY, l_acc = 0.0;
+    for (int c = 0; c < d; ++c) o[c] = 0.0;
+    int Tc = (n_kv + Bc - 1) / Bc;
+    for (int j = 1; j <= Tc; ++j) {
+        int kstart = (j - 1) * Bc;
+        int kend = j * Bc < n_kv ? j * Bc : n_kv;
+        double m_j = -INFINITY;
+        for (int n = kstart; n < kend; ++n) {
+            s[n - kstart] = score(q, K + (size_t)n * d, d, scale, dtype);
+            if (s[n - kstart] > m_j) m_j = s[n - kstart];
+        }
+        double l_j = 0.0;
+        for (int c = 0; c < d; ++c) pv[c] = 0.0;
+        for (int n = kstart; n < kend; ++n) {
+            double p = exp(s[n - kstart] - m_j);
+            l_j += p;
+            const uint16_t *v_row = V + (size_t)n * d;
+            for (int c = 0; c < d; ++c) pv[c] += p * widen(v_row[c], dtype);
+        }
+        double m_new = m_acc > m_j ? m_acc : m_j;
+        double alpha = exp(m_acc - m_new);
+        double beta = exp(m_j - m_new);
+        double l_new = alpha * l_acc + beta * l_j;
+        for (int c = 0; c < d; ++c)
+            o[c] = (alpha * l_acc * o[c] + beta * pv[c]) / l_new;
+        l_acc = l_new;
+        m_acc = m_new;
+    }
+}
+
+/* One (query row, head) pair by either method; Bc <= 0 selects the definition. */
+static void attention(const uint16_t *q, const uint16_t *K, const uint16_t *V,
+                      int n_kv, int d, double scale, int dtype, int Bc,
+                      double *o)
+{
+    if (Bc <= 0) {
+        double *s = (double *)malloc(sizeof(double) * (size_t)n_kv);
+        attention_definition(q, K, V, n_kv, d, scale, dtype, s, o);
+        free(s);
+    } else {
+        double *s = (double *)malloc(sizeof(double) * (size_t)Bc);
+        double *pv = (double *)malloc(sizeof(double) * (size_t)d);
+        attention_online(q, K, V, n_kv, d, scale, dtype, Bc, s, pv, o);
+        free(pv);
+        free(s);
+    }
+}
+
+/*
+ * Selective head decode over the full layout
+ *   Q, out : [B, H_q, d]        K, V : [B, H_kv, N_kv, d]
+ *   batch_head_index : [B, top_k], values are KV-head ids in [0, H_kv)
+ * G = H_q / H_kv query heads share one KV head (G = 1 is plain multi-head
+ * attention).  For every (b, k) with h = batch_head_index[b,k] in range, rows
+ * out[b, h*G + j, :], j < G, are overwritten; an id out of range writes
+ * nothing and is counted.  No other element of out is touched.
+ * Bc <= 0 uses the definition, Bc > 0 Algorithm 1's tiled recurrence.
+ * Returns the number of out-of-range ids, or -1 for inconsistent sizes.
+ */
+long long sha_oracle_decode(const uint16_t *Q, const uint16_t *K,
+                            const uint16_t *V, const int32_t *batch_head_index,
+                            int B, int H_q, int H_kv, int N_kv, int d,
+                            int top_k, double scale, int dtype, int Bc,
+                            double *out)
+{
+    if (B < 0 || H_kv <= 0 || H_q <= 0 || H_q % H_kv != 0 || N_kv <= 0 ||
+        d <= 0 || top_k < 0)
+        return -1;
+    int G = H_q / H_kv;
+    long long bad = 0;
+    long long units = (long long)B * top_k;
+#pragma omp parallel for schedule(dynamic, 1) reduction(+ : bad)
+    for (long long u = 0; u < units; ++u) {
+        long long b = u / top_k;
+        int h = batch_head_index[u];
+        if (h < 0 || h >= H_kv) {
+            bad += 1;
+            continue;
+        }
+        const uint16_t *K_bh = K + ((size_t)b * H_kv + h) * (size_t)N_kv * d;
+        const uint16_t *V_bh = V + ((size_t)b * H_kv + h) * (size_t)N_kv * d;
+        for (int j = 0; j < G; ++j) {
+            size_t row = ((size_t)b * H_q + (size_t)h * G + j) * (size_t)d;
+            attention(Q + row, K_bh, V_bh, N_kv, d, scale, dtype, Bc, out + row);
+        }
+    }
+    return bad;
+}
+
+/*
+ * The same per-unit computation on units already gathered by the caller:
+ *   Qu, out : [n_units, G, d]     Ku, Vu : [n_units, N_kv, d]
+ * (unit i is one selected (batch row, KV head) pair with its G query rows).
+ * Used to check sampled units of workloads too large to widen whole.
+ */
+int sha_oracle_units(const uint16_t *Qu, const uint16_t *Ku, const uint16_t *Vu,
+                     int n_units, int G, int N_kv, int d, double scale,
+                     int dtype, int Bc, double *out)
+{
+    if (n_units < 0 || G <= 0 || N_kv <= 0 || d <= 0) return -1;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int i = 0; i < n_units; ++i) {
+        const uint16_t *K_i = Ku + (size_t)i * N_kv * d;
+        const uint16_t *V_i = Vu + (size_t)i * N_kv * d;
+        for (int j = 0; j < G; ++j) {
+            size_t row = ((size_t)i * G + j) * (size_t)d;
+            attention(Qu + row, K_i, V_i, N_kv, d, scale, dtype, Bc, out + row);
+        }
+    }
+    return 0;
+}
+
+/* Number of host threads the parallel loops above use. */
+int sha_oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

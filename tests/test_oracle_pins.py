@@ -1,0 +1,253 @@
+"""Pins for the float64 oracle: checks against what the pages and the mathematics
+fix, not against the oracle itself.
+
+Each test is chosen so that a plausible slip in the oracle fails it:
+  * a wrong widening of fp16/bf16 bits        -> exhaustive conversion test
+  * a wrong sign in exp, a dropped scale,
+    dropped normalisation, K/V swapped,
+    a transposed K                             -> hand-derived golden values
+  * a wrong head / group / query-row mapping  -> golden routing, SDPA with GQA
+  * wrong online-softmax rescaling             -> online vs definition
+  * writing inactive rows                      -> untouched-row checks
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _half_bits(values, dtype="fp16"):
+    t = torch.tensor(values, dtype=torch.float64).to(workloads.TORCH_DTYPE[dtype])
+    return t
+
+
+def _rand(shape, seed, dtype="fp16", lo=None):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randn(shape, generator=g, dtype=torch.float32).to(workloads.TORCH_DTYPE[dtype])
+
+
+# ---------------------------------------------------------------- widening
+
+def test_fp16_widening_exhaustive():
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    got = np.array([oracle.widen(b, "fp16") for b in bits])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+    # signed zeros too
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(ref[~nan]))
+
+
+def test_bf16_widening_exhaustive():
+    bits = np.arange(1 << 16, dtype=np.uint32)
+    with np.errstate(invalid="ignore"):
+        ref = (bits << 16).astype(np.uint32).view(np.float32).astype(np.float64)
+    got = np.array([oracle.widen(int(b), "bf16") for b in bits])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+# ---------------------------------------------------------------- hand-derived
+
+def _frac(s):
+    return float(Fraction(s))
+
+
+@pytest.mark.parametrize("tile", [0, 1, 2, 3])
+def test_golden_single_unit(tile):
+    with open(os.path.join(GOLDEN, "hand_single_unit.json")) as f:
+        g = json.load(f)
+    assert g["scale"] == "ln2"
+    q = _half_bits(g["q"]).reshape(1, 1, -1)
+    K = _half_bits(g["K"]).reshape(1, 1, len(g["K"]), -1)
+    V = _half_bits(g["V"]).reshape(1, 1, len(g["V"]), -1)
+    out, bad = oracle.sha_decode(q, K, V, [[0]], math.log(2), "fp16", tile=tile)
+    assert bad == 0
+    want = np.array([_frac(s) for s in g["expected"]])
+    np.testing.assert_allclose(out[0, 0], want, rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("tile", [0, 1])
+def test_golden_gqa_routing(tile):
+    with open(os.path.join(GOLDEN, "hand_gqa_routing.json")) as f:
+        g = json.load(f)
+    Q = _half_bits(g["Q"])
+    K = _half_bits(g["K"])
+    V = _half_bits(g["V"])
+    out, bad = oracle.sha_decode(Q, K, V, g["batch_head_index"], math.log(2), "fp16",
+                                 tile=tile)
+    assert bad == 0
+    for key, vals in g["expected"].items():
+        b, h = map(int, key.split(","))
+        np.testing.assert_allclose(out[b, h], [_frac(s) for s in vals], rtol=0, atol=1e-13)
+    for key in g["untouched"]:
+        b, h = map(int, key.split(","))
+        assert np.isnan(out[b, h]).all()
+
+
+# ---------------------------------------------------------------- library routine
+
+@pytest.mark.parametrize("G", [1, 2, 8])
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_all_heads_active_equals_sdpa(G, dtype):
+    """With every head selected (layer 0 runs dense) the result is plain attention:
+    torch's scaled_dot_product_attention in float64 on the CPU."""
+    B, H_kv, N_kv, d = 3, 4, 37, 16
+    H_q = H_kv * G
+    q = _rand((B, H_q, d), 1, dtype)
+    k = _rand((B, H_kv, N_kv, d), 2, dtype)
+    v = _rand((B, H_kv, N_kv, d), 3, dtype)
+    # every head, in a different order per row
+    idx = np.stack([np.random.default_rng(b).permutation(H_kv) for b in range(B)])
+    scale = 0.37
+    out, bad = oracle.sha_decode(q, k, v, idx, scale, dtype)
+    assert bad == 0
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q.double().unsqueeze(2), k.double(), v.double(), scale=scale,
+        enable_gqa=(G > 1)).squeeze(2)
+    np.testing.assert_allclose(out, ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_sparse_rows_equal_sdpa_rows_and_rest_untouched():
+    w = workloads.CONFIGS["tiny_mha"]
+    q, k, v = workloads.make_qkv(w)
+    idx = workloads.make_index(w)
+    out, bad = oracle.sha_decode(q, k, v, idx, w.scale, w.dtype)
+    assert bad == 0
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q.double().unsqueeze(2), k.double(), v.double(), scale=w.scale).squeeze(2).numpy()
+    active = np.zeros((w.B, w.H_q), dtype=bool)
+    for b in range(w.B):
+        for h in idx[b].tolist():
+            active[b, h] = True
+    np.testing.assert_allclose(out[active], ref[active], rtol=0, atol=1e-12)
+    assert np.isnan(out[~active]).all()
+
+
+# ---------------------------------------------------------------- closed forms
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_single_key_returns_value_row(dtype):
+    """N_kv = 1: softmax of one score is 1, so O = V exactly."""
+    q = _rand((2, 3, 8), 4, dtype)
+    k = _rand((2, 3, 1, 8), 5, dtype)
+    v = _rand((2, 3, 1, 8), 6, dtype)
+    out, _ = oracle.sha_decode(q, k, v, [[0, 1, 2], [2, 1, 0]], 0.5, dtype)
+    assert np.array_equal(out, v.double().squeeze(2).numpy())
+
+
+def test_identical_keys_give_mean_value():
+    N, d = 29, 8
+    q = _rand((1, 1, d), 7)
+    k = _rand((1, 1, 1, d), 8).expand(1, 1, N, d).contiguous()
+    v = _rand((1, 1, N, d), 9)
+    out, _ = oracle.sha_decode(q, k, v, [[0]], 0.9, "fp16")
+    np.testing.assert_allclose(out[0, 0], v.double()[0, 0].mean(0).numpy(), rtol=0, atol=1e-13)
+
+
+def test_zero_scale_gives_mean_value():
+    N, d = 31, 8
+    q, k, v = _rand((1, 1, d), 10), _rand((1, 1, N, d), 11), _rand((1, 1, N, d), 12)
+    out, _ = oracle.sha_decode(q, k, v, [[0]], 0.0, "fp16")
+    np.testing.assert_allclose(out[0, 0], v.double()[0, 0].mean(0).numpy(), rtol=0, atol=1e-13)
+
+
+def test_dominant_key_selects_its_value():
+    """One score 60 above all others: O = V[n*] up to e^-60 relative weight."""
+    N, d = 16, 4
+    k = torch.zeros((1, 1, N, d), dtype=torch.float16)
+    k[0, 0, 5, 0] = 60.0
+    q = torch.tensor([[[1.0, 0, 0, 0]]], dtype=torch.float16)
+    v = _rand((1, 1, N, d), 13)
+    out, _ = oracle.sha_decode(q, k, v, [[0]], 1.0, "fp16")
+    np.testing.assert_allclose(out[0, 0], v.double()[0, 0, 5].numpy(), rtol=0, atol=1e-20)
+
+
+# ---------------------------------------------------------------- invariants
+
+@pytest.mark.parametrize("tile", [1, 3, 16, 100, 128, 500])
+def test_online_recurrence_equals_definition(tile):
+    """Algorithm 1's tiled recurrence (renormalised per tile) is an exact
+    reorganisation of the two-pass softmax."""
+    B, H, N, d = 2, 3, 128, 32
+    q, k, v = _rand((B, H, d), 14), _rand((B, H, N, d), 15), _rand((B, H, N, d), 16)
+    idx = [[2, 0], [1, 2]]
+    two_pass, _ = oracle.sha_decode(q, k, v, idx, 0.2, "fp16", tile=0)
+    online, _ = oracle.sha_decode(q, k, v, idx, 0.2, "fp16", tile=tile)
+    np.testing.assert_allclose(online, two_pass, rtol=0, atol=1e-13, equal_nan=True)
+
+
+def test_joint_permutation_of_keys_and_values():
+    N, d = 50, 16
+    q, k, v = _rand((1, 1, d), 17), _rand((1, 1, N, d), 18), _rand((1, 1, N, d), 19)
+    perm = torch.randperm(N, generator=torch.Generator().manual_seed(3))
+    a, _ = oracle.sha_decode(q, k, v, [[0]], 0.3, "fp16")
+    b, _ = oracle.sha_decode(q, k[:, :, perm].contiguous(), v[:, :, perm].contiguous(),
+                             [[0]], 0.3, "fp16")
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-13)
+
+
+def test_shift_of_all_scores_changes_nothing():
+    """Adding c to every key adds scale*q.c to every score: softmax is unchanged.
+    Values are multiples of 1/8 so every shifted key is exact in fp16."""
+    N, d = 20, 8
+    g = torch.Generator().manual_seed(20)
+    k = (torch.randint(-16, 16, (1, 1, N, d), generator=g) / 8.0).to(torch.float16)
+    c = (torch.randint(-16, 16, (d,), generator=g) / 8.0)
+    q = (torch.randint(-8, 8, (1, 1, d), generator=g) / 8.0).to(torch.float16)
+    v = _rand((1, 1, N, d), 21)
+    a, _ = oracle.sha_decode(q, k, v, [[0]], 0.7, "fp16")
+    b, _ = oracle.sha_decode(q, (k.double() + c.double()).to(torch.float16), v, [[0]], 0.7,
+                             "fp16")
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+def test_output_is_a_convex_combination_of_values():
+    N, d = 64, 32
+    q, k, v = _rand((1, 1, d), 22), _rand((1, 1, N, d), 23), _rand((1, 1, N, d), 24)
+    out, _ = oracle.sha_decode(q, k, v, [[0]], 2.0, "fp16")
+    vv = v.double()[0, 0].numpy()
+    assert (out[0, 0] >= vv.min(0) - 1e-15).all() and (out[0, 0] <= vv.max(0) + 1e-15).all()
+
+
+# ---------------------------------------------------------------- routing edges
+
+def test_out_of_range_ids_are_skipped_and_counted():
+    q, k, v = _rand((2, 4, 8), 25), _rand((2, 4, 9, 8), 26), _rand((2, 4, 9, 8), 27)
+    out, bad = oracle.sha_decode(q, k, v, [[0, 7], [-1, 3]], 0.5, "fp16")
+    assert bad == 2
+    assert not np.isnan(out[0, 0]).any() and not np.isnan(out[1, 3]).any()
+    for b, h in [(0, 1), (0, 2), (0, 3), (1, 0), (1, 1), (1, 2)]:
+        assert np.isnan(out[b, h]).all()
+
+
+def test_zero_top_k_writes_nothing():
+    q, k, v = _rand((2, 4, 8), 28), _rand((2, 4, 9, 8), 29), _rand((2, 4, 9, 8), 30)
+    out, bad = oracle.sha_decode(q, k, v, np.zeros((2, 0), np.int32), 0.5, "fp16")
+    assert bad == 0 and np.isnan(out).all()
+
+
+def test_units_entry_matches_full_layout():
+    w = workloads.CONFIGS["tiny_mha"].with_(H_q=8, H_kv=4)   # G = 2
+    q, k, v = workloads.make_qkv(w)
+    idx = workloads.make_index(w)
+    full, _ = oracle.sha_decode(q, k, v, idx, w.scale, w.dtype)
+    bs = np.repeat(np.arange(w.B), w.top_k)
+    hs = idx.reshape(-1).numpy()
+    qu = torch.stack([q[b, h * w.G:(h + 1) * w.G] for b, h in zip(bs, hs)])
+    ku = torch.stack([k[b, h] for b, h in zip(bs, hs)])
+    vu = torch.stack([v[b, h] for b, h in zip(bs, hs)])
+    per_unit = oracle.sha_units(qu, ku, vu, w.scale, w.dtype)
+    for i, (b, h) in enumerate(zip(bs, hs)):
+        assert np.array_equal(per_unit[i], full[b, h * w.G:(h + 1) * w.G])
