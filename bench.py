@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Selective Head Attention decode benchmark (one JSON line on stdout, rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config NAME]
+
+A step is one selective-head decode call over a whole batch (one attention
+layer, one decode token per sequence) on the OPT-66B-shaped workload: B=64,
+H=72, d=128, N_kv=1920, top_k=22 (30 % head density), fp16, N(0,1) data.
+Inputs are resident in HBM when the timed region starts; the active K/V of a
+step (1.39 GB) is 11x the 126 MB L2, so no flush is needed between steps.
+
+value    = algorithmic bytes of all ranks' steps / max-over-ranks device time
+           (active K+V, active Q rows read, active O rows written, the index)
+roofline = the same bytes per launch / mean launch time, against the measured
+           HBM copy bandwidth of this GPU pool (MEASURED_PEAKS.json, else the
+           fallback figure), and beside a copy kernel timed in this run
+e2e      = the same metric through the public API with the step's per-token
+           inputs (q, index) copied from pinned host memory and the output
+           copied back inside the timed region; the KV cache is model state
+           and stays resident
+cpu_baseline = the float64 oracle on the host cores, on a sample of units
+
+With --gpus N (torchrun, one process per GPU) every rank decodes its own
+batch (weak scaling: the path needs no exchange between GPUs).
+--impl reference times the float64 CPU oracle on the same workload instead.
+"""
+import argparse
+import datetime
+import glob
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = ("SHA decode: achieved HBM GB/s (% of B200 peak) and decode steps/sec vs density")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=4000)
+    p.add_argument("--warmup", type=int, default=100)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--config", default="opt66b", choices=sorted(workloads.CONFIGS))
+    p.add_argument("--batch", type=int, default=None,
+                   help="override the workload's batch size (small ncu captures)")
+    p.add_argument("--no-extras", action="store_true",
+                   help="skip the density sweep, e2e and CPU baseline (used for ncu)")
+    p.add_argument("--cpu-budget", type=float, default=10.0,
+                   help="seconds of oracle work for cpu_baseline")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------- environment
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback (no MEASURED_PEAKS.json)"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "head_sparse_decode_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    current = kernel_source_hash()
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        text = open(path).read()
+        m_hash = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
+        m_val = re.search(r"traffic_bytes_per_launch\[" + re.escape(workload) + r"\]:\s*(\d+)",
+                          text)
+        if m_hash and m_val and m_hash.group(1) == current:
+            return int(m_val.group(1))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples, stamped with wall time."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.samples = []
+        self.proc = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", uuid, "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, RuntimeError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) == 7:
+                self.samples.append((time.time(), parts))
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        window = [s for t, s in self.samples if t0 <= t <= t1] or [s for _, s in self.samples]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for s in window for i in range(4)
+                          if s[3 + i].lower().startswith("active")})
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(s[0]) for s in window if num(s[0]) is not None]
+        mx = [num(s[1]) for s in window if num(s[1]) is not None]
+        pw = [num(s[2]) for s in window if num(s[2]) is not None]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None,
+                "samples": len(window), "reasons": reasons}
+
+
+# ---------------------------------------------------------------- oracle timing
+
+def gather_units(w, q, k, v, idx, units):
+    idx_h = idx.cpu().numpy()
+    pairs = [(int(u) // w.top_k, int(idx_h[int(u) // w.top_k, int(u) % w.top_k])) for u in units]
+    G = w.G
+    qu = torch.stack([q[b, h * G:(h + 1) * G].cpu() for b, h in pairs])
+    ku = torch.stack([k[b, h].cpu() for b, h in pairs])
+    vu = torch.stack([v[b, h].cpu() for b, h in pairs])
+    return qu, ku, vu
+
+
+def cpu_baseline(w, q, k, v, idx, budget_s, max_units=128):
+    import oracle
+    rng = np.random.default_rng(0)
+    units = rng.choice(w.units, size=min(max_units, w.units), replace=False)
+    qu, ku, vu = gather_units(w, q, k, v, idx, units)
+    per_unit = w.algorithmic_bytes() / w.units
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.sha_units(qu, ku, vu, w.scale, w.dtype)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= budget_s:
+            break
+    return {"value": per_unit * len(units) * reps / dt / 1e9, "unit": "GB/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{len(units)} seeded-random (batch row, head) units of {w.name} "
+                      f"x {reps} passes, {dt:.1f} s, float64 C oracle with OpenMP"}
+
+
+# ---------------------------------------------------------------- timing helpers
+
+def timed(fn, steps, stream):
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        fn()
+    end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end) / 1e3   # seconds
+
+
+def sync_all(world, local):
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[local])
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- arms
+
+def run_ours(args, rank, world, local):
+    import head_sparse_decode_b200 as sha
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    base = workloads.CONFIGS[args.config]
+    if args.batch:
+        base = base.with_(B=args.batch)
+    w = base.with_(seed=base.seed + 100 * rank)     # each rank decodes its own batch
+    q, k, v = workloads.make_qkv(w, device=dev)
+    idx = workloads.make_index(w).to(dev)
+    out = workloads.make_out(w, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        sha.decode(q, k, v, idx, w.scale, out)
+
+    # same-run HBM copy probe (1 GiB read + 1 GiB written)
+    src = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
+    dst = torch.empty_like(src)
+    src.fill_(1)
+    for _ in range(3):
+        sha.sha_copy_bandwidth_probe(dst, src)
+    t = timed(lambda: sha.sha_copy_bandwidth_probe(dst, src), 20, stream)
+    copy_gbs = 2 * src.numel() * 20 / t / 1e9
+    del src, dst
+    torch.cuda.empty_cache()
+
+    sampler = ClockSampler(dev)
+    for _ in range(args.warmup):
+        step()
+    sync_all(world, local)
+    t0 = time.time()
+    elapsed = timed(step, args.steps, stream)
+    t1 = time.time()
+    sync_all(world, local)
+    clocks = sampler.stop(t0, t1)
+    status = sha.sha_get_device_status()
+    if status != sha.SHA_OK:
+        raise RuntimeError(f"device status after timing: {sha.sha_status_string(status)}")
+
+    t_max = max_over_ranks(elapsed, world)
+    bytes_step = w.algorithmic_bytes()
+    total_bytes = sum_over_ranks(bytes_step * args.steps, world)
+    value = total_bytes / t_max / 1e9
+    launch_s = elapsed / args.steps
+    achieved = bytes_step / launch_s / 1e9
+    peak, peak_src = measured_peak()
+
+    extras = {}
+    if not args.no_extras:
+        extras["density_sweep"] = density_sweep(sha, w, q, k, v, dev, stream, peak)
+        extras["e2e"] = e2e(sha, w, q, k, v, idx, out, dev, stream, args)
+    plan = sha.sha_decode_plan(w.B, w.H_q, w.H_kv, w.N_kv, w.d, w.top_k,
+                               num_sms=torch.cuda.get_device_properties(dev).multi_processor_count)
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(t_max / args.steps * 1e3, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic N(0,1), seeded",
+        "config": {**w.describe(), "parallelism": f"replicas x{world} (batch sharded by rank)",
+                   "accumulation": "fp32", "l2": "no flush: active K/V per step "
+                   f"{w.units * 2 * w.N_kv * w.d * 2 / 1e9:.2f} GB > 126 MB L2",
+                   "blocks": plan["blocks"], "tile_keys": plan["tile_keys"]},
+        "steps_per_s": round(args.steps / t_max, 2),
+        "tokens_per_s": round(world * w.B * args.steps / t_max, 1),
+        "hbm_frac_of_measured": round(achieved / peak, 4),
+        "copy_probe_gbs": round(copy_gbs, 1),
+        "clocks": clocks,
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": profiled_traffic(w.name), "peak_source": peak_src,
+                     "kernel": "sha_mha_decode_kernel", "launch_us": round(launch_s * 1e6, 3),
+                     "bytes_per_launch": bytes_step},
+    }
+    if "e2e" in extras:
+        line["e2e"] = extras.pop("e2e")
+    line.update(extras)
+    if rank == 0 and world == 1 and not args.no_extras:
+        line["cpu_baseline"] = cpu_baseline(w, q, k, v, idx, args.cpu_budget)
+    return line
+
+
+def density_sweep(sha, w, q, k, v, dev, stream, peak):
+    """Same shape at 25/50/75/100 % head density (100 % = the dense reference)."""
+    res = []
+    for frac in (0.25, 0.5, 0.75, 1.0):
+        top_k = max(1, round(frac * w.H_kv))
+        wk = w.with_(top_k=top_k)
+        idx = workloads.make_index(wk).to(dev)
+        out = workloads.make_out(wk, dev)
+        for _ in range(20):
+            sha.decode(q, k, v, idx, w.scale, out)
+        steps = 300
+        t = timed(lambda: sha.decode(q, k, v, idx, w.scale, out), steps, stream)
+        gbs = wk.algorithmic_bytes() * steps / t / 1e9
+        res.append({"top_k": top_k, "density": round(top_k / w.H_kv, 4),
+                    "us_per_step": round(t / steps * 1e6, 2), "gbs": round(gbs, 1),
+                    "frac": round(gbs / peak, 4), "steps_per_s": round(steps / t, 1)})
+    dense = res[-1]["us_per_step"]
+    for r in res:
+        r["time_vs_dense"] = round(r["us_per_step"] / dense, 4)
+    return res
+
+
+def e2e(sha, w, q, k, v, idx, out, dev, stream, args):
+    q_h = q.cpu().pin_memory()
+    idx_h = idx.cpu().pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def step():
+        q.copy_(q_h, non_blocking=True)
+        idx.copy_(idx_h, non_blocking=True)
+        sha.decode(q, k, v, idx, w.scale, out)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(10):
+        step()
+    steps = max(10, min(args.steps, 2000))
+    t = timed(step, steps, stream)
+    h2d = q.numel() * q.element_size() + idx.numel() * idx.element_size()
+    d2h = out.numel() * out.element_size()
+    return {"value": round(w.algorithmic_bytes() * steps / t / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(t / steps * 1e3, 5), "steps": steps}
+
+
+def run_reference(args):
+    """The float64 CPU oracle as a bench arm, on bounded samples of the workload."""
+    import oracle
+
+    w = workloads.CONFIGS[args.config]
+    dev = torch.device("cuda", 0) if torch.cuda.is_available() else torch.device("cpu")
+    q, k, v = workloads.make_qkv(w, device=dev)
+    idx = workloads.make_index(w)
+    rng = np.random.default_rng(1)
+    pool = rng.choice(w.units, size=min(64, w.units), replace=False)
+    qu, ku, vu = gather_units(w, q, k, v, idx, pool)
+    del q, k, v
+    per_unit = w.algorithmic_bytes() / w.units
+    oracle.sha_units(qu[:1], ku[:1], vu[:1], w.scale, w.dtype)
+    t0 = time.perf_counter()
+    oracle.sha_units(qu[:8], ku[:8], vu[:8], w.scale, w.dtype)
+    t_unit = (time.perf_counter() - t0) / 8
+    budget = 90.0 / max(1, args.steps + args.warmup)
+    n = int(max(1, min(len(pool), budget // max(t_unit, 1e-9))))
+
+    def step(i):
+        s = (i * n) % len(pool)
+        sel = [(s + j) % len(pool) for j in range(n)]
+        oracle.sha_units(qu[sel], ku[sel], vu[sel], w.scale, w.dtype)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    dt = time.perf_counter() - t0
+    value = per_unit * n * args.steps / dt / 1e9
+    cores = oracle.num_threads()
+    sample = (f"each step: {n} of a fixed pool of {len(pool)} seeded-random units of {w.name} "
+              f"(float64 C oracle, OpenMP)")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic N(0,1), seeded",
+        "config": {**w.describe(), "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main():
+    args = parse_args()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=torch.device("cuda", local))
+    try:
+        line = run_ours(args, rank, world, local)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,238 @@
+"""Selective Head Attention (SHA) decode on B200 -- Python binding.
+
+A thin ctypes layer over ``libsha_decode.so`` (the C ABI declared in
+``include/sha_decode.h``): it checks tensor properties, converts them to
+pointers and sizes, and calls the library.  Every step of the computation
+runs in the library's CUDA kernels; there is no fallback.  Importing this
+package fails loudly if the library has not been built
+(``python head_sparse_decode_b200/build.py``).
+
+    out = sha_decode(q, k, v, batch_head_index, scale, out)      # fp16
+    out = sha_decode_bf16(q, k, v, batch_head_index, scale, out) # bf16
+    out = decode(q, k, v, batch_head_index, out=out)             # either dtype
+
+Shapes: q, out [B, H_q, d] (or [B, H_q, 1, d]); k, v [B, H_kv, N_kv, d];
+batch_head_index [B, top_k] int32 on the same device.  Rows of out whose head
+is not selected are left exactly as they were.
+"""
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIBRARY_PATH = os.path.join(_PKG, "libsha_decode.so")
+
+if not os.path.exists(LIBRARY_PATH):
+    raise ImportError(
+        f"{LIBRARY_PATH} is missing: build the CUDA library first "
+        "(python head_sparse_decode_b200/build.py)")
+
+_lib = ctypes.CDLL(LIBRARY_PATH)
+
+SHA_OK = 0
+SHA_ERR_INVALID_ARG = 1
+SHA_ERR_UNSUPPORTED = 2
+SHA_ERR_MISALIGNED = 3
+SHA_ERR_LAUNCH = 4
+SHA_ERR_BAD_INDEX = 5
+SHA_ERR_TIMEOUT = 6
+SHA_ERR_WORKSPACE = 7
+SHA_FP16 = 0
+SHA_BF16 = 1
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_DECODE_ARGS = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_float, _vp, _vp]
+_lib.sha_decode.argtypes = _DECODE_ARGS
+_lib.sha_decode.restype = _i
+_lib.sha_decode_bf16.argtypes = _DECODE_ARGS
+_lib.sha_decode_bf16.restype = _i
+_lib.sha_decode_ex.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_float, _vp,
+                               _i, _vp, ctypes.c_size_t, _i, _vp]
+_lib.sha_decode_ex.restype = _i
+_lib.sha_decode_workspace_size.argtypes = [_i, _i, _i, _i, _i, _i, _i]
+_lib.sha_decode_workspace_size.restype = ctypes.c_size_t
+_lib.sha_get_device_status.argtypes = [_vp]
+_lib.sha_get_device_status.restype = _i
+_lib.sha_status_string.argtypes = [_i]
+_lib.sha_status_string.restype = ctypes.c_char_p
+_lib.sha_last_cuda_error.argtypes = []
+_lib.sha_last_cuda_error.restype = ctypes.c_char_p
+_lib.sha_decode_plan.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(ctypes.c_int64)]
+_lib.sha_decode_plan.restype = _i
+_lib.sha_copy_bandwidth_probe.argtypes = [_vp, _vp, ctypes.c_size_t, _vp]
+_lib.sha_copy_bandwidth_probe.restype = _i
+
+
+class ShaError(RuntimeError):
+    def __init__(self, status):
+        msg = sha_status_string(status)
+        if status == SHA_ERR_LAUNCH:
+            msg += ": " + _lib.sha_last_cuda_error().decode()
+        super().__init__(msg)
+        self.status = status
+
+
+def sha_status_string(status):
+    return _lib.sha_status_string(int(status)).decode()
+
+
+def _check(status):
+    if status != SHA_OK:
+        raise ShaError(status)
+
+
+def _stream_handle(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _shapes(q, k, v, batch_head_index, out):
+    if k.dim() != 4 or v.shape != k.shape:
+        raise ValueError("k and v must both be [B, H_kv, N_kv, d]")
+    B, H_kv, N_kv, d = k.shape
+    if q.dim() == 4:
+        if q.shape[2] != 1:
+            raise ValueError("decode takes one query token: q must be [B, H_q, 1, d]")
+    elif q.dim() != 3:
+        raise ValueError("q must be [B, H_q, d] or [B, H_q, 1, d]")
+    if q.shape[0] != B or q.shape[-1] != d:
+        raise ValueError("q does not match k's batch or head dim")
+    H_q = q.shape[1]
+    if out.numel() != B * H_q * d:
+        raise ValueError("out must hold [B, H_q, d] elements")
+    if batch_head_index.dim() != 2 or batch_head_index.shape[0] != B:
+        raise ValueError("batch_head_index must be [B, top_k]")
+    top_k = batch_head_index.shape[1]
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out),
+                    ("batch_head_index", batch_head_index)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if t.device != k.device:
+            raise ValueError(f"{name} is on {t.device}, k on {k.device}")
+    if batch_head_index.dtype != torch.int32:
+        raise TypeError("batch_head_index must be int32")
+    for name, t in (("q", q), ("v", v), ("out", out)):
+        if t.dtype != k.dtype:
+            raise TypeError(f"{name} has dtype {t.dtype}, k has {k.dtype}")
+    return B, H_q, H_kv, N_kv, d, top_k
+
+
+def _default_scale(scale, d):
+    return 1.0 / math.sqrt(d) if scale is None else float(scale)
+
+
+def _decode_args(q, k, v, batch_head_index, scale, out, stream):
+    B, H_q, H_kv, N_kv, d, top_k = _shapes(q, k, v, batch_head_index, out)
+    return ([q.data_ptr(), k.data_ptr(), v.data_ptr(), batch_head_index.data_ptr(),
+             B, H_q, H_kv, N_kv, d, top_k, _default_scale(scale, d), out.data_ptr()],
+            _stream_handle(stream, k.device))
+
+
+def sha_decode(q, k, v, batch_head_index, scale, out, stream=None):
+    """fp16 selective head decode into ``out`` (library-managed workspace)."""
+    if k.dtype != torch.float16:
+        raise TypeError("sha_decode takes float16 tensors; use sha_decode_bf16 for bfloat16")
+    args, s = _decode_args(q, k, v, batch_head_index, scale, out, stream)
+    with torch.cuda.device(k.device):
+        _check(_lib.sha_decode(*args, s))
+    return out
+
+
+def sha_decode_bf16(q, k, v, batch_head_index, scale, out, stream=None):
+    """bf16 selective head decode into ``out`` (library-managed workspace)."""
+    if k.dtype != torch.bfloat16:
+        raise TypeError("sha_decode_bf16 takes bfloat16 tensors")
+    args, s = _decode_args(q, k, v, batch_head_index, scale, out, stream)
+    with torch.cuda.device(k.device):
+        _check(_lib.sha_decode_bf16(*args, s))
+    return out
+
+
+def _dtype_code(dtype):
+    if dtype == torch.float16:
+        return SHA_FP16
+    if dtype == torch.bfloat16:
+        return SHA_BF16
+    raise TypeError(f"unsupported dtype {dtype}")
+
+
+def sha_decode_workspace_size(B, H_q, H_kv, N_kv, d, top_k, num_splits=0, device=None):
+    """Workspace bytes sha_decode_ex needs for these sizes on ``device``."""
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        return int(_lib.sha_decode_workspace_size(B, H_q, H_kv, N_kv, d, top_k, num_splits))
+
+
+def alloc_workspace(q, k, batch_head_index, num_splits=0):
+    """A zero-filled workspace tensor sized for sha_decode_ex with these inputs."""
+    B, H_kv, N_kv, d = k.shape
+    nbytes = sha_decode_workspace_size(B, q.shape[1], H_kv, N_kv, d,
+                                       batch_head_index.shape[1], num_splits, k.device)
+    return torch.zeros(max(nbytes, 1), dtype=torch.uint8, device=k.device)
+
+
+def sha_decode_ex(q, k, v, batch_head_index, scale, out, workspace=None, num_splits=0,
+                  stream=None):
+    """Selective head decode with a caller-owned workspace and a forced split count
+    (0 = automatic).  ``workspace`` is a zero-initialised CUDA uint8 tensor of at
+    least sha_decode_workspace_size(...) bytes (see alloc_workspace); every call
+    leaves it zeroed again."""
+    args, s = _decode_args(q, k, v, batch_head_index, scale, out, stream)
+    ws_ptr, ws_bytes = (0, 0) if workspace is None else (workspace.data_ptr(),
+                                                         workspace.numel() * workspace.element_size())
+    with torch.cuda.device(k.device):
+        _check(_lib.sha_decode_ex(*args, _dtype_code(k.dtype), ws_ptr, ws_bytes,
+                                  int(num_splits), s))
+    return out
+
+
+def decode(q, k, v, batch_head_index, scale=None, out=None, stream=None):
+    """Selective head decode for either dtype; allocates ``out`` if not given
+    (rows of unselected heads are then uninitialised)."""
+    if out is None:
+        out = torch.empty((q.shape[0], q.shape[1], q.shape[-1]), dtype=q.dtype, device=q.device)
+    if k.dtype == torch.float16:
+        return sha_decode(q, k, v, batch_head_index, scale, out, stream)
+    return sha_decode_bf16(q, k, v, batch_head_index, scale, out, stream)
+
+
+def sha_decode_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits=0, num_sms=148):
+    """Host-side plan of a call: dict with tiles_per_head, total_tiles, blocks,
+    workspace_bytes, tile_keys.  Raises ShaError for sizes the library rejects."""
+    plan = (ctypes.c_int64 * 5)()
+    _check(_lib.sha_decode_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits, num_sms, plan))
+    return {"tiles_per_head": plan[0], "total_tiles": plan[1], "blocks": plan[2],
+            "workspace_bytes": plan[3], "tile_keys": plan[4]}
+
+
+def sha_get_device_status(stream=None, device=None):
+    """Synchronise ``stream`` and read-and-clear the device's sticky flags; returns a
+    status code (SHA_OK, SHA_ERR_BAD_INDEX or SHA_ERR_TIMEOUT)."""
+    dev = device if device is not None else torch.cuda.current_device()
+    with torch.cuda.device(dev):
+        return int(_lib.sha_get_device_status(_stream_handle(stream, dev)))
+
+
+def sha_copy_bandwidth_probe(dst, src, stream=None):
+    """dst.copy_(src) with the library's 16-byte vectorised copy kernel (bandwidth probe)."""
+    nbytes = src.numel() * src.element_size()
+    if dst.numel() * dst.element_size() < nbytes:
+        raise ValueError("dst is smaller than src")
+    with torch.cuda.device(src.device):
+        _check(_lib.sha_copy_bandwidth_probe(dst.data_ptr(), src.data_ptr(), nbytes,
+                                             _stream_handle(stream, src.device)))
+    return dst
+
+
+__all__ = [
+    "sha_decode", "sha_decode_bf16", "sha_decode_ex", "sha_decode_workspace_size",
+    "sha_get_device_status", "sha_status_string", "sha_decode_plan", "sha_copy_bandwidth_probe", "decode",
+    "alloc_workspace", "ShaError", "LIBRARY_PATH",
+]

@@ -1,0 +1,329 @@
+// sha_decode.cu -- C ABI of the Selective Head Attention decode library:
+// argument checks, the work planner, workspace handling and kernel launches.
+// The operation and every argument are specified in include/sha_decode.h.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "sha_decode.h"
+#include "sha_device.cuh"
+#include "sha_mha_kernel.cuh"
+#include "sha_schedule.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxG = 16;
+
+thread_local char g_last_cuda_error[256] = "no error";
+
+sha_status_t launch_error(cudaError_t e)
+{
+    std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "%s: %s", cudaGetErrorName(e),
+                  cudaGetErrorString(e));
+    return SHA_ERR_LAUNCH;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Shape checks shared by every entry point; no CUDA call is made here.
+sha_status_t check_shape(int B, int H_q, int H_kv, int N_kv, int d, int top_k, float scale)
+{
+    if (B < 0 || H_q < 1 || H_kv < 1 || N_kv < 1 || top_k < 0 || top_k > H_kv)
+        return SHA_ERR_INVALID_ARG;
+    if (H_q % H_kv != 0) return SHA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return SHA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return SHA_ERR_UNSUPPORTED;
+    if (H_q / H_kv > kMaxG) return SHA_ERR_UNSUPPORTED;
+    return SHA_OK;
+}
+
+struct DeviceInfo {
+    int num_sms = 0;
+};
+
+std::mutex g_mutex;
+DeviceInfo g_devices[kMaxDevices];
+
+sha_status_t current_device(int *dev, DeviceInfo **info)
+{
+    cudaError_t e = cudaGetDevice(dev);
+    if (e != cudaSuccess) return launch_error(e);
+    if (*dev < 0 || *dev >= kMaxDevices) return SHA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo &di = g_devices[*dev];
+    if (di.num_sms == 0) {
+        e = cudaDeviceGetAttribute(&di.num_sms, cudaDevAttrMultiProcessorCount, *dev);
+        if (e != cudaSuccess) {
+            di.num_sms = 0;
+            return launch_error(e);
+        }
+    }
+    *info = &di;
+    return SHA_OK;
+}
+
+// The call's plan: tile schedule and workspace layout.
+struct Plan {
+    sha::Schedule sched;
+    int slot_floats;
+    size_t counter_bytes;   // [units] int32, rounded up to 256 bytes
+    size_t slot_bytes;      // 2*num_ctas slots
+    size_t workspace_bytes() const { return counter_bytes + slot_bytes; }
+};
+
+constexpr int kTileKeys = 64;          // keys per tile (both kernels)
+constexpr int kBlocksPerSm = 1;
+
+Plan make_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int num_splits,
+               int num_sms)
+{
+    Plan pl;
+    const int G = H_q / H_kv;
+    const long long units = (long long)B * top_k;
+    pl.sched.tiles_per_unit = (N_kv + kTileKeys - 1) / kTileKeys;
+    pl.sched.total_tiles = units * pl.sched.tiles_per_unit;
+    long long ctas = num_splits > 0 ? num_splits : (long long)num_sms * kBlocksPerSm;
+    if (ctas > pl.sched.total_tiles) ctas = pl.sched.total_tiles;
+    if (ctas < 1) ctas = 1;
+    pl.sched.num_ctas = (int)ctas;
+    // one partial state: G rows of (O[d], m, l), padded to 128 bytes
+    pl.slot_floats = ((G * (d + 2)) + 31) / 32 * 32;
+    pl.counter_bytes = ((size_t)units * sizeof(int) + 255) / 256 * 256;
+    pl.slot_bytes = (size_t)2 * pl.sched.num_ctas * pl.slot_floats * sizeof(float);
+    // every unit held whole by one block: no partial state is needed
+    if (pl.sched.total_tiles % pl.sched.num_ctas == 0 &&
+        (pl.sched.total_tiles / pl.sched.num_ctas) % pl.sched.tiles_per_unit == 0) {
+        pl.counter_bytes = 0;
+        pl.slot_bytes = 0;
+    }
+    return pl;
+}
+
+template <typename T, int D>
+sha_status_t launch_mha(const sha::DecodeParams &prm, int dev, cudaStream_t stream)
+{
+    using C = sha::MhaConfig<D>;
+    static bool configured[kMaxDevices] = {};
+    if (!configured[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(sha::sha_mha_decode_kernel<T, D>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::kSmemBytes);
+        if (e != cudaSuccess) return launch_error(e);
+        configured[dev] = true;
+    }
+    sha::sha_mha_decode_kernel<T, D>
+        <<<prm.sched.num_ctas, C::kThreads, C::kSmemBytes, stream>>>(prm);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return launch_error(e);
+    return SHA_OK;
+}
+
+sha_status_t decode_impl(const void *q, const void *k, const void *v, const int32_t *idx,
+                         int B, int H_q, int H_kv, int N_kv, int d, int top_k, float scale,
+                         void *out, sha_dtype_t dtype, void *workspace,
+                         size_t workspace_bytes, int num_splits, void *stream,
+                         bool library_workspace)
+{
+    if (dtype != SHA_FP16 && dtype != SHA_BF16) return SHA_ERR_UNSUPPORTED;
+    sha_status_t st = check_shape(B, H_q, H_kv, N_kv, d, top_k, scale);
+    if (st != SHA_OK) return st;
+    if (num_splits < 0) return SHA_ERR_INVALID_ARG;
+    if (B == 0 || top_k == 0) return SHA_OK;
+    if (!q || !k || !v || !idx || !out) return SHA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        !aligned(idx, 4))
+        return SHA_ERR_MISALIGNED;
+    if (workspace && !aligned(workspace, 256)) return SHA_ERR_MISALIGNED;
+    const int G = H_q / H_kv;
+    if (G != 1) return SHA_ERR_UNSUPPORTED;   // grouped-query kernel: not built yet
+
+    int dev;
+    DeviceInfo *info;
+    st = current_device(&dev, &info);
+    if (st != SHA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const Plan pl = make_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits, info->num_sms);
+    const size_t need = pl.workspace_bytes();
+
+    if (library_workspace && need > 0) {
+        static struct {
+            void *ptr;
+            size_t bytes;
+        } owned[kMaxDevices] = {};
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (owned[dev].bytes < need) {
+            size_t bytes = need < (1u << 20) ? (1u << 20) : need;
+            if (owned[dev].ptr) {
+                cudaError_t e = cudaFree(owned[dev].ptr);
+                owned[dev].ptr = nullptr;
+                owned[dev].bytes = 0;
+                if (e != cudaSuccess) return launch_error(e);
+            }
+            cudaError_t e = cudaMalloc(&owned[dev].ptr, bytes);
+            if (e != cudaSuccess) return launch_error(e);
+            e = cudaMemsetAsync(owned[dev].ptr, 0, bytes, s);
+            if (e != cudaSuccess) return launch_error(e);
+            owned[dev].bytes = bytes;
+        }
+        workspace = owned[dev].ptr;
+        workspace_bytes = owned[dev].bytes;
+    }
+    if (need > 0 && (!workspace || workspace_bytes < need)) return SHA_ERR_WORKSPACE;
+
+    sha::DecodeParams prm;
+    prm.q = q;
+    prm.k = k;
+    prm.v = v;
+    prm.idx = idx;
+    prm.out = out;
+    prm.B = B;
+    prm.H_q = H_q;
+    prm.H_kv = H_kv;
+    prm.N_kv = N_kv;
+    prm.top_k = top_k;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.sched = pl.sched;
+    prm.slot_floats = pl.slot_floats;
+    prm.counters = need ? static_cast<int *>(workspace) : nullptr;
+    prm.slots = need ? reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                                 pl.counter_bytes)
+                     : nullptr;
+
+    if (dtype == SHA_FP16)
+        return d == 128 ? launch_mha<__half, 128>(prm, dev, s) : launch_mha<__half, 64>(prm, dev, s);
+    return d == 128 ? launch_mha<__nv_bfloat16, 128>(prm, dev, s)
+                    : launch_mha<__nv_bfloat16, 64>(prm, dev, s);
+}
+
+__global__ void copy_probe_kernel(uint4 *__restrict__ dst, const uint4 *__restrict__ src,
+                                  size_t n)
+{
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    for (; i + 3 * stride < n; i += 4 * stride) {
+        const uint4 a = __ldcs(src + i);
+        const uint4 b = __ldcs(src + i + stride);
+        const uint4 c = __ldcs(src + i + 2 * stride);
+        const uint4 d = __ldcs(src + i + 3 * stride);
+        __stcs(dst + i, a);
+        __stcs(dst + i + stride, b);
+        __stcs(dst + i + 2 * stride, c);
+        __stcs(dst + i + 3 * stride, d);
+    }
+    for (; i < n; i += stride) __stcs(dst + i, __ldcs(src + i));
+}
+
+}  // namespace
+
+extern "C" {
+
+sha_status_t sha_decode(const void *q, const void *k, const void *v,
+                        const int32_t *batch_head_index, int B, int H_q, int H_kv, int N_kv,
+                        int d, int top_k, float scale, void *out, void *stream)
+{
+    return decode_impl(q, k, v, batch_head_index, B, H_q, H_kv, N_kv, d, top_k, scale, out,
+                       SHA_FP16, nullptr, 0, 0, stream, true);
+}
+
+sha_status_t sha_decode_bf16(const void *q, const void *k, const void *v,
+                             const int32_t *batch_head_index, int B, int H_q, int H_kv,
+                             int N_kv, int d, int top_k, float scale, void *out, void *stream)
+{
+    return decode_impl(q, k, v, batch_head_index, B, H_q, H_kv, N_kv, d, top_k, scale, out,
+                       SHA_BF16, nullptr, 0, 0, stream, true);
+}
+
+sha_status_t sha_decode_ex(const void *q, const void *k, const void *v,
+                           const int32_t *batch_head_index, int B, int H_q, int H_kv,
+                           int N_kv, int d, int top_k, float scale, void *out,
+                           sha_dtype_t dtype, void *workspace, size_t workspace_bytes,
+                           int num_splits, void *stream)
+{
+    return decode_impl(q, k, v, batch_head_index, B, H_q, H_kv, N_kv, d, top_k, scale, out,
+                       dtype, workspace, workspace_bytes, num_splits, stream, false);
+}
+
+size_t sha_decode_workspace_size(int B, int H_q, int H_kv, int N_kv, int d, int top_k,
+                                 int num_splits)
+{
+    if (check_shape(B, H_q, H_kv, N_kv, d, top_k, 1.0f) != SHA_OK || num_splits < 0) return 0;
+    if (B == 0 || top_k == 0) return 0;
+    int dev;
+    DeviceInfo *info;
+    if (current_device(&dev, &info) != SHA_OK) return 0;
+    return make_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits, info->num_sms)
+        .workspace_bytes();
+}
+
+sha_status_t sha_decode_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k,
+                             int num_splits, int num_sms, int64_t plan[5])
+{
+    sha_status_t st = check_shape(B, H_q, H_kv, N_kv, d, top_k, 1.0f);
+    if (st != SHA_OK) return st;
+    if (num_splits < 0 || num_sms < 1 || !plan) return SHA_ERR_INVALID_ARG;
+    if (B == 0 || top_k == 0) {
+        plan[0] = (N_kv + kTileKeys - 1) / kTileKeys;
+        plan[1] = plan[2] = plan[3] = 0;
+        plan[4] = kTileKeys;
+        return SHA_OK;
+    }
+    const Plan pl = make_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits, num_sms);
+    plan[0] = pl.sched.tiles_per_unit;
+    plan[1] = pl.sched.total_tiles;
+    plan[2] = pl.sched.num_ctas;
+    plan[3] = (int64_t)pl.workspace_bytes();
+    plan[4] = kTileKeys;
+    return SHA_OK;
+}
+
+sha_status_t sha_get_device_status(void *stream)
+{
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return launch_error(e);
+    unsigned int flags = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&flags, sha::g_sha_status, sizeof flags);
+    if (e != cudaSuccess) return launch_error(e);
+    e = cudaMemcpyToSymbol(sha::g_sha_status, &zero, sizeof zero);
+    if (e != cudaSuccess) return launch_error(e);
+    if (flags & sha::kStatusTimeout) return SHA_ERR_TIMEOUT;
+    if (flags & sha::kStatusBadIndex) return SHA_ERR_BAD_INDEX;
+    return SHA_OK;
+}
+
+const char *sha_status_string(sha_status_t status)
+{
+    switch (status) {
+    case SHA_OK: return "SHA_OK";
+    case SHA_ERR_INVALID_ARG: return "SHA_ERR_INVALID_ARG";
+    case SHA_ERR_UNSUPPORTED: return "SHA_ERR_UNSUPPORTED";
+    case SHA_ERR_MISALIGNED: return "SHA_ERR_MISALIGNED";
+    case SHA_ERR_LAUNCH: return "SHA_ERR_LAUNCH";
+    case SHA_ERR_BAD_INDEX: return "SHA_ERR_BAD_INDEX";
+    case SHA_ERR_TIMEOUT: return "SHA_ERR_TIMEOUT";
+    case SHA_ERR_WORKSPACE: return "SHA_ERR_WORKSPACE";
+    }
+    return "unknown sha_status_t";
+}
+
+const char *sha_last_cuda_error(void) { return g_last_cuda_error; }
+
+sha_status_t sha_copy_bandwidth_probe(void *dst, const void *src, size_t bytes, void *stream)
+{
+    if (!dst || !src || bytes % 16 != 0) return SHA_ERR_INVALID_ARG;
+    if (!aligned(dst, 16) || !aligned(src, 16)) return SHA_ERR_MISALIGNED;
+    if (bytes == 0) return SHA_OK;
+    int dev;
+    DeviceInfo *info;
+    sha_status_t st = current_device(&dev, &info);
+    if (st != SHA_OK) return st;
+    copy_probe_kernel<<<info->num_sms * 4, 512, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint4 *>(dst), static_cast<const uint4 *>(src), bytes / 16);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return launch_error(e);
+    return SHA_OK;
+}
+
+}  // extern "C"

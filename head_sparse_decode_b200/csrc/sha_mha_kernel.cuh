@@ -1,0 +1,358 @@
+// sha_mha_kernel.cuh -- selective head decode for multi-head attention (G = 1).
+//
+// What one thread block does.  It owns a contiguous range of key tiles (see
+// sha_schedule.cuh) and walks it one unit (batch row b, selected head h) at a
+// time, as in Algorithm 1, "Selective Head Flash Attention (Decode)" (Polar
+// Sparsity, ri.k117.org reproducibility record): head id lookup
+// h = batch_head_index[b, k], query row Q[b, h], then the tiles of
+// K[b, h], V[b, h] with an online softmax, and finally O written to
+// out[b, h] only.  Heads that are not selected are never touched.
+//
+// How, on sm_100a.  The kernel is bound by HBM bandwidth (about one flop per
+// byte), so the design is about keeping bytes in flight:
+//   * one producer lane issues 1-D bulk async copies (cp.async.bulk) of each
+//     K and V tile -- kTile rows of the head's contiguous [N_kv, d] block --
+//     into a kStages-deep shared-memory ring, completion counted on an
+//     mbarrier per stage; the ring refills while consumers compute and
+//     across unit boundaries;
+//   * kConsumerWarps warps each take kTile/kConsumerWarps rows of every tile
+//     and keep their OWN running (m, l, O) state for the unit, so a tile
+//     needs no block-wide reduction; the warps' states are merged once per
+//     unit (log-sum-exp);
+//   * scores q.k: 8 lanes per key row, each lane holding 8*(d/64) elements of
+//     q in registers, reduced with 3 shuffles; the 16-byte shared loads of 8
+//     lanes cover 128 consecutive bytes, so they are free of bank conflicts;
+//   * P.V: d/8 lanes per row, one 16-byte vector each, fp32 accumulators;
+//   * q is pre-multiplied by scale*log2(e) so every weight is one exp2f.
+// The pages' Algorithm 1 renormalises O after every tile; this kernel keeps
+// O unnormalised and divides once at the end, which is the same quantity.
+#pragma once
+
+#include "sha_device.cuh"
+#include "sha_schedule.cuh"
+
+namespace sha {
+
+// Sticky device status (one per device per loaded library).
+static __device__ unsigned int g_sha_status;
+
+struct DecodeParams {
+    const void *q;
+    const void *k;
+    const void *v;
+    const int32_t *idx;
+    void *out;
+    int B, H_q, H_kv, N_kv, top_k;
+    float scale_log2;        // scale * log2(e)
+    Schedule sched;
+    float *slots;            // 2*num_ctas partial states of slot_floats floats
+    int slot_floats;
+    int *counters;           // one arrival counter per unit, zero between calls
+};
+
+template <int D>
+struct MhaConfig {
+    static constexpr int kConsumerWarps = 8;
+    static constexpr int kConsumers = kConsumerWarps * 32;
+    static constexpr int kThreads = kConsumers + 32;   // + one producer warp
+    static constexpr int kTile = 64;                   // keys per tile
+    static constexpr int kStages = 4;
+    static constexpr int kRowsPerWarp = kTile / kConsumerWarps;
+    static constexpr int kPasses = kRowsPerWarp / 4;   // score passes of 4 rows
+    static constexpr int kQkChunks = D / 64;           // 16-byte chunks per lane (scores)
+    static constexpr int kPvLanesPerRow = D / 8;
+    static constexpr int kPvRowsPerIter = 32 / kPvLanesPerRow;
+    static constexpr int kPvIters = kRowsPerWarp / kPvRowsPerIter;
+    static constexpr int kRowBytes = D * 2;
+    static constexpr int kTileBytes = kTile * kRowBytes;
+    static constexpr int kStateFloats = D + 2;         // O[0..D), m, l
+    static constexpr int kKOffset = 0;
+    static constexpr int kVOffset = kStages * kTileBytes;
+    static constexpr int kBarOffset = 2 * kStages * kTileBytes;
+    static constexpr int kFlagOffset = kBarOffset + 2 * kStages * 8;
+    static constexpr int kStateOffset = kFlagOffset + 16;
+    static constexpr int kSmemBytes = kStateOffset + kConsumerWarps * kStateFloats * 4;
+    static_assert(kRowsPerWarp % 4 == 0, "score passes cover 4 rows");
+    static_assert(kRowsPerWarp % kPvRowsPerIter == 0, "P.V iterations");
+    static_assert(kConsumers >= D, "one consumer thread per output element");
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(MhaConfig<D>::kThreads, 1)
+    sha_mha_decode_kernel(const DecodeParams p)
+{
+    using C = MhaConfig<D>;
+    extern __shared__ __align__(1024) unsigned char smem[];
+    unsigned char *k_ring = smem + C::kKOffset;
+    unsigned char *v_ring = smem + C::kVOffset;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOffset);
+    uint64_t *empty = full + C::kStages;
+    volatile int *flags = reinterpret_cast<volatile int *>(smem + C::kFlagOffset);
+    float *wstate = reinterpret_cast<float *>(smem + C::kStateOffset);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], C::kConsumerWarps);
+        }
+        flags[0] = 0;   // abort: a wait gave up
+        flags[1] = 0;   // this block merges the current unit
+        mbar_init_fence();
+    }
+    __syncthreads();
+
+    const Schedule S = p.sched;
+    const long long t_begin = S.begin(blockIdx.x);
+    const long long t_end = S.begin(blockIdx.x + 1);
+
+    // ------------------------------------------------------------ producer
+    if (warp == C::kConsumerWarps) {
+        if (lane != 0) return;
+        const uint64_t policy = l2_policy_evict_first();
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t last_parity = 0, used = 0;   // per-stage parity of the last copy, stages used
+        bool ok = true;
+        for (long long t = t_begin; t < t_end && ok;) {
+            const Segment seg = segment_at(S, t, t_end);
+            t += seg.num_tiles;
+            const int b = (int)(seg.unit / p.top_k);
+            const int h = p.idx[seg.unit];
+            if ((unsigned)h >= (unsigned)p.H_kv) continue;
+            const size_t head = ((size_t)b * p.H_kv + h) * (size_t)p.N_kv * D;
+            const T *kbase = static_cast<const T *>(p.k) + head;
+            const T *vbase = static_cast<const T *>(p.v) + head;
+            for (int j = seg.first_tile; j < seg.first_tile + seg.num_tiles; ++j) {
+                if (flags[0]) { ok = false; break; }
+                if (!mbar_wait(&empty[stage], phase ^ 1)) {
+                    atomicOr(&g_sha_status, kStatusTimeout);
+                    flags[0] = 1;
+                    ok = false;
+                    break;
+                }
+                const int n0 = j * C::kTile;
+                const int rows = min(C::kTile, p.N_kv - n0);
+                const uint32_t bytes = (uint32_t)rows * C::kRowBytes;
+                mbar_arrive_expect_tx(&full[stage], 2 * bytes);
+                bulk_copy_g2s(k_ring + stage * C::kTileBytes, kbase + (size_t)n0 * D, bytes,
+                              &full[stage], policy);
+                bulk_copy_g2s(v_ring + stage * C::kTileBytes, vbase + (size_t)n0 * D, bytes,
+                              &full[stage], policy);
+                last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+                used |= 1u << stage;
+                if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+            }
+        }
+        // Never leave the block with a copy still landing in shared memory.
+        for (int s = 0; s < C::kStages; ++s)
+            if (used & (1u << s)) mbar_wait(&full[s], (last_parity >> s) & 1u);
+        return;
+    }
+
+    // ------------------------------------------------------------ consumers
+    const int tid = threadIdx.x;            // 0 .. kConsumers-1
+    const int part = lane & 7;              // score lanes: 8 per row
+    const int grp = lane >> 3;
+    const int pv_chunk = lane % C::kPvLanesPerRow;
+    const int pv_row = lane / C::kPvLanesPerRow;
+    const unsigned FULL = 0xffffffffu;
+
+    int stage = 0;
+    uint32_t phase = 0;
+
+    for (long long t = t_begin; t < t_end;) {
+        const Segment seg = segment_at(S, t, t_end);
+        t += seg.num_tiles;
+        const long long u = seg.unit;
+        const int b = (int)(u / p.top_k);
+        const int h = p.idx[u];
+        if ((unsigned)h >= (unsigned)p.H_kv) {
+            if (tid == 0) atomicOr(&g_sha_status, kStatusBadIndex);
+            continue;
+        }
+
+        // query row of head h, pre-scaled by scale*log2(e)
+        float q[C::kQkChunks * 8];
+        {
+            const T *qrow = static_cast<const T *>(p.q) + ((size_t)b * p.H_q + h) * D;
+#pragma unroll
+            for (int i = 0; i < C::kQkChunks; ++i) {
+                const uint4 raw = *reinterpret_cast<const uint4 *>(qrow + (part + 8 * i) * 8);
+                float f[8];
+                widen8<T>(raw, f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) q[i * 8 + e] = f[e] * p.scale_log2;
+            }
+        }
+
+        float m_run = -INFINITY, l_run = 0.f;
+        float o[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] = 0.f;
+
+        for (int j = seg.first_tile; j < seg.first_tile + seg.num_tiles; ++j) {
+            bool live = !__any_sync(FULL, flags[0] != 0);
+            if (live) {
+                live = __all_sync(FULL, mbar_wait(&full[stage], phase));
+                if (!live && lane == 0) {
+                    atomicOr(&g_sha_status, kStatusTimeout);
+                    flags[0] = 1;
+                }
+            }
+            if (live) {
+                const int rows = min(C::kTile, p.N_kv - j * C::kTile);
+                const unsigned char *kt = k_ring + stage * C::kTileBytes;
+                const unsigned char *vt = v_ring + stage * C::kTileBytes;
+                const int row0 = warp * C::kRowsPerWarp;
+
+                // scores, already in log2 units
+                float sc[C::kPasses];
+#pragma unroll
+                for (int ps = 0; ps < C::kPasses; ++ps) {
+                    const int r = row0 + ps * 4 + grp;
+                    float acc = 0.f;
+#pragma unroll
+                    for (int i = 0; i < C::kQkChunks; ++i) {
+                        const uint4 raw = *reinterpret_cast<const uint4 *>(
+                            kt + r * C::kRowBytes + (part + 8 * i) * 16);
+                        float f[8];
+                        widen8<T>(raw, f);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) acc = fmaf(q[i * 8 + e], f[e], acc);
+                    }
+                    acc += __shfl_xor_sync(FULL, acc, 1);
+                    acc += __shfl_xor_sync(FULL, acc, 2);
+                    acc += __shfl_xor_sync(FULL, acc, 4);
+                    sc[ps] = (r < rows) ? acc : -INFINITY;
+                }
+
+                // online softmax over this warp's rows of the tile
+                float mt = sc[0];
+#pragma unroll
+                for (int ps = 1; ps < C::kPasses; ++ps) mt = fmaxf(mt, sc[ps]);
+                mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 8));
+                mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 16));
+                const float m_new = fmaxf(m_run, mt);
+                const float m_ref = (m_new == -INFINITY) ? 0.f : m_new;
+                const float alpha = exp2f(m_run - m_ref);
+                float pw[C::kPasses];
+                float ls = 0.f;
+#pragma unroll
+                for (int ps = 0; ps < C::kPasses; ++ps) {
+                    pw[ps] = exp2f(sc[ps] - m_ref);
+                    ls += pw[ps];
+                }
+                ls += __shfl_xor_sync(FULL, ls, 8);
+                ls += __shfl_xor_sync(FULL, ls, 16);
+                l_run = l_run * alpha + ls;
+                m_run = m_new;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o[e] *= alpha;
+
+                // O += P V over this warp's rows
+#pragma unroll
+                for (int it = 0; it < C::kPvIters; ++it) {
+                    const int lr = it * C::kPvRowsPerIter + pv_row;
+                    const int ps = (it * C::kPvRowsPerIter) / 4;
+                    const float pr = __shfl_sync(FULL, pw[ps], (lr & 3) * 8);
+                    const int r = row0 + lr;
+                    if (r < rows) {
+                        const uint4 raw = *reinterpret_cast<const uint4 *>(
+                            vt + r * C::kRowBytes + pv_chunk * 16);
+                        float f[8];
+                        widen8<T>(raw, f);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) o[e] = fmaf(pr, f[e], o[e]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+            if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+        }
+
+        // ---- merge: lanes of one warp, then the warps, then (maybe) blocks
+#pragma unroll
+        for (int off = C::kPvLanesPerRow; off < 32; off <<= 1)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) o[e] += __shfl_xor_sync(FULL, o[e], off);
+        float *ws = wstate + warp * C::kStateFloats;
+        if (lane < C::kPvLanesPerRow) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ws[lane * 8 + e] = o[e];
+        }
+        if (lane == 0) {
+            ws[D] = m_run;
+            ws[D + 1] = l_run;
+        }
+        named_barrier(1, C::kConsumers);
+
+        const bool aborted = flags[0] != 0;
+        if (tid < D && !aborted) {
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < C::kConsumerWarps; ++w) M = fmaxf(M, wstate[w * C::kStateFloats + D]);
+            const float M_ref = (M == -INFINITY) ? 0.f : M;
+            float L = 0.f, O = 0.f;
+#pragma unroll
+            for (int w = 0; w < C::kConsumerWarps; ++w) {
+                const float c = exp2f(wstate[w * C::kStateFloats + D] - M_ref);
+                L = fmaf(c, wstate[w * C::kStateFloats + D + 1], L);
+                O = fmaf(c, wstate[w * C::kStateFloats + tid], O);
+            }
+            if (seg.whole) {
+                T *orow = static_cast<T *>(p.out) + ((size_t)b * p.H_q + h) * D;
+                orow[tid] = Elem<T>::from_float(O / L);
+            } else {
+                float *slot = p.slots + (size_t)S.slot_of(blockIdx.x, u) * p.slot_floats;
+                slot[tid] = O;
+                if (tid == 0) {
+                    slot[D] = M;
+                    slot[D + 1] = L;
+                }
+                __threadfence();
+            }
+        }
+        named_barrier(1, C::kConsumers);
+
+        if (!seg.whole) {
+            const int first = S.cta_of(u * S.tiles_per_unit);
+            const int last = S.cta_of((u + 1) * S.tiles_per_unit - 1);
+            if (tid == 0) {
+                int merge = 0;
+                if (!flags[0]) {
+                    const int prev = atomicAdd(&p.counters[u], 1);
+                    merge = (prev == last - first);
+                }
+                flags[1] = merge;
+            }
+            named_barrier(1, C::kConsumers);
+            if (flags[1]) {
+                // Last block to finish its piece: merge all pieces in block order.
+                __threadfence();
+                if (tid < D) {
+                    float M = -INFINITY;
+                    for (int c = first; c <= last; ++c) {
+                        const float *slot = p.slots + (size_t)S.slot_of(c, u) * p.slot_floats;
+                        M = fmaxf(M, __ldcg(slot + D));
+                    }
+                    float L = 0.f, O = 0.f;
+                    for (int c = first; c <= last; ++c) {
+                        const float *slot = p.slots + (size_t)S.slot_of(c, u) * p.slot_floats;
+                        const float w = exp2f(__ldcg(slot + D) - M);
+                        L = fmaf(w, __ldcg(slot + D + 1), L);
+                        O = fmaf(w, __ldcg(slot + tid), O);
+                    }
+                    T *orow = static_cast<T *>(p.out) + ((size_t)b * p.H_q + h) * D;
+                    orow[tid] = Elem<T>::from_float(O / L);
+                }
+                if (tid == 0) p.counters[u] = 0;
+            }
+        }
+    }
+}
+
+}  // namespace sha

@@ -1,0 +1,72 @@
+// sha_schedule.cuh -- how one call's work is cut across thread blocks.
+//
+// The work of a call is B*top_k units (one per selected (batch row, head));
+// each unit's N_kv keys are cut into tiles of kTile keys (the last one
+// partial, as in the pages' tiling of Algorithm 1, "Selective Head Flash
+// Attention (Decode)": kend = min(j*Bc, N_kv)).  All tiles of all units are
+// numbered unit-major, t = unit*tiles_per_unit + j, and the range [0, total)
+// is cut into num_ctas contiguous pieces of equal size (to within one tile),
+// one per thread block.  Every block therefore streams the same number of
+// K/V bytes whatever B, top_k and N_kv are.  A unit whose tiles fall in more
+// than one piece is finished by a log-sum-exp merge of the pieces' partial
+// (m, l, O) states (see the kernels).
+//
+// Everything here is integer arithmetic shared by the host planner and the
+// device code, so both agree on every boundary.
+#pragma once
+
+#include <stdint.h>
+
+namespace sha {
+
+struct Schedule {
+    int tiles_per_unit;      // ceil(N_kv / kTile)
+    long long total_tiles;   // units * tiles_per_unit
+    int num_ctas;            // 1 <= num_ctas <= total_tiles
+
+    // First tile of block c (c in [0, num_ctas]); begin(num_ctas) == total_tiles.
+    __host__ __device__ __forceinline__ long long begin(int c) const
+    {
+        return (long long)c * total_tiles / num_ctas;
+    }
+    // The block whose range holds tile t: the largest c with begin(c) <= t.
+    __host__ __device__ __forceinline__ int cta_of(long long t) const
+    {
+        return (int)(((t + 1) * (long long)num_ctas - 1) / total_tiles);
+    }
+    __host__ __device__ __forceinline__ long long unit_of(long long t) const
+    {
+        return t / tiles_per_unit;
+    }
+    // Partial-state slot of block c's piece of unit u.  A block holds at most
+    // two pieces that are not whole units: the tail of the unit it starts in
+    // (slot 2c) and the head of the unit it ends in (slot 2c+1).
+    __host__ __device__ __forceinline__ int slot_of(int c, long long u) const
+    {
+        return 2 * c + (unit_of(begin(c)) == u ? 0 : 1);
+    }
+};
+
+// One maximal run of a block's tiles that belongs to a single unit.
+struct Segment {
+    long long unit;
+    int first_tile;   // tile index within the unit
+    int num_tiles;
+    bool whole;       // the run covers the whole unit
+};
+
+__host__ __device__ __forceinline__ Segment segment_at(const Schedule &s, long long t,
+                                                       long long t_end)
+{
+    Segment seg;
+    seg.unit = s.unit_of(t);
+    long long unit_begin = seg.unit * s.tiles_per_unit;
+    long long unit_end = unit_begin + s.tiles_per_unit;
+    long long end = unit_end < t_end ? unit_end : t_end;
+    seg.first_tile = (int)(t - unit_begin);
+    seg.num_tiles = (int)(end - t);
+    seg.whole = (t == unit_begin) && (end == unit_end);
+    return seg;
+}
+
+}  // namespace sha

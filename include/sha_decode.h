@@ -1,0 +1,166 @@
+/*
+ * sha_decode.h -- C ABI of the Selective Head Attention (SHA) decode library
+ * (libsha_decode.so, CUDA kernels for sm_100a).
+ *
+ * The operation.  Polar Sparsity (papernotes.org summary, section "Selective
+ * Head Attention (SHA) Kernel"; ri.k117.org reproducibility record,
+ * "Pseudocode" row, Algorithm 1 "Selective Head Flash Attention (Decode)"):
+ * for every batch row b and every slot k < top_k the kernel reads
+ * h = batch_head_index[b, k], streams only that head's K/V cache and writes
+ *
+ *     out[b, h*G + j, :] = softmax(scale * q K^T) V,   q = Q[b, h*G + j, :],
+ *     K = K[b, h, :, :],  V = V[b, h, :, :],  j = 0 .. G-1,  G = H_q / H_kv,
+ *
+ * i.e. the attention equation under "Attention Head 稀疏性" (papernotes.org
+ * summary) for one decode token.  G = 1 is multi-head attention with head
+ * sparsity; G > 1 is grouped-query attention with group sparsity (the pages:
+ * GQA models select KV groups, and a selected group computes all of its query
+ * heads).  Rows of heads that are not selected are neither read nor written:
+ * they keep the caller's contents bit for bit.
+ *
+ * Layout (all row-major, contiguous, one dtype for q, k, v and out):
+ *     q   : [B, H_q, d]            (the decode token's query; [B, H_q, 1, d] is the same memory)
+ *     k,v : [B, H_kv, N_kv, d]     (KV cache)
+ *     out : [B, H_q, d]
+ *     batch_head_index : [B, top_k] int32, KV-head (group) ids in [0, H_kv)
+ * All pointers are DEVICE pointers owned by the caller and must be 16-byte
+ * aligned.  Arithmetic: fp32 accumulation; the result is rounded to the
+ * tensor dtype (round to nearest even).
+ *
+ * Asynchrony.  Every launching call enqueues its kernel(s) on `stream`
+ * (a cudaStream_t; NULL = the legacy default stream) and returns without
+ * synchronising.  Argument errors are detected on the host before any launch
+ * and nothing is enqueued then.
+ *
+ * Head ids out of [0, H_kv) are a device-side condition: that (b, k) slot is
+ * skipped (nothing read, nothing written) and a sticky flag is raised, which
+ * sha_get_device_status() reports.  No kernel traps.
+ */
+#ifndef SHA_DECODE_H
+#define SHA_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SHA_OK = 0,
+    SHA_ERR_INVALID_ARG = 1,   /* null pointer, negative or inconsistent size, non-finite scale */
+    SHA_ERR_UNSUPPORTED = 2,   /* d not in {64, 128}, G = H_q/H_kv > 16, unknown dtype */
+    SHA_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned */
+    SHA_ERR_LAUNCH = 4,        /* a CUDA runtime call failed (see sha_last_cuda_error) */
+    SHA_ERR_BAD_INDEX = 5,     /* device flag: a head id was out of range */
+    SHA_ERR_TIMEOUT = 6,       /* device flag: a pipeline wait gave up (should never happen) */
+    SHA_ERR_WORKSPACE = 7      /* caller workspace too small */
+} sha_status_t;
+
+typedef enum { SHA_FP16 = 0, SHA_BF16 = 1 } sha_dtype_t;
+
+/*
+ * sha_decode -- fp16 selective head decode, the operation above.
+ *   q, k, v, out       : device pointers, fp16, layout above.
+ *   batch_head_index   : device pointer, int32 [B, top_k].
+ *   B >= 0, H_q >= 1, H_kv >= 1 with H_q % H_kv == 0 and H_q / H_kv <= 16,
+ *   N_kv >= 1, d in {64, 128}, 0 <= top_k <= H_kv, scale finite
+ *   (1/sqrt(d) reproduces the pages' softmax(Q K^T / sqrt(d_h))).
+ *   B == 0 or top_k == 0 is a no-op returning SHA_OK.
+ * Scratch: the call may split one head's key range across thread blocks and
+ * then needs a small device workspace (sha_decode_workspace_size bytes); this
+ * entry point keeps one per device, allocated on the first call that needs
+ * it (or a larger one) and reused after.  Calls that share a device and
+ * overlap in time on different streams therefore race on it; use
+ * sha_decode_ex with one workspace per stream for that.
+ * Returns SHA_OK once the kernel is enqueued.
+ */
+sha_status_t sha_decode(const void *q, const void *k, const void *v,
+                        const int32_t *batch_head_index, int B, int H_q,
+                        int H_kv, int N_kv, int d, int top_k, float scale,
+                        void *out, void *stream);
+
+/* sha_decode_bf16 -- the same operation on bfloat16 tensors. */
+sha_status_t sha_decode_bf16(const void *q, const void *k, const void *v,
+                             const int32_t *batch_head_index, int B, int H_q,
+                             int H_kv, int N_kv, int d, int top_k, float scale,
+                             void *out, void *stream);
+
+/*
+ * sha_decode_ex -- explicit dtype, caller-owned workspace, forced partition count.
+ *   dtype           : SHA_FP16 or SHA_BF16.
+ *   workspace       : device pointer, 256-byte aligned, at least
+ *                     sha_decode_workspace_size(...) bytes for the same sizes
+ *                     and num_splits, or NULL when that size is 0.  Its
+ *                     counter area must be zero before the first use; every
+ *                     call leaves it zero again when it completes, so one
+ *                     cudaMemset after allocation is enough.  Calls that use
+ *                     one workspace must not overlap on the device.
+ *   num_splits      : 0 = automatic.  Otherwise the B*top_k*ceil(N_kv/tile)
+ *                     key tiles of the call are cut into exactly this many
+ *                     contiguous, equal (to within one tile) ranges, one per
+ *                     thread block (clamped to the tile count).  A head whose
+ *                     tiles straddle ranges is finished by the last block to
+ *                     complete its part (log-sum-exp merge of the parts, in a
+ *                     fixed order, so results do not depend on timing).
+ * The library allocates nothing here.
+ */
+sha_status_t sha_decode_ex(const void *q, const void *k, const void *v,
+                           const int32_t *batch_head_index, int B, int H_q,
+                           int H_kv, int N_kv, int d, int top_k, float scale,
+                           void *out, sha_dtype_t dtype, void *workspace,
+                           size_t workspace_bytes, int num_splits,
+                           void *stream);
+
+/*
+ * sha_decode_workspace_size -- bytes of workspace sha_decode_ex needs for
+ * these sizes and num_splits (0 = automatic) on the current device.  Host
+ * only; reads the device's SM count.  Returns 0 for sizes sha_decode_ex
+ * would reject.
+ */
+size_t sha_decode_workspace_size(int B, int H_q, int H_kv, int N_kv, int d,
+                                 int top_k, int num_splits);
+
+/*
+ * sha_decode_plan -- how a call with these sizes is cut into thread blocks on
+ * a device with num_sms SMs (host only, no CUDA call).  Writes
+ *   plan[0] = key tiles per selected head   (ceil(N_kv / tile))
+ *   plan[1] = key tiles of the whole call   (B * top_k * plan[0])
+ *   plan[2] = thread blocks launched        (one contiguous tile range each)
+ *   plan[3] = workspace bytes               (0: every head lies in one range)
+ *   plan[4] = keys per tile
+ * Returns the status sha_decode_ex would return for these sizes before any
+ * launch (SHA_OK when they are valid).
+ */
+sha_status_t sha_decode_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k,
+                             int num_splits, int num_sms, int64_t plan[5]);
+
+/*
+ * sha_get_device_status -- synchronises `stream`, then reads and clears the
+ * current device's sticky flags: SHA_ERR_BAD_INDEX if any call since the last
+ * read met an out-of-range head id, SHA_ERR_TIMEOUT if a pipeline wait gave
+ * up, SHA_OK otherwise (SHA_ERR_LAUNCH if the read itself failed).
+ */
+sha_status_t sha_get_device_status(void *stream);
+
+/* Static, human-readable name of a status code. */
+const char *sha_status_string(sha_status_t status);
+
+/* The CUDA error string behind the last SHA_ERR_LAUNCH on this thread. */
+const char *sha_last_cuda_error(void);
+
+/*
+ * sha_copy_bandwidth_probe -- not part of the method: a plain 16-byte
+ * vectorised device copy dst[i] = src[i] over `bytes` bytes (a multiple of
+ * 16, both pointers 16-byte aligned), grid sized to the SM count.  The
+ * benchmark times it in the same process to measure the HBM bandwidth the
+ * SHA kernels are compared against.
+ */
+sha_status_t sha_copy_bandwidth_probe(void *dst, const void *src, size_t bytes,
+                                      void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SHA_DECODE_H */

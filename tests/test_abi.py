@@ -1,0 +1,97 @@
+"""The C-ABI library loads, exports every entry point its header declares, and
+rejects bad arguments on the host before touching a GPU (no compute here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER_DIR = os.path.join(ROOT, "include")
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(HEADER_DIR):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(HEADER_DIR, fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w \*]*?\b(sha_\w+)\s*\(", text, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import head_sparse_decode_b200 as h
+    return h._lib
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for must in ("sha_decode", "sha_decode_bf16", "sha_decode_ex", "sha_decode_workspace_size",
+                 "sha_decode_plan", "sha_get_device_status", "sha_status_string"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    import head_sparse_decode_b200 as h
+    raw = ctypes.CDLL(h.LIBRARY_PATH)
+    for name in _declared_functions():
+        assert hasattr(raw, name), f"{name} declared in include/ but not exported"
+
+
+def test_status_strings(lib):
+    import head_sparse_decode_b200 as h
+    for code in range(8):
+        assert h.sha_status_string(code).startswith("SHA_")
+
+
+_P = ctypes.c_void_p
+
+
+def _call(lib, B=2, H_q=4, H_kv=4, N_kv=16, d=64, top_k=2, scale=0.125, ptr=0x1000,
+          dtype=0, num_splits=0):
+    return lib.sha_decode_ex(ptr, ptr, ptr, ptr, B, H_q, H_kv, N_kv, d, top_k,
+                             ctypes.c_float(scale), ptr, dtype, None, 0, num_splits, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=96), 2), (dict(d=256), 2),                   # unsupported head dim
+    (dict(H_q=6, H_kv=4), 1),                            # H_q not a multiple of H_kv
+    (dict(H_q=68, H_kv=4), 2),                           # G = 17 > 16
+    (dict(top_k=5), 1), (dict(top_k=-1), 1),             # top_k outside [0, H_kv]
+    (dict(N_kv=0), 1), (dict(B=-1), 1),
+    (dict(scale=float("nan")), 1), (dict(scale=float("inf")), 1),
+    (dict(dtype=7), 2),
+    (dict(num_splits=-3), 1),
+    (dict(ptr=0x1008), 3),                               # not 16-byte aligned
+    (dict(ptr=0), 1),                                    # null
+])
+def test_host_rejects_bad_arguments_before_any_launch(lib, kw, code):
+    assert _call(lib, **kw) == code
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(top_k=0), dict(B=0, ptr=0)])
+def test_empty_problem_is_a_no_op(lib, kw):
+    assert _call(lib, **kw) == 0
+
+
+def test_plan_tiles_and_blocks():
+    import head_sparse_decode_b200 as h
+    p = h.sha_decode_plan(64, 72, 72, 1920, 128, 22, num_sms=148)
+    assert p["tiles_per_head"] == -(-1920 // p["tile_keys"])
+    assert p["total_tiles"] == 64 * 22 * p["tiles_per_head"]
+    assert p["blocks"] == 148
+    # forced splits are clamped to the number of tiles
+    p = h.sha_decode_plan(1, 4, 4, 10, 64, 1, num_splits=50, num_sms=148)
+    assert p["total_tiles"] == 1 and p["blocks"] == 1 and p["workspace_bytes"] == 0
+    # one block per head exactly: no partial states, no workspace
+    p = h.sha_decode_plan(4, 8, 8, 640, 128, 2, num_splits=8, num_sms=148)
+    assert p["workspace_bytes"] == 0
+    # heads straddling blocks need counters and partial states
+    p = h.sha_decode_plan(4, 8, 8, 640, 128, 2, num_splits=3, num_sms=148)
+    assert p["workspace_bytes"] > 0
+    with pytest.raises(h.ShaError):
+        h.sha_decode_plan(1, 4, 4, 10, 96, 1)

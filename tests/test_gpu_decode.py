@@ -1,0 +1,183 @@
+"""GPU parity of the CUDA selective-head decode against the float64 oracle,
+called through the C ABI (ctypes binding)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from parity import TOLERANCE, active_mask, check_against_oracle, check_sampled_units, out_bits
+
+pytestmark = pytest.mark.gpu
+
+W = workloads.Workload
+
+
+@pytest.fixture(scope="module")
+def sha():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import head_sparse_decode_b200 as h
+    return h
+
+
+def _on_gpu(w):
+    q, k, v = workloads.make_qkv(w)            # CPU generator: host-reproducible
+    idx = workloads.make_index(w)
+    dev = torch.device("cuda")
+    return q.to(dev), k.to(dev), v.to(dev), idx.to(dev)
+
+
+def _run(sha, w, q, k, v, idx, num_splits=None, out=None):
+    out = workloads.make_out(w, "cuda") if out is None else out
+    if num_splits is None:
+        sha.decode(q, k, v, idx, w.scale, out)
+    else:
+        ws = sha.alloc_workspace(q, k, idx, num_splits)
+        sha.sha_decode_ex(q, k, v, idx, w.scale, out, ws, num_splits)
+    torch.cuda.synchronize()
+    assert sha.sha_get_device_status() == sha.SHA_OK
+    return out
+
+
+def test_tiny_mha(sha):
+    w = workloads.CONFIGS["tiny_mha"]
+    q, k, v, idx = _on_gpu(w)
+    out = _run(sha, w, q, k, v, idx)
+    check_against_oracle(w, q, k, v, idx, out)
+
+
+# several tiles and a ragged tail, both head dims and dtypes
+CASES = [
+    W("mha_a", B=3, H_q=8, H_kv=8, N_kv=200, d=128, top_k=3, dtype="fp16", seed=11),
+    W("mha_b", B=5, H_q=6, H_kv=6, N_kv=1000, d=64, top_k=2, dtype="fp16", seed=12),
+    W("mha_c", B=2, H_q=16, H_kv=16, N_kv=513, d=128, top_k=16, dtype="bf16", seed=13),
+    W("mha_d", B=7, H_q=4, H_kv=4, N_kv=65, d=64, top_k=1, dtype="bf16", seed=14),
+    W("mha_e", B=1, H_q=12, H_kv=12, N_kv=63, d=128, top_k=5, dtype="fp16", seed=15),
+    W("mha_f", B=4, H_q=8, H_kv=8, N_kv=2049, d=128, top_k=4, dtype="fp16", seed=16,
+      index="zipf"),
+]
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_parity_ragged(sha, w):
+    q, k, v, idx = _on_gpu(w)
+    out = _run(sha, w, q, k, v, idx)
+    check_against_oracle(w, q, k, v, idx, out)
+
+
+@pytest.mark.parametrize("splits", [1, 2, 3, 7, 29, 148, 10_000])
+def test_forced_splits_match_oracle(sha, splits):
+    w = W("splits", B=3, H_q=8, H_kv=8, N_kv=777, d=128, top_k=3, dtype="fp16", seed=21)
+    q, k, v, idx = _on_gpu(w)
+    expected, _ = oracle.sha_decode(q.cpu(), k.cpu(), v.cpu(), idx.cpu().numpy(), w.scale,
+                                    w.dtype)
+    out = _run(sha, w, q, k, v, idx, num_splits=splits)
+    check_against_oracle(w, q, k, v, idx, out, expected)
+
+
+def test_workspace_counters_return_to_zero(sha):
+    w = W("ws", B=2, H_q=4, H_kv=4, N_kv=300, d=64, top_k=3, dtype="bf16", seed=22)
+    q, k, v, idx = _on_gpu(w)
+    ws = sha.alloc_workspace(q, k, idx, num_splits=5)
+    out = workloads.make_out(w, "cuda")
+    plan = sha.sha_decode_plan(w.B, w.H_q, w.H_kv, w.N_kv, w.d, w.top_k, 5)
+    assert plan["workspace_bytes"] > 0
+    for _ in range(3):
+        sha.sha_decode_ex(q, k, v, idx, w.scale, out, ws, 5)
+        torch.cuda.synchronize()
+        counters = ws[: 4 * w.units].view(torch.int32)
+        assert int(counters.abs().sum()) == 0
+    check_against_oracle(w, q, k, v, idx, out)
+
+
+def test_repeat_calls_are_bit_identical(sha):
+    w = W("det", B=4, H_q=8, H_kv=8, N_kv=900, d=128, top_k=5, dtype="fp16", seed=23)
+    q, k, v, idx = _on_gpu(w)
+    a = out_bits(_run(sha, w, q, k, v, idx))
+    b = out_bits(_run(sha, w, q, k, v, idx))
+    assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_single_key_returns_value_rows_exactly(sha, dtype):
+    w = W("n1", B=3, H_q=8, H_kv=8, N_kv=1, d=128, top_k=4, dtype=dtype, seed=24)
+    q, k, v, idx = _on_gpu(w)
+    out = _run(sha, w, q, k, v, idx)
+    bits = out_bits(out).reshape(w.B, w.H_q, w.d)
+    vbits = out_bits(v).reshape(w.B, w.H_kv, w.d)
+    for b, row in enumerate(idx.cpu().numpy()):
+        for h in row:
+            assert np.array_equal(bits[b, h], vbits[b, h])
+
+
+def test_top_k_zero_writes_nothing(sha):
+    w = W("k0", B=2, H_q=4, H_kv=4, N_kv=64, d=64, top_k=0, dtype="fp16", seed=25)
+    q, k, v, _ = _on_gpu(w.with_(top_k=1))
+    idx = torch.zeros((w.B, 0), dtype=torch.int32, device="cuda")
+    out = _run(sha, w, q, k, v, idx)
+    assert (out_bits(out) == np.uint16(workloads.SENTINEL["fp16"])).all()
+
+
+def test_all_heads_active_is_dense_attention(sha):
+    """top_k = H (layer 0 runs dense): equal to dense attention everywhere."""
+    w = W("dense", B=2, H_q=8, H_kv=8, N_kv=300, d=128, top_k=8, dtype="fp16", seed=26)
+    q, k, v, idx = _on_gpu(w)
+    out = _run(sha, w, q, k, v, idx)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q.cpu().double().unsqueeze(2), k.cpu().double(), v.cpu().double(),
+        scale=w.scale).squeeze(2)
+    err = (out.cpu().double() - ref).abs().max().item()
+    assert err <= TOLERANCE["fp16"]
+
+
+def test_out_of_range_ids_skip_the_slot_and_raise_the_flag(sha):
+    w = W("bad", B=3, H_q=8, H_kv=8, N_kv=130, d=64, top_k=2, dtype="fp16", seed=27)
+    q, k, v, idx = _on_gpu(w)
+    idx[1, 0] = 8
+    idx[2, 1] = -3
+    out = workloads.make_out(w, "cuda")
+    sha.decode(q, k, v, idx, w.scale, out)
+    assert sha.sha_get_device_status() == sha.SHA_ERR_BAD_INDEX
+    assert sha.sha_get_device_status() == sha.SHA_OK          # read clears it
+    check_against_oracle(w, q, k, v, idx, out)
+
+
+def test_index_order_within_a_row_does_not_matter(sha):
+    w = W("perm", B=4, H_q=8, H_kv=8, N_kv=400, d=128, top_k=4, dtype="fp16", seed=28)
+    q, k, v, idx = _on_gpu(w)
+    a = _run(sha, w, q, k, v, idx)
+    b = _run(sha, w, q, k, v, idx.flip(1).contiguous())
+    # same rows written; values agree to rounding (the block split depends on order)
+    assert np.array_equal(out_bits(a) == workloads.SENTINEL["fp16"],
+                          out_bits(b) == workloads.SENTINEL["fp16"])
+    assert (a.double() - b.double()).abs().max().item() <= TOLERANCE["fp16"]
+
+
+def test_rows_of_other_tensors_are_not_read(sha):
+    """Unselected heads' K/V may hold anything (here NaN): results are unaffected."""
+    w = W("nan", B=2, H_q=8, H_kv=8, N_kv=256, d=128, top_k=3, dtype="fp16", seed=29)
+    q, k, v, idx = _on_gpu(w)
+    expected, _ = oracle.sha_decode(q.cpu(), k.cpu(), v.cpu(), idx.cpu().numpy(), w.scale,
+                                    w.dtype)
+    mask = active_mask(idx.cpu().numpy(), w.B, w.H_kv, 1)
+    k2, v2 = k.clone(), v.clone()
+    k2[torch.from_numpy(~mask).cuda()] = float("nan")
+    v2[torch.from_numpy(~mask).cuda()] = float("nan")
+    out = _run(sha, w, q, k2, v2, idx)
+    check_against_oracle(w, q, k, v, idx, out, expected)
+
+
+# ---------------------------------------------------------------- full-size configs
+
+@pytest.mark.parametrize("name", ["opt66b", "opt66b_dense", "llama2_7b"])
+def test_full_size_config_sampled(sha, name):
+    w = workloads.CONFIGS[name]
+    q, k, v = workloads.make_qkv(w, device="cuda")
+    idx = workloads.make_index(w).cuda()
+    out = workloads.make_out(w, "cuda")
+    sha.decode(q, k, v, idx, w.scale, out)
+    torch.cuda.synchronize()
+    assert sha.sha_get_device_status() == sha.SHA_OK
+    err, n = check_sampled_units(w, q, k, v, idx, out, n_random=48)
+    assert n >= 48
