@@ -46,6 +46,13 @@ struct DeviceInfo {
 std::mutex g_mutex;
 DeviceInfo g_devices[kMaxDevices];
 
+// Workspace of sha_decode / sha_decode_bf16, one per device, grown on demand.
+struct OwnedWorkspace {
+    void *ptr;
+    size_t bytes;
+};
+OwnedWorkspace g_owned[kMaxDevices];
+
 sha_status_t current_device(int *dev, DeviceInfo **info)
 {
     cudaError_t e = cudaGetDevice(dev);
@@ -68,7 +75,7 @@ sha_status_t current_device(int *dev, DeviceInfo **info)
 struct Plan {
     sha::Schedule sched;
     int slot_floats;
-    size_t counter_bytes;   // [units] int32, rounded up to 256 bytes
+    size_t counter_bytes;   // fixed region of sha::kMaxBlocks int32 counters
     size_t slot_bytes;      // 2*num_ctas slots
     size_t workspace_bytes() const { return counter_bytes + slot_bytes; }
 };
@@ -85,12 +92,13 @@ Plan make_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int num_spl
     pl.sched.tiles_per_unit = (N_kv + kTileKeys - 1) / kTileKeys;
     pl.sched.total_tiles = units * pl.sched.tiles_per_unit;
     long long ctas = num_splits > 0 ? num_splits : (long long)num_sms * kBlocksPerSm;
+    if (ctas > sha::kMaxBlocks) ctas = sha::kMaxBlocks;
     if (ctas > pl.sched.total_tiles) ctas = pl.sched.total_tiles;
     if (ctas < 1) ctas = 1;
     pl.sched.num_ctas = (int)ctas;
     // one partial state: G rows of (O[d], m, l), padded to 128 bytes
     pl.slot_floats = ((G * (d + 2)) + 31) / 32 * 32;
-    pl.counter_bytes = ((size_t)units * sizeof(int) + 255) / 256 * 256;
+    pl.counter_bytes = sha::kCounterBytes;
     pl.slot_bytes = (size_t)2 * pl.sched.num_ctas * pl.slot_floats * sizeof(float);
     // every unit held whole by one block: no partial state is needed
     if (pl.sched.total_tiles % pl.sched.num_ctas == 0 &&
@@ -148,10 +156,7 @@ sha_status_t decode_impl(const void *q, const void *k, const void *v, const int3
     const size_t need = pl.workspace_bytes();
 
     if (library_workspace && need > 0) {
-        static struct {
-            void *ptr;
-            size_t bytes;
-        } owned[kMaxDevices] = {};
+        OwnedWorkspace *owned = g_owned;
         std::lock_guard<std::mutex> lock(g_mutex);
         if (owned[dev].bytes < need) {
             size_t bytes = need < (1u << 20) ? (1u << 20) : need;
@@ -288,7 +293,15 @@ sha_status_t sha_get_device_status(void *stream)
     if (e != cudaSuccess) return launch_error(e);
     e = cudaMemcpyToSymbol(sha::g_sha_status, &zero, sizeof zero);
     if (e != cudaSuccess) return launch_error(e);
-    if (flags & sha::kStatusTimeout) return SHA_ERR_TIMEOUT;
+    if (flags & sha::kStatusTimeout) {
+        // an abandoned merge can leave arrival counters raised: clear them
+        int dev;
+        if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices) {
+            std::lock_guard<std::mutex> lock(g_mutex);
+            if (g_owned[dev].ptr) cudaMemset(g_owned[dev].ptr, 0, sha::kCounterBytes);
+        }
+        return SHA_ERR_TIMEOUT;
+    }
     if (flags & sha::kStatusBadIndex) return SHA_ERR_BAD_INDEX;
     return SHA_OK;
 }

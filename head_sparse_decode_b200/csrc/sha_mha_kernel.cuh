@@ -47,7 +47,7 @@ struct DecodeParams {
     Schedule sched;
     float *slots;            // 2*num_ctas partial states of slot_floats floats
     int slot_floats;
-    int *counters;           // one arrival counter per unit, zero between calls
+    int *counters;           // arrival counters, one per block, zero between calls
 };
 
 template <int D>
@@ -324,7 +324,8 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, 1)
             if (tid == 0) {
                 int merge = 0;
                 if (!flags[0]) {
-                    const int prev = atomicAdd(&p.counters[u], 1);
+                    // a split unit's first block is unique to it: its counter slot
+                    const int prev = atomicAdd(&p.counters[first], 1);
                     merge = (prev == last - first);
                 }
                 flags[1] = merge;
@@ -349,7 +350,7 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, 1)
                     T *orow = static_cast<T *>(p.out) + ((size_t)b * p.H_q + h) * D;
                     orow[tid] = Elem<T>::from_float(O / L);
                 }
-                if (tid == 0) p.counters[u] = 0;
+                if (tid == 0) p.counters[first] = 0;
             }
         }
     }

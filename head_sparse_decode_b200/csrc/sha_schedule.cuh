@@ -11,6 +11,14 @@
 // than one piece is finished by a log-sum-exp merge of the pieces' partial
 // (m, l, O) states (see the kernels).
 //
+// A unit split across blocks c_first..c_last is merged by whichever of them
+// finishes last, found with an arrival counter.  Counter c_first belongs to
+// it alone: a block can be the first of at most one split unit (two units
+// starting inside one block's range would put the earlier one wholly inside
+// it).  So one counter per block suffices, in a fixed-size region at the
+// start of the workspace that only ever holds counters, whatever the shape
+// of the call that used the workspace before.
+//
 // Everything here is integer arithmetic shared by the host planner and the
 // device code, so both agree on every boundary.
 #pragma once
@@ -18,6 +26,9 @@
 #include <stdint.h>
 
 namespace sha {
+
+constexpr int kMaxBlocks = 4096;                       // cap on blocks of one call
+constexpr int kCounterBytes = kMaxBlocks * 4;          // counter region, zero between calls
 
 struct Schedule {
     int tiles_per_unit;      // ceil(N_kv / kTile)

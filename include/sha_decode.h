@@ -92,14 +92,18 @@ sha_status_t sha_decode_bf16(const void *q, const void *k, const void *v,
  *   workspace       : device pointer, 256-byte aligned, at least
  *                     sha_decode_workspace_size(...) bytes for the same sizes
  *                     and num_splits, or NULL when that size is 0.  Its
- *                     counter area must be zero before the first use; every
- *                     call leaves it zero again when it completes, so one
- *                     cudaMemset after allocation is enough.  Calls that use
- *                     one workspace must not overlap on the device.
+ *                     first 16 KiB hold arrival counters that must be zero
+ *                     before the first use; every call leaves them zero
+ *                     again when it completes (whatever the sizes of the
+ *                     calls that share the workspace), so one cudaMemset
+ *                     after allocation is enough -- unless a call reported
+ *                     SHA_ERR_TIMEOUT, after which the workspace must be
+ *                     zeroed again.  Calls that use one workspace must not
+ *                     overlap on the device.
  *   num_splits      : 0 = automatic.  Otherwise the B*top_k*ceil(N_kv/tile)
  *                     key tiles of the call are cut into exactly this many
  *                     contiguous, equal (to within one tile) ranges, one per
- *                     thread block (clamped to the tile count).  A head whose
+ *                     thread block (clamped to the tile count and to 4096).  A head whose
  *                     tiles straddle ranges is finished by the last block to
  *                     complete its part (log-sum-exp merge of the parts, in a
  *                     fixed order, so results do not depend on timing).
