@@ -193,6 +193,23 @@ def sha_decode_ex(q, k, v, batch_head_index, scale, out, workspace=None, num_spl
     return out
 
 
+_lib.sha_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_float,
+                                    _vp, _i, _i, _vp]
+_lib.sha_decode_noalloc.restype = _i
+NOALLOC_SCRATCH_BYTES = 512 * 1024
+
+
+def sha_decode_noalloc(q, k, v, batch_head_index, scale, out, num_splits=0, stream=None):
+    """Multi-head decode for callers that cannot allocate device memory: the
+    library keeps the split-merge scratch in a fixed 512 KiB device array
+    instead of a workspace, so the call allocates nothing.  Calls on one device
+    share that array: do not let them overlap on the GPU."""
+    args, s = _decode_args(q, k, v, batch_head_index, scale, out, stream)
+    with torch.cuda.device(k.device):
+        _check(_lib.sha_decode_noalloc(*args, _dtype_code(k.dtype), int(num_splits), s))
+    return out
+
+
 def decode(q, k, v, batch_head_index, scale=None, out=None, stream=None):
     """Selective head decode for either dtype; allocates ``out`` if not given
     (rows of unselected heads are then uninitialised)."""
@@ -234,5 +251,5 @@ def sha_copy_bandwidth_probe(dst, src, stream=None):
 __all__ = [
     "sha_decode", "sha_decode_bf16", "sha_decode_ex", "sha_decode_workspace_size",
     "sha_get_device_status", "sha_status_string", "sha_decode_plan", "sha_copy_bandwidth_probe", "decode",
-    "alloc_workspace", "ShaError", "LIBRARY_PATH",
+    "alloc_workspace", "ShaError", "LIBRARY_PATH", "sha_decode_noalloc",
 ]

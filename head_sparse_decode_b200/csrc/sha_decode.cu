@@ -340,3 +340,71 @@ sha_status_t sha_copy_bandwidth_probe(void *dst, const void *src, size_t bytes, 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode without allocation: the multi-head kernel with its split-merge
+// scratch (arrival counters + partial states) in a fixed static device array
+// instead of a cudaMalloc'd workspace.  Every GPU that loads this library
+// holds the array until the process exits.
+
+namespace {
+
+// Scratch of sha_decode_noalloc.  In host code this name is only a stand-in
+// for the symbol: the device address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SHA_NOALLOC_SCRATCH_BYTES];
+
+void *g_noalloc_scratch_ptr[kMaxDevices];
+
+// Once per device, with that device current: the array's device address.
+sha_status_t noalloc_scratch_address(int dev, void **ptr)
+{
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!g_noalloc_scratch_ptr[dev]) {
+        void *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return launch_error(e);
+        g_noalloc_scratch_ptr[dev] = p;
+    }
+    *ptr = g_noalloc_scratch_ptr[dev];
+    return SHA_OK;
+}
+
+}  // namespace
+
+extern "C" sha_status_t sha_decode_noalloc(const void *q, const void *k, const void *v,
+                                           const int32_t *batch_head_index, int B, int H_q,
+                                           int H_kv, int N_kv, int d, int top_k, float scale,
+                                           void *out, sha_dtype_t dtype, int num_splits,
+                                           void *stream)
+{
+    // every host-side check before the first CUDA call
+    if (dtype != SHA_FP16 && dtype != SHA_BF16) return SHA_ERR_UNSUPPORTED;
+    sha_status_t st = check_shape(B, H_q, H_kv, N_kv, d, top_k, scale);
+    if (st != SHA_OK) return st;
+    if (num_splits < 0) return SHA_ERR_INVALID_ARG;
+    if (H_q != H_kv) return SHA_ERR_UNSUPPORTED;   // the multi-head kernel only
+    if (B == 0 || top_k == 0) return SHA_OK;
+    if (!q || !k || !v || !batch_head_index || !out) return SHA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        !aligned(batch_head_index, 4))
+        return SHA_ERR_MISALIGNED;
+
+    int dev;
+    DeviceInfo *info;
+    st = current_device(&dev, &info);
+    if (st != SHA_OK) return st;
+    const Plan pl = make_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits, info->num_sms);
+    const size_t need = pl.workspace_bytes();
+    if (need > (size_t)SHA_NOALLOC_SCRATCH_BYTES) return SHA_ERR_WORKSPACE;
+    void *scratch = nullptr;
+    st = noalloc_scratch_address(dev, &scratch);
+    if (st != SHA_OK) return st;
+    if (need > 0) {
+        // the arrival counters must start at zero whatever an earlier call left
+        cudaError_t e = cudaMemsetAsync(scratch, 0, (size_t)pl.sched.num_ctas * sizeof(int),
+                                        static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return launch_error(e);
+    }
+    return decode_impl(q, k, v, batch_head_index, B, H_q, H_kv, N_kv, d, top_k, scale, out,
+                       dtype, scratch, SHA_NOALLOC_SCRATCH_BYTES, num_splits, stream, false);
+}

@@ -163,6 +163,43 @@ const char *sha_last_cuda_error(void);
 sha_status_t sha_copy_bandwidth_probe(void *dst, const void *src, size_t bytes,
                                       void *stream);
 
+/*
+ * sha_decode_noalloc -- the multi-head (H_q == H_kv) decode above for callers
+ * that cannot allocate device memory: for example a serving engine whose
+ * allocator has reserved all of HBM for its KV cache and hands out nothing
+ * else, or a caller that must not pay cudaMalloc's device-wide
+ * synchronisation and latency inside a decode step.  The polar-sparsity
+ * pages have no counterpart to this entry point; it exists only for them.
+ *
+ * It computes what sha_decode_ex computes with the same arguments, but the
+ * scratch that merges a head split across thread blocks lives in a fixed
+ * device array of SHA_NOALLOC_SCRATCH_BYTES inside this library (each GPU
+ * that loads the library holds it until the process exits).  The call makes
+ * no cudaMalloc, cudaFree or other allocating call; q, k, v, the index and
+ * out are still the caller's device buffers, as for sha_decode.
+ *   dtype, num_splits : as for sha_decode_ex.
+ * Limits and rules:
+ *   - G = H_q / H_kv must be 1 (SHA_ERR_UNSUPPORTED otherwise);
+ *   - a call whose scratch (sha_decode_workspace_size for the same sizes and
+ *     num_splits) exceeds SHA_NOALLOC_SCRATCH_BYTES is rejected with
+ *     SHA_ERR_WORKSPACE before anything is enqueued; with num_splits = 0 this
+ *     happens only on GPUs with more than 396 SMs (d = 128);
+ *   - the first call on a device looks the array's address up once
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture;
+ *   - every call on a device shares the one array, which keeps whatever the
+ *     last call left in it.  Each call clears the arrival counters it uses
+ *     (a cudaMemsetAsync on `stream`) before its kernel; partial states need
+ *     no clearing.  Calls that overlap on the GPU (other streams, other host
+ *     threads) race on the array and give wrong results: serialise them.
+ */
+#define SHA_NOALLOC_SCRATCH_BYTES (512 * 1024)
+sha_status_t sha_decode_noalloc(const void *q, const void *k, const void *v,
+                                const int32_t *batch_head_index, int B, int H_q,
+                                int H_kv, int N_kv, int d, int top_k, float scale,
+                                void *out, sha_dtype_t dtype, int num_splits,
+                                void *stream);
+
 #ifdef __cplusplus
 }
 #endif
