@@ -9,6 +9,8 @@ layer, one decode token per sequence) on the OPT-66B-shaped workload: B=64,
 H=72, d=128, N_kv=1920, top_k=22 (30 % head density), fp16, N(0,1) data.
 Inputs are resident in HBM when the timed region starts; the active K/V of a
 step (1.39 GB) is 11x the 126 MB L2, so no flush is needed between steps.
+Device-timed steps are launched by replaying CUDA graphs of 100 steps, as the
+pages measure decode throughput under CUDA graphs; e2e calls the API eagerly.
 
 value    = algorithmic bytes of all ranks' steps / max-over-ranks device time
            (active K+V, active Q rows read, active O rows written, the index)
@@ -202,6 +204,34 @@ def timed(fn, steps, stream):
     return start.elapsed_time(end) / 1e3   # seconds
 
 
+def capture_graph(fn, n, dev):
+    """n calls of fn captured into one CUDA graph (fn already warmed up)."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(n):
+            fn()
+    return g
+
+
+def timed_graphs(fn, steps, dev, stream, chunk=100):
+    """Exactly `steps` calls of fn, launched by replaying CUDA graphs of up to
+    `chunk` calls (the pages measure decode throughput under CUDA graphs), timed
+    with events on `stream`.  Returns seconds."""
+    chunk = max(1, min(chunk, steps))
+    g_main = capture_graph(fn, chunk, dev)
+    rem = steps % chunk
+    g_rem = capture_graph(fn, rem, dev) if rem else None
+    g_main.replay()                       # first replay uploads the graph
+    torch.cuda.synchronize(dev)
+
+    def run():
+        for _ in range(steps // chunk):
+            g_main.replay()
+        if g_rem is not None:
+            g_rem.replay()
+    return timed(run, 1, stream)
+
+
 def sync_all(world, local):
     torch.cuda.synchronize()
     if world > 1:
@@ -263,7 +293,7 @@ def run_ours(args, rank, world, local):
         step()
     sync_all(world, local)
     t0 = time.time()
-    elapsed = timed(step, args.steps, stream)
+    elapsed = timed_graphs(step, args.steps, dev, stream)
     t1 = time.time()
     sync_all(world, local)
     clocks = sampler.stop(t0, t1)
@@ -283,6 +313,7 @@ def run_ours(args, rank, world, local):
     if not args.no_extras:
         extras["density_sweep"] = density_sweep(sha, w, q, k, v, dev, stream, peak)
         extras["e2e"] = e2e(sha, w, q, k, v, idx, out, dev, stream, args)
+        extras["other_configs"] = other_configs(sha, w, dev, stream, peak, rank)
     plan = sha.sha_decode_plan(w.B, w.H_q, w.H_kv, w.N_kv, w.d, w.top_k,
                                num_sms=torch.cuda.get_device_properties(dev).multi_processor_count)
     line = {
@@ -294,7 +325,8 @@ def run_ours(args, rank, world, local):
         "config": {**w.describe(), "parallelism": f"replicas x{world} (batch sharded by rank)",
                    "accumulation": "fp32", "l2": "no flush: active K/V per step "
                    f"{w.units * 2 * w.N_kv * w.d * 2 / 1e9:.2f} GB > 126 MB L2",
-                   "blocks": plan["blocks"], "tile_keys": plan["tile_keys"]},
+                   "blocks": plan["blocks"], "tile_keys": plan["tile_keys"],
+                   "launch": "CUDA graph replay, 100 steps per graph"},
         "steps_per_s": round(args.steps / t_max, 2),
         "tokens_per_s": round(world * w.B * args.steps / t_max, 1),
         "hbm_frac_of_measured": round(achieved / peak, 4),
@@ -304,7 +336,8 @@ def run_ours(args, rank, world, local):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": profiled_traffic(w.name), "peak_source": peak_src,
-                     "kernel": "sha_mha_decode_kernel", "launch_us": round(launch_s * 1e6, 3),
+                     "kernel": "sha_mha_decode_kernel" if w.G == 1 else "sha_gqa_decode_kernel",
+                     "launch_us": round(launch_s * 1e6, 3),
                      "bytes_per_launch": bytes_step},
     }
     if "e2e" in extras:
@@ -326,7 +359,7 @@ def density_sweep(sha, w, q, k, v, dev, stream, peak):
         for _ in range(20):
             sha.decode(q, k, v, idx, w.scale, out)
         steps = 300
-        t = timed(lambda: sha.decode(q, k, v, idx, w.scale, out), steps, stream)
+        t = timed_graphs(lambda: sha.decode(q, k, v, idx, w.scale, out), steps, dev, stream)
         gbs = wk.algorithmic_bytes() * steps / t / 1e9
         res.append({"top_k": top_k, "density": round(top_k / w.H_kv, 4),
                     "us_per_step": round(t / steps * 1e6, 2), "gbs": round(gbs, 1),
@@ -334,6 +367,31 @@ def density_sweep(sha, w, q, k, v, dev, stream, peak):
     dense = res[-1]["us_per_step"]
     for r in res:
         r["time_vs_dense"] = round(r["us_per_step"] / dense, 4)
+    return res
+
+
+def other_configs(sha, w_main, dev, stream, peak, rank):
+    """The other full-size workloads, timed the same way (fewer steps)."""
+    res = []
+    for name in ("llama2_7b", "llama31_70b_gqa"):
+        if name == w_main.name:
+            continue
+        w = workloads.CONFIGS[name]
+        w = w.with_(seed=w.seed + 100 * rank)
+        q, k, v = workloads.make_qkv(w, device=dev)
+        idx = workloads.make_index(w).to(dev)
+        out = workloads.make_out(w, dev)
+        for _ in range(20):
+            sha.decode(q, k, v, idx, w.scale, out)
+        steps = 500
+        t = timed_graphs(lambda: sha.decode(q, k, v, idx, w.scale, out), steps, dev, stream)
+        gbs = w.algorithmic_bytes() * steps / t / 1e9
+        res.append({"workload": name, "us_per_step": round(t / steps * 1e6, 2),
+                    "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
+                    "steps_per_s": round(steps / t, 1), "G": w.G, "dtype": w.dtype,
+                    "bytes_per_step": w.algorithmic_bytes()})
+        del q, k, v, idx, out
+        torch.cuda.empty_cache()
     return res
 
 

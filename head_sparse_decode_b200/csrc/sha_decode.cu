@@ -6,8 +6,11 @@
 #include <cstring>
 #include <mutex>
 
+#include <cudaTypedefs.h>
+
 #include "sha_decode.h"
 #include "sha_device.cuh"
+#include "sha_gqa_kernel.cuh"
 #include "sha_mha_kernel.cuh"
 #include "sha_schedule.cuh"
 
@@ -94,6 +97,13 @@ Plan make_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int num_spl
     long long ctas = num_splits > 0 ? num_splits : (long long)num_sms * kBlocksPerSm;
     if (ctas > sha::kMaxBlocks) ctas = sha::kMaxBlocks;
     if (ctas > pl.sched.total_tiles) ctas = pl.sched.total_tiles;
+    // every block gets at least ceil((Tu-1)/(kMaxMergeParts-1)) tiles, so a
+    // unit of Tu tiles is shared by at most kMaxMergeParts blocks
+    const long long min_tiles =
+        (pl.sched.tiles_per_unit - 1 + sha::kMaxMergeParts - 2) / (sha::kMaxMergeParts - 1);
+    if (min_tiles > 1 && ctas > pl.sched.total_tiles / min_tiles)
+        ctas = pl.sched.total_tiles / min_tiles;
+    if (ctas < 1) ctas = 1;
     if (ctas < 1) ctas = 1;
     pl.sched.num_ctas = (int)ctas;
     // one partial state: G rows of (O[d], m, l), padded to 128 bytes
@@ -107,6 +117,81 @@ Plan make_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int num_spl
         pl.slot_bytes = 0;
     }
     return pl;
+}
+
+static_assert(sha::MhaConfig<128>::kTile == kTileKeys && sha::GqaConfig<128>::kTile == kTileKeys,
+              "host plan and kernels agree on the tile");
+
+// cuTensorMapEncodeTiled from the driver, found through the runtime so the
+// library does not link against libcuda.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 3-D view [B*H_kv][N_kv][d] of a K or V cache, 64x64-element boxes with
+// 128-byte swizzle; rows past N_kv read as zero.
+sha_status_t kv_tensor_map(CUtensorMap *map, const void *base, sha_dtype_t dtype, int d,
+                           int N_kv, long long planes)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+    if (!encode) {
+        std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error,
+                      "cuTensorMapEncodeTiled is not available from the driver");
+        return SHA_ERR_LAUNCH;
+    }
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N_kv, (cuuint64_t)planes};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N_kv * d * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)kTileKeys, 1};
+    cuuint32_t elem[3] = {1, 1, 1};
+    CUresult r = encode(map,
+                        dtype == SHA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                          : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                        3, const_cast<void *>(base), dims, strides, box, elem,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error,
+                      "cuTensorMapEncodeTiled failed with CUresult %d", (int)r);
+        return SHA_ERR_LAUNCH;
+    }
+    return SHA_OK;
+}
+
+template <typename T, int D>
+sha_status_t launch_gqa(const sha::DecodeParams &prm, sha_dtype_t dtype, int dev,
+                        cudaStream_t stream)
+{
+    using C = sha::GqaConfig<D>;
+    static bool configured[kMaxDevices] = {};
+    if (!configured[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(sha::sha_gqa_decode_kernel<T, D>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::kSmemBytes);
+        if (e != cudaSuccess) return launch_error(e);
+        configured[dev] = true;
+    }
+    CUtensorMap tm_k, tm_v;
+    const long long planes = (long long)prm.B * prm.H_kv;
+    sha_status_t st = kv_tensor_map(&tm_k, prm.k, dtype, D, prm.N_kv, planes);
+    if (st != SHA_OK) return st;
+    st = kv_tensor_map(&tm_v, prm.v, dtype, D, prm.N_kv, planes);
+    if (st != SHA_OK) return st;
+    sha::sha_gqa_decode_kernel<T, D>
+        <<<prm.sched.num_ctas, C::kThreads, C::kSmemBytes, stream>>>(prm, tm_k, tm_v);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return launch_error(e);
+    return SHA_OK;
 }
 
 template <typename T, int D>
@@ -145,7 +230,6 @@ sha_status_t decode_impl(const void *q, const void *k, const void *v, const int3
         return SHA_ERR_MISALIGNED;
     if (workspace && !aligned(workspace, 256)) return SHA_ERR_MISALIGNED;
     const int G = H_q / H_kv;
-    if (G != 1) return SHA_ERR_UNSUPPORTED;   // grouped-query kernel: not built yet
 
     int dev;
     DeviceInfo *info;
@@ -196,6 +280,13 @@ sha_status_t decode_impl(const void *q, const void *k, const void *v, const int3
                                                  pl.counter_bytes)
                      : nullptr;
 
+    if (G > 1) {
+        if (dtype == SHA_FP16)
+            return d == 128 ? launch_gqa<__half, 128>(prm, dtype, dev, s)
+                            : launch_gqa<__half, 64>(prm, dtype, dev, s);
+        return d == 128 ? launch_gqa<__nv_bfloat16, 128>(prm, dtype, dev, s)
+                        : launch_gqa<__nv_bfloat16, 64>(prm, dtype, dev, s);
+    }
     if (dtype == SHA_FP16)
         return d == 128 ? launch_mha<__half, 128>(prm, dev, s) : launch_mha<__half, 64>(prm, dev, s);
     return d == 128 ? launch_mha<__nv_bfloat16, 128>(prm, dev, s)

@@ -1,0 +1,428 @@
+// sha_gqa_kernel.cuh -- selective decode for grouped-query attention (G > 1).
+//
+// What one thread block does.  As in the multi-head kernel, it walks a
+// contiguous range of key tiles (sha_schedule.cuh).  Here a unit is a batch
+// row b and a selected KV group h (Polar Sparsity, papernotes.org summary,
+// "Selective Head Attention (SHA) Kernel": GQA models select groups); all G
+// query heads h*G .. h*G+G-1 of the group are computed from each K/V tile
+// while it is in shared memory, so the group's cache is read from HBM once.
+//
+// How, on sm_100a.  With G query rows sharing every key, a tile is a small
+// dense contraction (about G flops per byte: 8 for LLaMA-3.1-70B), so the
+// scores and P.V run on the tensor cores with fp32 accumulation:
+//   * one producer lane loads each K and V tile with TMA tensor copies
+//     (cp.async.bulk.tensor, a 3-D map [planes = B*H_kv][N_kv][d] with
+//     64-element boxes and 128-byte swizzle) into a kStages-deep ring; keys
+//     past N_kv are outside the map and arrive as zeros;
+//   * 4 consumer warps take 16 keys of each 64-key tile each and keep their
+//     own online-softmax state for up to 16 query rows;
+//   * S = Q K^T: mma.sync m16n8k16 with Q (G rows, zero-padded to 16) as the
+//     A operand held in registers and K fragments read by ldmatrix from the
+//     swizzled tile (conflict-free);
+//   * P V: the S accumulators, exponentiated, are reused in registers as the
+//     A operand (16 keys = one k-step); V fragments come from ldmatrix.trans;
+//   * warps merge once per unit; units split across blocks merge in the
+//     workspace exactly as in the multi-head kernel.
+#pragma once
+
+#include <cuda.h>
+
+#include "sha_device.cuh"
+#include "sha_merge.cuh"
+#include "sha_mha_kernel.cuh"
+#include "sha_schedule.cuh"
+
+namespace sha {
+
+template <int D>
+struct GqaConfig {
+    static constexpr int kConsumerWarps = 4;
+    static constexpr int kConsumers = kConsumerWarps * 32;
+    static constexpr int kThreads = kConsumers + 32;
+    static constexpr int kTile = 64;                   // keys per tile
+    static constexpr int kKeysPerWarp = kTile / kConsumerWarps;   // 16: one m16n8k16 k-step
+    static constexpr int kStages = 4;
+    static constexpr int kRows = 16;                   // query rows per MMA (G padded)
+    static constexpr int kBoxes = D / 64;              // 128-byte boxes across d
+    static constexpr int kBoxBytes = kTile * 128;
+    static constexpr int kTileBytes = kBoxes * kBoxBytes;
+    static constexpr int kKSteps = D / 16;
+    static constexpr int kONTiles = D / 8;
+    static constexpr int kStateFloats = kRows * (D + 2);
+    static constexpr int kAlignPad = 1024;             // 128-byte swizzle wants 1 KiB alignment
+    static constexpr int kKOffset = 0;
+    static constexpr int kVOffset = kStages * kTileBytes;
+    static constexpr int kBarOffset = 2 * kStages * kTileBytes;
+    static constexpr int kFlagOffset = kBarOffset + 2 * kStages * 8;
+    static constexpr int kStateOffset = kFlagOffset + 16;
+    static constexpr int kSmemBytes =
+        kAlignPad + kStateOffset + kConsumerWarps * kStateFloats * 4;
+    static_assert(kKeysPerWarp == 16, "one k-step of 16 keys per warp");
+    static_assert(kBoxBytes % 1024 == 0, "boxes stay 1 KiB aligned");
+    static_assert(kConsumerWarps * kStateFloats >= 3 * kMaxMergeParts * kRows,
+                  "merge staging fits");
+};
+
+// TMA tiled load of one box of a 3-D tensor map into shared memory.
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int x, int y,
+                                            int z, uint64_t *bar, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar)),
+        "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t (&r)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t (&r)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+// D(16x8, f32) += A(16x16) * B(16x8), 16-bit inputs of type T.
+template <typename T>
+__device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1);
+
+template <>
+__device__ __forceinline__ void mma_16816<__half>(float (&c)[4], const uint32_t (&a)[4],
+                                                  uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7},"
+        " {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <>
+__device__ __forceinline__ void mma_16816<__nv_bfloat16>(float (&c)[4], const uint32_t (&a)[4],
+                                                         uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7},"
+        " {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Two fp32 values rounded to T and packed low/high into one 32-bit register.
+template <typename T> __device__ __forceinline__ uint32_t pack2(float lo, float hi);
+template <> __device__ __forceinline__ uint32_t pack2<__half>(float lo, float hi)
+{
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+template <> __device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float lo, float hi)
+{
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Shared address of 16-byte chunk `chunk` (of d/8) of key row `key` in a
+// tile stored as 128-byte-swizzled boxes of 64 elements.
+template <int D>
+__device__ __forceinline__ uint32_t swizzled(uint32_t tile, int key, int chunk)
+{
+    using C = GqaConfig<D>;
+    const int box = chunk >> 3, c = chunk & 7;
+    return tile + box * C::kBoxBytes + key * 128 + ((c ^ (key & 7)) << 4);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
+    sha_gqa_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v)
+{
+    using C = GqaConfig<D>;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char *k_ring = smem + C::kKOffset;
+    unsigned char *v_ring = smem + C::kVOffset;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOffset);
+    uint64_t *empty = full + C::kStages;
+    volatile int *flags = reinterpret_cast<volatile int *>(smem + C::kFlagOffset);
+    float *wstate = reinterpret_cast<float *>(smem + C::kStateOffset);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int G = p.H_q / p.H_kv;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], C::kConsumerWarps);
+        }
+        flags[0] = 0;
+        flags[1] = 0;
+        mbar_init_fence();
+    }
+    __syncthreads();
+
+    const Schedule S = p.sched;
+    const long long t_begin = S.begin(blockIdx.x);
+    const long long t_end = S.begin(blockIdx.x + 1);
+
+    // ------------------------------------------------------------ producer
+    if (warp == C::kConsumerWarps) {
+        if (lane != 0) return;
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k))
+                     : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v))
+                     : "memory");
+        const uint64_t policy = l2_policy_evict_first();
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t last_parity = 0, used = 0;
+        bool ok = true;
+        for (long long t = t_begin; t < t_end && ok;) {
+            const Segment seg = segment_at(S, t, t_end);
+            t += seg.num_tiles;
+            const int b = (int)(seg.unit / p.top_k);
+            const int h = p.idx[seg.unit];
+            if ((unsigned)h >= (unsigned)p.H_kv) continue;
+            const int plane = b * p.H_kv + h;
+            for (int j = seg.first_tile; j < seg.first_tile + seg.num_tiles; ++j) {
+                if (flags[0]) { ok = false; break; }
+                if (!mbar_wait(&empty[stage], phase ^ 1)) {
+                    atomicOr(&g_sha_status, kStatusTimeout);
+                    flags[0] = 1;
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&full[stage], 2 * C::kTileBytes);
+#pragma unroll
+                for (int bx = 0; bx < C::kBoxes; ++bx) {
+                    tma_load_3d(k_ring + stage * C::kTileBytes + bx * C::kBoxBytes, &tm_k,
+                                bx * 64, j * C::kTile, plane, &full[stage], policy);
+                    tma_load_3d(v_ring + stage * C::kTileBytes + bx * C::kBoxBytes, &tm_v,
+                                bx * 64, j * C::kTile, plane, &full[stage], policy);
+                }
+                last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+                used |= 1u << stage;
+                if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+            }
+        }
+        for (int s = 0; s < C::kStages; ++s)
+            if (used & (1u << s)) mbar_wait(&full[s], (last_parity >> s) & 1u);
+        return;
+    }
+
+    // ------------------------------------------------------------ consumers
+    const int tid = threadIdx.x;
+    const int g = lane >> 2;          // accumulator rows g and g+8
+    const int qd = lane & 3;          // column pair within an 8-wide n-tile
+    const unsigned FULL = 0xffffffffu;
+    const uint32_t k_base = smem_addr(k_ring), v_base = smem_addr(v_ring);
+    // ldmatrix row addresses: lane -> (matrix lane>>3, row lane&7)
+    const int mi = lane >> 3, mr = lane & 7;
+    const int key_k = warp * C::kKeysPerWarp + (mi >> 1) * 8 + mr;   // K: matrices (keys, d-chunk)
+    const int key_v = warp * C::kKeysPerWarp + (mi & 1) * 8 + mr;    // V: matrices (keys, d-chunk)
+
+    int stage = 0;
+    uint32_t phase = 0;
+
+    for (long long t = t_begin; t < t_end;) {
+        const Segment seg = segment_at(S, t, t_end);
+        t += seg.num_tiles;
+        const long long u = seg.unit;
+        const int b = (int)(u / p.top_k);
+        const int h = p.idx[u];
+        if ((unsigned)h >= (unsigned)p.H_kv) {
+            if (tid == 0) atomicOr(&g_sha_status, kStatusBadIndex);
+            continue;
+        }
+
+        // Q of the group as the MMA's A operand: rows g, g+8 (zero past G)
+        uint32_t qa[C::kKSteps][4];
+        {
+            const T *qg = static_cast<const T *>(p.q) + ((size_t)b * p.H_q + (size_t)h * G) * D;
+            const bool r0 = g < G, r1 = g + 8 < G;
+#pragma unroll
+            for (int ks = 0; ks < C::kKSteps; ++ks) {
+                const int c0 = ks * 16 + qd * 2;
+                qa[ks][0] = r0 ? *reinterpret_cast<const uint32_t *>(qg + g * D + c0) : 0u;
+                qa[ks][1] = r1 ? *reinterpret_cast<const uint32_t *>(qg + (g + 8) * D + c0) : 0u;
+                qa[ks][2] = r0 ? *reinterpret_cast<const uint32_t *>(qg + g * D + c0 + 8) : 0u;
+                qa[ks][3] =
+                    r1 ? *reinterpret_cast<const uint32_t *>(qg + (g + 8) * D + c0 + 8) : 0u;
+            }
+        }
+
+        float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+        float o[C::kONTiles][4];
+#pragma unroll
+        for (int n = 0; n < C::kONTiles; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+
+        for (int j = seg.first_tile; j < seg.first_tile + seg.num_tiles; ++j) {
+            bool live = !__any_sync(FULL, flags[0] != 0);
+            if (live) {
+                live = __all_sync(FULL, mbar_wait(&full[stage], phase));
+                if (!live && lane == 0) {
+                    atomicOr(&g_sha_status, kStatusTimeout);
+                    flags[0] = 1;
+                }
+            }
+            if (live) {
+                const uint32_t kt = k_base + stage * C::kTileBytes;
+                const uint32_t vt = v_base + stage * C::kTileBytes;
+                const int rows = min(C::kTile, p.N_kv - j * C::kTile);
+
+                // S = Q K^T over this warp's 16 keys: two 8-key n-tiles
+                float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+                for (int ks = 0; ks < C::kKSteps; ++ks) {
+                    uint32_t kb[4];
+                    ldmatrix_x4(swizzled<D>(kt, key_k, ks * 2 + (mi & 1)), kb);
+                    mma_16816<T>(s[0], qa[ks], kb[0], kb[1]);
+                    mma_16816<T>(s[1], qa[ks], kb[2], kb[3]);
+                }
+
+                // online softmax on rows g (entries 0,1) and g+8 (entries 2,3)
+                float mt[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int key = warp * C::kKeysPerWarp + nt * 8 + qd * 2 + (e & 1);
+                        s[nt][e] = key < rows ? s[nt][e] * p.scale_log2 : -INFINITY;
+                        mt[e >> 1] = fmaxf(mt[e >> 1], s[nt][e]);
+                    }
+                float alpha[2], ref[2];
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    mt[r] = fmaxf(mt[r], __shfl_xor_sync(FULL, mt[r], 1));
+                    mt[r] = fmaxf(mt[r], __shfl_xor_sync(FULL, mt[r], 2));
+                    const float m_new = fmaxf(m_run[r], mt[r]);
+                    ref[r] = (m_new == -INFINITY) ? 0.f : m_new;
+                    alpha[r] = exp2f(m_run[r] - ref[r]);
+                    m_run[r] = m_new;
+                    l_run[r] *= alpha[r];
+                }
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        s[nt][e] = exp2f(s[nt][e] - ref[e >> 1]);
+                        l_run[e >> 1] += s[nt][e];
+                    }
+#pragma unroll
+                for (int n = 0; n < C::kONTiles; ++n) {
+                    o[n][0] *= alpha[0];
+                    o[n][1] *= alpha[0];
+                    o[n][2] *= alpha[1];
+                    o[n][3] *= alpha[1];
+                }
+                uint32_t pa[4];
+                pa[0] = pack2<T>(s[0][0], s[0][1]);
+                pa[1] = pack2<T>(s[0][2], s[0][3]);
+                pa[2] = pack2<T>(s[1][0], s[1][1]);
+                pa[3] = pack2<T>(s[1][2], s[1][3]);
+
+                // O += P V: 16 keys x d, two 8-wide n-tiles per ldmatrix
+#pragma unroll
+                for (int dn = 0; dn < D / 16; ++dn) {
+                    uint32_t vb[4];
+                    ldmatrix_x4_trans(swizzled<D>(vt, key_v, dn * 2 + (mi >> 1)), vb);
+                    mma_16816<T>(o[2 * dn], pa, vb[0], vb[1]);
+                    mma_16816<T>(o[2 * dn + 1], pa, vb[2], vb[3]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+            if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+        }
+
+        // ---- merge: the quad's partial sums, then warps, then (maybe) blocks
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            l_run[r] += __shfl_xor_sync(FULL, l_run[r], 1);
+            l_run[r] += __shfl_xor_sync(FULL, l_run[r], 2);
+        }
+        float *ws = wstate + warp * C::kStateFloats;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int row = g + 8 * r;
+            if (row < G) {
+#pragma unroll
+                for (int n = 0; n < C::kONTiles; ++n) {
+                    ws[row * (D + 2) + n * 8 + qd * 2] = o[n][2 * r];
+                    ws[row * (D + 2) + n * 8 + qd * 2 + 1] = o[n][2 * r + 1];
+                }
+                if (qd == 0) {
+                    ws[row * (D + 2) + D] = m_run[r];
+                    ws[row * (D + 2) + D + 1] = l_run[r];
+                }
+            }
+        }
+        named_barrier(1, C::kConsumers);
+
+        T *out_g = static_cast<T *>(p.out) + ((size_t)b * p.H_q + (size_t)h * G) * D;
+        const bool aborted = flags[0] != 0;
+        float *slot = p.slots ? p.slots + (size_t)S.slot_of(blockIdx.x, u) * p.slot_floats
+                              : nullptr;
+        if (!aborted) {
+            for (int e = tid; e < G * D; e += C::kConsumers) {
+                const int row = e / D, c = e - row * D;
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < C::kConsumerWarps; ++w)
+                    M = fmaxf(M, wstate[w * C::kStateFloats + row * (D + 2) + D]);
+                const float M_ref = (M == -INFINITY) ? 0.f : M;
+                float L = 0.f, O = 0.f;
+#pragma unroll
+                for (int w = 0; w < C::kConsumerWarps; ++w) {
+                    const float *st = wstate + w * C::kStateFloats + row * (D + 2);
+                    const float cw = exp2f(st[D] - M_ref);
+                    L = fmaf(cw, st[D + 1], L);
+                    O = fmaf(cw, st[c], O);
+                }
+                if (seg.whole) {
+                    out_g[e] = Elem<T>::from_float(O / L);
+                } else {
+                    slot[e] = O;
+                    if (c == 0) {
+                        slot[G * D + row] = M;
+                        slot[G * D + G + row] = L;
+                    }
+                }
+            }
+            if (!seg.whole) __threadfence();
+        }
+        named_barrier(1, C::kConsumers);
+
+        if (!seg.whole) {
+            const int first = S.cta_of(u * S.tiles_per_unit);
+            const int last = S.cta_of((u + 1) * S.tiles_per_unit - 1);
+            if (tid == 0) {
+                int merge = 0;
+                if (!flags[0]) {
+                    const int prev = atomicAdd(&p.counters[first], 1);
+                    merge = (prev == last - first);
+                }
+                flags[1] = merge;
+            }
+            named_barrier(1, C::kConsumers);
+            if (flags[1]) {
+                __threadfence();
+                merge_parts<T, D, C::kConsumers>(p.slots, p.slot_floats, first,
+                                                  S.slot_of(first, u), last - first + 1, G,
+                                                  out_g, wstate, tid);
+                if (tid == 0) p.counters[first] = 0;
+            }
+        }
+    }
+}
+
+}  // namespace sha

@@ -29,6 +29,7 @@
 #pragma once
 
 #include "sha_device.cuh"
+#include "sha_merge.cuh"
 #include "sha_schedule.cuh"
 
 namespace sha {
@@ -75,6 +76,7 @@ struct MhaConfig {
     static_assert(kRowsPerWarp % 4 == 0, "score passes cover 4 rows");
     static_assert(kRowsPerWarp % kPvRowsPerIter == 0, "P.V iterations");
     static_assert(kConsumers >= D, "one consumer thread per output element");
+    static_assert(kConsumerWarps * kStateFloats >= 3 * kMaxMergeParts, "merge staging fits");
 };
 
 template <typename T, int D>
@@ -334,22 +336,10 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, 1)
             if (flags[1]) {
                 // Last block to finish its piece: merge all pieces in block order.
                 __threadfence();
-                if (tid < D) {
-                    float M = -INFINITY;
-                    for (int c = first; c <= last; ++c) {
-                        const float *slot = p.slots + (size_t)S.slot_of(c, u) * p.slot_floats;
-                        M = fmaxf(M, __ldcg(slot + D));
-                    }
-                    float L = 0.f, O = 0.f;
-                    for (int c = first; c <= last; ++c) {
-                        const float *slot = p.slots + (size_t)S.slot_of(c, u) * p.slot_floats;
-                        const float w = exp2f(__ldcg(slot + D) - M);
-                        L = fmaf(w, __ldcg(slot + D + 1), L);
-                        O = fmaf(w, __ldcg(slot + tid), O);
-                    }
-                    T *orow = static_cast<T *>(p.out) + ((size_t)b * p.H_q + h) * D;
-                    orow[tid] = Elem<T>::from_float(O / L);
-                }
+                T *orow = static_cast<T *>(p.out) + ((size_t)b * p.H_q + h) * D;
+                merge_parts<T, D, C::kConsumers>(p.slots, p.slot_floats, first,
+                                                  S.slot_of(first, u), last - first + 1, 1,
+                                                  orow, wstate, tid);
                 if (tid == 0) p.counters[first] = 0;
             }
         }

@@ -201,3 +201,81 @@ def test_full_size_config_sampled(sha, name):
     assert sha.sha_get_device_status() == sha.SHA_OK
     err, n = check_sampled_units(w, q, k, v, idx, out, n_random=48)
     assert n >= 48
+
+
+# ---------------------------------------------------------------- grouped-query (G > 1)
+
+GQA_CASES = [
+    W("gqa_g8", B=3, H_q=64, H_kv=8, N_kv=300, d=128, top_k=5, dtype="bf16", seed=41),
+    W("gqa_g2", B=4, H_q=8, H_kv=4, N_kv=129, d=64, top_k=2, dtype="fp16", seed=42),
+    W("gqa_g4", B=2, H_q=32, H_kv=8, N_kv=1000, d=128, top_k=3, dtype="fp16", seed=43),
+    W("gqa_g16", B=2, H_q=64, H_kv=4, N_kv=200, d=128, top_k=4, dtype="bf16", seed=44),
+    W("gqa_g7", B=3, H_q=28, H_kv=4, N_kv=65, d=64, top_k=2, dtype="bf16", seed=45),
+    W("gqa_short", B=5, H_q=16, H_kv=2, N_kv=17, d=128, top_k=1, dtype="fp16", seed=46),
+]
+
+
+@pytest.mark.parametrize("w", GQA_CASES, ids=lambda w: w.name)
+def test_gqa_parity(sha, w):
+    q, k, v, idx = _on_gpu(w)
+    out = _run(sha, w, q, k, v, idx)
+    check_against_oracle(w, q, k, v, idx, out)
+
+
+@pytest.mark.parametrize("splits", [1, 3, 7, 64, 10_000])
+def test_gqa_forced_splits(sha, splits):
+    w = W("gqa_splits", B=2, H_q=32, H_kv=4, N_kv=900, d=128, top_k=3, dtype="bf16", seed=47)
+    q, k, v, idx = _on_gpu(w)
+    out = _run(sha, w, q, k, v, idx, num_splits=splits)
+    check_against_oracle(w, q, k, v, idx, out)
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_gqa_single_key_returns_value_rows_exactly(sha, dtype):
+    w = W("gqa_n1", B=2, H_q=16, H_kv=4, N_kv=1, d=128, top_k=2, dtype=dtype, seed=48)
+    q, k, v, idx = _on_gpu(w)
+    out = _run(sha, w, q, k, v, idx)
+    bits = out_bits(out).reshape(w.B, w.H_q, w.d)
+    vbits = out_bits(v).reshape(w.B, w.H_kv, w.d)
+    for b, row in enumerate(idx.cpu().numpy()):
+        for h in row:
+            for j in range(w.G):
+                assert np.array_equal(bits[b, h * w.G + j], vbits[b, h])
+
+
+def test_gqa_unselected_groups_are_not_read(sha):
+    w = W("gqa_nan", B=2, H_q=32, H_kv=8, N_kv=190, d=128, top_k=3, dtype="bf16", seed=49)
+    q, k, v, idx = _on_gpu(w)
+    expected, _ = oracle.sha_decode(q.cpu(), k.cpu(), v.cpu(), idx.cpu().numpy(), w.scale,
+                                    w.dtype)
+    sel = np.zeros((w.B, w.H_kv), dtype=bool)
+    for b, row in enumerate(idx.cpu().numpy()):
+        sel[b, row] = True
+    k2, v2 = k.clone(), v.clone()
+    k2[torch.from_numpy(~sel).cuda()] = float("nan")
+    v2[torch.from_numpy(~sel).cuda()] = float("nan")
+    out = _run(sha, w, q, k2, v2, idx)
+    check_against_oracle(w, q, k, v, idx, out, expected)
+
+
+def test_gqa_out_of_range_group_ids(sha):
+    w = W("gqa_bad", B=3, H_q=32, H_kv=8, N_kv=130, d=128, top_k=2, dtype="bf16", seed=50)
+    q, k, v, idx = _on_gpu(w)
+    idx[0, 1] = 8
+    idx[2, 0] = -1
+    out = workloads.make_out(w, "cuda")
+    sha.decode(q, k, v, idx, w.scale, out)
+    assert sha.sha_get_device_status() == sha.SHA_ERR_BAD_INDEX
+    check_against_oracle(w, q, k, v, idx, out)
+
+
+def test_gqa_full_size_config_sampled(sha):
+    w = workloads.CONFIGS["llama31_70b_gqa"]
+    q, k, v = workloads.make_qkv(w, device="cuda")
+    idx = workloads.make_index(w).cuda()
+    out = workloads.make_out(w, "cuda")
+    sha.decode(q, k, v, idx, w.scale, out)
+    torch.cuda.synchronize()
+    assert sha.sha_get_device_status() == sha.SHA_OK
+    err, n = check_sampled_units(w, q, k, v, idx, out, n_random=48)
+    assert n >= 48
