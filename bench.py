@@ -240,22 +240,37 @@ def sync_all(world, local):
     torch.cuda.synchronize()
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device="cuda"):
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def sum_over_ranks(x, world):
+def sum_over_ranks(x, world, device="cuda"):
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def rank_workload(config, rank, batch=None):
+    """The batch shard rank `rank` decodes: the config's shape, its own seed."""
+    base = workloads.CONFIGS[config]
+    if batch:
+        base = base.with_(B=batch)
+    return base.with_(seed=base.seed + 100 * rank)
+
+
+def aggregate(bytes_per_step, steps, elapsed_s, world, device="cuda"):
+    """Whole-job GB/s (all ranks' bytes / slowest rank's time) and that time."""
+    t_max = max_over_ranks(elapsed_s, world, device)
+    total = sum_over_ranks(bytes_per_step * steps, world, device)
+    return total / t_max / 1e9, t_max
 
 
 # ---------------------------------------------------------------- arms
@@ -265,10 +280,7 @@ def run_ours(args, rank, world, local):
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    base = workloads.CONFIGS[args.config]
-    if args.batch:
-        base = base.with_(B=args.batch)
-    w = base.with_(seed=base.seed + 100 * rank)     # each rank decodes its own batch
+    w = rank_workload(args.config, rank, args.batch)   # each rank decodes its own batch
     q, k, v = workloads.make_qkv(w, device=dev)
     idx = workloads.make_index(w).to(dev)
     out = workloads.make_out(w, dev)
@@ -301,10 +313,8 @@ def run_ours(args, rank, world, local):
     if status != sha.SHA_OK:
         raise RuntimeError(f"device status after timing: {sha.sha_status_string(status)}")
 
-    t_max = max_over_ranks(elapsed, world)
     bytes_step = w.algorithmic_bytes()
-    total_bytes = sum_over_ranks(bytes_step * args.steps, world)
-    value = total_bytes / t_max / 1e9
+    value, t_max = aggregate(bytes_step, args.steps, elapsed, world)
     launch_s = elapsed / args.steps
     achieved = bytes_step / launch_s / 1e9
     peak, peak_src = measured_peak()
