@@ -28,19 +28,23 @@ def _sources():
                   + [os.path.join(INCLUDE, "sha_decode.h")])
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile the library unless it is newer than every source file."""
-    if not force and os.path.exists(LIBRARY):
+def build(force: bool = False, verbose: bool = False, defines=(), output=None) -> str:
+    """Compile the library unless it is newer than every source file.
+
+    defines: extra -D settings (the kernels' build-time tuning knobs);
+    output:  another path for the library (builds with non-default knobs)."""
+    library = output or LIBRARY
+    if not force and os.path.exists(library):
         newest = max(os.path.getmtime(p) for p in _sources())
-        if os.path.getmtime(LIBRARY) >= newest:
-            return LIBRARY
-    cmd = [NVCC, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC]
+        if os.path.getmtime(library) >= newest:
+            return library
+    cmd = [NVCC, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, *[f"-D{d}" for d in defines]]
     if verbose:
         cmd += ["-Xptxas", "-v"]
-    cmd += ["-o", LIBRARY + ".tmp", os.path.join(CSRC, "sha_decode.cu")]
+    cmd += ["-o", library + ".tmp", os.path.join(CSRC, "sha_decode.cu")]
     subprocess.run(cmd, check=True)
-    os.replace(LIBRARY + ".tmp", LIBRARY)
-    return LIBRARY
+    os.replace(library + ".tmp", library)
+    return library
 
 
 if __name__ == "__main__":

@@ -83,8 +83,10 @@ struct Plan {
     size_t workspace_bytes() const { return counter_bytes + slot_bytes; }
 };
 
-constexpr int kTileKeys = 64;          // keys per tile (both kernels)
 constexpr int kBlocksPerSm = 1;
+
+// keys per tile of the kernel that serves G query heads per KV head
+int tile_keys(int G) { return G == 1 ? sha::MhaConfig<128>::kTile : sha::GqaConfig<128>::kTile; }
 
 Plan make_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int num_splits,
                int num_sms)
@@ -92,7 +94,8 @@ Plan make_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int num_spl
     Plan pl;
     const int G = H_q / H_kv;
     const long long units = (long long)B * top_k;
-    pl.sched.tiles_per_unit = (N_kv + kTileKeys - 1) / kTileKeys;
+    const int tile = tile_keys(G);
+    pl.sched.tiles_per_unit = (N_kv + tile - 1) / tile;
     pl.sched.total_tiles = units * pl.sched.tiles_per_unit;
     long long ctas = num_splits > 0 ? num_splits : (long long)num_sms * kBlocksPerSm;
     if (ctas > sha::kMaxBlocks) ctas = sha::kMaxBlocks;
@@ -119,8 +122,9 @@ Plan make_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int num_spl
     return pl;
 }
 
-static_assert(sha::MhaConfig<128>::kTile == kTileKeys && sha::GqaConfig<128>::kTile == kTileKeys,
-              "host plan and kernels agree on the tile");
+static_assert(sha::MhaConfig<128>::kTile == sha::MhaConfig<64>::kTile &&
+                  sha::GqaConfig<128>::kTile == sha::GqaConfig<64>::kTile,
+              "one tile size per kernel, whatever d");
 
 // cuTensorMapEncodeTiled from the driver, found through the runtime so the
 // library does not link against libcuda.
@@ -152,7 +156,7 @@ sha_status_t kv_tensor_map(CUtensorMap *map, const void *base, sha_dtype_t dtype
     }
     cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N_kv, (cuuint64_t)planes};
     cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N_kv * d * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)kTileKeys, 1};
+    cuuint32_t box[3] = {64, (cuuint32_t)sha::GqaConfig<128>::kTile, 1};
     cuuint32_t elem[3] = {1, 1, 1};
     CUresult r = encode(map,
                         dtype == SHA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -359,10 +363,11 @@ sha_status_t sha_decode_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_
     sha_status_t st = check_shape(B, H_q, H_kv, N_kv, d, top_k, 1.0f);
     if (st != SHA_OK) return st;
     if (num_splits < 0 || num_sms < 1 || !plan) return SHA_ERR_INVALID_ARG;
+    const int tile = tile_keys(H_q / H_kv);
     if (B == 0 || top_k == 0) {
-        plan[0] = (N_kv + kTileKeys - 1) / kTileKeys;
+        plan[0] = (N_kv + tile - 1) / tile;
         plan[1] = plan[2] = plan[3] = 0;
-        plan[4] = kTileKeys;
+        plan[4] = tile;
         return SHA_OK;
     }
     const Plan pl = make_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits, num_sms);
@@ -370,7 +375,7 @@ sha_status_t sha_decode_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_
     plan[1] = pl.sched.total_tiles;
     plan[2] = pl.sched.num_ctas;
     plan[3] = (int64_t)pl.workspace_bytes();
-    plan[4] = kTileKeys;
+    plan[4] = tile;
     return SHA_OK;
 }
 

@@ -14,8 +14,8 @@
 //     (cp.async.bulk.tensor, a 3-D map [planes = B*H_kv][N_kv][d] with
 //     64-element boxes and 128-byte swizzle) into a kStages-deep ring; keys
 //     past N_kv are outside the map and arrive as zeros;
-//   * 4 consumer warps take 16 keys of each 64-key tile each and keep their
-//     own online-softmax state for up to 16 query rows;
+//   * 4 consumer warps take 16 keys of every 64-key slice of a tile each and
+//     keep their own online-softmax state for up to 16 query rows;
 //   * S = Q K^T: mma.sync m16n8k16 with Q (G rows, zero-padded to 16) as the
 //     A operand held in registers and K fragments read by ldmatrix from the
 //     swizzled tile (conflict-free);
@@ -34,14 +34,23 @@
 
 namespace sha {
 
+// Build-time tuning of the grouped-query kernel (default measured best on B200).
+#ifndef SHA_GQA_TILE_KEYS
+#define SHA_GQA_TILE_KEYS 128
+#endif
+#ifndef SHA_GQA_STAGES
+#define SHA_GQA_STAGES 3
+#endif
+
 template <int D>
 struct GqaConfig {
     static constexpr int kConsumerWarps = 4;
     static constexpr int kConsumers = kConsumerWarps * 32;
     static constexpr int kThreads = kConsumers + 32;
-    static constexpr int kTile = 64;                   // keys per tile
-    static constexpr int kKeysPerWarp = kTile / kConsumerWarps;   // 16: one m16n8k16 k-step
-    static constexpr int kStages = 4;
+    static constexpr int kTile = SHA_GQA_TILE_KEYS;    // keys per tile (one pipeline stage)
+    static constexpr int kSlices = kTile / 64;         // 64-key slices per tile
+    static constexpr int kKeysPerWarp = 64 / kConsumerWarps;      // 16 per slice: one m16n8k16 k-step
+    static constexpr int kStages = SHA_GQA_STAGES;
     static constexpr int kRows = 16;                   // query rows per MMA (G padded)
     static constexpr int kBoxes = D / 64;              // 128-byte boxes across d
     static constexpr int kBoxBytes = kTile * 128;
@@ -57,7 +66,8 @@ struct GqaConfig {
     static constexpr int kStateOffset = kFlagOffset + 16;
     static constexpr int kSmemBytes =
         kAlignPad + kStateOffset + kConsumerWarps * kStateFloats * 4;
-    static_assert(kKeysPerWarp == 16, "one k-step of 16 keys per warp");
+    static_assert(kKeysPerWarp == 16, "one k-step of 16 keys per warp and slice");
+    static_assert(kTile % 64 == 0 && kTile <= 256, "whole 64-key slices, TMA box <= 256 rows");
     static_assert(kBoxBytes % 1024 == 0, "boxes stay 1 KiB aligned");
     static_assert(kConsumerWarps * kStateFloats >= 3 * kMaxMergeParts * kRows,
                   "merge staging fits");
@@ -279,26 +289,36 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
                 const uint32_t vt = v_base + stage * C::kTileBytes;
                 const int rows = min(C::kTile, p.N_kv - j * C::kTile);
 
-                // S = Q K^T over this warp's 16 keys: two 8-key n-tiles
-                float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                // S = Q K^T over this warp's 16 keys of each 64-key slice:
+                // two 8-key n-tiles per slice
+                float s[C::kSlices][2][4];
 #pragma unroll
-                for (int ks = 0; ks < C::kKSteps; ++ks) {
-                    uint32_t kb[4];
-                    ldmatrix_x4(swizzled<D>(kt, key_k, ks * 2 + (mi & 1)), kb);
-                    mma_16816<T>(s[0], qa[ks], kb[0], kb[1]);
-                    mma_16816<T>(s[1], qa[ks], kb[2], kb[3]);
+                for (int sl = 0; sl < C::kSlices; ++sl) {
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+                        s[sl][nt][0] = s[sl][nt][1] = s[sl][nt][2] = s[sl][nt][3] = 0.f;
+#pragma unroll
+                    for (int ks = 0; ks < C::kKSteps; ++ks) {
+                        uint32_t kb[4];
+                        ldmatrix_x4(swizzled<D>(kt, sl * 64 + key_k, ks * 2 + (mi & 1)), kb);
+                        mma_16816<T>(s[sl][0], qa[ks], kb[0], kb[1]);
+                        mma_16816<T>(s[sl][1], qa[ks], kb[2], kb[3]);
+                    }
                 }
 
                 // online softmax on rows g (entries 0,1) and g+8 (entries 2,3)
                 float mt[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
+                for (int sl = 0; sl < C::kSlices; ++sl)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int key = warp * C::kKeysPerWarp + nt * 8 + qd * 2 + (e & 1);
-                        s[nt][e] = key < rows ? s[nt][e] * p.scale_log2 : -INFINITY;
-                        mt[e >> 1] = fmaxf(mt[e >> 1], s[nt][e]);
-                    }
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int key = sl * 64 + warp * C::kKeysPerWarp + nt * 8 + qd * 2 +
+                                            (e & 1);
+                            s[sl][nt][e] = key < rows ? s[sl][nt][e] * p.scale_log2 : -INFINITY;
+                            mt[e >> 1] = fmaxf(mt[e >> 1], s[sl][nt][e]);
+                        }
                 float alpha[2], ref[2];
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
@@ -311,12 +331,14 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
                     l_run[r] *= alpha[r];
                 }
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
+                for (int sl = 0; sl < C::kSlices; ++sl)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        s[nt][e] = exp2f(s[nt][e] - ref[e >> 1]);
-                        l_run[e >> 1] += s[nt][e];
-                    }
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            s[sl][nt][e] = exp2f(s[sl][nt][e] - ref[e >> 1]);
+                            l_run[e >> 1] += s[sl][nt][e];
+                        }
 #pragma unroll
                 for (int n = 0; n < C::kONTiles; ++n) {
                     o[n][0] *= alpha[0];
@@ -324,19 +346,22 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
                     o[n][2] *= alpha[1];
                     o[n][3] *= alpha[1];
                 }
-                uint32_t pa[4];
-                pa[0] = pack2<T>(s[0][0], s[0][1]);
-                pa[1] = pack2<T>(s[0][2], s[0][3]);
-                pa[2] = pack2<T>(s[1][0], s[1][1]);
-                pa[3] = pack2<T>(s[1][2], s[1][3]);
 
-                // O += P V: 16 keys x d, two 8-wide n-tiles per ldmatrix
+                // O += P V: per slice, 16 keys x d, two 8-wide n-tiles per ldmatrix
 #pragma unroll
-                for (int dn = 0; dn < D / 16; ++dn) {
-                    uint32_t vb[4];
-                    ldmatrix_x4_trans(swizzled<D>(vt, key_v, dn * 2 + (mi >> 1)), vb);
-                    mma_16816<T>(o[2 * dn], pa, vb[0], vb[1]);
-                    mma_16816<T>(o[2 * dn + 1], pa, vb[2], vb[3]);
+                for (int sl = 0; sl < C::kSlices; ++sl) {
+                    uint32_t pa[4];
+                    pa[0] = pack2<T>(s[sl][0][0], s[sl][0][1]);
+                    pa[1] = pack2<T>(s[sl][0][2], s[sl][0][3]);
+                    pa[2] = pack2<T>(s[sl][1][0], s[sl][1][1]);
+                    pa[3] = pack2<T>(s[sl][1][2], s[sl][1][3]);
+#pragma unroll
+                    for (int dn = 0; dn < D / 16; ++dn) {
+                        uint32_t vb[4];
+                        ldmatrix_x4_trans(swizzled<D>(vt, sl * 64 + key_v, dn * 2 + (mi >> 1)), vb);
+                        mma_16816<T>(o[2 * dn], pa, vb[0], vb[1]);
+                        mma_16816<T>(o[2 * dn + 1], pa, vb[2], vb[3]);
+                    }
                 }
             }
             __syncwarp();

@@ -51,13 +51,21 @@ struct DecodeParams {
     int *counters;           // arrival counters, one per block, zero between calls
 };
 
+// Build-time tuning of the multi-head kernel (defaults measured best on B200).
+#ifndef SHA_MHA_TILE_KEYS
+#define SHA_MHA_TILE_KEYS 128
+#endif
+#ifndef SHA_MHA_STAGES
+#define SHA_MHA_STAGES 3
+#endif
+
 template <int D>
 struct MhaConfig {
     static constexpr int kConsumerWarps = 8;
     static constexpr int kConsumers = kConsumerWarps * 32;
     static constexpr int kThreads = kConsumers + 32;   // + one producer warp
-    static constexpr int kTile = 64;                   // keys per tile
-    static constexpr int kStages = 4;
+    static constexpr int kTile = SHA_MHA_TILE_KEYS;    // keys per tile
+    static constexpr int kStages = SHA_MHA_STAGES;
     static constexpr int kRowsPerWarp = kTile / kConsumerWarps;
     static constexpr int kPasses = kRowsPerWarp / 4;   // score passes of 4 rows
     static constexpr int kQkChunks = D / 64;           // 16-byte chunks per lane (scores)
