@@ -66,6 +66,8 @@ def parse_args():
                    help="skip the density sweep, e2e and CPU baseline (used for ncu)")
     p.add_argument("--cpu-budget", type=float, default=10.0,
                    help="seconds of oracle work for cpu_baseline")
+    p.add_argument("--sweep", action="store_true",
+                   help="run the LLaMA-2-7B-shaped scaling sweep instead (one JSON line)")
     return p.parse_args()
 
 
@@ -476,9 +478,88 @@ def run_reference(args):
     }
 
 
+L2_BYTES = 126 * 1024 * 1024
+
+
+def linear_fit(xs, ys):
+    """Least-squares y = a + b x and its R^2."""
+    n = len(xs)
+    mx, my = sum(xs) / n, sum(ys) / n
+    sxx = sum((x - mx) ** 2 for x in xs)
+    sxy = sum((x - mx) * (y - my) for x, y in zip(xs, ys))
+    b = sxy / sxx
+    a = my - b * mx
+    ss_res = sum((y - a - b * x) ** 2 for x, y in zip(xs, ys))
+    ss_tot = sum((y - my) ** 2 for y in ys)
+    return a, b, (1.0 - ss_res / ss_tot) if ss_tot > 0 else 1.0
+
+
+def run_sweep(args):
+    """B x N_kv x density grid of the LLaMA-2-7B shape (H=32, d=128, fp16).
+
+    Where one copy of the inputs would sit in L2, the timed graph cycles
+    through enough independent copies (replicas) that every pass touches at
+    least 4x L2 of K/V, so the figures are HBM figures."""
+    import head_sparse_decode_b200 as sha
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peak, peak_src = measured_peak()
+    points, fits = [], []
+    pi = 0
+    for B in workloads.SWEEP_B:
+        for N in workloads.SWEEP_N:
+            w0 = workloads.sweep(B, N, workloads.SWEEP_TOPK[-1], pi)
+            kv_bytes = 2 * w0.B * w0.H_kv * w0.N_kv * w0.d * 2
+            reps = max(1, math.ceil(4 * L2_BYTES / kv_bytes))
+            data = [workloads.make_qkv(w0.with_(seed=w0.seed + 17 * r), device=dev)
+                    for r in range(reps)]
+            times = []
+            for top_k in workloads.SWEEP_TOPK:
+                w = w0.with_(top_k=top_k, name=f"sweep_B{B}_N{N}_k{top_k}")
+                idx = workloads.make_index(w).to(dev)
+                outs = [workloads.make_out(w, dev) for _ in range(reps)]
+                calls = [lambda q=q, k=k, v=v, o=o: sha.decode(q, k, v, idx, w.scale, o)
+                         for (q, k, v), o in zip(data, outs)]
+                for c in calls:
+                    c()
+
+                def one_pass():
+                    for c in calls:
+                        c()
+                est = w.algorithmic_bytes() / (0.8 * peak * 1e9)      # s per call
+                passes = int(min(200, max(5, math.ceil(0.02 / (est * reps)))))
+                t = timed_graphs(one_pass, passes, dev, stream, chunk=max(1, 100 // reps))
+                us = t / (passes * reps) * 1e6
+                gbs = w.algorithmic_bytes() / (us * 1e-6) / 1e9
+                times.append(us)
+                points.append({"B": B, "N_kv": N, "top_k": top_k,
+                               "density": round(top_k / w.H_kv, 4), "us_per_step": round(us, 3),
+                               "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
+                               "replicas": reps})
+                pi += 1
+            a, b, r2 = linear_fit(list(workloads.SWEEP_TOPK), times)
+            fits.append({"B": B, "N_kv": N, "intercept_us": round(a, 3),
+                         "us_per_head": round(b, 4), "r2": round(r2, 5),
+                         "t_over_dense": [round(t / times[-1], 4) for t in times]})
+            del data
+            torch.cuda.empty_cache()
+    return {"metric": METRIC, "sweep": "LLaMA-2-7B shape, H=32, d=128, fp16",
+            "unit": "GB/s", "peak": peak, "peak_source": peak_src,
+            "densities": [k / 32 for k in workloads.SWEEP_TOPK], "points": points,
+            "fits": fits,
+            "l2": "inputs rotated over >= 4x L2 of K/V per pass where one copy is smaller",
+            "launch": "CUDA graph replay"}
+
+
 def main():
     args = parse_args()
     rank, world, local = dist_env()
+    if args.sweep:
+        if rank == 0:
+            print(json.dumps(run_sweep(args)), flush=True)
+        return
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)

@@ -279,3 +279,29 @@ def test_gqa_full_size_config_sampled(sha):
     assert sha.sha_get_device_status() == sha.SHA_OK
     err, n = check_sampled_units(w, q, k, v, idx, out, n_random=48)
     assert n >= 48
+
+
+# ---------------------------------------------------------------- scaling-sweep points
+
+@pytest.mark.parametrize("B,N_kv,top_k", [(1, 8192, 8), (256, 512, 32), (32, 4096, 24),
+                                          (8, 1920, 16)])
+def test_sweep_points_sampled(sha, B, N_kv, top_k):
+    w = workloads.sweep(B, N_kv, top_k, point=B + N_kv + top_k)
+    q, k, v = workloads.make_qkv(w, device="cuda")
+    idx = workloads.make_index(w).cuda()
+    out = workloads.make_out(w, "cuda")
+    sha.decode(q, k, v, idx, w.scale, out)
+    torch.cuda.synchronize()
+    assert sha.sha_get_device_status() == sha.SHA_OK
+    check_sampled_units(w, q, k, v, idx, out, n_random=24)
+
+
+def test_long_context_16k_gqa_and_mha(sha):
+    """The pages evaluate contexts up to 16K tokens."""
+    for w in (W("ctx16k_mha", B=2, H_q=8, H_kv=8, N_kv=16384, d=128, top_k=3, dtype="fp16",
+                seed=61),
+              W("ctx16k_gqa", B=2, H_q=32, H_kv=4, N_kv=16384, d=128, top_k=2, dtype="bf16",
+                seed=62)):
+        q, k, v, idx = _on_gpu(w)
+        out = _run(sha, w, q, k, v, idx)
+        check_against_oracle(w, q, k, v, idx, out)
