@@ -5,6 +5,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include <cudaTypedefs.h>
 
@@ -126,6 +127,30 @@ static_assert(sha::MhaConfig<128>::kTile == sha::MhaConfig<64>::kTile &&
                   sha::GqaConfig<128>::kTile == sha::GqaConfig<64>::kTile,
               "one tile size per kernel, whatever d");
 
+#ifndef SHA_USE_PDL
+#define SHA_USE_PDL 1
+#endif
+
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel in the stream finishes, and waits for it on the
+// device (griddepcontrol.wait) before reading any input.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), int grid, int block, size_t smem,
+                          cudaStream_t stream, Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = SHA_USE_PDL;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // cuTensorMapEncodeTiled from the driver, found through the runtime so the
 // library does not link against libcuda.
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
@@ -191,9 +216,8 @@ sha_status_t launch_gqa(const sha::DecodeParams &prm, sha_dtype_t dtype, int dev
     if (st != SHA_OK) return st;
     st = kv_tensor_map(&tm_v, prm.v, dtype, D, prm.N_kv, planes);
     if (st != SHA_OK) return st;
-    sha::sha_gqa_decode_kernel<T, D>
-        <<<prm.sched.num_ctas, C::kThreads, C::kSmemBytes, stream>>>(prm, tm_k, tm_v);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_kernel(sha::sha_gqa_decode_kernel<T, D>, prm.sched.num_ctas,
+                                  C::kThreads, C::kSmemBytes, stream, prm, tm_k, tm_v);
     if (e != cudaSuccess) return launch_error(e);
     return SHA_OK;
 }
@@ -210,9 +234,8 @@ sha_status_t launch_mha(const sha::DecodeParams &prm, int dev, cudaStream_t stre
         if (e != cudaSuccess) return launch_error(e);
         configured[dev] = true;
     }
-    sha::sha_mha_decode_kernel<T, D>
-        <<<prm.sched.num_ctas, C::kThreads, C::kSmemBytes, stream>>>(prm);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_kernel(sha::sha_mha_decode_kernel<T, D>, prm.sched.num_ctas,
+                                  C::kThreads, C::kSmemBytes, stream, prm);
     if (e != cudaSuccess) return launch_error(e);
     return SHA_OK;
 }

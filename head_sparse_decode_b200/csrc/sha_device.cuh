@@ -106,6 +106,22 @@ __device__ __forceinline__ void named_barrier(int id, int threads)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// ---- programmatic dependent launch ------------------------------------------
+// A kernel launched with programmatic stream serialization may start while the
+// previous kernel in the stream is still running.  pdl_wait() blocks until that
+// kernel has completed and its memory is visible (a no-op otherwise): it must
+// come before the first read of anything a previous kernel may have written.
+// pdl_launch_dependents() lets the next kernel in the stream be scheduled as SMs
+// free up.
+__device__ __forceinline__ void pdl_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- element conversion ---------------------------------------------------
 
 template <typename T> struct Elem;

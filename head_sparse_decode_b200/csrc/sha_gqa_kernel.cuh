@@ -179,6 +179,9 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
         mbar_init_fence();
     }
     __syncthreads();
+    // inputs, workspace and the output may come from the previous kernel
+    pdl_wait();
+    pdl_launch_dependents();
 
     const Schedule S = p.sched;
     const long long t_begin = S.begin(blockIdx.x);
