@@ -13,8 +13,9 @@ float16 / bfloat16).
 What is computed, and which passage each function follows, is stated in
 ``sha_oracle.c``: the attention equation of the "Attention Head 稀疏性"
 section (papernotes.org summary of Polar Sparsity), Algorithm 1 "Selective
-Head Flash Attention (Decode)" (ri.k117.org reproducibility record) and the
-routing of the "Selective Head Attention (SHA) Kernel" section.
+Head Flash Attention (Decode)" (ri.k117.org reproducibility record), the
+routing of the "Selective Head Attention (SHA) Kernel" section, and the
+router's top-k head selection ("Router 训练").
 """
 import ctypes
 import os
@@ -48,6 +49,9 @@ def _load():
             ctypes.c_int, ctypes.c_double, ctypes.c_int, ctypes.c_int, f64p]
         lib.sha_oracle_widen.restype = ctypes.c_double
         lib.sha_oracle_widen.argtypes = [ctypes.c_uint16, ctypes.c_int]
+        lib.sha_oracle_select_heads.restype = ctypes.c_int
+        lib.sha_oracle_select_heads.argtypes = [
+            ctypes.POINTER(ctypes.c_float), ctypes.c_int, ctypes.c_int, ctypes.c_int, i32p]
         lib.sha_oracle_num_threads.restype = ctypes.c_int
         lib.sha_oracle_num_threads.argtypes = []
         _lib = lib
@@ -142,6 +146,21 @@ def sha_units(q_units, k_units, v_units, scale, dtype, tile=0):
         _ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16),
         n, G, N_kv, d, float(scale), _dtype_code(dtype), int(tile),
         _ptr(out, ctypes.c_double))
+    if rc != 0:
+        raise ValueError("inconsistent sizes")
+    return out
+
+
+def select_heads(scores, top_k):
+    """Per-row top-k head ids of router scores [B, H] (float32): decreasing score,
+    ties by increasing head id.  Returns int32 [B, top_k]."""
+    sc = np.ascontiguousarray(np.asarray(scores, dtype=np.float32))
+    if sc.ndim != 2:
+        raise ValueError("scores must be [B, H]")
+    B, H = sc.shape
+    out = np.empty((B, top_k), dtype=np.int32)
+    rc = _load().sha_oracle_select_heads(_ptr(sc, ctypes.c_float), B, H, int(top_k),
+                                         _ptr(out, ctypes.c_int32))
     if rc != 0:
         raise ValueError("inconsistent sizes")
     return out

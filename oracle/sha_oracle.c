@@ -252,3 +252,35 @@ int sha_oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/*
+ * Head selection: the step that turns the attention router's per-head scores
+ * into batch_head_index (papernotes.org summary, "Router 训练": the attention
+ * router is one fully connected layer whose top-k heads are kept; atlas.scime.ai
+ * summary: a router picks the top-k attention heads or GQA groups per token).
+ * For every row b the top_k heads with the largest scores[b, :] are written in
+ * order of decreasing score; equal scores are ordered by increasing head id.
+ * Done here by top_k rounds of "take the best head not yet taken".
+ * Returns -1 for inconsistent sizes.
+ */
+int sha_oracle_select_heads(const float *scores, int B, int H, int top_k,
+                            int32_t *batch_head_index)
+{
+    if (B < 0 || H <= 0 || top_k < 0 || top_k > H) return -1;
+    unsigned char *taken = (unsigned char *)malloc((size_t)H);
+    for (int b = 0; b < B; ++b) {
+        const float *row = scores + (size_t)b * H;
+        memset(taken, 0, (size_t)H);
+        for (int k = 0; k < top_k; ++k) {
+            int best = -1;
+            for (int h = 0; h < H; ++h) {
+                if (taken[h]) continue;
+                if (best < 0 || row[h] > row[best]) best = h;   /* ties keep the lower id */
+            }
+            taken[best] = 1;
+            batch_head_index[(size_t)b * top_k + k] = best;
+        }
+    }
+    free(taken);
+    return 0;
+}

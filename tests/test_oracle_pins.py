@@ -251,3 +251,23 @@ def test_units_entry_matches_full_layout():
     per_unit = oracle.sha_units(qu, ku, vu, w.scale, w.dtype)
     for i, (b, h) in enumerate(zip(bs, hs)):
         assert np.array_equal(per_unit[i], full[b, h * w.G:(h + 1) * w.G])
+
+
+# ---------------------------------------------------------------- head selection
+
+@pytest.mark.parametrize("B,H,top_k", [(5, 8, 3), (3, 72, 22), (4, 32, 32), (2, 256, 100),
+                                       (3, 1, 1), (2, 9, 0)])
+def test_select_heads_matches_stable_argsort(B, H, top_k):
+    """numpy's stable argsort of -score: decreasing score, ties by head id."""
+    rng = np.random.default_rng(B * 1000 + H)
+    scores = rng.integers(-4, 5, size=(B, H)).astype(np.float32)   # many ties
+    got = oracle.select_heads(scores, top_k)
+    want = np.argsort(-scores, axis=1, kind="stable")[:, :top_k].astype(np.int32)
+    assert np.array_equal(got, want)
+
+
+def test_select_heads_hand_example():
+    scores = np.array([[0.5, 2.0, -1.0, 2.0, 7.0]], dtype=np.float32)
+    assert oracle.select_heads(scores, 3).tolist() == [[4, 1, 3]]
+    neg = np.array([[-np.inf, -3.0, -np.inf]], dtype=np.float32)
+    assert oracle.select_heads(neg, 3).tolist() == [[1, 0, 2]]
