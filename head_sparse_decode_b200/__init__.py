@@ -229,6 +229,35 @@ def sha_decode_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits=0, num_sms=148):
             "workspace_bytes": plan[3], "tile_keys": plan[4]}
 
 
+_lib.sha_select_heads.argtypes = [_vp, _i, _i, _i, _vp, _vp]
+_lib.sha_select_heads.restype = _i
+
+
+def sha_select_heads(scores, top_k, out=None, stream=None):
+    """Per-row top-k of router scores [B, H] (float32, CUDA) into an int32
+    [B, top_k] index tensor on the same device (decreasing score, ties by head id)."""
+    if scores.dim() != 2 or not scores.is_cuda or not scores.is_contiguous():
+        raise ValueError("scores must be a contiguous CUDA tensor [B, H]")
+    if scores.dtype != torch.float32:
+        raise TypeError("scores must be float32")
+    B, H = scores.shape
+    if out is None:
+        out = torch.empty((B, top_k), dtype=torch.int32, device=scores.device)
+    if out.shape != (B, top_k) or out.dtype != torch.int32 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous int32 [B, top_k] tensor")
+    with torch.cuda.device(scores.device):
+        _check(_lib.sha_select_heads(scores.data_ptr(), B, H, int(top_k), out.data_ptr(),
+                                     _stream_handle(stream, scores.device)))
+    return out
+
+
+def decode_from_scores(q, k, v, scores, top_k, scale=None, out=None, stream=None):
+    """Head selection then selective decode, both on the device and on one stream:
+    the router scores [B, H_kv] pick each row's top_k heads (or groups)."""
+    idx = sha_select_heads(scores, top_k, stream=stream)
+    return decode(q, k, v, idx, scale, out, stream), idx
+
+
 def sha_get_device_status(stream=None, device=None):
     """Synchronise ``stream`` and read-and-clear the device's sticky flags; returns a
     status code (SHA_OK, SHA_ERR_BAD_INDEX or SHA_ERR_TIMEOUT)."""
@@ -250,6 +279,7 @@ def sha_copy_bandwidth_probe(dst, src, stream=None):
 
 __all__ = [
     "sha_decode", "sha_decode_bf16", "sha_decode_ex", "sha_decode_workspace_size",
-    "sha_get_device_status", "sha_status_string", "sha_decode_plan", "sha_copy_bandwidth_probe", "decode",
+    "sha_get_device_status", "sha_status_string", "sha_decode_plan", "sha_select_heads",
+    "decode_from_scores", "sha_copy_bandwidth_probe", "decode",
     "alloc_workspace", "ShaError", "LIBRARY_PATH", "sha_decode_noalloc",
 ]

@@ -14,6 +14,7 @@
 #include "sha_gqa_kernel.cuh"
 #include "sha_mha_kernel.cuh"
 #include "sha_schedule.cuh"
+#include "sha_select_kernel.cuh"
 
 namespace {
 
@@ -399,6 +400,23 @@ sha_status_t sha_decode_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_
     plan[2] = pl.sched.num_ctas;
     plan[3] = (int64_t)pl.workspace_bytes();
     plan[4] = tile;
+    return SHA_OK;
+}
+
+sha_status_t sha_select_heads(const float *scores, int B, int H, int top_k,
+                              int32_t *batch_head_index, void *stream)
+{
+    if (B < 0 || H < 1 || top_k < 0 || top_k > H) return SHA_ERR_INVALID_ARG;
+    if (H > sha::kSelectMaxHeads) return SHA_ERR_UNSUPPORTED;
+    if (B == 0 || top_k == 0) return SHA_OK;
+    if (!scores || !batch_head_index) return SHA_ERR_INVALID_ARG;
+    if (!aligned(scores, 4) || !aligned(batch_head_index, 4)) return SHA_ERR_MISALIGNED;
+    const int grid = (B + sha::kSelectRowsPerBlock - 1) / sha::kSelectRowsPerBlock;
+    cudaError_t e = launch_kernel(sha::sha_select_heads_kernel, grid,
+                                  sha::kSelectRowsPerBlock * 32, 0,
+                                  static_cast<cudaStream_t>(stream), scores, B, H, top_k,
+                                  batch_head_index);
+    if (e != cudaSuccess) return launch_error(e);
     return SHA_OK;
 }
 

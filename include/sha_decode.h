@@ -140,6 +140,21 @@ sha_status_t sha_decode_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_
                              int num_splits, int num_sms, int64_t plan[5]);
 
 /*
+ * sha_select_heads -- router scores to batch_head_index on the device.
+ * Polar Sparsity (papernotes.org summary, "Router 训练"; atlas.scime.ai
+ * summary): an attention router scores the heads (or GQA groups) of each
+ * token and the top_k are kept.  This call does that selection:
+ *   scores           : device pointer, fp32 [B, H] (finite or +-inf; no NaN)
+ *   batch_head_index : device pointer, int32 [B, top_k], written in order of
+ *                      decreasing score, equal scores by increasing head id
+ *   1 <= H <= 256 (SHA_ERR_UNSUPPORTED above), 0 <= top_k <= H.
+ * Enqueued on `stream`; a decode enqueued after it on the same stream reads
+ * the indices it wrote, with no host synchronisation in between.
+ */
+sha_status_t sha_select_heads(const float *scores, int B, int H, int top_k,
+                              int32_t *batch_head_index, void *stream);
+
+/*
  * sha_get_device_status -- synchronises `stream`, then reads and clears the
  * current device's sticky flags: SHA_ERR_BAD_INDEX if any call since the last
  * read met an out-of-range head id, SHA_ERR_TIMEOUT if a pipeline wait gave

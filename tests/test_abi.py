@@ -95,3 +95,11 @@ def test_plan_tiles_and_blocks():
     assert p["workspace_bytes"] > 0
     with pytest.raises(h.ShaError):
         h.sha_decode_plan(1, 4, 4, 10, 96, 1)
+
+
+@pytest.mark.parametrize("B,H,top_k,code", [(2, 300, 3, 2), (2, 8, 9, 1), (2, 0, 0, 1),
+                                             (-1, 8, 2, 1), (0, 8, 2, 0), (3, 8, 0, 0)])
+def test_select_heads_host_checks(lib, B, H, top_k, code):
+    lib.sha_select_heads.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                     ctypes.c_void_p, ctypes.c_void_p]
+    assert lib.sha_select_heads(0x1000, B, H, top_k, 0x2000, None) == code
