@@ -49,6 +49,10 @@ def _load():
             ctypes.c_int, ctypes.c_double, ctypes.c_int, ctypes.c_int, f64p]
         lib.sha_oracle_widen.restype = ctypes.c_double
         lib.sha_oracle_widen.argtypes = [ctypes.c_uint16, ctypes.c_int]
+        lib.sha_oracle_decode_varlen.restype = ctypes.c_longlong
+        lib.sha_oracle_decode_varlen.argtypes = [
+            u16p, u16p, u16p, i32p, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int, f64p]
         lib.sha_oracle_select_heads.restype = ctypes.c_int
         lib.sha_oracle_select_heads.argtypes = [
             ctypes.POINTER(ctypes.c_float), ctypes.c_int, ctypes.c_int, ctypes.c_int, i32p]
@@ -164,3 +168,25 @@ def select_heads(scores, top_k):
     if rc != 0:
         raise ValueError("inconsistent sizes")
     return out
+
+
+def sha_decode_varlen(q, k, v, batch_head_index, seqlens, scale, dtype, out=None):
+    """Selective head decode where row b uses only the first seqlens[b] keys of its
+    [N_max]-long cache.  Same conventions as sha_decode; rows with a length outside
+    [1, N_max] are skipped and counted.  Returns (out, count)."""
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, H_kv, N_max, d = kb.shape
+    qb = qb.reshape(B, -1, d)
+    H_q = qb.shape[1]
+    idx = np.ascontiguousarray(np.asarray(batch_head_index, dtype=np.int32).reshape(B, -1))
+    lens = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32).reshape(B))
+    top_k = idx.shape[1]
+    if out is None:
+        out = np.full((B, H_q, d), np.nan, dtype=np.float64)
+    bad = _load().sha_oracle_decode_varlen(
+        _ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16),
+        _ptr(idx, ctypes.c_int32), _ptr(lens, ctypes.c_int32), B, H_q, H_kv, N_max, d, top_k,
+        float(scale), _dtype_code(dtype), _ptr(out, ctypes.c_double))
+    if bad < 0:
+        raise ValueError("inconsistent sizes")
+    return out, int(bad)

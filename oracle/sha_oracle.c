@@ -284,3 +284,42 @@ int sha_oracle_select_heads(const float *scores, int B, int H, int top_k,
     free(taken);
     return 0;
 }
+
+/*
+ * Selective head decode when every batch row has its own cache length: row b
+ * attends to keys [0, seqlens[b]) of its [N_max]-long cache (a decode batch
+ * whose sequences have different lengths).  Each selected unit is exactly the
+ * operation of sha_oracle_decode on that row's first seqlens[b] keys.  Rows
+ * whose length is outside [1, N_max] are skipped and counted like out-of-range
+ * ids.  Returns the count, or -1 for inconsistent sizes.
+ */
+long long sha_oracle_decode_varlen(const uint16_t *Q, const uint16_t *K,
+                                   const uint16_t *V, const int32_t *batch_head_index,
+                                   const int32_t *seqlens, int B, int H_q, int H_kv,
+                                   int N_max, int d, int top_k, double scale, int dtype,
+                                   double *out)
+{
+    if (B < 0 || H_kv <= 0 || H_q <= 0 || H_q % H_kv != 0 || N_max <= 0 ||
+        d <= 0 || top_k < 0)
+        return -1;
+    int G = H_q / H_kv;
+    long long bad = 0;
+    long long units = (long long)B * top_k;
+#pragma omp parallel for schedule(dynamic, 1) reduction(+ : bad)
+    for (long long u = 0; u < units; ++u) {
+        long long b = u / top_k;
+        int h = batch_head_index[u];
+        int n = seqlens[b];
+        if (h < 0 || h >= H_kv || n < 1 || n > N_max) {
+            bad += 1;
+            continue;
+        }
+        const uint16_t *K_bh = K + ((size_t)b * H_kv + h) * (size_t)N_max * d;
+        const uint16_t *V_bh = V + ((size_t)b * H_kv + h) * (size_t)N_max * d;
+        for (int j = 0; j < G; ++j) {
+            size_t row = ((size_t)b * H_q + (size_t)h * G + j) * (size_t)d;
+            attention(Q + row, K_bh, V_bh, n, d, scale, dtype, 0, out + row);
+        }
+    }
+    return bad;
+}

@@ -271,3 +271,36 @@ def test_select_heads_hand_example():
     assert oracle.select_heads(scores, 3).tolist() == [[4, 1, 3]]
     neg = np.array([[-np.inf, -3.0, -np.inf]], dtype=np.float32)
     assert oracle.select_heads(neg, 3).tolist() == [[1, 0, 2]]
+
+
+# ---------------------------------------------------------------- per-row lengths
+
+def test_varlen_rows_equal_fixed_length_on_truncated_caches():
+    """Row b with length L is plain decode over the first L keys (checked against
+    the fixed-length path on a truncated copy, and against SDPA on that copy)."""
+    B, H, N, d = 4, 6, 90, 16
+    q, k, v = _rand((B, H, d), 31), _rand((B, H, N, d), 32), _rand((B, H, N, d), 33)
+    idx = np.array([[0, 5], [2, 3], [1, 4], [5, 0]])
+    lens = [1, 37, 90, 64]
+    got, bad = oracle.sha_decode_varlen(q, k, v, idx, lens, 0.25, "fp16")
+    assert bad == 0
+    for b, L in enumerate(lens):
+        kt, vt = k[b:b + 1, :, :L].contiguous(), v[b:b + 1, :, :L].contiguous()
+        ref, _ = oracle.sha_decode(q[b:b + 1], kt, vt, idx[b:b + 1], 0.25, "fp16")
+        np.testing.assert_array_equal(got[b], ref[0])
+        sd = torch.nn.functional.scaled_dot_product_attention(
+            q[b:b + 1].double().unsqueeze(2), kt.double(), vt.double(), scale=0.25).squeeze(2)
+        for h in idx[b]:
+            np.testing.assert_allclose(got[b, h], sd[0, h].numpy(), rtol=0, atol=1e-12)
+
+
+def test_varlen_full_lengths_equal_fixed_and_bad_lengths_are_skipped():
+    B, H, N, d = 3, 4, 20, 8
+    q, k, v = _rand((B, H, d), 34), _rand((B, H, N, d), 35), _rand((B, H, N, d), 36)
+    idx = np.array([[0, 1], [2, 3], [3, 0]])
+    fixed, _ = oracle.sha_decode(q, k, v, idx, 0.3, "fp16")
+    same, bad = oracle.sha_decode_varlen(q, k, v, idx, [N, N, N], 0.3, "fp16")
+    assert bad == 0 and np.array_equal(np.isnan(fixed), np.isnan(same))
+    np.testing.assert_array_equal(fixed[~np.isnan(fixed)], same[~np.isnan(same)])
+    out, bad = oracle.sha_decode_varlen(q, k, v, idx, [0, N + 1, 5], 0.3, "fp16")
+    assert bad == 4 and np.isnan(out[:2]).all() and not np.isnan(out[2, [3, 0]]).any()
