@@ -156,6 +156,24 @@ def sha_decode_bf16(q, k, v, batch_head_index, scale, out, stream=None):
     return out
 
 
+_lib.sha_decode_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                   ctypes.c_float, _vp, _i, _vp]
+_lib.sha_decode_varlen.restype = _i
+
+
+def sha_decode_varlen(q, k, v, batch_head_index, seqlens, scale, out, stream=None):
+    """Selective head decode where row b uses the first seqlens[b] keys of its
+    [N_max]-long cache (seqlens: int32 [B] on the device, each in [1, N_max])."""
+    args, s = _decode_args(q, k, v, batch_head_index, scale, out, stream)
+    if (seqlens.dim() != 1 or seqlens.shape[0] != k.shape[0] or seqlens.dtype != torch.int32
+            or not seqlens.is_contiguous() or seqlens.device != k.device):
+        raise ValueError("seqlens must be a contiguous int32 [B] tensor on k's device")
+    with torch.cuda.device(k.device):
+        _check(_lib.sha_decode_varlen(*args[:4], seqlens.data_ptr(), *args[4:],
+                                      _dtype_code(k.dtype), s))
+    return out
+
+
 def _dtype_code(dtype):
     if dtype == torch.float16:
         return SHA_FP16
@@ -280,6 +298,6 @@ def sha_copy_bandwidth_probe(dst, src, stream=None):
 __all__ = [
     "sha_decode", "sha_decode_bf16", "sha_decode_ex", "sha_decode_workspace_size",
     "sha_get_device_status", "sha_status_string", "sha_decode_plan", "sha_select_heads",
-    "decode_from_scores", "sha_copy_bandwidth_probe", "decode",
+    "decode_from_scores", "sha_decode_varlen", "sha_copy_bandwidth_probe", "decode",
     "alloc_workspace", "ShaError", "LIBRARY_PATH", "sha_decode_noalloc",
 ]

@@ -198,14 +198,30 @@ sha_status_t kv_tensor_map(CUtensorMap *map, const void *base, sha_dtype_t dtype
     return SHA_OK;
 }
 
-template <typename T, int D>
+// Per-row lengths: the kernel plans its own split from the lengths on the
+// device, using at most this many blocks; the workspace covers any split.
+Plan make_varlen_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int num_splits,
+                      int num_sms)
+{
+    Plan pl = make_plan(B, H_q, H_kv, N_kv, d, top_k, 0, num_sms);
+    long long ctas = num_splits > 0 ? num_splits : (long long)num_sms * kBlocksPerSm;
+    if (ctas > sha::kMaxBlocks) ctas = sha::kMaxBlocks;
+    if (ctas > pl.sched.total_tiles) ctas = pl.sched.total_tiles;
+    if (ctas < 1) ctas = 1;
+    pl.sched.num_ctas = (int)ctas;
+    pl.counter_bytes = sha::kCounterBytes;
+    pl.slot_bytes = (size_t)2 * pl.sched.num_ctas * pl.slot_floats * sizeof(float);
+    return pl;
+}
+
+template <typename T, int D, bool kVarlen>
 sha_status_t launch_gqa(const sha::DecodeParams &prm, sha_dtype_t dtype, int dev,
                         cudaStream_t stream)
 {
     using C = sha::GqaConfig<D>;
     static bool configured[kMaxDevices] = {};
     if (!configured[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(sha::sha_gqa_decode_kernel<T, D>,
+        cudaError_t e = cudaFuncSetAttribute(sha::sha_gqa_decode_kernel<T, D, kVarlen>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::kSmemBytes);
         if (e != cudaSuccess) return launch_error(e);
@@ -217,35 +233,55 @@ sha_status_t launch_gqa(const sha::DecodeParams &prm, sha_dtype_t dtype, int dev
     if (st != SHA_OK) return st;
     st = kv_tensor_map(&tm_v, prm.v, dtype, D, prm.N_kv, planes);
     if (st != SHA_OK) return st;
-    cudaError_t e = launch_kernel(sha::sha_gqa_decode_kernel<T, D>, prm.sched.num_ctas,
+    cudaError_t e = launch_kernel(sha::sha_gqa_decode_kernel<T, D, kVarlen>, prm.sched.num_ctas,
                                   C::kThreads, C::kSmemBytes, stream, prm, tm_k, tm_v);
     if (e != cudaSuccess) return launch_error(e);
     return SHA_OK;
 }
 
-template <typename T, int D>
+template <typename T, int D, bool kVarlen>
 sha_status_t launch_mha(const sha::DecodeParams &prm, int dev, cudaStream_t stream)
 {
     using C = sha::MhaConfig<D>;
     static bool configured[kMaxDevices] = {};
     if (!configured[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(sha::sha_mha_decode_kernel<T, D>,
+        cudaError_t e = cudaFuncSetAttribute(sha::sha_mha_decode_kernel<T, D, kVarlen>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::kSmemBytes);
         if (e != cudaSuccess) return launch_error(e);
         configured[dev] = true;
     }
-    cudaError_t e = launch_kernel(sha::sha_mha_decode_kernel<T, D>, prm.sched.num_ctas,
+    cudaError_t e = launch_kernel(sha::sha_mha_decode_kernel<T, D, kVarlen>, prm.sched.num_ctas,
                                   C::kThreads, C::kSmemBytes, stream, prm);
     if (e != cudaSuccess) return launch_error(e);
     return SHA_OK;
 }
 
+template <bool kVarlen>
+sha_status_t launch_decode(const sha::DecodeParams &prm, sha_dtype_t dtype, int d, int G,
+                           int dev, cudaStream_t s)
+{
+    if (G > 1) {
+        if (dtype == SHA_FP16)
+            return d == 128 ? launch_gqa<__half, 128, kVarlen>(prm, dtype, dev, s)
+                            : launch_gqa<__half, 64, kVarlen>(prm, dtype, dev, s);
+        return d == 128 ? launch_gqa<__nv_bfloat16, 128, kVarlen>(prm, dtype, dev, s)
+                        : launch_gqa<__nv_bfloat16, 64, kVarlen>(prm, dtype, dev, s);
+    }
+    if (dtype == SHA_FP16)
+        return d == 128 ? launch_mha<__half, 128, kVarlen>(prm, dev, s)
+                        : launch_mha<__half, 64, kVarlen>(prm, dev, s);
+    return d == 128 ? launch_mha<__nv_bfloat16, 128, kVarlen>(prm, dev, s)
+                    : launch_mha<__nv_bfloat16, 64, kVarlen>(prm, dev, s);
+}
+
+// seqlens == nullptr: every row has N_kv keys.  Otherwise row b has
+// seqlens[b] keys (device array) of an N_kv-long cache.
 sha_status_t decode_impl(const void *q, const void *k, const void *v, const int32_t *idx,
                          int B, int H_q, int H_kv, int N_kv, int d, int top_k, float scale,
                          void *out, sha_dtype_t dtype, void *workspace,
                          size_t workspace_bytes, int num_splits, void *stream,
-                         bool library_workspace)
+                         bool library_workspace, const int32_t *seqlens = nullptr)
 {
     if (dtype != SHA_FP16 && dtype != SHA_BF16) return SHA_ERR_UNSUPPORTED;
     sha_status_t st = check_shape(B, H_q, H_kv, N_kv, d, top_k, scale);
@@ -257,6 +293,7 @@ sha_status_t decode_impl(const void *q, const void *k, const void *v, const int3
         !aligned(idx, 4))
         return SHA_ERR_MISALIGNED;
     if (workspace && !aligned(workspace, 256)) return SHA_ERR_MISALIGNED;
+    if (seqlens && !aligned(seqlens, 4)) return SHA_ERR_MISALIGNED;
     const int G = H_q / H_kv;
 
     int dev;
@@ -264,7 +301,9 @@ sha_status_t decode_impl(const void *q, const void *k, const void *v, const int3
     st = current_device(&dev, &info);
     if (st != SHA_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const Plan pl = make_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits, info->num_sms);
+    const Plan pl = seqlens ? make_varlen_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits,
+                                               info->num_sms)
+                            : make_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits, info->num_sms);
     const size_t need = pl.workspace_bytes();
 
     if (library_workspace && need > 0) {
@@ -307,18 +346,9 @@ sha_status_t decode_impl(const void *q, const void *k, const void *v, const int3
     prm.slots = need ? reinterpret_cast<float *>(static_cast<char *>(workspace) +
                                                  pl.counter_bytes)
                      : nullptr;
-
-    if (G > 1) {
-        if (dtype == SHA_FP16)
-            return d == 128 ? launch_gqa<__half, 128>(prm, dtype, dev, s)
-                            : launch_gqa<__half, 64>(prm, dtype, dev, s);
-        return d == 128 ? launch_gqa<__nv_bfloat16, 128>(prm, dtype, dev, s)
-                        : launch_gqa<__nv_bfloat16, 64>(prm, dtype, dev, s);
-    }
-    if (dtype == SHA_FP16)
-        return d == 128 ? launch_mha<__half, 128>(prm, dev, s) : launch_mha<__half, 64>(prm, dev, s);
-    return d == 128 ? launch_mha<__nv_bfloat16, 128>(prm, dev, s)
-                    : launch_mha<__nv_bfloat16, 64>(prm, dev, s);
+    prm.seqlens = seqlens;
+    return seqlens ? launch_decode<true>(prm, dtype, d, G, dev, s)
+                   : launch_decode<false>(prm, dtype, d, G, dev, s);
 }
 
 __global__ void copy_probe_kernel(uint4 *__restrict__ dst, const uint4 *__restrict__ src,
@@ -367,6 +397,16 @@ sha_status_t sha_decode_ex(const void *q, const void *k, const void *v,
 {
     return decode_impl(q, k, v, batch_head_index, B, H_q, H_kv, N_kv, d, top_k, scale, out,
                        dtype, workspace, workspace_bytes, num_splits, stream, false);
+}
+
+sha_status_t sha_decode_varlen(const void *q, const void *k, const void *v,
+                               const int32_t *batch_head_index, const int32_t *seqlens, int B,
+                               int H_q, int H_kv, int N_max, int d, int top_k, float scale,
+                               void *out, sha_dtype_t dtype, void *stream)
+{
+    if (B > 0 && top_k > 0 && !seqlens) return SHA_ERR_INVALID_ARG;
+    return decode_impl(q, k, v, batch_head_index, B, H_q, H_kv, N_max, d, top_k, scale, out,
+                       dtype, nullptr, 0, 0, stream, true, seqlens);
 }
 
 size_t sha_decode_workspace_size(int B, int H_q, int H_kv, int N_kv, int d, int top_k,

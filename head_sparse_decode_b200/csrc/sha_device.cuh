@@ -14,6 +14,9 @@ namespace sha {
 // Sticky status bits, read and cleared by sha_get_device_status().
 enum : unsigned { kStatusBadIndex = 1u, kStatusTimeout = 2u };
 
+// Sticky device status (one per device per loaded library).
+static __device__ unsigned int g_sha_status;
+
 // A pipeline wait that has not completed after this long gives up, raises
 // kStatusTimeout and lets the kernel unwind.  Healthy waits last microseconds.
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;
@@ -98,6 +101,13 @@ __device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32
         " [%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(dst)),
         "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
         : "memory");
+}
+
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy (bulk copy / TMA) accesses of the same bytes.
+__device__ __forceinline__ void fence_proxy_async_shared()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // Named barrier over `threads` threads (a multiple of 32), id 1..15.

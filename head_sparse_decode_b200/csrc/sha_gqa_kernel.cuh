@@ -27,10 +27,13 @@
 
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "sha_device.cuh"
 #include "sha_merge.cuh"
 #include "sha_mha_kernel.cuh"
 #include "sha_schedule.cuh"
+#include "sha_walk.cuh"
 
 namespace sha {
 
@@ -63,9 +66,11 @@ struct GqaConfig {
     static constexpr int kVOffset = kStages * kTileBytes;
     static constexpr int kBarOffset = 2 * kStages * kTileBytes;
     static constexpr int kFlagOffset = kBarOffset + 2 * kStages * 8;
-    static constexpr int kStateOffset = kFlagOffset + 16;
+    static constexpr int kPlanOffset = kFlagOffset + 16;       // 32 longs: per-row-length plan
+    static constexpr int kStateOffset = kPlanOffset + 256;
     static constexpr int kSmemBytes =
         kAlignPad + kStateOffset + kConsumerWarps * kStateFloats * 4;
+    static_assert(2 * (kThreads / 32) + 8 <= 32, "plan scratch fits");
     static_assert(kKeysPerWarp == 16, "one k-step of 16 keys per warp and slice");
     static_assert(kTile % 64 == 0 && kTile <= 256, "whole 64-key slices, TMA box <= 256 rows");
     static_assert(kBoxBytes % 1024 == 0, "boxes stay 1 KiB aligned");
@@ -149,11 +154,12 @@ __device__ __forceinline__ uint32_t swizzled(uint32_t tile, int key, int chunk)
     return tile + box * C::kBoxBytes + key * 128 + ((c ^ (key & 7)) << 4);
 }
 
-template <typename T, int D>
+template <typename T, int D, bool kVarlen>
 __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
     sha_gqa_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v)
 {
+    using Walk = typename std::conditional<kVarlen, VarlenWalk, UniformWalk>::type;
     using C = GqaConfig<D>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = reinterpret_cast<unsigned char *>(
@@ -183,9 +189,19 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
     pdl_wait();
     pdl_launch_dependents();
 
-    const Schedule S = p.sched;
-    const long long t_begin = S.begin(blockIdx.x);
-    const long long t_end = S.begin(blockIdx.x + 1);
+    Schedule S = p.sched;
+    Walk walk;
+    if constexpr (kVarlen) {
+        if (!varlen_plan<C::kThreads>(p.seqlens, p.B, p.top_k, p.N_kv, C::kTile, gridDim.x,
+                                      reinterpret_cast<long long *>(smem + C::kPlanOffset), S,
+                                      walk))
+            return;
+    } else {
+        walk.S = S;
+        walk.t = S.begin(blockIdx.x);
+        walk.t_end = S.begin(blockIdx.x + 1);
+        walk.n_keys = p.N_kv;
+    }
 
     // ------------------------------------------------------------ producer
     if (warp == C::kConsumerWarps) {
@@ -199,9 +215,9 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
         uint32_t phase = 0;
         uint32_t last_parity = 0, used = 0;
         bool ok = true;
-        for (long long t = t_begin; t < t_end && ok;) {
-            const Segment seg = segment_at(S, t, t_end);
-            t += seg.num_tiles;
+        Walk wk = walk;
+        Seg seg;
+        while (ok && wk.next(seg)) {
             const int b = (int)(seg.unit / p.top_k);
             const int h = p.idx[seg.unit];
             if ((unsigned)h >= (unsigned)p.H_kv) continue;
@@ -246,9 +262,9 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
 
-    for (long long t = t_begin; t < t_end;) {
-        const Segment seg = segment_at(S, t, t_end);
-        t += seg.num_tiles;
+    Walk wk = walk;
+    Seg seg;
+    for (bool first_seg = true; wk.next(seg); first_seg = false) {
         const long long u = seg.unit;
         const int b = (int)(u / p.top_k);
         const int h = p.idx[u];
@@ -290,7 +306,24 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
             if (live) {
                 const uint32_t kt = k_base + stage * C::kTileBytes;
                 const uint32_t vt = v_base + stage * C::kTileBytes;
-                const int rows = min(C::kTile, p.N_kv - j * C::kTile);
+                const int rows = min(C::kTile, seg.n_keys - j * C::kTile);
+                if constexpr (kVarlen) {
+                    // keys past this row's length but inside the cache hold stale
+                    // values: zero this warp's V rows there (0 * NaN would poison P V)
+                    if (rows < C::kTile) {
+                        unsigned char *vtile = v_ring + stage * C::kTileBytes;
+                        for (int i = lane; i < C::kSlices * 16 * C::kBoxes * 8; i += 32) {
+                            const int chunk = i & 7, bx = (i >> 3) % C::kBoxes;
+                            const int rr = (i >> 3) / C::kBoxes;      // 0 .. kSlices*16-1
+                            const int key = (rr >> 4) * 64 + warp * C::kKeysPerWarp + (rr & 15);
+                            if (key >= rows)
+                                *reinterpret_cast<uint4 *>(vtile + bx * C::kBoxBytes + key * 128 +
+                                                           chunk * 16) = make_uint4(0, 0, 0, 0);
+                        }
+                        fence_proxy_async_shared();   // before the stage is refilled by TMA
+                        __syncwarp();
+                    }
+                }
 
                 // S = Q K^T over this warp's 16 keys of each 64-key slice:
                 // two 8-key n-tiles per slice
@@ -398,7 +431,9 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
 
         T *out_g = static_cast<T *>(p.out) + ((size_t)b * p.H_q + (size_t)h * G) * D;
         const bool aborted = flags[0] != 0;
-        float *slot = p.slots ? p.slots + (size_t)S.slot_of(blockIdx.x, u) * p.slot_floats
+        // this block's first unit goes to slot 2c, any later partial one to 2c+1
+        float *slot = p.slots ? p.slots + (size_t)(2 * blockIdx.x + (first_seg ? 0 : 1)) *
+                                              p.slot_floats
                               : nullptr;
         if (!aborted) {
             for (int e = tid; e < G * D; e += C::kConsumers) {
@@ -431,8 +466,8 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
         named_barrier(1, C::kConsumers);
 
         if (!seg.whole) {
-            const int first = S.cta_of(u * S.tiles_per_unit);
-            const int last = S.cta_of((u + 1) * S.tiles_per_unit - 1);
+            int first, last, first_slot;
+            unit_parts(S, seg, first, last, first_slot);
             if (tid == 0) {
                 int merge = 0;
                 if (!flags[0]) {
@@ -444,9 +479,8 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
             named_barrier(1, C::kConsumers);
             if (flags[1]) {
                 __threadfence();
-                merge_parts<T, D, C::kConsumers>(p.slots, p.slot_floats, first,
-                                                  S.slot_of(first, u), last - first + 1, G,
-                                                  out_g, wstate, tid);
+                merge_parts<T, D, C::kConsumers>(p.slots, p.slot_floats, first, first_slot,
+                                                  last - first + 1, G, out_g, wstate, tid);
                 if (tid == 0) p.counters[first] = 0;
             }
         }

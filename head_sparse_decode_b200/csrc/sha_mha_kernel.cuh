@@ -28,14 +28,14 @@
 // O unnormalised and divides once at the end, which is the same quantity.
 #pragma once
 
+#include <type_traits>
+
 #include "sha_device.cuh"
 #include "sha_merge.cuh"
 #include "sha_schedule.cuh"
+#include "sha_walk.cuh"
 
 namespace sha {
-
-// Sticky device status (one per device per loaded library).
-static __device__ unsigned int g_sha_status;
 
 struct DecodeParams {
     const void *q;
@@ -49,6 +49,7 @@ struct DecodeParams {
     float *slots;            // 2*num_ctas partial states of slot_floats floats
     int slot_floats;
     int *counters;           // arrival counters, one per block, zero between calls
+    const int32_t *seqlens;  // per-row cache lengths (variable-length calls), else null
 };
 
 // Build-time tuning of the multi-head kernel (defaults measured best on B200).
@@ -79,18 +80,21 @@ struct MhaConfig {
     static constexpr int kVOffset = kStages * kTileBytes;
     static constexpr int kBarOffset = 2 * kStages * kTileBytes;
     static constexpr int kFlagOffset = kBarOffset + 2 * kStages * 8;
-    static constexpr int kStateOffset = kFlagOffset + 16;
+    static constexpr int kPlanOffset = kFlagOffset + 16;       // 32 longs: per-row-length plan
+    static constexpr int kStateOffset = kPlanOffset + 256;
     static constexpr int kSmemBytes = kStateOffset + kConsumerWarps * kStateFloats * 4;
+    static_assert(2 * (kThreads / 32) + 8 <= 32, "plan scratch fits");
     static_assert(kRowsPerWarp % 4 == 0, "score passes cover 4 rows");
     static_assert(kRowsPerWarp % kPvRowsPerIter == 0, "P.V iterations");
     static_assert(kConsumers >= D, "one consumer thread per output element");
     static_assert(kConsumerWarps * kStateFloats >= 3 * kMaxMergeParts, "merge staging fits");
 };
 
-template <typename T, int D>
+template <typename T, int D, bool kVarlen>
 __global__ void __launch_bounds__(MhaConfig<D>::kThreads, 1)
     sha_mha_decode_kernel(const DecodeParams p)
 {
+    using Walk = typename std::conditional<kVarlen, VarlenWalk, UniformWalk>::type;
     using C = MhaConfig<D>;
     extern __shared__ __align__(1024) unsigned char smem[];
     unsigned char *k_ring = smem + C::kKOffset;
@@ -117,9 +121,19 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, 1)
     pdl_wait();
     pdl_launch_dependents();
 
-    const Schedule S = p.sched;
-    const long long t_begin = S.begin(blockIdx.x);
-    const long long t_end = S.begin(blockIdx.x + 1);
+    Schedule S = p.sched;
+    Walk walk;
+    if constexpr (kVarlen) {
+        if (!varlen_plan<C::kThreads>(p.seqlens, p.B, p.top_k, p.N_kv, C::kTile, gridDim.x,
+                                      reinterpret_cast<long long *>(smem + C::kPlanOffset), S,
+                                      walk))
+            return;
+    } else {
+        walk.S = S;
+        walk.t = S.begin(blockIdx.x);
+        walk.t_end = S.begin(blockIdx.x + 1);
+        walk.n_keys = p.N_kv;
+    }
 
     // ------------------------------------------------------------ producer
     if (warp == C::kConsumerWarps) {
@@ -129,9 +143,9 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, 1)
         uint32_t phase = 0;
         uint32_t last_parity = 0, used = 0;   // per-stage parity of the last copy, stages used
         bool ok = true;
-        for (long long t = t_begin; t < t_end && ok;) {
-            const Segment seg = segment_at(S, t, t_end);
-            t += seg.num_tiles;
+        Walk wk = walk;
+        Seg seg;
+        while (ok && wk.next(seg)) {
             const int b = (int)(seg.unit / p.top_k);
             const int h = p.idx[seg.unit];
             if ((unsigned)h >= (unsigned)p.H_kv) continue;
@@ -147,7 +161,7 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, 1)
                     break;
                 }
                 const int n0 = j * C::kTile;
-                const int rows = min(C::kTile, p.N_kv - n0);
+                const int rows = min(C::kTile, seg.n_keys - n0);
                 const uint32_t bytes = (uint32_t)rows * C::kRowBytes;
                 mbar_arrive_expect_tx(&full[stage], 2 * bytes);
                 bulk_copy_g2s(k_ring + stage * C::kTileBytes, kbase + (size_t)n0 * D, bytes,
@@ -176,9 +190,9 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
 
-    for (long long t = t_begin; t < t_end;) {
-        const Segment seg = segment_at(S, t, t_end);
-        t += seg.num_tiles;
+    Walk wk = walk;
+    Seg seg;
+    for (bool first_seg = true; wk.next(seg); first_seg = false) {
         const long long u = seg.unit;
         const int b = (int)(u / p.top_k);
         const int h = p.idx[u];
@@ -216,7 +230,7 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, 1)
                 }
             }
             if (live) {
-                const int rows = min(C::kTile, p.N_kv - j * C::kTile);
+                const int rows = min(C::kTile, seg.n_keys - j * C::kTile);
                 const unsigned char *kt = k_ring + stage * C::kTileBytes;
                 const unsigned char *vt = v_ring + stage * C::kTileBytes;
                 const int row0 = warp * C::kRowsPerWarp;
@@ -320,7 +334,9 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, 1)
                 T *orow = static_cast<T *>(p.out) + ((size_t)b * p.H_q + h) * D;
                 orow[tid] = Elem<T>::from_float(O / L);
             } else {
-                float *slot = p.slots + (size_t)S.slot_of(blockIdx.x, u) * p.slot_floats;
+                // this block's first unit goes to slot 2c, any later partial one to 2c+1
+                float *slot = p.slots + (size_t)(2 * blockIdx.x + (first_seg ? 0 : 1)) *
+                                            p.slot_floats;
                 slot[tid] = O;
                 if (tid == 0) {
                     slot[D] = M;
@@ -332,8 +348,8 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, 1)
         named_barrier(1, C::kConsumers);
 
         if (!seg.whole) {
-            const int first = S.cta_of(u * S.tiles_per_unit);
-            const int last = S.cta_of((u + 1) * S.tiles_per_unit - 1);
+            int first, last, first_slot;
+            unit_parts(S, seg, first, last, first_slot);
             if (tid == 0) {
                 int merge = 0;
                 if (!flags[0]) {
@@ -348,9 +364,8 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, 1)
                 // Last block to finish its piece: merge all pieces in block order.
                 __threadfence();
                 T *orow = static_cast<T *>(p.out) + ((size_t)b * p.H_q + h) * D;
-                merge_parts<T, D, C::kConsumers>(p.slots, p.slot_floats, first,
-                                                  S.slot_of(first, u), last - first + 1, 1,
-                                                  orow, wstate, tid);
+                merge_parts<T, D, C::kConsumers>(p.slots, p.slot_floats, first, first_slot,
+                                                  last - first + 1, 1, orow, wstate, tid);
                 if (tid == 0) p.counters[first] = 0;
             }
         }

@@ -117,6 +117,25 @@ sha_status_t sha_decode_ex(const void *q, const void *k, const void *v,
                            void *stream);
 
 /*
+ * sha_decode_varlen -- the same operation when every batch row has its own
+ * cache length, as in a decode batch of sequences of different lengths:
+ * row b attends to keys [0, seqlens[b]) of its cache.
+ *   k, v     : [B, H_kv, N_max, d] (rows padded to N_max; keys at or past
+ *              seqlens[b] are never used and may hold anything)
+ *   seqlens  : device pointer, int32 [B], each in [1, N_max]; a row whose
+ *              length is outside that range is skipped (its outputs stay
+ *              untouched) and raises the SHA_ERR_BAD_INDEX flag
+ *   dtype    : SHA_FP16 or SHA_BF16; other arguments as for sha_decode.
+ * The lengths stay on the device: the kernel plans its own balanced split
+ * from them (every block streams the same number of key tiles).  Uses the
+ * library-owned per-device workspace, like sha_decode.
+ */
+sha_status_t sha_decode_varlen(const void *q, const void *k, const void *v,
+                               const int32_t *batch_head_index, const int32_t *seqlens,
+                               int B, int H_q, int H_kv, int N_max, int d, int top_k,
+                               float scale, void *out, sha_dtype_t dtype, void *stream);
+
+/*
  * sha_decode_workspace_size -- bytes of workspace sha_decode_ex needs for
  * these sizes and num_splits (0 = automatic) on the current device.  Host
  * only; reads the device's SM count.  Returns 0 for sizes sha_decode_ex
