@@ -326,6 +326,7 @@ def run_ours(args, rank, world, local):
         extras["density_sweep"] = density_sweep(sha, w, q, k, v, dev, stream, peak)
         extras["e2e"] = e2e(sha, w, q, k, v, idx, out, dev, stream, args)
         extras["other_configs"] = other_configs(sha, w, dev, stream, peak, rank)
+        extras["other_configs"].append(varlen_config(sha, dev, stream, peak, rank))
     plan = sha.sha_decode_plan(w.B, w.H_q, w.H_kv, w.N_kv, w.d, w.top_k,
                                num_sms=torch.cuda.get_device_properties(dev).multi_processor_count)
     line = {
@@ -404,6 +405,36 @@ def other_configs(sha, w_main, dev, stream, peak, rank):
                     "bytes_per_step": w.algorithmic_bytes()})
         del q, k, v, idx, out
         torch.cuda.empty_cache()
+    return res
+
+
+def varlen_config(sha, dev, stream, peak, rank):
+    """LLaMA-2-7B shape with per-row cache lengths drawn uniformly from [1, 4096]
+    (a decode batch of sequences of different lengths)."""
+    w = workloads.CONFIGS["llama2_7b"].with_(N_kv=4096, seed=2500 + 100 * rank)
+    q, k, v = workloads.make_qkv(w, device=dev)
+    idx = workloads.make_index(w).to(dev)
+    out = workloads.make_out(w, dev)
+    g = torch.Generator().manual_seed(w.seed + 11)
+    lens = torch.randint(1, w.N_kv + 1, (w.B,), generator=g, dtype=torch.int32)
+    lens_d = lens.to(dev)
+    # algorithmic bytes: active K+V of each row's own length, Q/O rows, index, lengths
+    kv = sum(2 * int(L) * w.d * 2 * w.top_k for L in lens.tolist())
+    nbytes = kv + 2 * w.units * w.G * w.d * 2 + 4 * w.units + 4 * w.B
+
+    def call():
+        sha.sha_decode_varlen(q, k, v, idx, lens_d, w.scale, out)
+    for _ in range(20):
+        call()
+    steps = 500
+    t = timed_graphs(call, steps, dev, stream)
+    gbs = nbytes * steps / t / 1e9
+    res = {"workload": "llama2_7b_varlen", "lengths": "uniform [1, 4096], seeded",
+           "mean_len": round(float(lens.float().mean()), 1), "us_per_step": round(t / steps * 1e6, 2),
+           "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
+           "steps_per_s": round(steps / t, 1), "bytes_per_step": nbytes}
+    del q, k, v
+    torch.cuda.empty_cache()
     return res
 
 

@@ -305,3 +305,32 @@ def test_long_context_16k_gqa_and_mha(sha):
         q, k, v, idx = _on_gpu(w)
         out = _run(sha, w, q, k, v, idx)
         check_against_oracle(w, q, k, v, idx, out)
+
+
+# ---------------------------------------------------------------- CUDA-graph capture
+
+def test_select_and_decode_captured_in_a_cuda_graph(sha):
+    """Head selection + decode captured once and replayed with new inputs copied
+    into the captured buffers: every replay matches an eager call."""
+    w = W("graph", B=16, H_q=32, H_kv=8, N_kv=1000, d=128, top_k=3, dtype="bf16", seed=91)
+    q, k, v, _ = _on_gpu(w)
+    scores = torch.randn((w.B, w.H_kv), device="cuda")
+    out = workloads.make_out(w, "cuda")
+    sha.decode_from_scores(q, k, v, scores, w.top_k, w.scale, out)      # warm-up, workspace
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        _, idx_g = sha.decode_from_scores(q, k, v, scores, w.top_k, w.scale, out)
+    for step in range(3):
+        gen = torch.Generator(device="cuda").manual_seed(100 + step)
+        q.copy_(torch.randn(q.shape, generator=gen, device="cuda").to(q.dtype))
+        scores.copy_(torch.randn(scores.shape, generator=gen, device="cuda"))
+        out.view(torch.int16).fill_(workloads.SENTINEL["bf16"])
+        graph.replay()
+        torch.cuda.synchronize()
+        ref = workloads.make_out(w, "cuda")
+        ref, idx_e = sha.decode_from_scores(q, k, v, scores, w.top_k, w.scale, ref)
+        torch.cuda.synchronize()
+        assert torch.equal(idx_g, idx_e)
+        assert np.array_equal(out_bits(out), out_bits(ref))
+    check_against_oracle(w, q, k, v, idx_e, out)
