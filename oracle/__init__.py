@@ -53,6 +53,11 @@ def _load():
         lib.sha_oracle_decode_varlen.argtypes = [
             u16p, u16p, u16p, i32p, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int, f64p]
+        lib.sha_oracle_decode_paged.restype = ctypes.c_longlong
+        lib.sha_oracle_decode_paged.argtypes = [
+            u16p, u16p, u16p, i32p, i32p, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_double, ctypes.c_int, f64p]
         lib.sha_oracle_select_heads.restype = ctypes.c_int
         lib.sha_oracle_select_heads.argtypes = [
             ctypes.POINTER(ctypes.c_float), ctypes.c_int, ctypes.c_int, ctypes.c_int, i32p]
@@ -187,6 +192,31 @@ def sha_decode_varlen(q, k, v, batch_head_index, seqlens, scale, dtype, out=None
         _ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16),
         _ptr(idx, ctypes.c_int32), _ptr(lens, ctypes.c_int32), B, H_q, H_kv, N_max, d, top_k,
         float(scale), _dtype_code(dtype), _ptr(out, ctypes.c_double))
+    if bad < 0:
+        raise ValueError("inconsistent sizes")
+    return out, int(bad)
+
+
+def sha_decode_paged(q, k_pages, v_pages, batch_head_index, seqlens, block_table, scale, dtype,
+                     out=None):
+    """Selective head decode over a paged cache: k/v_pages [num_pages, H_kv, page_size, d],
+    block_table [B, max_pages], seqlens [B].  Returns (out, count of skipped units)."""
+    qb, kb, vb = _bits(q), _bits(k_pages), _bits(v_pages)
+    num_pages, H_kv, page_size, d = kb.shape
+    bt = np.ascontiguousarray(np.asarray(block_table, dtype=np.int32))
+    B, max_pages = bt.shape
+    qb = qb.reshape(B, -1, d)
+    H_q = qb.shape[1]
+    idx = np.ascontiguousarray(np.asarray(batch_head_index, dtype=np.int32).reshape(B, -1))
+    lens = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32).reshape(B))
+    top_k = idx.shape[1]
+    if out is None:
+        out = np.full((B, H_q, d), np.nan, dtype=np.float64)
+    bad = _load().sha_oracle_decode_paged(
+        _ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16),
+        _ptr(idx, ctypes.c_int32), _ptr(lens, ctypes.c_int32), _ptr(bt, ctypes.c_int32),
+        B, H_q, H_kv, num_pages, page_size, max_pages, d, top_k, float(scale),
+        _dtype_code(dtype), _ptr(out, ctypes.c_double))
     if bad < 0:
         raise ValueError("inconsistent sizes")
     return out, int(bad)

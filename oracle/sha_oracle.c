@@ -323,3 +323,59 @@ long long sha_oracle_decode_varlen(const uint16_t *Q, const uint16_t *K,
     }
     return bad;
 }
+
+/*
+ * Selective head decode over a paged KV cache (the serving layout in which a
+ * sequence's keys live in fixed-size pages of a shared pool):
+ *   K, V        : [num_pages, H_kv, page_size, d]
+ *   block_table : [B, max_pages]; key n of row b is at page
+ *                 block_table[b, n / page_size], position n % page_size
+ *   seqlens     : [B]; row b attends to keys [0, seqlens[b])
+ * Each unit gathers its row's keys and values through the block table and is
+ * then exactly the per-row-length decode.  A row whose length is outside
+ * [1, max_pages * page_size], or that needs a page id outside [0, num_pages),
+ * is skipped and counted with the out-of-range head ids.
+ */
+long long sha_oracle_decode_paged(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
+                                  const int32_t *batch_head_index, const int32_t *seqlens,
+                                  const int32_t *block_table, int B, int H_q, int H_kv,
+                                  int num_pages, int page_size, int max_pages, int d,
+                                  int top_k, double scale, int dtype, double *out)
+{
+    if (B < 0 || H_kv <= 0 || H_q <= 0 || H_q % H_kv != 0 || num_pages <= 0 ||
+        page_size <= 0 || max_pages <= 0 || d <= 0 || top_k < 0)
+        return -1;
+    int G = H_q / H_kv;
+    long long bad = 0;
+    long long units = (long long)B * top_k;
+#pragma omp parallel for schedule(dynamic, 1) reduction(+ : bad)
+    for (long long u = 0; u < units; ++u) {
+        long long b = u / top_k;
+        int h = batch_head_index[u];
+        int n = seqlens[b];
+        int ok = h >= 0 && h < H_kv && n >= 1 && n <= max_pages * page_size;
+        for (int p = 0; ok && p < (n + page_size - 1) / page_size; ++p) {
+            int page = block_table[b * (long long)max_pages + p];
+            if (page < 0 || page >= num_pages) ok = 0;
+        }
+        if (!ok) {
+            bad += 1;
+            continue;
+        }
+        uint16_t *Kg = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)n * d);
+        uint16_t *Vg = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)n * d);
+        for (int key = 0; key < n; ++key) {
+            int page = block_table[b * (long long)max_pages + key / page_size];
+            size_t src = (((size_t)page * H_kv + h) * page_size + key % page_size) * (size_t)d;
+            memcpy(Kg + (size_t)key * d, K + src, sizeof(uint16_t) * (size_t)d);
+            memcpy(Vg + (size_t)key * d, V + src, sizeof(uint16_t) * (size_t)d);
+        }
+        for (int j = 0; j < G; ++j) {
+            size_t row = ((size_t)b * H_q + (size_t)h * G + j) * (size_t)d;
+            attention(Q + row, Kg, Vg, n, d, scale, dtype, 0, out + row);
+        }
+        free(Vg);
+        free(Kg);
+    }
+    return bad;
+}

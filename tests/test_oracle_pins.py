@@ -304,3 +304,47 @@ def test_varlen_full_lengths_equal_fixed_and_bad_lengths_are_skipped():
     np.testing.assert_array_equal(fixed[~np.isnan(fixed)], same[~np.isnan(same)])
     out, bad = oracle.sha_decode_varlen(q, k, v, idx, [0, N + 1, 5], 0.3, "fp16")
     assert bad == 4 and np.isnan(out[:2]).all() and not np.isnan(out[2, [3, 0]]).any()
+
+
+# ---------------------------------------------------------------- paged cache
+
+def _to_pages(k, page_size, perm):
+    """[B, H, N, d] contiguous cache -> [B*N/ps, H, ps, d] pages, page i of row b stored
+    at pool slot perm[b*P + i]; returns (pool, block_table)."""
+    B, H, N, d = k.shape
+    P = N // page_size
+    pool = torch.empty((B * P, H, page_size, d), dtype=k.dtype)
+    table = np.empty((B, P), dtype=np.int32)
+    for b in range(B):
+        for i in range(P):
+            slot = int(perm[b * P + i])
+            pool[slot] = k[b, :, i * page_size:(i + 1) * page_size]
+            table[b, i] = slot
+    return pool, table
+
+
+@pytest.mark.parametrize("page_size", [1, 16, 64])
+def test_paged_equals_contiguous_varlen_for_any_page_placement(page_size):
+    B, H, N, d = 3, 4, 128, 16
+    q, k, v = _rand((B, H, d), 41), _rand((B, H, N, d), 42), _rand((B, H, N, d), 43)
+    idx = np.array([[0, 3], [2, 1], [3, 2]])
+    lens = [1, 77, 128]
+    perm = np.random.default_rng(page_size).permutation(B * N // page_size)
+    kp, table = _to_pages(k, page_size, perm)
+    vp, _ = _to_pages(v, page_size, perm)
+    want, _ = oracle.sha_decode_varlen(q, k, v, idx, lens, 0.3, "fp16")
+    got, bad = oracle.sha_decode_paged(q, kp, vp, idx, lens, table, 0.3, "fp16")
+    assert bad == 0
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(want))
+    np.testing.assert_array_equal(got[~np.isnan(got)], want[~np.isnan(want)])
+
+
+def test_paged_rows_with_bad_pages_or_lengths_are_skipped():
+    B, H, N, d, ps = 3, 2, 32, 8, 16
+    q, k, v = _rand((B, H, d), 44), _rand((B, H, N, d), 45), _rand((B, H, N, d), 46)
+    kp, table = _to_pages(k, ps, np.arange(B * N // ps))
+    vp, _ = _to_pages(v, ps, np.arange(B * N // ps))
+    table[1, 1] = 999                           # row 1 needs page 1 (length 20)
+    out, bad = oracle.sha_decode_paged(q, kp, vp, [[0], [1], [0]], [5, 20, 33], table, 0.5,
+                                       "fp16")
+    assert bad == 2 and not np.isnan(out[0, 0]).any() and np.isnan(out[1:]).all()
