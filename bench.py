@@ -327,6 +327,7 @@ def run_ours(args, rank, world, local):
         extras["e2e"] = e2e(sha, w, q, k, v, idx, out, dev, stream, args)
         extras["other_configs"] = other_configs(sha, w, dev, stream, peak, rank)
         extras["other_configs"].append(varlen_config(sha, dev, stream, peak, rank))
+        extras["other_configs"].append(paged_config(sha, dev, stream, peak, rank))
     plan = sha.sha_decode_plan(w.B, w.H_q, w.H_kv, w.N_kv, w.d, w.top_k,
                                num_sms=torch.cuda.get_device_properties(dev).multi_processor_count)
     line = {
@@ -434,6 +435,40 @@ def varlen_config(sha, dev, stream, peak, rank):
            "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
            "steps_per_s": round(steps / t, 1), "bytes_per_step": nbytes}
     del q, k, v
+    torch.cuda.empty_cache()
+    return res
+
+
+def paged_config(sha, dev, stream, peak, rank, page_size=16):
+    """OPT-66B shape with its cache in 16-key pages scattered over a pool in
+    random order (the serving layout), every row 1920 long."""
+    w = workloads.CONFIGS["opt66b"].with_(seed=1500 + 100 * rank)
+    P = -(-w.N_kv // page_size)
+    n_pages = w.B * P
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed)
+    q = torch.randn((w.B, w.H_q, w.d), generator=g, device=dev).half()
+    kp = torch.randn((n_pages, w.H_kv, page_size, w.d), generator=g, device=dev).half()
+    vp = torch.randn((n_pages, w.H_kv, page_size, w.d), generator=g, device=dev).half()
+    gc = torch.Generator().manual_seed(w.seed + 3)
+    table = torch.randperm(n_pages, generator=gc).to(torch.int32).view(w.B, P).to(dev)
+    lens = torch.full((w.B,), w.N_kv, dtype=torch.int32, device=dev)
+    idx = workloads.make_index(w).to(dev)
+    out = workloads.make_out(w, dev)
+    nbytes = w.algorithmic_bytes() + 4 * w.B + 4 * w.B * P
+
+    def call():
+        sha.sha_decode_paged(q, kp, vp, idx, lens, table, w.scale, out)
+    for _ in range(20):
+        call()
+    steps = 500
+    t = timed_graphs(call, steps, dev, stream)
+    gbs = nbytes * steps / t / 1e9
+    res = {"workload": f"opt66b_paged{page_size}", "page_size": page_size,
+           "us_per_step": round(t / steps * 1e6, 2), "gbs": round(gbs, 1),
+           "frac": round(gbs / peak, 4), "steps_per_s": round(steps / t, 1),
+           "bytes_per_step": nbytes}
+    del q, kp, vp
     torch.cuda.empty_cache()
     return res
 

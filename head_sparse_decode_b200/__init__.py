@@ -174,6 +174,41 @@ def sha_decode_varlen(q, k, v, batch_head_index, seqlens, scale, out, stream=Non
     return out
 
 
+_lib.sha_decode_paged.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
+                                  ctypes.c_float, _vp, _i, _vp]
+_lib.sha_decode_paged.restype = _i
+
+
+def sha_decode_paged(q, k_pages, v_pages, batch_head_index, seqlens, block_table, scale, out,
+                     stream=None):
+    """Selective head decode over a paged cache: k/v_pages [num_pages, H_kv, page_size, d],
+    block_table int32 [B, max_pages], seqlens int32 [B] (all on one device)."""
+    if k_pages.dim() != 4 or v_pages.shape != k_pages.shape:
+        raise ValueError("k_pages and v_pages must both be [num_pages, H_kv, page_size, d]")
+    num_pages, H_kv, page_size, d = k_pages.shape
+    B = q.shape[0]
+    H_q = q.shape[1]
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("block_table must be [B, max_pages]")
+    max_pages = block_table.shape[1]
+    for name, t, dt in (("block_table", block_table, torch.int32), ("seqlens", seqlens, torch.int32),
+                        ("batch_head_index", batch_head_index, torch.int32),
+                        ("q", q, k_pages.dtype), ("v_pages", v_pages, k_pages.dtype),
+                        ("out", out, k_pages.dtype)):
+        if t.dtype != dt or not t.is_contiguous() or t.device != k_pages.device:
+            raise ValueError(f"{name} must be a contiguous {dt} tensor on {k_pages.device}")
+    if seqlens.shape != (B,) or q.shape[-1] != d or out.numel() != B * H_q * d:
+        raise ValueError("inconsistent shapes")
+    top_k = batch_head_index.shape[1]
+    with torch.cuda.device(k_pages.device):
+        _check(_lib.sha_decode_paged(
+            q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), batch_head_index.data_ptr(),
+            seqlens.data_ptr(), block_table.data_ptr(), B, H_q, H_kv, num_pages, page_size,
+            max_pages, d, top_k, _default_scale(scale, d), out.data_ptr(),
+            _dtype_code(k_pages.dtype), _stream_handle(stream, k_pages.device)))
+    return out
+
+
 def _dtype_code(dtype):
     if dtype == torch.float16:
         return SHA_FP16
@@ -298,6 +333,6 @@ def sha_copy_bandwidth_probe(dst, src, stream=None):
 __all__ = [
     "sha_decode", "sha_decode_bf16", "sha_decode_ex", "sha_decode_workspace_size",
     "sha_get_device_status", "sha_status_string", "sha_decode_plan", "sha_select_heads",
-    "decode_from_scores", "sha_decode_varlen", "sha_copy_bandwidth_probe", "decode",
+    "decode_from_scores", "sha_decode_varlen", "sha_decode_paged", "sha_copy_bandwidth_probe", "decode",
     "alloc_workspace", "ShaError", "LIBRARY_PATH", "sha_decode_noalloc",
 ]

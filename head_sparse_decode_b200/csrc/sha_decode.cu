@@ -172,7 +172,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 // 3-D view [B*H_kv][N_kv][d] of a K or V cache, 64x64-element boxes with
 // 128-byte swizzle; rows past N_kv read as zero.
 sha_status_t kv_tensor_map(CUtensorMap *map, const void *base, sha_dtype_t dtype, int d,
-                           int N_kv, long long planes)
+                           int N_kv, long long planes, int box_rows)
 {
     PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
     if (!encode) {
@@ -182,7 +182,7 @@ sha_status_t kv_tensor_map(CUtensorMap *map, const void *base, sha_dtype_t dtype
     }
     cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N_kv, (cuuint64_t)planes};
     cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N_kv * d * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)sha::GqaConfig<128>::kTile, 1};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
     cuuint32_t elem[3] = {1, 1, 1};
     CUresult r = encode(map,
                         dtype == SHA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -214,75 +214,86 @@ Plan make_varlen_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int 
     return pl;
 }
 
-template <typename T, int D, bool kVarlen>
+template <typename T, int D, int kLayout>
 sha_status_t launch_gqa(const sha::DecodeParams &prm, sha_dtype_t dtype, int dev,
                         cudaStream_t stream)
 {
     using C = sha::GqaConfig<D>;
     static bool configured[kMaxDevices] = {};
     if (!configured[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(sha::sha_gqa_decode_kernel<T, D, kVarlen>,
+        cudaError_t e = cudaFuncSetAttribute(sha::sha_gqa_decode_kernel<T, D, kLayout>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::kSmemBytes);
         if (e != cudaSuccess) return launch_error(e);
         configured[dev] = true;
     }
     CUtensorMap tm_k, tm_v;
-    const long long planes = (long long)prm.B * prm.H_kv;
-    sha_status_t st = kv_tensor_map(&tm_k, prm.k, dtype, D, prm.N_kv, planes);
+    // a padded cache: [B*H_kv][N_kv][d]; a page pool: [num_pages*H_kv][page_size][d]
+    const bool paged = kLayout == sha::kLayoutPaged;
+    const long long planes = paged ? (long long)prm.num_pages * prm.H_kv : (long long)prm.B * prm.H_kv;
+    const int rows = paged ? prm.page_size : prm.N_kv;
+    const int box_rows = paged && prm.page_size < C::kTile ? prm.page_size : C::kTile;
+    sha_status_t st = kv_tensor_map(&tm_k, prm.k, dtype, D, rows, planes, box_rows);
     if (st != SHA_OK) return st;
-    st = kv_tensor_map(&tm_v, prm.v, dtype, D, prm.N_kv, planes);
+    st = kv_tensor_map(&tm_v, prm.v, dtype, D, rows, planes, box_rows);
     if (st != SHA_OK) return st;
-    cudaError_t e = launch_kernel(sha::sha_gqa_decode_kernel<T, D, kVarlen>, prm.sched.num_ctas,
+    cudaError_t e = launch_kernel(sha::sha_gqa_decode_kernel<T, D, kLayout>, prm.sched.num_ctas,
                                   C::kThreads, C::kSmemBytes, stream, prm, tm_k, tm_v);
     if (e != cudaSuccess) return launch_error(e);
     return SHA_OK;
 }
 
-template <typename T, int D, bool kVarlen>
+template <typename T, int D, int kLayout>
 sha_status_t launch_mha(const sha::DecodeParams &prm, int dev, cudaStream_t stream)
 {
     using C = sha::MhaConfig<D>;
     static bool configured[kMaxDevices] = {};
     if (!configured[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(sha::sha_mha_decode_kernel<T, D, kVarlen>,
+        cudaError_t e = cudaFuncSetAttribute(sha::sha_mha_decode_kernel<T, D, kLayout>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::kSmemBytes);
         if (e != cudaSuccess) return launch_error(e);
         configured[dev] = true;
     }
-    cudaError_t e = launch_kernel(sha::sha_mha_decode_kernel<T, D, kVarlen>, prm.sched.num_ctas,
+    cudaError_t e = launch_kernel(sha::sha_mha_decode_kernel<T, D, kLayout>, prm.sched.num_ctas,
                                   C::kThreads, C::kSmemBytes, stream, prm);
     if (e != cudaSuccess) return launch_error(e);
     return SHA_OK;
 }
 
-template <bool kVarlen>
+template <int kLayout>
 sha_status_t launch_decode(const sha::DecodeParams &prm, sha_dtype_t dtype, int d, int G,
                            int dev, cudaStream_t s)
 {
     if (G > 1) {
         if (dtype == SHA_FP16)
-            return d == 128 ? launch_gqa<__half, 128, kVarlen>(prm, dtype, dev, s)
-                            : launch_gqa<__half, 64, kVarlen>(prm, dtype, dev, s);
-        return d == 128 ? launch_gqa<__nv_bfloat16, 128, kVarlen>(prm, dtype, dev, s)
-                        : launch_gqa<__nv_bfloat16, 64, kVarlen>(prm, dtype, dev, s);
+            return d == 128 ? launch_gqa<__half, 128, kLayout>(prm, dtype, dev, s)
+                            : launch_gqa<__half, 64, kLayout>(prm, dtype, dev, s);
+        return d == 128 ? launch_gqa<__nv_bfloat16, 128, kLayout>(prm, dtype, dev, s)
+                        : launch_gqa<__nv_bfloat16, 64, kLayout>(prm, dtype, dev, s);
     }
     if (dtype == SHA_FP16)
-        return d == 128 ? launch_mha<__half, 128, kVarlen>(prm, dev, s)
-                        : launch_mha<__half, 64, kVarlen>(prm, dev, s);
-    return d == 128 ? launch_mha<__nv_bfloat16, 128, kVarlen>(prm, dev, s)
-                    : launch_mha<__nv_bfloat16, 64, kVarlen>(prm, dev, s);
+        return d == 128 ? launch_mha<__half, 128, kLayout>(prm, dev, s)
+                        : launch_mha<__half, 64, kLayout>(prm, dev, s);
+    return d == 128 ? launch_mha<__nv_bfloat16, 128, kLayout>(prm, dev, s)
+                    : launch_mha<__nv_bfloat16, 64, kLayout>(prm, dev, s);
 }
 
-// seqlens == nullptr: every row has N_kv keys.  Otherwise row b has
-// seqlens[b] keys (device array) of an N_kv-long cache.
+// Where the keys of a call live beyond the plain [B, H_kv, N_kv, d] cache.
+struct KvLayout {
+    const int32_t *seqlens = nullptr;       // per-row lengths (device), or null
+    const int32_t *block_table = nullptr;   // paged pool: [B, max_pages] (device), or null
+    int page_size = 0, max_pages = 0, num_pages = 0;
+};
+
+// N_kv is the padded length (per-row lengths) or max_pages * page_size (paged).
 sha_status_t decode_impl(const void *q, const void *k, const void *v, const int32_t *idx,
                          int B, int H_q, int H_kv, int N_kv, int d, int top_k, float scale,
                          void *out, sha_dtype_t dtype, void *workspace,
                          size_t workspace_bytes, int num_splits, void *stream,
-                         bool library_workspace, const int32_t *seqlens = nullptr)
+                         bool library_workspace, const KvLayout &lay = KvLayout())
 {
+    const int32_t *seqlens = lay.seqlens;
     if (dtype != SHA_FP16 && dtype != SHA_BF16) return SHA_ERR_UNSUPPORTED;
     sha_status_t st = check_shape(B, H_q, H_kv, N_kv, d, top_k, scale);
     if (st != SHA_OK) return st;
@@ -294,6 +305,7 @@ sha_status_t decode_impl(const void *q, const void *k, const void *v, const int3
         return SHA_ERR_MISALIGNED;
     if (workspace && !aligned(workspace, 256)) return SHA_ERR_MISALIGNED;
     if (seqlens && !aligned(seqlens, 4)) return SHA_ERR_MISALIGNED;
+    if (lay.block_table && !aligned(lay.block_table, 4)) return SHA_ERR_MISALIGNED;
     const int G = H_q / H_kv;
 
     int dev;
@@ -347,8 +359,13 @@ sha_status_t decode_impl(const void *q, const void *k, const void *v, const int3
                                                  pl.counter_bytes)
                      : nullptr;
     prm.seqlens = seqlens;
-    return seqlens ? launch_decode<true>(prm, dtype, d, G, dev, s)
-                   : launch_decode<false>(prm, dtype, d, G, dev, s);
+    prm.block_table = lay.block_table;
+    prm.page_size = lay.page_size;
+    prm.max_pages = lay.max_pages;
+    prm.num_pages = lay.num_pages;
+    if (lay.block_table) return launch_decode<sha::kLayoutPaged>(prm, dtype, d, G, dev, s);
+    if (seqlens) return launch_decode<sha::kLayoutVarlen>(prm, dtype, d, G, dev, s);
+    return launch_decode<sha::kLayoutFixed>(prm, dtype, d, G, dev, s);
 }
 
 __global__ void copy_probe_kernel(uint4 *__restrict__ dst, const uint4 *__restrict__ src,
@@ -405,8 +422,33 @@ sha_status_t sha_decode_varlen(const void *q, const void *k, const void *v,
                                void *out, sha_dtype_t dtype, void *stream)
 {
     if (B > 0 && top_k > 0 && !seqlens) return SHA_ERR_INVALID_ARG;
+    KvLayout lay;
+    lay.seqlens = seqlens;
     return decode_impl(q, k, v, batch_head_index, B, H_q, H_kv, N_max, d, top_k, scale, out,
-                       dtype, nullptr, 0, 0, stream, true, seqlens);
+                       dtype, nullptr, 0, 0, stream, true, lay);
+}
+
+sha_status_t sha_decode_paged(const void *q, const void *k_pages, const void *v_pages,
+                              const int32_t *batch_head_index, const int32_t *seqlens,
+                              const int32_t *block_table, int B, int H_q, int H_kv,
+                              int num_pages, int page_size, int max_pages, int d, int top_k,
+                              float scale, void *out, sha_dtype_t dtype, void *stream)
+{
+    if (num_pages < 1 || page_size < 1 || max_pages < 1) return SHA_ERR_INVALID_ARG;
+    if ((long long)max_pages * page_size > (1 << 30)) return SHA_ERR_INVALID_ARG;
+    if (H_kv >= 1 && H_q % H_kv == 0 && H_q / H_kv > 1 &&
+        (page_size < 8 || (page_size & (page_size - 1)) != 0))
+        return SHA_ERR_UNSUPPORTED;   // TMA boxes of whole pages: powers of two >= 8
+    if (B > 0 && top_k > 0 && (!seqlens || !block_table)) return SHA_ERR_INVALID_ARG;
+    KvLayout lay;
+    lay.seqlens = seqlens;
+    lay.block_table = block_table;
+    lay.page_size = page_size;
+    lay.max_pages = max_pages;
+    lay.num_pages = num_pages;
+    return decode_impl(q, k_pages, v_pages, batch_head_index, B, H_q, H_kv,
+                       max_pages * page_size, d, top_k, scale, out, dtype, nullptr, 0, 0,
+                       stream, true, lay);
 }
 
 size_t sha_decode_workspace_size(int B, int H_q, int H_kv, int N_kv, int d, int top_k,

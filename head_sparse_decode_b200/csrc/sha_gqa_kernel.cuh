@@ -154,11 +154,12 @@ __device__ __forceinline__ uint32_t swizzled(uint32_t tile, int key, int chunk)
     return tile + box * C::kBoxBytes + key * 128 + ((c ^ (key & 7)) << 4);
 }
 
-template <typename T, int D, bool kVarlen>
+template <typename T, int D, int kLayout>
 __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
     sha_gqa_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v)
 {
+    constexpr bool kVarlen = kLayout != kLayoutFixed;
     using Walk = typename std::conditional<kVarlen, VarlenWalk, UniformWalk>::type;
     using C = GqaConfig<D>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -230,13 +231,43 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
                     ok = false;
                     break;
                 }
-                mbar_arrive_expect_tx(&full[stage], 2 * C::kTileBytes);
+                if constexpr (kLayout == kLayoutPaged) {
+                    // boxes of min(page_size, tile) keys, each inside one page,
+                    // landing at 1 KiB-aligned rows of the swizzled tile
+                    const int n0 = j * C::kTile;
+                    const int rows = min(C::kTile, seg.n_keys - n0);
+                    const int box_rows = min(p.page_size, C::kTile);
+                    const int chunks = (rows + box_rows - 1) / box_rows;
+                    mbar_arrive_expect_tx(&full[stage],
+                                          (uint32_t)(2 * chunks * C::kBoxes * box_rows * 128));
+                    const int32_t *bt = p.block_table + (size_t)b * p.max_pages;
+                    for (int c = 0; c < chunks; ++c) {
+                        const int key = n0 + c * box_rows;
+                        const int pi = key / p.page_size, off = key - pi * p.page_size;
+                        int page = bt[pi];
+                        if ((unsigned)page >= (unsigned)p.num_pages) {
+                            atomicOr(&g_sha_status, kStatusBadIndex);
+                            page = 0;                   // stay inside the pool
+                        }
+                        const int pplane = page * p.H_kv + h;
+                        for (int bx = 0; bx < C::kBoxes; ++bx) {
+                            tma_load_3d(k_ring + stage * C::kTileBytes + bx * C::kBoxBytes +
+                                            c * box_rows * 128,
+                                        &tm_k, bx * 64, off, pplane, &full[stage], policy);
+                            tma_load_3d(v_ring + stage * C::kTileBytes + bx * C::kBoxBytes +
+                                            c * box_rows * 128,
+                                        &tm_v, bx * 64, off, pplane, &full[stage], policy);
+                        }
+                    }
+                } else {
+                    mbar_arrive_expect_tx(&full[stage], 2 * C::kTileBytes);
 #pragma unroll
-                for (int bx = 0; bx < C::kBoxes; ++bx) {
-                    tma_load_3d(k_ring + stage * C::kTileBytes + bx * C::kBoxBytes, &tm_k,
-                                bx * 64, j * C::kTile, plane, &full[stage], policy);
-                    tma_load_3d(v_ring + stage * C::kTileBytes + bx * C::kBoxBytes, &tm_v,
-                                bx * 64, j * C::kTile, plane, &full[stage], policy);
+                    for (int bx = 0; bx < C::kBoxes; ++bx) {
+                        tma_load_3d(k_ring + stage * C::kTileBytes + bx * C::kBoxBytes, &tm_k,
+                                    bx * 64, j * C::kTile, plane, &full[stage], policy);
+                        tma_load_3d(v_ring + stage * C::kTileBytes + bx * C::kBoxBytes, &tm_v,
+                                    bx * 64, j * C::kTile, plane, &full[stage], policy);
+                    }
                 }
                 last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
                 used |= 1u << stage;

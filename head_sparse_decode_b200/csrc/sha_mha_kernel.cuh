@@ -50,7 +50,15 @@ struct DecodeParams {
     int slot_floats;
     int *counters;           // arrival counters, one per block, zero between calls
     const int32_t *seqlens;  // per-row cache lengths (variable-length calls), else null
+    // paged cache: k, v are page pools [num_pages, H_kv, page_size, d] and key n
+    // of row b sits in page block_table[b, n / page_size]
+    const int32_t *block_table;
+    int page_size, max_pages, num_pages;
 };
+
+// How K/V of a unit are found: one padded [N_kv] block per (b, h) with every
+// row N_kv long or with per-row lengths, or pages of a shared pool.
+enum : int { kLayoutFixed = 0, kLayoutVarlen = 1, kLayoutPaged = 2 };
 
 // Build-time tuning of the multi-head kernel (defaults measured best on B200).
 #ifndef SHA_MHA_TILE_KEYS
@@ -90,10 +98,11 @@ struct MhaConfig {
     static_assert(kConsumerWarps * kStateFloats >= 3 * kMaxMergeParts, "merge staging fits");
 };
 
-template <typename T, int D, bool kVarlen>
+template <typename T, int D, int kLayout>
 __global__ void __launch_bounds__(MhaConfig<D>::kThreads, 1)
     sha_mha_decode_kernel(const DecodeParams p)
 {
+    constexpr bool kVarlen = kLayout != kLayoutFixed;
     using Walk = typename std::conditional<kVarlen, VarlenWalk, UniformWalk>::type;
     using C = MhaConfig<D>;
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -164,10 +173,34 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, 1)
                 const int rows = min(C::kTile, seg.n_keys - n0);
                 const uint32_t bytes = (uint32_t)rows * C::kRowBytes;
                 mbar_arrive_expect_tx(&full[stage], 2 * bytes);
-                bulk_copy_g2s(k_ring + stage * C::kTileBytes, kbase + (size_t)n0 * D, bytes,
-                              &full[stage], policy);
-                bulk_copy_g2s(v_ring + stage * C::kTileBytes, vbase + (size_t)n0 * D, bytes,
-                              &full[stage], policy);
+                if constexpr (kLayout == kLayoutPaged) {
+                    // one copy per run of keys that lie in one page
+                    const int32_t *bt = p.block_table + (size_t)b * p.max_pages;
+                    for (int key = n0, dst = 0; dst < rows;) {
+                        const int pi = key / p.page_size, off = key - pi * p.page_size;
+                        const int run = min(rows - dst, p.page_size - off);
+                        int page = bt[pi];
+                        if ((unsigned)page >= (unsigned)p.num_pages) {
+                            atomicOr(&g_sha_status, kStatusBadIndex);
+                            page = 0;                   // stay inside the pool
+                        }
+                        const size_t src =
+                            (((size_t)page * p.H_kv + h) * p.page_size + off) * D;
+                        bulk_copy_g2s(k_ring + stage * C::kTileBytes + dst * C::kRowBytes,
+                                      static_cast<const T *>(p.k) + src,
+                                      (uint32_t)run * C::kRowBytes, &full[stage], policy);
+                        bulk_copy_g2s(v_ring + stage * C::kTileBytes + dst * C::kRowBytes,
+                                      static_cast<const T *>(p.v) + src,
+                                      (uint32_t)run * C::kRowBytes, &full[stage], policy);
+                        key += run;
+                        dst += run;
+                    }
+                } else {
+                    bulk_copy_g2s(k_ring + stage * C::kTileBytes, kbase + (size_t)n0 * D,
+                                  bytes, &full[stage], policy);
+                    bulk_copy_g2s(v_ring + stage * C::kTileBytes, vbase + (size_t)n0 * D,
+                                  bytes, &full[stage], policy);
+                }
                 last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
                 used |= 1u << stage;
                 if (++stage == C::kStages) { stage = 0; phase ^= 1; }

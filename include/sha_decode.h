@@ -136,6 +136,28 @@ sha_status_t sha_decode_varlen(const void *q, const void *k, const void *v,
                                float scale, void *out, sha_dtype_t dtype, void *stream);
 
 /*
+ * sha_decode_paged -- the same operation over a paged KV cache, the serving
+ * layout in which each sequence's keys live in fixed-size pages of a pool:
+ *   k_pages, v_pages : [num_pages, H_kv, page_size, d]
+ *   block_table      : device pointer, int32 [B, max_pages]; key n of row b
+ *                      sits at page block_table[b, n / page_size], position
+ *                      n % page_size
+ *   seqlens          : device pointer, int32 [B], each in
+ *                      [1, max_pages * page_size]
+ *   page_size >= 1; for G = H_q/H_kv > 1 a power of two >= 8
+ *   (SHA_ERR_UNSUPPORTED otherwise).
+ * Rows with a bad length are skipped and flagged as in sha_decode_varlen.
+ * A page id outside [0, num_pages) is bad input: the flag is raised, no
+ * memory outside the pool is read, and that unit's output is unspecified.
+ * Uses the library-owned per-device workspace, like sha_decode.
+ */
+sha_status_t sha_decode_paged(const void *q, const void *k_pages, const void *v_pages,
+                              const int32_t *batch_head_index, const int32_t *seqlens,
+                              const int32_t *block_table, int B, int H_q, int H_kv,
+                              int num_pages, int page_size, int max_pages, int d, int top_k,
+                              float scale, void *out, sha_dtype_t dtype, void *stream);
+
+/*
  * sha_decode_workspace_size -- bytes of workspace sha_decode_ex needs for
  * these sizes and num_splits (0 = automatic) on the current device.  Host
  * only; reads the device's SM count.  Returns 0 for sizes sha_decode_ex
