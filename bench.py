@@ -87,11 +87,17 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback (no MEASURED_PEAKS.json)"
 
 
+# the sources the selective-head decode kernels are built from (kernels, their
+# helpers and the launch path); a change to any of them voids a stored capture
+DECODE_SOURCES = ("sha_decode.cu", "sha_device.cuh", "sha_gqa_kernel.cuh", "sha_merge.cuh",
+                  "sha_mha_kernel.cuh", "sha_schedule.cuh", "sha_walk.cuh")
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "head_sparse_decode_b200", "csrc", "*"))):
-        with open(p, "rb") as f:
-            h.update(os.path.basename(p).encode() + b"\0" + f.read())
+    for name in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "head_sparse_decode_b200", "csrc", name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()
 
 

@@ -206,7 +206,10 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
 
     // ------------------------------------------------------------ producer
     if (warp == C::kConsumerWarps) {
-        if (lane != 0) return;
+        // A paged cache needs several page ids per tile: the whole warp gathers
+        // them (one page box per lane).  Otherwise one lane drives the pipeline.
+        constexpr bool kWarpProducer = kLayout == kLayoutPaged;
+        if (!kWarpProducer && lane != 0) return;
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k))
                      : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v))
@@ -224,13 +227,18 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
             if ((unsigned)h >= (unsigned)p.H_kv) continue;
             const int plane = b * p.H_kv + h;
             for (int j = seg.first_tile; j < seg.first_tile + seg.num_tiles; ++j) {
-                if (flags[0]) { ok = false; break; }
-                if (!mbar_wait(&empty[stage], phase ^ 1)) {
-                    atomicOr(&g_sha_status, kStatusTimeout);
-                    flags[0] = 1;
-                    ok = false;
-                    break;
+                bool go = true;
+                if (lane == 0) {
+                    if (flags[0]) {
+                        go = false;
+                    } else if (!mbar_wait(&empty[stage], phase ^ 1)) {
+                        atomicOr(&g_sha_status, kStatusTimeout);
+                        flags[0] = 1;
+                        go = false;
+                    }
                 }
+                if constexpr (kWarpProducer) go = __shfl_sync(0xffffffffu, go, 0);
+                if (!go) { ok = false; break; }
                 if constexpr (kLayout == kLayoutPaged) {
                     // boxes of min(page_size, tile) keys, each inside one page,
                     // landing at 1 KiB-aligned rows of the swizzled tile
@@ -238,10 +246,12 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
                     const int rows = min(C::kTile, seg.n_keys - n0);
                     const int box_rows = min(p.page_size, C::kTile);
                     const int chunks = (rows + box_rows - 1) / box_rows;
-                    mbar_arrive_expect_tx(&full[stage],
-                                          (uint32_t)(2 * chunks * C::kBoxes * box_rows * 128));
+                    if (lane == 0)
+                        mbar_arrive_expect_tx(
+                            &full[stage], (uint32_t)(2 * chunks * C::kBoxes * box_rows * 128));
+                    __syncwarp();
                     const int32_t *bt = p.block_table + (size_t)b * p.max_pages;
-                    for (int c = 0; c < chunks; ++c) {
+                    for (int c = lane; c < chunks; c += 32) {
                         const int key = n0 + c * box_rows;
                         const int pi = key / p.page_size, off = key - pi * p.page_size;
                         int page = bt[pi];
@@ -274,8 +284,10 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
                 if (++stage == C::kStages) { stage = 0; phase ^= 1; }
             }
         }
-        for (int s = 0; s < C::kStages; ++s)
-            if (used & (1u << s)) mbar_wait(&full[s], (last_parity >> s) & 1u);
+        if (lane == 0)
+            for (int s = 0; s < C::kStages; ++s)
+                if (used & (1u << s)) mbar_wait(&full[s], (last_parity >> s) & 1u);
+        if constexpr (kWarpProducer) __syncwarp();
         return;
     }
 

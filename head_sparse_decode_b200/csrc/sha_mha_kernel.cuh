@@ -146,7 +146,11 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, 1)
 
     // ------------------------------------------------------------ producer
     if (warp == C::kConsumerWarps) {
-        if (lane != 0) return;
+        // A paged cache needs several page ids per tile: the whole warp gathers
+        // them (one page run per lane) so a tile costs one round trip to the
+        // block table.  Otherwise one lane drives the pipeline.
+        constexpr bool kWarpProducer = kLayout == kLayoutPaged;
+        if (!kWarpProducer && lane != 0) return;
         const uint64_t policy = l2_policy_evict_first();
         int stage = 0;
         uint32_t phase = 0;
@@ -162,38 +166,45 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, 1)
             const T *kbase = static_cast<const T *>(p.k) + head;
             const T *vbase = static_cast<const T *>(p.v) + head;
             for (int j = seg.first_tile; j < seg.first_tile + seg.num_tiles; ++j) {
-                if (flags[0]) { ok = false; break; }
-                if (!mbar_wait(&empty[stage], phase ^ 1)) {
-                    atomicOr(&g_sha_status, kStatusTimeout);
-                    flags[0] = 1;
-                    ok = false;
-                    break;
+                bool go = true;
+                if (lane == 0) {
+                    if (flags[0]) {
+                        go = false;
+                    } else if (!mbar_wait(&empty[stage], phase ^ 1)) {
+                        atomicOr(&g_sha_status, kStatusTimeout);
+                        flags[0] = 1;
+                        go = false;
+                    }
                 }
+                if constexpr (kWarpProducer) go = __shfl_sync(0xffffffffu, go, 0);
+                if (!go) { ok = false; break; }
                 const int n0 = j * C::kTile;
                 const int rows = min(C::kTile, seg.n_keys - n0);
                 const uint32_t bytes = (uint32_t)rows * C::kRowBytes;
-                mbar_arrive_expect_tx(&full[stage], 2 * bytes);
+                if (lane == 0) mbar_arrive_expect_tx(&full[stage], 2 * bytes);
                 if constexpr (kLayout == kLayoutPaged) {
-                    // one copy per run of keys that lie in one page
+                    // one copy per run of keys that lie in one page, a run per lane
+                    __syncwarp();
                     const int32_t *bt = p.block_table + (size_t)b * p.max_pages;
-                    for (int key = n0, dst = 0; dst < rows;) {
-                        const int pi = key / p.page_size, off = key - pi * p.page_size;
-                        const int run = min(rows - dst, p.page_size - off);
+                    const int ps = p.page_size;
+                    const int pi0 = n0 / ps, runs = (n0 + rows - 1) / ps - pi0 + 1;
+                    for (int r = lane; r < runs; r += 32) {
+                        const int pi = pi0 + r;
+                        const int k0 = max(n0, pi * ps), k1 = min(n0 + rows, (pi + 1) * ps);
                         int page = bt[pi];
                         if ((unsigned)page >= (unsigned)p.num_pages) {
                             atomicOr(&g_sha_status, kStatusBadIndex);
                             page = 0;                   // stay inside the pool
                         }
                         const size_t src =
-                            (((size_t)page * p.H_kv + h) * p.page_size + off) * D;
+                            (((size_t)page * p.H_kv + h) * ps + (k0 - pi * ps)) * D;
+                        const int dst = k0 - n0;
                         bulk_copy_g2s(k_ring + stage * C::kTileBytes + dst * C::kRowBytes,
                                       static_cast<const T *>(p.k) + src,
-                                      (uint32_t)run * C::kRowBytes, &full[stage], policy);
+                                      (uint32_t)(k1 - k0) * C::kRowBytes, &full[stage], policy);
                         bulk_copy_g2s(v_ring + stage * C::kTileBytes + dst * C::kRowBytes,
                                       static_cast<const T *>(p.v) + src,
-                                      (uint32_t)run * C::kRowBytes, &full[stage], policy);
-                        key += run;
-                        dst += run;
+                                      (uint32_t)(k1 - k0) * C::kRowBytes, &full[stage], policy);
                     }
                 } else {
                     bulk_copy_g2s(k_ring + stage * C::kTileBytes, kbase + (size_t)n0 * D,
@@ -207,8 +218,10 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, 1)
             }
         }
         // Never leave the block with a copy still landing in shared memory.
-        for (int s = 0; s < C::kStages; ++s)
-            if (used & (1u << s)) mbar_wait(&full[s], (last_parity >> s) & 1u);
+        if (lane == 0)
+            for (int s = 0; s < C::kStages; ++s)
+                if (used & (1u << s)) mbar_wait(&full[s], (last_parity >> s) & 1u);
+        if constexpr (kWarpProducer) __syncwarp();
         return;
     }
 
