@@ -58,6 +58,13 @@ def _load():
             u16p, u16p, u16p, i32p, i32p, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_double, ctypes.c_int, f64p]
+        lib.sha_oracle_mlp_union.restype = ctypes.c_int
+        lib.sha_oracle_mlp_union.argtypes = [ctypes.POINTER(ctypes.c_uint8), ctypes.c_int,
+                                             ctypes.c_int, i32p]
+        lib.sha_oracle_selective_mlp.restype = ctypes.c_int
+        lib.sha_oracle_selective_mlp.argtypes = [
+            u16p, u16p, u16p, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, f64p]
         lib.sha_oracle_select_heads.restype = ctypes.c_int
         lib.sha_oracle_select_heads.argtypes = [
             ctypes.POINTER(ctypes.c_float), ctypes.c_int, ctypes.c_int, ctypes.c_int, i32p]
@@ -220,3 +227,31 @@ def sha_decode_paged(q, k_pages, v_pages, batch_head_index, seqlens, block_table
     if bad < 0:
         raise ValueError("inconsistent sizes")
     return out, int(bad)
+
+
+def mlp_union(active):
+    """Sorted ids of the neurons active for any row: active [B, D] (bool/uint8)."""
+    a = np.ascontiguousarray(np.asarray(active).astype(np.uint8))
+    B, D = a.shape
+    S = np.empty(D, dtype=np.int32)
+    n = _load().sha_oracle_mlp_union(_ptr(a, ctypes.c_uint8), B, D, _ptr(S, ctypes.c_int32))
+    if n < 0:
+        raise ValueError("inconsistent sizes")
+    return S[:n].copy()
+
+
+def selective_mlp(x, W1t, W2t, S, dtype, act="relu"):
+    """sigma(x W1[:, S]) W2[:, S]^T in float64; x [B, d], W1t/W2t [D, d] (neuron-major),
+    S sorted neuron ids.  Returns float64 [B, d]."""
+    xb, w1, w2 = _bits(x), _bits(W1t), _bits(W2t)
+    B, d = xb.shape
+    D = w1.shape[0]
+    Sa = np.ascontiguousarray(np.asarray(S, dtype=np.int32))
+    y = np.empty((B, d), dtype=np.float64)
+    rc = _load().sha_oracle_selective_mlp(
+        _ptr(xb, ctypes.c_uint16), _ptr(w1, ctypes.c_uint16), _ptr(w2, ctypes.c_uint16),
+        _ptr(Sa, ctypes.c_int32), len(Sa), B, d, D, 1 if act == "relu" else 0,
+        _dtype_code(dtype), _ptr(y, ctypes.c_double))
+    if rc != 0:
+        raise ValueError("inconsistent sizes")
+    return y

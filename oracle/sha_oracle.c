@@ -379,3 +379,45 @@ long long sha_oracle_decode_paged(const uint16_t *Q, const uint16_t *K, const ui
     }
     return bad;
 }
+
+/*
+ * Selective GEMM -- the MLP half of Polar Sparsity (papernotes.org summary,
+ * "MLP 层动态稀疏"): for a decode batch x [B, d] and the union S_B of the
+ * neurons active for any row of the batch,
+ *     MLP_{S_B}(x) = sigma(x W1[:, S_B]) W2[:, S_B]^T,
+ * with W1, W2 of shape [d, D].  Both are passed transposed, neuron-major:
+ * W1t = W1^T and W2t = W2^T, [D, d], so neuron j's weights are row j.
+ * sigma is ReLU (act = 1) or the identity (act = 0).
+ */
+int sha_oracle_mlp_union(const uint8_t *active, int B, int D, int32_t *S)
+{
+    if (B < 0 || D <= 0) return -1;
+    int n = 0;
+    for (int j = 0; j < D; ++j) {
+        int any = 0;
+        for (int b = 0; b < B; ++b) any |= active[(size_t)b * D + j] != 0;
+        if (any) S[n++] = j;
+    }
+    return n;
+}
+
+int sha_oracle_selective_mlp(const uint16_t *x, const uint16_t *W1t, const uint16_t *W2t,
+                             const int32_t *S, int n_S, int B, int d, int D, int act,
+                             int dtype, double *y)
+{
+    if (B < 0 || d <= 0 || D <= 0 || n_S < 0 || n_S > D) return -1;
+#pragma omp parallel for schedule(static)
+    for (int b = 0; b < B; ++b) {
+        double *yb = y + (size_t)b * d;
+        for (int c = 0; c < d; ++c) yb[c] = 0.0;
+        for (int t = 0; t < n_S; ++t) {
+            const int j = S[t];
+            const uint16_t *w1 = W1t + (size_t)j * d, *w2 = W2t + (size_t)j * d;
+            double pre = 0.0;
+            for (int i = 0; i < d; ++i) pre += widen(x[(size_t)b * d + i], dtype) * widen(w1[i], dtype);
+            const double h = (act == 1 && pre < 0.0) ? 0.0 : pre;
+            for (int c = 0; c < d; ++c) yb[c] += h * widen(w2[c], dtype);
+        }
+    }
+    return 0;
+}

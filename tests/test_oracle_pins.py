@@ -348,3 +348,38 @@ def test_paged_rows_with_bad_pages_or_lengths_are_skipped():
     out, bad = oracle.sha_decode_paged(q, kp, vp, [[0], [1], [0]], [5, 20, 33], table, 0.5,
                                        "fp16")
     assert bad == 2 and not np.isnan(out[0, 0]).any() and np.isnan(out[1:]).all()
+
+
+# ---------------------------------------------------------------- selective GEMM (MLP)
+
+def test_mlp_union_matches_numpy():
+    rng = np.random.default_rng(5)
+    active = rng.random((7, 300)) < 0.05
+    assert np.array_equal(oracle.mlp_union(active), np.nonzero(active.any(0))[0])
+    assert len(oracle.mlp_union(np.zeros((3, 10), bool))) == 0
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_selective_mlp_all_neurons_is_the_dense_mlp(dtype):
+    """S = every neuron: relu(x W1) W2^T with torch in float64."""
+    B, d, D = 5, 24, 40
+    x, W1t, W2t = _rand((B, d), 51, dtype), _rand((D, d), 52, dtype), _rand((D, d), 53, dtype)
+    y = oracle.selective_mlp(x, W1t, W2t, np.arange(D), dtype)
+    ref = torch.relu(x.double() @ W1t.double().T) @ W2t.double()
+    np.testing.assert_allclose(y, ref.numpy(), rtol=0, atol=1e-11)
+
+
+def test_selective_mlp_equals_dense_with_unselected_neurons_removed():
+    B, d, D = 4, 16, 50
+    x, W1t, W2t = _rand((B, d), 54), _rand((D, d), 55), _rand((D, d), 56)
+    S = np.array([1, 7, 8, 20, 49])
+    y = oracle.selective_mlp(x, W1t, W2t, S, "fp16")
+    keep = torch.zeros(D, dtype=torch.float64)
+    keep[S] = 1.0
+    ref = (torch.relu(x.double() @ W1t.double().T) * keep) @ W2t.double()
+    np.testing.assert_allclose(y, ref.numpy(), rtol=0, atol=1e-12)
+    # identity activation, and the empty set
+    y_lin = oracle.selective_mlp(x, W1t, W2t, S, "fp16", act="identity")
+    ref_lin = ((x.double() @ W1t.double().T) * keep) @ W2t.double()
+    np.testing.assert_allclose(y_lin, ref_lin.numpy(), rtol=0, atol=1e-12)
+    assert (oracle.selective_mlp(x, W1t, W2t, [], "fp16") == 0).all()
