@@ -311,6 +311,72 @@ def decode_from_scores(q, k, v, scores, top_k, scale=None, out=None, stream=None
     return decode(q, k, v, idx, scale, out, stream), idx
 
 
+_lib.sha_mlp_union_workspace_size.argtypes = [_i]
+_lib.sha_mlp_union_workspace_size.restype = ctypes.c_size_t
+_lib.sha_mlp_union.argtypes = [_vp, _i, _i, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+_lib.sha_mlp_union.restype = _i
+_lib.sha_selective_mlp_workspace_size.argtypes = [_i, _i, _i]
+_lib.sha_selective_mlp_workspace_size.restype = ctypes.c_size_t
+_lib.sha_selective_mlp.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp,
+                                   ctypes.c_size_t, _vp]
+_lib.sha_selective_mlp.restype = _i
+
+
+def sha_mlp_union(active, S=None, n_S=None, workspace=None, stream=None):
+    """Union of active neurons over the batch: active [B, D] uint8/bool (CUDA) ->
+    (S int32 [D], n_S int32 [1]); the first n_S entries of S are the ids."""
+    if active.dtype == torch.bool:
+        active = active.view(torch.uint8)
+    if active.dim() != 2 or active.dtype != torch.uint8 or not active.is_contiguous():
+        raise ValueError("active must be a contiguous uint8/bool CUDA tensor [B, D]")
+    B, D = active.shape
+    dev = active.device
+    S = torch.empty(D, dtype=torch.int32, device=dev) if S is None else S
+    n_S = torch.empty(1, dtype=torch.int32, device=dev) if n_S is None else n_S
+    with torch.cuda.device(dev):
+        nbytes = int(_lib.sha_mlp_union_workspace_size(D))
+        if workspace is None:
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        _check(_lib.sha_mlp_union(active.data_ptr(), B, D, S.data_ptr(), n_S.data_ptr(),
+                                  workspace.data_ptr(), workspace.numel(),
+                                  _stream_handle(stream, dev)))
+    return S, n_S
+
+
+def sha_selective_mlp_workspace_size(B, d, D, device=None):
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        return int(_lib.sha_selective_mlp_workspace_size(B, d, D))
+
+
+def sha_selective_mlp(x, W1t, W2t, S, n_S, y=None, activation="relu", workspace=None,
+                      stream=None):
+    """Selective GEMM: y = sigma(x W1t[S]^T) W2t[S] over the first n_S ids of S.
+    x [B, d]; W1t, W2t [D, d] neuron-major; S int32 [>= n_S]; n_S int32 [1] (all CUDA)."""
+    B, d = x.shape
+    D = W1t.shape[0]
+    for name, t in (("x", x), ("W1t", W1t), ("W2t", W2t)):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != x.dtype:
+            raise ValueError(f"{name} must be a contiguous CUDA tensor of x's dtype")
+    if W1t.shape != (D, d) or W2t.shape != (D, d):
+        raise ValueError("W1t and W2t must both be [D, d]")
+    if S.dtype != torch.int32 or n_S.dtype != torch.int32:
+        raise TypeError("S and n_S must be int32")
+    dev = x.device
+    if y is None:
+        y = torch.empty((B, d), dtype=x.dtype, device=dev)
+    with torch.cuda.device(dev):
+        if workspace is None:
+            nbytes = int(_lib.sha_selective_mlp_workspace_size(B, d, D))
+            if nbytes == 0:
+                raise ShaError(SHA_ERR_UNSUPPORTED)
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        _check(_lib.sha_selective_mlp(
+            x.data_ptr(), W1t.data_ptr(), W2t.data_ptr(), S.data_ptr(), n_S.data_ptr(), B, d, D,
+            1 if activation == "relu" else 0, _dtype_code(x.dtype), y.data_ptr(),
+            workspace.data_ptr(), workspace.numel(), _stream_handle(stream, dev)))
+    return y
+
+
 def sha_get_device_status(stream=None, device=None):
     """Synchronise ``stream`` and read-and-clear the device's sticky flags; returns a
     status code (SHA_OK, SHA_ERR_BAD_INDEX or SHA_ERR_TIMEOUT)."""
@@ -333,6 +399,7 @@ def sha_copy_bandwidth_probe(dst, src, stream=None):
 __all__ = [
     "sha_decode", "sha_decode_bf16", "sha_decode_ex", "sha_decode_workspace_size",
     "sha_get_device_status", "sha_status_string", "sha_decode_plan", "sha_select_heads",
-    "decode_from_scores", "sha_decode_varlen", "sha_decode_paged", "sha_copy_bandwidth_probe", "decode",
+    "decode_from_scores", "sha_decode_varlen", "sha_decode_paged", "sha_mlp_union",
+    "sha_selective_mlp", "sha_selective_mlp_workspace_size", "sha_copy_bandwidth_probe", "decode",
     "alloc_workspace", "ShaError", "LIBRARY_PATH", "sha_decode_noalloc",
 ]

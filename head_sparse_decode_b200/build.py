@@ -41,7 +41,7 @@ def build(force: bool = False, verbose: bool = False, defines=(), output=None) -
     cmd = [NVCC, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, *[f"-D{d}" for d in defines]]
     if verbose:
         cmd += ["-Xptxas", "-v"]
-    cmd += ["-o", library + ".tmp", os.path.join(CSRC, "sha_decode.cu")]
+    cmd += ["-o", library + ".tmp", *sorted(glob.glob(os.path.join(CSRC, "*.cu")))]
     subprocess.run(cmd, check=True)
     os.replace(library + ".tmp", library)
     return library

@@ -502,6 +502,8 @@ sha_status_t sha_select_heads(const float *scores, int B, int H, int top_k,
     return SHA_OK;
 }
 
+unsigned sha_mlp_take_status();   // sha_mlp.cu
+
 sha_status_t sha_get_device_status(void *stream)
 {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -512,6 +514,7 @@ sha_status_t sha_get_device_status(void *stream)
     if (e != cudaSuccess) return launch_error(e);
     e = cudaMemcpyToSymbol(sha::g_sha_status, &zero, sizeof zero);
     if (e != cudaSuccess) return launch_error(e);
+    flags |= sha_mlp_take_status();
     if (flags & sha::kStatusTimeout) {
         // an abandoned merge can leave arrival counters raised: clear them
         int dev;

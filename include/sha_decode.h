@@ -196,6 +196,49 @@ sha_status_t sha_select_heads(const float *scores, int B, int H, int top_k,
                               int32_t *batch_head_index, void *stream);
 
 /*
+ * ---- Selective GEMM (the MLP half of Polar Sparsity) ----------------------
+ * papernotes.org summary, "MLP 层动态稀疏": for a decode batch x [B, d] and the
+ * union S_B of the neurons active for any of its rows,
+ *     MLP_{S_B}(x) = sigma(x W1[:, S_B]) W2[:, S_B]^T,
+ * read only the selected neurons' weights, the index gather fused into the
+ * GEMMs.  Weights are neuron-major: W1t = W1^T and W2t = W2^T, each [D, d]
+ * row-major, so neuron j's weights are row j.
+ */
+
+/* Bytes of workspace sha_mlp_union needs for D neurons. */
+size_t sha_mlp_union_workspace_size(int D);
+
+/*
+ * sha_mlp_union -- S_B from per-row activity: active [B, D] (uint8, nonzero =
+ * active, e.g. a router's thresholded predictions) -> S [D] int32 holding the
+ * ids of neurons active in any row in increasing order (first *n_S entries),
+ * and n_S (one int32 on the device).  All pointers are device pointers; the
+ * union size stays on the device for sha_selective_mlp.  Enqueued on `stream`.
+ */
+sha_status_t sha_mlp_union(const uint8_t *active, int B, int D, int32_t *S, int32_t *n_S,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/* Bytes of workspace sha_selective_mlp needs (current device); 0 if unsupported. */
+size_t sha_selective_mlp_workspace_size(int B, int d, int D);
+
+/*
+ * sha_selective_mlp -- y [B, d] = sigma(x W1t[S]^T) W2t[S] over the first *n_S
+ * ids of S (device memory; typically written by sha_mlp_union on the same
+ * stream, so no host synchronisation is needed).
+ *   x, y      : device, [B, d], fp16 or bf16 (dtype); W1t, W2t: [D, d]
+ *   1 <= B <= 64, d a multiple of 256 (SHA_ERR_UNSUPPORTED otherwise)
+ *   activation: 1 = ReLU (OPT's MLP), 0 = identity
+ *   workspace : device, 256-byte aligned, >= sha_selective_mlp_workspace_size
+ * The hidden activations are rounded to the input dtype before the second
+ * product (tensor-core operands); all sums are fp32.  Ids outside [0, D) are
+ * bad input: the flag is raised, no memory outside the weights is read.
+ */
+sha_status_t sha_selective_mlp(const void *x, const void *W1t, const void *W2t,
+                               const int32_t *S, const int32_t *n_S, int B, int d, int D,
+                               int activation, sha_dtype_t dtype, void *y, void *workspace,
+                               size_t workspace_bytes, void *stream);
+
+/*
  * sha_get_device_status -- synchronises `stream`, then reads and clears the
  * current device's sticky flags: SHA_ERR_BAD_INDEX if any call since the last
  * read met an out-of-range head id, SHA_ERR_TIMEOUT if a pipeline wait gave

@@ -64,7 +64,7 @@ def _load():
         lib.sha_oracle_selective_mlp.restype = ctypes.c_int
         lib.sha_oracle_selective_mlp.argtypes = [
             u16p, u16p, u16p, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-            ctypes.c_int, ctypes.c_int, f64p]
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, f64p]
         lib.sha_oracle_select_heads.restype = ctypes.c_int
         lib.sha_oracle_select_heads.argtypes = [
             ctypes.POINTER(ctypes.c_float), ctypes.c_int, ctypes.c_int, ctypes.c_int, i32p]
@@ -241,16 +241,20 @@ def mlp_union(active):
 
 
 def selective_mlp(x, W1t, W2t, S, dtype, act="relu"):
-    """sigma(x W1[:, S]) W2[:, S]^T in float64; x [B, d], W1t/W2t [D, d] (neuron-major),
-    S sorted neuron ids.  Returns float64 [B, d]."""
+    """sigma(x W1[:, S]) W2[:, S]^T in float64; x [B, d], W1t [D, d], W2t [D, d_out]
+    (neuron-major; d_out < d computes a subset of output columns), S neuron ids.
+    Returns float64 [B, d_out]."""
     xb, w1, w2 = _bits(x), _bits(W1t), _bits(W2t)
     B, d = xb.shape
     D = w1.shape[0]
+    if w1.shape != (D, d) or w2.ndim != 2 or w2.shape[0] != D:
+        raise ValueError("W1t must be [D, d] and W2t [D, d_out]")
+    d_out = w2.shape[1]
     Sa = np.ascontiguousarray(np.asarray(S, dtype=np.int32))
-    y = np.empty((B, d), dtype=np.float64)
+    y = np.empty((B, d_out), dtype=np.float64)
     rc = _load().sha_oracle_selective_mlp(
         _ptr(xb, ctypes.c_uint16), _ptr(w1, ctypes.c_uint16), _ptr(w2, ctypes.c_uint16),
-        _ptr(Sa, ctypes.c_int32), len(Sa), B, d, D, 1 if act == "relu" else 0,
+        _ptr(Sa, ctypes.c_int32), len(Sa), B, d, d_out, D, 1 if act == "relu" else 0,
         _dtype_code(dtype), _ptr(y, ctypes.c_double))
     if rc != 0:
         raise ValueError("inconsistent sizes")

@@ -401,22 +401,26 @@ int sha_oracle_mlp_union(const uint8_t *active, int B, int D, int32_t *S)
     return n;
 }
 
+/* W2t may hold a subset of the output columns: [D, d_out], y [B, d_out]
+ * (output columns are independent, so this is the same sum restricted). */
 int sha_oracle_selective_mlp(const uint16_t *x, const uint16_t *W1t, const uint16_t *W2t,
-                             const int32_t *S, int n_S, int B, int d, int D, int act,
-                             int dtype, double *y)
+                             const int32_t *S, int n_S, int B, int d, int d_out, int D,
+                             int act, int dtype, double *y)
 {
-    if (B < 0 || d <= 0 || D <= 0 || n_S < 0 || n_S > D) return -1;
+    if (B < 0 || d <= 0 || d_out <= 0 || D <= 0 || n_S < 0 || n_S > D) return -1;
+    for (int t = 0; t < n_S; ++t)
+        if (S[t] < 0 || S[t] >= D) return -1;
 #pragma omp parallel for schedule(static)
     for (int b = 0; b < B; ++b) {
-        double *yb = y + (size_t)b * d;
-        for (int c = 0; c < d; ++c) yb[c] = 0.0;
+        double *yb = y + (size_t)b * d_out;
+        for (int c = 0; c < d_out; ++c) yb[c] = 0.0;
         for (int t = 0; t < n_S; ++t) {
             const int j = S[t];
-            const uint16_t *w1 = W1t + (size_t)j * d, *w2 = W2t + (size_t)j * d;
+            const uint16_t *w1 = W1t + (size_t)j * d, *w2 = W2t + (size_t)j * d_out;
             double pre = 0.0;
             for (int i = 0; i < d; ++i) pre += widen(x[(size_t)b * d + i], dtype) * widen(w1[i], dtype);
             const double h = (act == 1 && pre < 0.0) ? 0.0 : pre;
-            for (int c = 0; c < d; ++c) yb[c] += h * widen(w2[c], dtype);
+            for (int c = 0; c < d_out; ++c) yb[c] += h * widen(w2[c], dtype);
         }
     }
     return 0;

@@ -1,0 +1,105 @@
+"""Selective GEMM on the GPU against the float64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from parity import TOLERANCE
+
+pytestmark = pytest.mark.gpu
+M = workloads.MlpWorkload
+
+
+@pytest.fixture(scope="module")
+def sha():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import head_sparse_decode_b200 as h
+    return h
+
+
+@pytest.mark.parametrize("B,D,p", [(1, 300, 0.1), (8, 5000, 0.02), (64, 2048, 0.5),
+                                   (3, 1, 1.0), (5, 1024, 0.0)])
+def test_union_bit_exact(sha, B, D, p):
+    g = torch.Generator().manual_seed(B * 100 + D)
+    active = (torch.rand((B, D), generator=g) < p).to(torch.uint8)
+    S, n_S = sha.sha_mlp_union(active.cuda())
+    torch.cuda.synchronize()
+    want = oracle.mlp_union(active.numpy())
+    n = int(n_S.item())
+    assert n == len(want)
+    assert np.array_equal(S[:n].cpu().numpy(), want)
+
+
+CASES = [
+    M("m1", B=1, d=256, D=1024, density=0.1, dtype="fp16", seed=1),
+    M("m2", B=8, d=512, D=2048, density=0.3, dtype="bf16", seed=2),
+    M("m3", B=64, d=256, D=1500, density=0.7, dtype="fp16", seed=3),
+    M("m4", B=17, d=768, D=3072, density=1.0, dtype="bf16", seed=4),
+    M("m5", B=5, d=256, D=4096, density=0.003, dtype="fp16", seed=5),
+]
+
+
+def _run(sha, w, act="relu"):
+    x, W1t, W2t, active = workloads.make_mlp(w)
+    dev = torch.device("cuda")
+    S, n_S = sha.sha_mlp_union(active.to(dev))
+    y = sha.sha_selective_mlp(x.to(dev), W1t.to(dev), W2t.to(dev), S, n_S, activation=act)
+    torch.cuda.synchronize()
+    assert sha.sha_get_device_status() == sha.SHA_OK
+    want_S = oracle.mlp_union(active.numpy())
+    assert int(n_S.item()) == len(want_S)
+    want = oracle.selective_mlp(x, W1t, W2t, want_S, w.dtype, act=act)
+    err = np.abs(y.cpu().double().numpy() - want).max()
+    return err, want
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_selective_mlp_parity(sha, w):
+    err, _ = _run(sha, w)
+    assert err <= TOLERANCE[w.dtype], err
+
+
+def test_selective_mlp_identity_activation(sha):
+    err, _ = _run(sha, CASES[1].with_(seed=21), act="identity")
+    assert err <= TOLERANCE["bf16"], err
+
+
+def test_empty_union_gives_zero(sha):
+    w = CASES[0]
+    x, W1t, W2t, _ = workloads.make_mlp(w)
+    dev = torch.device("cuda")
+    S = torch.zeros(w.D, dtype=torch.int32, device=dev)
+    n_S = torch.zeros(1, dtype=torch.int32, device=dev)
+    y = sha.sha_selective_mlp(x.to(dev), W1t.to(dev), W2t.to(dev), S, n_S)
+    torch.cuda.synchronize()
+    assert (y == 0).all()
+
+
+def test_out_of_range_ids_are_flagged_not_read(sha):
+    w = CASES[0]
+    x, W1t, W2t, _ = workloads.make_mlp(w)
+    dev = torch.device("cuda")
+    S = torch.tensor([3, 10**6, 7], dtype=torch.int32, device=dev)
+    n_S = torch.tensor([3], dtype=torch.int32, device=dev)
+    sha.sha_selective_mlp(x.to(dev), W1t.to(dev), W2t.to(dev), S, n_S)
+    assert sha.sha_get_device_status() == sha.SHA_ERR_BAD_INDEX
+
+
+def test_opt66b_mlp_shape_sampled(sha):
+    """The OPT-66B MLP at batch 8 and a 30 % union: sampled output columns."""
+    w = workloads.MLP_CONFIGS["opt66b_mlp"]
+    dev = torch.device("cuda")
+    x, W1t, W2t, active = workloads.make_mlp(w, device=dev)
+    S, n_S = sha.sha_mlp_union(active)
+    y = sha.sha_selective_mlp(x, W1t, W2t, S, n_S)
+    torch.cuda.synchronize()
+    assert sha.sha_get_device_status() == sha.SHA_OK
+    n = int(n_S.item())
+    Sh = S[:n].cpu().numpy()
+    assert np.array_equal(Sh, oracle.mlp_union(active.cpu().numpy()))
+    cols = np.sort(np.random.default_rng(0).choice(w.d, 256, replace=False))
+    want = oracle.selective_mlp(x.cpu(), W1t.cpu(), W2t[:, cols].cpu().contiguous(), Sh, w.dtype)
+    err = np.abs(y[:, cols].cpu().double().numpy() - want).max()
+    assert err <= TOLERANCE[w.dtype], err

@@ -383,3 +383,13 @@ def test_selective_mlp_equals_dense_with_unselected_neurons_removed():
     ref_lin = ((x.double() @ W1t.double().T) * keep) @ W2t.double()
     np.testing.assert_allclose(y_lin, ref_lin.numpy(), rtol=0, atol=1e-12)
     assert (oracle.selective_mlp(x, W1t, W2t, [], "fp16") == 0).all()
+
+
+def test_selective_mlp_column_subset_is_the_same_sum():
+    B, d, D = 3, 16, 30
+    x, W1t, W2t = _rand((B, d), 57), _rand((D, d), 58), _rand((D, d), 59)
+    S = [2, 5, 11, 29]
+    full = oracle.selective_mlp(x, W1t, W2t, S, "fp16")
+    cols = [1, 7, 15]
+    sub = oracle.selective_mlp(x, W1t, W2t[:, cols].contiguous(), S, "fp16")
+    np.testing.assert_array_equal(sub, full[:, cols])

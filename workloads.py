@@ -146,3 +146,58 @@ def make_out(w: Workload, device="cpu"):
     out.view(torch.int16).fill_(SENTINEL[w.dtype] - (1 << 16) if SENTINEL[w.dtype] >= 1 << 15
                                 else SENTINEL[w.dtype])
     return out
+
+
+# ---------------------------------------------------------------- selective GEMM (MLP)
+
+@dataclass(frozen=True)
+class MlpWorkload:
+    """One decoder MLP at decode time: batch B, hidden d, D = 4d neurons (OPT).
+    `density` is the fraction of neurons in the union of the batch's active sets."""
+    name: str
+    B: int
+    d: int
+    D: int
+    density: float
+    dtype: str = "fp16"
+    seed: int = 0
+
+    def with_(self, **kw):
+        return replace(self, **kw)
+
+    def n_union(self):
+        return max(1, int(round(self.density * self.D)))
+
+    def algorithmic_bytes(self):
+        """Selected rows of W1t and W2t, x read, y written, the active mask, S."""
+        n = self.n_union()
+        return 2 * n * self.d * 2 + 2 * self.B * self.d * 2 + self.B * self.D + 4 * self.D
+
+
+MLP_CONFIGS = {
+    # OPT-66B MLP (hidden 9216, 36864 neurons) at a small decode batch
+    "opt66b_mlp": MlpWorkload("opt66b_mlp", B=8, d=9216, D=36864, density=0.3, dtype="fp16",
+                              seed=5000),
+}
+
+
+def make_mlp(w: MlpWorkload, device="cpu"):
+    """x [B, d] ~ N(0,1); W1t [D, d] ~ N(0, 1/d); W2t [D, d] ~ N(0, 1/n_union), so
+    hidden pre-activations and outputs are O(1).  active [B, D] uint8: a seeded
+    union of n_union neurons, each of which is active in at least one row (rows
+    pick random subsets of the union)."""
+    dt = TORCH_DTYPE[w.dtype]
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed)
+    x = torch.randn((w.B, w.d), generator=g, device=device).to(dt)
+    W1t = (torch.randn((w.D, w.d), generator=g, device=device) / w.d ** 0.5).to(dt)
+    W2t = (torch.randn((w.D, w.d), generator=g, device=device) / w.n_union() ** 0.5).to(dt)
+    gc = torch.Generator().manual_seed(w.seed + 7)
+    union = torch.randperm(w.D, generator=gc)[: w.n_union()]
+    owner = torch.randint(0, w.B, (len(union),), generator=gc)
+    extra = torch.rand((w.B, len(union)), generator=gc) < 0.3
+    active = torch.zeros((w.B, w.D), dtype=torch.uint8)
+    active[owner, union] = 1
+    cols = union.unsqueeze(0).expand(w.B, -1)
+    active[extra.nonzero(as_tuple=True)[0], cols[extra]] = 1
+    return x, W1t, W2t, active.to(device)
