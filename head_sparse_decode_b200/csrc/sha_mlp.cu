@@ -13,15 +13,18 @@
 //
 // Kernels (each launched with programmatic stream serialization):
 //   mlp_union_flags / mlp_union_write -- S_B as sorted neuron ids + n_S
-//   mlp_up    -- P[split] = x . W1t[S]^T over a range of d (fp32 partials):
-//                M = 128 gathered neurons, N = batch, K = d in 128-wide tiles
-//   mlp_act   -- H = sigma(sum of the splits), rounded to the input dtype
-//   mlp_down  -- Q[split] = H . W2t[S] over a range of neurons (fp32):
-//                M = batch, N = 256 output columns, K = neurons in 64-row tiles
-//   mlp_out   -- y = sum of the splits, in a fixed order
-// The GEMMs stream weight rows with 1-D bulk copies (one per row) into
-// shared-memory rows padded by 16 bytes, so ldmatrix reads are free of bank
-// conflicts, and run on the tensor cores (mma.sync m16n8k16, fp32 accumulate).
+//   mlp_up    -- partial x . W1t[S]^T (fp32): M = 16 gathered neurons, N =
+//                batch, K = d streamed in 2 KiB row segments
+//   mlp_act   -- Ht = sigma(sum of the partials), rounded to the input dtype,
+//                neuron-major
+//   mlp_down  -- partial Ht^T . W2t[S] over a range of neurons (fp32): M =
+//                batch, N = up to 1024 output columns, K = neurons
+//   mlp_out   -- y = sum of the partials, in a fixed order
+// The GEMMs stream weight-row segments with 1-D bulk copies (one per row)
+// into shared-memory rows padded by 16 bytes, so ldmatrix reads are free of
+// bank conflicts, and run on the tensor cores (mma.sync m16n8k16, fp32
+// accumulate).  Segments are long (2 KiB for batches up to 16) so DRAM sees
+// contiguous runs of each selected row.
 // They are bound by HBM: every selected weight byte is read once, and the
 // arithmetic intensity is about B flops per weight byte.
 #include <cmath>
@@ -122,39 +125,56 @@ __device__ __forceinline__ int neuron_id(const int32_t *S, int t, int D)
 }
 
 // ---------------------------------------------------------------- up-projection
+//
+// An item is kUpRows gathered neurons x the whole hidden width d (or a range
+// of it when the union is too small to give every block several items).
+// Each stage holds kUpRows weight-row segments and the matching x segments,
+// kstage elements long (2 KiB for batches up to 16), so DRAM sees long
+// contiguous runs of each selected row.  The four consumer warps split a
+// stage's columns; their partial products go to the workspace separately
+// and the activation kernel adds them up.
 
+constexpr int kUpRows = 16;
+
+template <int BP>
 struct UpCfg {
     static constexpr int kConsumerWarps = 4;
     static constexpr int kThreads = (kConsumerWarps + 1) * 32;
-    static constexpr int kM = 128;                      // gathered neurons per item
-    static constexpr int kK = 128;                      // d per tile
+    static constexpr int kKMax = BP == 16 ? 1024 : (BP == 32 ? 512 : 256);  // d per stage
     static constexpr int kStages = 3;
-    static constexpr int kRow = kK * 2 + 16;            // padded row: conflict-free ldmatrix
-    static constexpr int kWBytes = kM * kRow;
-    static constexpr int kXBytes = kMlpMaxBatch * kRow;
-    static constexpr int kStage = kWBytes + kXBytes;
+    static constexpr int kRow = kKMax * 2 + 16;        // padded row: conflict-free ldmatrix
+    static constexpr int kStage = (kUpRows + BP) * kRow;
     static constexpr int kBarOffset = kStages * kStage;
     static constexpr int kSmemBytes = kBarOffset + 2 * kStages * 8;
 };
 
-// Work of the up-projection for n_S selected neurons on `blocks` blocks:
-// chunks of kM neurons, each split over `splits` ranges of d.
-__device__ __forceinline__ void up_plan(int n_S, int d, int blocks, int &chunks, int &splits)
+// d per stage: the largest of 1024/512/256 that divides d and fits the batch.
+__host__ __device__ __forceinline__ int stage_width(int d, int kmax)
 {
-    chunks = (n_S + UpCfg::kM - 1) / UpCfg::kM;
-    const int ktiles = d / UpCfg::kK;
-    splits = chunks > 0 ? (blocks + chunks - 1) / chunks : 1;
+    int k = kmax;
+    while (k > 256 && d % k != 0) k >>= 1;
+    return k;
+}
+
+// Items of the up-projection: groups of kUpRows neurons, each over `splits`
+// ranges of d; the partial buffer holds splits * 4 (warps) sums per neuron.
+__host__ __device__ __forceinline__ void up_plan(int n_S, int d, int kstage, int blocks,
+                                                 int &groups, int &splits)
+{
+    groups = (n_S + kUpRows - 1) / kUpRows;
+    const int ktiles = d / kstage;
+    splits = groups > 0 ? (4 * blocks + groups - 1) / groups : 1;
     if (splits > ktiles) splits = ktiles;
     if (splits < 1) splits = 1;
 }
 
-template <typename T>
-__global__ void __launch_bounds__(UpCfg::kThreads, 1)
+template <typename T, int BP>
+__global__ void __launch_bounds__(UpCfg<BP>::kThreads, 1)
     mlp_up_kernel(const T *__restrict__ x, const T *__restrict__ W1t,
                   const int32_t *__restrict__ S, const int32_t *__restrict__ n_S_ptr, int B,
                   int d, int D, float *__restrict__ part)
 {
-    using C = UpCfg;
+    using C = UpCfg<BP>;
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOffset);
     uint64_t *empty = full + C::kStages;
@@ -171,27 +191,24 @@ __global__ void __launch_bounds__(UpCfg::kThreads, 1)
     pdl_launch_dependents();
 
     const int n_S = union_size(n_S_ptr, D);
-    int chunks, splits;
-    up_plan(n_S, d, gridDim.x, chunks, splits);
-    const int items = chunks * splits, ktiles = d / C::kK;
-    const int n_pad = chunks * C::kM;
+    const int kstage = stage_width(d, C::kKMax);
+    int groups, splits;
+    up_plan(n_S, d, kstage, gridDim.x, groups, splits);
+    const int items = groups * splits, ktiles = d / kstage;
+    const int n_pad = groups * kUpRows;
 
     if (warp == C::kConsumerWarps) {
-        // producer warp: lanes gather weight rows and batch rows of each tile
+        // producer warp: lanes 0..15 fetch weight-row segments, all lanes x rows
         const uint64_t policy = l2_policy_evict_first();
         int stage = 0;
         uint32_t phase = 0, last_parity = 0, used = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
-            const int chunk = item / splits, split = item % splits;
+            const int grp = item / splits, split = item % splits;
             const int kt0 = split * ktiles / splits, kt1 = (split + 1) * ktiles / splits;
-            int ids[C::kM / 32];
-#pragma unroll
-            for (int i = 0; i < C::kM / 32; ++i) {
-                const int t = chunk * C::kM + lane + 32 * i;
-                ids[i] = t < n_S ? neuron_id(S, t, D) : -1;
-            }
-            int valid = min(C::kM, n_S - chunk * C::kM);
+            const int t = grp * kUpRows + lane;
+            const int id = (lane < kUpRows && t < n_S) ? neuron_id(S, t, D) : -1;
+            const int valid = min(kUpRows, n_S - grp * kUpRows);
             for (int kt = kt0; kt < kt1; ++kt) {
                 bool go = true;
                 if (lane == 0 && !mbar_wait(&empty[stage], phase ^ 1)) {
@@ -201,18 +218,16 @@ __global__ void __launch_bounds__(UpCfg::kThreads, 1)
                 go = __shfl_sync(0xffffffffu, go, 0);
                 if (!go) { ok = false; break; }
                 if (lane == 0)
-                    mbar_arrive_expect_tx(&full[stage], (uint32_t)((valid + B) * C::kK * 2));
+                    mbar_arrive_expect_tx(&full[stage], (uint32_t)((valid + B) * kstage * 2));
                 __syncwarp();
                 unsigned char *ws = smem + stage * C::kStage;
-                unsigned char *xs = ws + C::kWBytes;
-                const size_t k0 = (size_t)kt * C::kK;
-#pragma unroll
-                for (int i = 0; i < C::kM / 32; ++i)
-                    if (ids[i] >= 0)
-                        bulk_copy_g2s(ws + (lane + 32 * i) * C::kRow, W1t + (size_t)ids[i] * d + k0,
-                                      C::kK * 2, &full[stage], policy);
+                unsigned char *xs = ws + kUpRows * C::kRow;
+                const size_t k0 = (size_t)kt * kstage;
+                if (id >= 0)
+                    bulk_copy_g2s(ws + lane * C::kRow, W1t + (size_t)id * d + k0, kstage * 2,
+                                  &full[stage], policy);
                 for (int b = lane; b < B; b += 32)
-                    bulk_copy_g2s(xs + b * C::kRow, x + (size_t)b * d + k0, C::kK * 2,
+                    bulk_copy_g2s(xs + b * C::kRow, x + (size_t)b * d + k0, kstage * 2,
                                   &full[stage], policy);
                 last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
                 used |= 1u << stage;
@@ -226,46 +241,37 @@ __global__ void __launch_bounds__(UpCfg::kThreads, 1)
         return;
     }
 
-    // consumers: warp w computes neurons [32w, 32w+32) of the chunk x all batch rows
-    const int g = lane >> 2, qd = lane & 3;
-    const int ntiles = (B + 7) / 8;          // 8-row batch tiles in use
+    // consumers: all kUpRows neurons x the batch, over a quarter of each stage
+    const int g = lane >> 2, qd = lane & 3, mi = lane >> 3;
+    constexpr int kNT = BP / 8;                       // 8-row batch tiles
+    const int ntiles = (B + 7) / 8;
+    const int k16_per_warp = kstage / 16 / C::kConsumerWarps;
     int stage = 0;
     uint32_t phase = 0;
     const uint32_t base = smem_addr(smem);
     for (int item = blockIdx.x; item < items; item += gridDim.x) {
-        const int chunk = item / splits, split = item % splits;
+        const int grp = item / splits, split = item % splits;
         const int kt0 = split * ktiles / splits, kt1 = (split + 1) * ktiles / splits;
-        float acc[2][8][4];
+        float acc[kNT][4];
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = acc[mt][nt][2] =
-                                                acc[mt][nt][3] = 0.f;
+        for (int nt = 0; nt < kNT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
         for (int kt = kt0; kt < kt1; ++kt) {
             const bool live = __all_sync(0xffffffffu, mbar_wait(&full[stage], phase));
             if (live) {
-                const uint32_t ws = base + stage * C::kStage, xs = ws + C::kWBytes;
+                const uint32_t ws = base + stage * C::kStage, xs = ws + kUpRows * C::kRow;
+                for (int kk = 0; kk < k16_per_warp; ++kk) {
+                    const int k16 = warp * k16_per_warp + kk;
+                    uint32_t a[4];
+                    ldmatrix_x4(ws + (lane & 15) * C::kRow + (k16 * 16 + (lane >> 4) * 8) * 2, a);
 #pragma unroll
-                for (int k16 = 0; k16 < C::kK / 16; ++k16) {
-                    uint32_t a[2][4];
-#pragma unroll
-                    for (int mt = 0; mt < 2; ++mt)
-                        ldmatrix_x4(ws + (warp * 32 + mt * 16 + (lane & 15)) * C::kRow +
-                                        (k16 * 16 + (lane >> 4) * 8) * 2,
-                                    a[mt]);
-#pragma unroll
-                    for (int np = 0; np < 4; ++np) {
+                    for (int np = 0; np < kNT / 2; ++np) {
                         if (np * 2 >= ntiles) break;                 // warp-uniform
-                        const int mi = lane >> 3;
                         uint32_t kb[4];
                         ldmatrix_x4(xs + (np * 16 + (mi >> 1) * 8 + (lane & 7)) * C::kRow +
                                         (k16 * 16 + (mi & 1) * 8) * 2,
                                     kb);
-#pragma unroll
-                        for (int mt = 0; mt < 2; ++mt) {
-                            mma_16816<T>(acc[mt][2 * np], a[mt], kb[0], kb[1]);
-                            mma_16816<T>(acc[mt][2 * np + 1], a[mt], kb[2], kb[3]);
-                        }
+                        mma_16816<T>(acc[2 * np], a, kb[0], kb[1]);
+                        mma_16816<T>(acc[2 * np + 1], a, kb[2], kb[3]);
                     }
                 }
             } else if (lane == 0) {
@@ -275,70 +281,78 @@ __global__ void __launch_bounds__(UpCfg::kThreads, 1)
             if (lane == 0) mbar_arrive(&empty[stage]);
             if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
-        // partial sums of this range of d: part[split][neuron][batch]
+        // part[(split*4 + warp)][neuron][batch], batch padded to BP
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
+        for (int r = 0; r < 2; ++r) {
+            const int t = grp * kUpRows + g + 8 * r;
+            if (t >= n_S) continue;
+            float *dst = part + ((size_t)(split * C::kConsumerWarps + warp) * n_pad + t) * BP;
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int t = chunk * C::kM + warp * 32 + mt * 16 + g + 8 * r;
-                if (t >= n_S) continue;
-                float *dst = part + ((size_t)split * n_pad + t) * kMlpMaxBatch;
-#pragma unroll
-                for (int nt = 0; nt < 8; ++nt)
-                    if (nt < ntiles)
-                        *reinterpret_cast<float2 *>(dst + nt * 8 + qd * 2) =
-                            make_float2(acc[mt][nt][2 * r], acc[mt][nt][2 * r + 1]);
-            }
+            for (int nt = 0; nt < kNT; ++nt)
+                if (nt < ntiles)
+                    *reinterpret_cast<float2 *>(dst + nt * 8 + qd * 2) =
+                        make_float2(acc[nt][2 * r], acc[nt][2 * r + 1]);
+        }
     }
 }
 
-// H[b, t] = sigma(sum over splits), rounded to T; zero outside the batch and the union.
-template <typename T>
+// Ht[t, b] = sigma(sum of the partial products), rounded to T, neuron-major
+// ([n rows][BP]); zero outside the batch and the union.
+template <typename T, int BP>
 __global__ void mlp_act_kernel(const float *__restrict__ part, const int32_t *__restrict__ n_S_ptr,
-                               int B, int d, int D, int h_stride, int up_blocks, int act,
-                               T *__restrict__ H)
+                               int B, int d, int D, int h_rows, int up_blocks, int act,
+                               T *__restrict__ Ht)
 {
     pdl_wait();
     pdl_launch_dependents();
     const int n_S = union_size(n_S_ptr, D);
-    int chunks, splits;
-    up_plan(n_S, d, up_blocks, chunks, splits);
-    const int n_pad = chunks * UpCfg::kM;
-    const int t = blockIdx.x * blockDim.x + threadIdx.x;
-    const int b = blockIdx.y;
-    if (t >= h_stride) return;
+    const int kstage = stage_width(d, UpCfg<BP>::kKMax);
+    int groups, splits;
+    up_plan(n_S, d, kstage, up_blocks, groups, splits);
+    const int n_pad = groups * kUpRows;
+    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (size_t)h_rows * BP) return;
+    const int t = (int)(i / BP), b = (int)(i % BP);
     float v = 0.f;
     if (t < n_S && b < B) {
-        for (int s = 0; s < splits; ++s) v += part[((size_t)s * n_pad + t) * kMlpMaxBatch + b];
+        for (int s = 0; s < splits * UpCfg<BP>::kConsumerWarps; ++s)
+            v += part[((size_t)s * n_pad + t) * BP + b];
         if (act == 1) v = fmaxf(v, 0.f);
     }
-    H[(size_t)b * h_stride + t] = Elem<T>::from_float(v);
+    Ht[i] = Elem<T>::from_float(v);
 }
 
 // ---------------------------------------------------------------- down-projection
+//
+// An item is a range of wc output columns (2 KiB of each weight row for
+// batches up to 16) over a range of the union's neurons; stages hold
+// kDownRows weight-row segments and the matching kDownRows x BP block of the
+// neuron-major activations (one contiguous copy).  Eight consumer warps own
+// wc/8 columns each.  Partial sums over the neuron ranges go to the workspace
+// and mlp_out adds them in a fixed order.
 
+constexpr int kDownRows = 32;
+
+template <int BP>
 struct DownCfg {
     static constexpr int kConsumerWarps = 8;
     static constexpr int kThreads = (kConsumerWarps + 1) * 32;
-    static constexpr int kN = 256;                      // output columns per item
-    static constexpr int kK = 64;                       // neurons per tile
-    static constexpr int kStages = 4;
-    static constexpr int kWRow = kN * 2 + 16;           // padded rows
-    static constexpr int kHRow = kK * 2 + 16;
-    static constexpr int kWBytes = kK * kWRow;
-    static constexpr int kHBytes = kMlpMaxBatch * kHRow;
-    static constexpr int kStage = kWBytes + kHBytes;
+    static constexpr int kWMax = BP == 16 ? 1024 : (BP == 32 ? 512 : 256);   // columns per item
+    static constexpr int kStages = 3;
+    static constexpr int kWRow = kWMax * 2 + 16;       // padded rows
+    static constexpr int kHBytes = kDownRows * BP * 2;
+    static constexpr int kStage = kDownRows * kWRow + kHBytes;
     static constexpr int kBarOffset = kStages * kStage;
     static constexpr int kSmemBytes = kBarOffset + 2 * kStages * 8;
 };
 
-template <typename T>
-__global__ void __launch_bounds__(DownCfg::kThreads, 1)
-    mlp_down_kernel(const T *__restrict__ H, const T *__restrict__ W2t,
+template <typename T, int BP>
+__global__ void __launch_bounds__(DownCfg<BP>::kThreads, 1)
+    mlp_down_kernel(const T *__restrict__ Ht, const T *__restrict__ W2t,
                     const int32_t *__restrict__ S, const int32_t *__restrict__ n_S_ptr, int B,
-                    int d, int D, int h_stride, int splits, float *__restrict__ part)
+                    int d, int D, int splits, float *__restrict__ part)
 {
-    using C = DownCfg;
+    using C = DownCfg<BP>;
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOffset);
     uint64_t *empty = full + C::kStages;
@@ -355,9 +369,10 @@ __global__ void __launch_bounds__(DownCfg::kThreads, 1)
     pdl_launch_dependents();
 
     const int n_S = union_size(n_S_ptr, D);
-    const int ktiles = (n_S + C::kK - 1) / C::kK;
-    const int dchunks = d / C::kN;
-    const int items = dchunks * splits;
+    const int wc = stage_width(d, C::kWMax);
+    const int ktiles = (n_S + kDownRows - 1) / kDownRows;
+    const int wchunks = d / wc;
+    const int items = wchunks * splits;
 
     if (warp == C::kConsumerWarps) {
         const uint64_t policy = l2_policy_evict_first();
@@ -365,9 +380,9 @@ __global__ void __launch_bounds__(DownCfg::kThreads, 1)
         uint32_t phase = 0, last_parity = 0, used = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
-            const int dc = item / splits, split = item % splits;
+            const int wcn = item / splits, split = item % splits;
             const int kt0 = split * ktiles / splits, kt1 = (split + 1) * ktiles / splits;
-            const size_t c0 = (size_t)dc * C::kN;
+            const size_t c0 = (size_t)wcn * wc;
             for (int kt = kt0; kt < kt1; ++kt) {
                 bool go = true;
                 if (lane == 0 && !mbar_wait(&empty[stage], phase ^ 1)) {
@@ -378,21 +393,19 @@ __global__ void __launch_bounds__(DownCfg::kThreads, 1)
                 if (!go) { ok = false; break; }
                 if (lane == 0)
                     mbar_arrive_expect_tx(&full[stage],
-                                          (uint32_t)(C::kK * C::kN * 2 + kMlpMaxBatch * C::kK * 2));
+                                          (uint32_t)(kDownRows * wc * 2 + C::kHBytes));
                 __syncwarp();
                 unsigned char *ws = smem + stage * C::kStage;
-                unsigned char *hs = ws + C::kWBytes;
-                const int t0 = kt * C::kK;
-                for (int r = lane; r < C::kK; r += 32) {
-                    // rows past the union repeat its last neuron: finite values
-                    // times H = 0 add nothing (stale shared memory could be NaN)
-                    const int t = min(t0 + r, n_S - 1);
-                    bulk_copy_g2s(ws + r * C::kWRow, W2t + (size_t)neuron_id(S, t, D) * d + c0,
-                                  C::kN * 2, &full[stage], policy);
-                }
-                for (int b = lane; b < kMlpMaxBatch; b += 32)
-                    bulk_copy_g2s(hs + b * C::kHRow, H + (size_t)b * h_stride + t0, C::kK * 2,
-                                  &full[stage], policy);
+                unsigned char *hs = ws + kDownRows * C::kWRow;
+                const int t0 = kt * kDownRows;
+                // rows past the union repeat its last neuron: finite values
+                // times an activation of 0 add nothing (stale shared memory
+                // could be NaN)
+                const int t = min(t0 + lane, n_S - 1);
+                bulk_copy_g2s(ws + lane * C::kWRow, W2t + (size_t)neuron_id(S, t, D) * d + c0,
+                              wc * 2, &full[stage], policy);
+                if (lane == 0)
+                    bulk_copy_g2s(hs, Ht + (size_t)t0 * BP, C::kHBytes, &full[stage], policy);
                 last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
                 used |= 1u << stage;
                 if (++stage == C::kStages) { stage = 0; phase ^= 1; }
@@ -405,44 +418,51 @@ __global__ void __launch_bounds__(DownCfg::kThreads, 1)
         return;
     }
 
-    // consumers: warp w owns output columns [32w, 32w+32) of the item x all batch rows
+    // consumers: warp w owns output columns [w*wc/8, (w+1)*wc/8) x the batch
     const int g = lane >> 2, qd = lane & 3, mi = lane >> 3;
+    constexpr int kMT = BP / 16;                    // 16-row batch tiles
+    constexpr int kNT = C::kWMax / C::kConsumerWarps / 8;   // 8-column tiles per warp
     const int mtiles = (B + 15) / 16;
+    const int nt_used = wc / C::kConsumerWarps / 8;
     int stage = 0;
     uint32_t phase = 0;
     const uint32_t base = smem_addr(smem);
     for (int item = blockIdx.x; item < items; item += gridDim.x) {
-        const int dc = item / splits, split = item % splits;
+        const int wcn = item / splits, split = item % splits;
         const int kt0 = split * ktiles / splits, kt1 = (split + 1) * ktiles / splits;
-        float acc[4][4][4];
+        float acc[kMT][kNT][4];
 #pragma unroll
-        for (int mt = 0; mt < 4; ++mt)
+        for (int mt = 0; mt < kMT; ++mt)
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = acc[mt][nt][2] =
+            for (int nt = 0; nt < kNT; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = acc[mt][nt][2] =
                                                 acc[mt][nt][3] = 0.f;
+        const int col0 = warp * (wc / C::kConsumerWarps);
         for (int kt = kt0; kt < kt1; ++kt) {
             const bool live = __all_sync(0xffffffffu, mbar_wait(&full[stage], phase));
             if (live) {
-                const uint32_t ws = base + stage * C::kStage, hs = ws + C::kWBytes;
+                const uint32_t ws = base + stage * C::kStage, hs = ws + kDownRows * C::kWRow;
 #pragma unroll
-                for (int k16 = 0; k16 < C::kK / 16; ++k16) {
-                    uint32_t vb[2][4];
+                for (int k16 = 0; k16 < kDownRows / 16; ++k16) {
+                    // activations, neuron-major in shared memory: A = Ht^T via ldmatrix.trans
+                    uint32_t a[kMT][4];
 #pragma unroll
-                    for (int np = 0; np < 2; ++np)
+                    for (int mt = 0; mt < kMT; ++mt)
+                        if (mt < mtiles)
+                            ldmatrix_x4_trans(hs + (k16 * 16 + (mi >> 1) * 8 + (lane & 7)) * BP * 2 +
+                                                  (mt * 16 + (mi & 1) * 8) * 2,
+                                              a[mt]);
+#pragma unroll
+                    for (int np = 0; np < kNT / 2; ++np) {
+                        if (np * 2 >= nt_used) break;               // warp-uniform
+                        uint32_t vb[4];
                         ldmatrix_x4_trans(ws + (k16 * 16 + (mi & 1) * 8 + (lane & 7)) * C::kWRow +
-                                              (warp * 32 + np * 16 + (mi >> 1) * 8) * 2,
-                                          vb[np]);
+                                              (col0 + np * 16 + (mi >> 1) * 8) * 2,
+                                          vb);
 #pragma unroll
-                    for (int mt = 0; mt < 4; ++mt) {
-                        if (mt >= mtiles) break;                     // warp-uniform
-                        uint32_t a[4];
-                        ldmatrix_x4(hs + (mt * 16 + (lane & 15)) * C::kHRow +
-                                        (k16 * 16 + (lane >> 4) * 8) * 2,
-                                    a);
-#pragma unroll
-                        for (int np = 0; np < 2; ++np) {
-                            mma_16816<T>(acc[mt][2 * np], a, vb[np][0], vb[np][1]);
-                            mma_16816<T>(acc[mt][2 * np + 1], a, vb[np][2], vb[np][3]);
+                        for (int mt = 0; mt < kMT; ++mt) {
+                            if (mt >= mtiles) break;                 // warp-uniform
+                            mma_16816<T>(acc[mt][2 * np], a[mt], vb[0], vb[1]);
+                            mma_16816<T>(acc[mt][2 * np + 1], a[mt], vb[2], vb[3]);
                         }
                     }
                 }
@@ -455,17 +475,17 @@ __global__ void __launch_bounds__(DownCfg::kThreads, 1)
         }
         // partial sums of this range of neurons: part[split][b][column]
 #pragma unroll
-        for (int mt = 0; mt < 4; ++mt)
+        for (int mt = 0; mt < kMT; ++mt)
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
                 const int b = mt * 16 + g + 8 * r;
                 if (b >= B) continue;
-                float *dst = part + ((size_t)split * kMlpMaxBatch + b) * d + (size_t)dc * C::kN +
-                             warp * 32;
+                float *dst = part + ((size_t)split * kMlpMaxBatch + b) * d + (size_t)wcn * wc + col0;
 #pragma unroll
-                for (int nt = 0; nt < 4; ++nt)
-                    *reinterpret_cast<float2 *>(dst + nt * 8 + qd * 2) =
-                        make_float2(acc[mt][nt][2 * r], acc[mt][nt][2 * r + 1]);
+                for (int nt = 0; nt < kNT; ++nt)
+                    if (nt < nt_used)
+                        *reinterpret_cast<float2 *>(dst + nt * 8 + qd * 2) =
+                            make_float2(acc[mt][nt][2 * r], acc[mt][nt][2 * r + 1]);
             }
     }
 }
@@ -526,24 +546,74 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Workspace of sha_selective_mlp for these sizes on a device with `sms` SMs.
 struct MlpPlan {
-    int h_stride;          // padded union length (H row stride)
-    int down_splits;
+    int bp;                // batch padded to 16, 32 or 64
+    int h_rows;            // rows of the neuron-major activations (union padded)
+    int down_splits, down_blocks;
     size_t up_bytes, h_bytes, down_bytes;
     size_t total() const { return up_bytes + h_bytes + down_bytes; }
 };
 
-MlpPlan mlp_plan(int d, int D, int sms)
+int batch_pad(int B) { return B <= 16 ? 16 : (B <= 32 ? 32 : 64); }
+
+MlpPlan mlp_plan(int B, int d, int D, int sms)
 {
     MlpPlan pl;
-    pl.h_stride = (int)round_up((size_t)D, UpCfg::kM);
-    const int max_chunks = pl.h_stride / UpCfg::kM;
-    // splits * chunks <= blocks + chunks for any union size
-    pl.up_bytes = round_up((size_t)(sms + max_chunks) * UpCfg::kM * kMlpMaxBatch * 4, 256);
-    pl.h_bytes = round_up((size_t)kMlpMaxBatch * pl.h_stride * 2, 256);
-    const int dchunks = d / DownCfg::kN;
-    pl.down_splits = sms / dchunks > 0 ? sms / dchunks : 1;
+    pl.bp = batch_pad(B);
+    const int kmax = pl.bp == 16 ? 1024 : (pl.bp == 32 ? 512 : 256);
+    pl.h_rows = (int)round_up((size_t)D, (size_t)kDownRows);
+    // up partials: splits * 4 warps sums of n_pad neurons; splits * groups <= 4*sms + groups
+    const size_t max_groups = (D + kUpRows - 1) / kUpRows;
+    pl.up_bytes = round_up((4 * (size_t)sms + max_groups) * 4 * kUpRows * pl.bp * 4, 256);
+    pl.h_bytes = round_up((size_t)pl.h_rows * pl.bp * 2, 256);
+    const int wc = stage_width(d, kmax);
+    const int wchunks = d / wc;
+    pl.down_splits = sms / wchunks > 0 ? sms / wchunks : 1;
+    const int items = wchunks * pl.down_splits;
+    pl.down_blocks = items < sms ? items : sms;
     pl.down_bytes = round_up((size_t)pl.down_splits * kMlpMaxBatch * d * 4, 256);
     return pl;
+}
+
+template <typename T, int BP>
+sha_status_t run_mlp_bp(const void *x, const void *W1t, const void *W2t, const int32_t *S,
+                        const int32_t *n_S, int B, int d, int D, int act, void *y, void *ws,
+                        int dev, int sms, cudaStream_t s)
+{
+    static bool configured[kMaxDevicesMlp] = {};
+    if (!configured[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(mlp_up_kernel<T, BP>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             UpCfg<BP>::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(mlp_down_kernel<T, BP>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     DownCfg<BP>::kSmemBytes);
+        if (e != cudaSuccess) return mlp_launch_error(e);
+        configured[dev] = true;
+    }
+    const MlpPlan pl = mlp_plan(B, d, D, sms);
+    char *w = static_cast<char *>(ws);
+    float *up_part = reinterpret_cast<float *>(w);
+    T *Ht = reinterpret_cast<T *>(w + pl.up_bytes);
+    float *down_part = reinterpret_cast<float *>(w + pl.up_bytes + pl.h_bytes);
+
+    cudaError_t e = launch_pdl(mlp_up_kernel<T, BP>, dim3(sms), UpCfg<BP>::kThreads,
+                               UpCfg<BP>::kSmemBytes, s, static_cast<const T *>(x),
+                               static_cast<const T *>(W1t), S, n_S, B, d, D, up_part);
+    if (e != cudaSuccess) return mlp_launch_error(e);
+    const size_t hn = (size_t)pl.h_rows * BP;
+    e = launch_pdl(mlp_act_kernel<T, BP>, dim3((unsigned)((hn + 255) / 256)), 256, 0, s,
+                   (const float *)up_part, n_S, B, d, D, pl.h_rows, sms, act, Ht);
+    if (e != cudaSuccess) return mlp_launch_error(e);
+    e = launch_pdl(mlp_down_kernel<T, BP>, dim3(pl.down_blocks), DownCfg<BP>::kThreads,
+                   DownCfg<BP>::kSmemBytes, s, (const T *)Ht, static_cast<const T *>(W2t), S, n_S,
+                   B, d, D, pl.down_splits, down_part);
+    if (e != cudaSuccess) return mlp_launch_error(e);
+    const size_t n = (size_t)B * d;
+    e = launch_pdl(mlp_out_kernel<T>, dim3((unsigned)((n + 255) / 256)), 256, 0, s,
+                   (const float *)down_part, B, d, pl.down_splits, static_cast<T *>(y));
+    if (e != cudaSuccess) return mlp_launch_error(e);
+    return SHA_OK;
 }
 
 template <typename T>
@@ -551,41 +621,11 @@ sha_status_t run_mlp(const void *x, const void *W1t, const void *W2t, const int3
                      const int32_t *n_S, int B, int d, int D, int act, void *y, void *ws,
                      int dev, int sms, cudaStream_t s)
 {
-    static bool configured[kMaxDevicesMlp] = {};
-    if (!configured[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(mlp_up_kernel<T>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             UpCfg::kSmemBytes);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(mlp_down_kernel<T>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     DownCfg::kSmemBytes);
-        if (e != cudaSuccess) return mlp_launch_error(e);
-        configured[dev] = true;
+    switch (batch_pad(B)) {
+    case 16: return run_mlp_bp<T, 16>(x, W1t, W2t, S, n_S, B, d, D, act, y, ws, dev, sms, s);
+    case 32: return run_mlp_bp<T, 32>(x, W1t, W2t, S, n_S, B, d, D, act, y, ws, dev, sms, s);
+    default: return run_mlp_bp<T, 64>(x, W1t, W2t, S, n_S, B, d, D, act, y, ws, dev, sms, s);
     }
-    const MlpPlan pl = mlp_plan(d, D, sms);
-    char *w = static_cast<char *>(ws);
-    float *up_part = reinterpret_cast<float *>(w);
-    T *H = reinterpret_cast<T *>(w + pl.up_bytes);
-    float *down_part = reinterpret_cast<float *>(w + pl.up_bytes + pl.h_bytes);
-
-    cudaError_t e = launch_pdl(mlp_up_kernel<T>, dim3(sms), UpCfg::kThreads, UpCfg::kSmemBytes, s,
-                               static_cast<const T *>(x), static_cast<const T *>(W1t), S, n_S, B, d,
-                               D, up_part);
-    if (e != cudaSuccess) return mlp_launch_error(e);
-    e = launch_pdl(mlp_act_kernel<T>, dim3((pl.h_stride + 255) / 256, kMlpMaxBatch), 256, 0, s,
-                   (const float *)up_part, n_S, B, d, D, pl.h_stride, sms, act, H);
-    if (e != cudaSuccess) return mlp_launch_error(e);
-    const int items = (d / DownCfg::kN) * pl.down_splits;
-    e = launch_pdl(mlp_down_kernel<T>, dim3(items < sms ? items : sms), DownCfg::kThreads,
-                   DownCfg::kSmemBytes, s, (const T *)H, static_cast<const T *>(W2t), S, n_S, B,
-                   d, D, pl.h_stride, pl.down_splits, down_part);
-    if (e != cudaSuccess) return mlp_launch_error(e);
-    const size_t n = (size_t)B * d;
-    e = launch_pdl(mlp_out_kernel<T>, dim3((unsigned)((n + 255) / 256)), 256, 0, s,
-                   (const float *)down_part, B, d, pl.down_splits, static_cast<T *>(y));
-    if (e != cudaSuccess) return mlp_launch_error(e);
-    return SHA_OK;
 }
 
 }  // namespace
@@ -631,11 +671,11 @@ sha_status_t sha_mlp_union(const uint8_t *active, int B, int D, int32_t *S, int3
 
 size_t sha_selective_mlp_workspace_size(int B, int d, int D)
 {
-    if (B < 1 || B > kMlpMaxBatch || d < DownCfg::kN || d % DownCfg::kN || D < 1) return 0;
+    if (B < 1 || B > kMlpMaxBatch || d < 256 || d % 256 || D < 1) return 0;
     int dev;
     const int sms = device_sms(&dev);
     if (sms == 0) return 0;
-    return mlp_plan(d, D, sms).total();
+    return mlp_plan(B, d, D, sms).total();
 }
 
 sha_status_t sha_selective_mlp(const void *x, const void *W1t, const void *W2t,
@@ -646,7 +686,7 @@ sha_status_t sha_selective_mlp(const void *x, const void *W1t, const void *W2t,
     if (dtype != SHA_FP16 && dtype != SHA_BF16) return SHA_ERR_UNSUPPORTED;
     if (B < 1 || D < 1 || d < 1 || (activation != 0 && activation != 1))
         return SHA_ERR_INVALID_ARG;
-    if (B > kMlpMaxBatch || d % DownCfg::kN != 0) return SHA_ERR_UNSUPPORTED;
+    if (B > kMlpMaxBatch || d % 256 != 0) return SHA_ERR_UNSUPPORTED;
     if (!x || !W1t || !W2t || !S || !n_S || !y || !workspace) return SHA_ERR_INVALID_ARG;
     if (!aligned_to(x, 16) || !aligned_to(W1t, 16) || !aligned_to(W2t, 16) ||
         !aligned_to(y, 16) || !aligned_to(S, 4) || !aligned_to(n_S, 4) ||
@@ -655,7 +695,7 @@ sha_status_t sha_selective_mlp(const void *x, const void *W1t, const void *W2t,
     int dev;
     const int sms = device_sms(&dev);
     if (sms == 0 || dev >= kMaxDevicesMlp) return SHA_ERR_LAUNCH;
-    if (workspace_bytes < mlp_plan(d, D, sms).total()) return SHA_ERR_WORKSPACE;
+    if (workspace_bytes < mlp_plan(B, d, D, sms).total()) return SHA_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (dtype == SHA_FP16)
         return run_mlp<__half>(x, W1t, W2t, S, n_S, B, d, D, activation, y, workspace, dev, sms, s);
