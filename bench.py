@@ -336,6 +336,9 @@ def run_ours(args, rank, world, local):
         extras["other_configs"] = other_configs(sha, w, dev, stream, peak, rank)
         extras["other_configs"].append(varlen_config(sha, dev, stream, peak, rank))
         extras["other_configs"].append(paged_config(sha, dev, stream, peak, rank))
+        mlp = run_mlp(argparse.Namespace(batch=None))
+        extras["selective_mlp"] = {"config": mlp["config"], "cublas_dense_us": mlp["cublas_dense_us"],
+                                   "points": mlp["points"]}
     plan = sha.sha_decode_plan(w.B, w.H_q, w.H_kv, w.N_kv, w.d, w.top_k,
                                num_sms=torch.cuda.get_device_properties(dev).multi_processor_count)
     line = {
@@ -568,6 +571,8 @@ def run_mlp(args):
     base = workloads.MLP_CONFIGS["opt66b_mlp"]
     if args.batch:
         base = base.with_(B=args.batch)
+    sampler = ClockSampler(dev)
+    t_start = time.time()
     x, W1t, W2t, _ = workloads.make_mlp(base.with_(density=1.0), device=dev)
     ws = torch.empty(sha.sha_selective_mlp_workspace_size(base.B, base.d, base.D, dev),
                      dtype=torch.uint8, device=dev)
@@ -602,10 +607,14 @@ def run_mlp(args):
         cublas()
     t = timed_graphs(cublas, 200, dev, stream, chunk=50)
     cublas_us = t / 200 * 1e6
+    clocks = sampler.stop(t_start, time.time())
     for p in points:
         p["speedup_vs_dense_selective"] = round(dense_us / p["us_per_layer"], 3)
         p["speedup_vs_cublas_dense"] = round(cublas_us / p["us_per_layer"], 3)
+    del x, W1t, W2t
+    torch.cuda.empty_cache()
     return {"metric": "Selective GEMM (OPT-66B MLP): achieved HBM GB/s and speedup vs dense",
+            "clocks": clocks,
             "unit": "GB/s", "peak": peak, "peak_source": peak_src,
             "config": {"B": base.B, "d": base.d, "D": base.D, "dtype": base.dtype,
                        "activation": "relu", "launch": "CUDA graph replay (union + MLP)",

@@ -40,6 +40,10 @@ namespace {
 
 using namespace sha;
 
+#ifndef SHA_USE_PDL
+#define SHA_USE_PDL 1
+#endif
+
 constexpr int kMaxDevicesMlp = 64;
 constexpr int kMlpMaxBatch = 64;        // batch rows per call (MMA tiles cover 64)
 constexpr int kUnionChunk = 1024;       // neurons per block in the union kernels
@@ -525,7 +529,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, int block, size_t sm
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[0].val.programmaticStreamSerializationAllowed = SHA_USE_PDL;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
