@@ -336,7 +336,7 @@ def run_ours(args, rank, world, local):
         extras["other_configs"] = other_configs(sha, w, dev, stream, peak, rank)
         extras["other_configs"].append(varlen_config(sha, dev, stream, peak, rank))
         extras["other_configs"].append(paged_config(sha, dev, stream, peak, rank))
-        mlp = run_mlp(argparse.Namespace(batch=None))
+        mlp = run_mlp(argparse.Namespace(batch=None), dev)
         extras["selective_mlp"] = {"config": mlp["config"], "cublas_dense_us": mlp["cublas_dense_us"],
                                    "points": mlp["points"]}
     plan = sha.sha_decode_plan(w.B, w.H_q, w.H_kv, w.N_kv, w.d, w.top_k,
@@ -558,13 +558,13 @@ def run_reference(args):
 L2_BYTES = 126 * 1024 * 1024
 
 
-def run_mlp(args):
+def run_mlp(args, dev=None):
     """Selective GEMM on the OPT-66B MLP (hidden 9216, 36864 neurons) at decode
     batch B: union densities 10-100 %, against the same kernels at 100 % and
     against a dense cuBLAS MLP (torch.matmul) on the same weights."""
     import head_sparse_decode_b200 as sha
 
-    dev = torch.device("cuda", 0)
+    dev = dev if dev is not None else torch.device("cuda", dist_env()[2])
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     peak, peak_src = measured_peak()
@@ -643,7 +643,7 @@ def run_sweep(args):
     least 4x L2 of K/V, so the figures are HBM figures."""
     import head_sparse_decode_b200 as sha
 
-    dev = torch.device("cuda", 0)
+    dev = torch.device("cuda", dist_env()[2])
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     peak, peak_src = measured_peak()
