@@ -1,6 +1,7 @@
 // sha_decode.cu -- C ABI of the Selective Head Attention decode library:
 // argument checks, the work planner, workspace handling and kernel launches.
 // The operation and every argument are specified in include/sha_decode.h.
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -219,13 +220,13 @@ sha_status_t launch_gqa(const sha::DecodeParams &prm, sha_dtype_t dtype, int dev
                         cudaStream_t stream)
 {
     using C = sha::GqaConfig<D>;
-    static bool configured[kMaxDevices] = {};
-    if (!configured[dev]) {
+    static std::atomic<bool> configured[kMaxDevices];
+    if (!configured[dev].load(std::memory_order_acquire)) {
         cudaError_t e = cudaFuncSetAttribute(sha::sha_gqa_decode_kernel<T, D, kLayout>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::kSmemBytes);
         if (e != cudaSuccess) return launch_error(e);
-        configured[dev] = true;
+        configured[dev].store(true, std::memory_order_release);
     }
     CUtensorMap tm_k, tm_v;
     // a padded cache: [B*H_kv][N_kv][d]; a page pool: [num_pages*H_kv][page_size][d]
@@ -247,13 +248,13 @@ template <typename T, int D, int kLayout>
 sha_status_t launch_mha(const sha::DecodeParams &prm, int dev, cudaStream_t stream)
 {
     using C = sha::MhaConfig<D>;
-    static bool configured[kMaxDevices] = {};
-    if (!configured[dev]) {
+    static std::atomic<bool> configured[kMaxDevices];
+    if (!configured[dev].load(std::memory_order_acquire)) {
         cudaError_t e = cudaFuncSetAttribute(sha::sha_mha_decode_kernel<T, D, kLayout>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::kSmemBytes);
         if (e != cudaSuccess) return launch_error(e);
-        configured[dev] = true;
+        configured[dev].store(true, std::memory_order_release);
     }
     cudaError_t e = launch_kernel(sha::sha_mha_decode_kernel<T, D, kLayout>, prm.sched.num_ctas,
                                   C::kThreads, C::kSmemBytes, stream, prm);

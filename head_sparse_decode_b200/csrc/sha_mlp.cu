@@ -27,6 +27,7 @@
 // contiguous runs of each selected row.
 // They are bound by HBM: every selected weight byte is read once, and the
 // arithmetic intensity is about B flops per weight byte.
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <mutex>
@@ -144,8 +145,8 @@ template <int BP>
 struct UpCfg {
     static constexpr int kConsumerWarps = 4;
     static constexpr int kThreads = (kConsumerWarps + 1) * 32;
-    static constexpr int kKMax = BP == 16 ? 1024 : (BP == 32 ? 512 : 256);  // d per stage
-    static constexpr int kStages = 3;
+    static constexpr int kKMax = BP <= 16 ? 1024 : (BP == 32 ? 512 : 256);  // d per stage
+    static constexpr int kStages = BP == 8 ? 4 : 3;    // small batches: more weight bytes in flight
     static constexpr int kRow = kKMax * 2 + 16;        // padded row: conflict-free ldmatrix
     static constexpr int kStage = (kUpRows + BP) * kRow;
     static constexpr int kBarOffset = kStages * kStage;
@@ -249,6 +250,7 @@ __global__ void __launch_bounds__(UpCfg<BP>::kThreads, 1)
     const int g = lane >> 2, qd = lane & 3, mi = lane >> 3;
     constexpr int kNT = BP / 8;                       // 8-row batch tiles
     const int ntiles = (B + 7) / 8;
+    static_assert(BP == 8 || kNT % 2 == 0, "batch tiles come in pairs above 8 rows");
     const int k16_per_warp = kstage / 16 / C::kConsumerWarps;
     int stage = 0;
     uint32_t phase = 0;
@@ -267,15 +269,23 @@ __global__ void __launch_bounds__(UpCfg<BP>::kThreads, 1)
                     const int k16 = warp * k16_per_warp + kk;
                     uint32_t a[4];
                     ldmatrix_x4(ws + (lane & 15) * C::kRow + (k16 * 16 + (lane >> 4) * 8) * 2, a);
-#pragma unroll
-                    for (int np = 0; np < kNT / 2; ++np) {
-                        if (np * 2 >= ntiles) break;                 // warp-uniform
-                        uint32_t kb[4];
-                        ldmatrix_x4(xs + (np * 16 + (mi >> 1) * 8 + (lane & 7)) * C::kRow +
-                                        (k16 * 16 + (mi & 1) * 8) * 2,
+                    if constexpr (BP == 8) {
+                        // one 8-row batch tile: x rows 0-7 at k and k+8
+                        uint32_t kb[2];
+                        ldmatrix_x2(xs + (lane & 7) * C::kRow + (k16 * 16 + ((lane >> 3) & 1) * 8) * 2,
                                     kb);
-                        mma_16816<T>(acc[2 * np], a, kb[0], kb[1]);
-                        mma_16816<T>(acc[2 * np + 1], a, kb[2], kb[3]);
+                        mma_16816<T>(acc[0], a, kb[0], kb[1]);
+                    } else {
+#pragma unroll
+                        for (int np = 0; np < kNT / 2; ++np) {
+                            if (np * 2 >= ntiles) break;             // warp-uniform
+                            uint32_t kb[4];
+                            ldmatrix_x4(xs + (np * 16 + (mi >> 1) * 8 + (lane & 7)) * C::kRow +
+                                            (k16 * 16 + (mi & 1) * 8) * 2,
+                                        kb);
+                            mma_16816<T>(acc[2 * np], a, kb[0], kb[1]);
+                            mma_16816<T>(acc[2 * np + 1], a, kb[2], kb[3]);
+                        }
                     }
                 }
             } else if (lane == 0) {
@@ -341,7 +351,7 @@ template <int BP>
 struct DownCfg {
     static constexpr int kConsumerWarps = 8;
     static constexpr int kThreads = (kConsumerWarps + 1) * 32;
-    static constexpr int kWMax = BP == 16 ? 1024 : (BP == 32 ? 512 : 256);   // columns per item
+    static constexpr int kWMax = BP <= 16 ? 1024 : (BP == 32 ? 512 : 256);   // columns per item
     static constexpr int kStages = 3;
     static constexpr int kWRow = kWMax * 2 + 16;       // padded rows
     static constexpr int kHBytes = kDownRows * BP * 2;
@@ -424,7 +434,7 @@ __global__ void __launch_bounds__(DownCfg<BP>::kThreads, 1)
 
     // consumers: warp w owns output columns [w*wc/8, (w+1)*wc/8) x the batch
     const int g = lane >> 2, qd = lane & 3, mi = lane >> 3;
-    constexpr int kMT = BP / 16;                    // 16-row batch tiles
+    constexpr int kMT = BP >= 16 ? BP / 16 : 1;     // 16-row batch tiles (8 rows padded)
     constexpr int kNT = C::kWMax / C::kConsumerWarps / 8;   // 8-column tiles per warp
     const int mtiles = (B + 15) / 16;
     const int nt_used = wc / C::kConsumerWarps / 8;
@@ -449,12 +459,23 @@ __global__ void __launch_bounds__(DownCfg<BP>::kThreads, 1)
                 for (int k16 = 0; k16 < kDownRows / 16; ++k16) {
                     // activations, neuron-major in shared memory: A = Ht^T via ldmatrix.trans
                     uint32_t a[kMT][4];
+                    if constexpr (BP == 8) {
+                        // batch rows 0-7 only: the A rows 8-15 are zero
+                        uint32_t h2[2];
+                        ldmatrix_x2_trans(hs + (k16 * 16 + ((lane >> 3) & 1) * 8 + (lane & 7)) * BP * 2,
+                                          h2);
+                        a[0][0] = h2[0];
+                        a[0][1] = 0u;
+                        a[0][2] = h2[1];
+                        a[0][3] = 0u;
+                    } else {
 #pragma unroll
-                    for (int mt = 0; mt < kMT; ++mt)
-                        if (mt < mtiles)
-                            ldmatrix_x4_trans(hs + (k16 * 16 + (mi >> 1) * 8 + (lane & 7)) * BP * 2 +
-                                                  (mt * 16 + (mi & 1) * 8) * 2,
-                                              a[mt]);
+                        for (int mt = 0; mt < kMT; ++mt)
+                            if (mt < mtiles)
+                                ldmatrix_x4_trans(hs + (k16 * 16 + (mi >> 1) * 8 + (lane & 7)) * BP * 2 +
+                                                      (mt * 16 + (mi & 1) * 8) * 2,
+                                                  a[mt]);
+                    }
 #pragma unroll
                     for (int np = 0; np < kNT / 2; ++np) {
                         if (np * 2 >= nt_used) break;               // warp-uniform
@@ -557,13 +578,13 @@ struct MlpPlan {
     size_t total() const { return up_bytes + h_bytes + down_bytes; }
 };
 
-int batch_pad(int B) { return B <= 16 ? 16 : (B <= 32 ? 32 : 64); }
+int batch_pad(int B) { return B <= 8 ? 8 : (B <= 16 ? 16 : (B <= 32 ? 32 : 64)); }
 
 MlpPlan mlp_plan(int B, int d, int D, int sms)
 {
     MlpPlan pl;
     pl.bp = batch_pad(B);
-    const int kmax = pl.bp == 16 ? 1024 : (pl.bp == 32 ? 512 : 256);
+    const int kmax = pl.bp <= 16 ? 1024 : (pl.bp == 32 ? 512 : 256);
     pl.h_rows = (int)round_up((size_t)D, (size_t)kDownRows);
     // up partials: splits * 4 warps sums of n_pad neurons; splits * groups <= 4*sms + groups
     const size_t max_groups = (D + kUpRows - 1) / kUpRows;
@@ -583,8 +604,8 @@ sha_status_t run_mlp_bp(const void *x, const void *W1t, const void *W2t, const i
                         const int32_t *n_S, int B, int d, int D, int act, void *y, void *ws,
                         int dev, int sms, cudaStream_t s)
 {
-    static bool configured[kMaxDevicesMlp] = {};
-    if (!configured[dev]) {
+    static std::atomic<bool> configured[kMaxDevicesMlp];
+    if (!configured[dev].load(std::memory_order_acquire)) {
         cudaError_t e = cudaFuncSetAttribute(mlp_up_kernel<T, BP>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              UpCfg<BP>::kSmemBytes);
@@ -593,7 +614,7 @@ sha_status_t run_mlp_bp(const void *x, const void *W1t, const void *W2t, const i
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      DownCfg<BP>::kSmemBytes);
         if (e != cudaSuccess) return mlp_launch_error(e);
-        configured[dev] = true;
+        configured[dev].store(true, std::memory_order_release);
     }
     const MlpPlan pl = mlp_plan(B, d, D, sms);
     char *w = static_cast<char *>(ws);
@@ -626,6 +647,7 @@ sha_status_t run_mlp(const void *x, const void *W1t, const void *W2t, const int3
                      int dev, int sms, cudaStream_t s)
 {
     switch (batch_pad(B)) {
+    case 8: return run_mlp_bp<T, 8>(x, W1t, W2t, S, n_S, B, d, D, act, y, ws, dev, sms, s);
     case 16: return run_mlp_bp<T, 16>(x, W1t, W2t, S, n_S, B, d, D, act, y, ws, dev, sms, s);
     case 32: return run_mlp_bp<T, 32>(x, W1t, W2t, S, n_S, B, d, D, act, y, ws, dev, sms, s);
     default: return run_mlp_bp<T, 64>(x, W1t, W2t, S, n_S, B, d, D, act, y, ws, dev, sms, s);

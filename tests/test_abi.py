@@ -103,3 +103,37 @@ def test_select_heads_host_checks(lib, B, H, top_k, code):
     lib.sha_select_heads.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                      ctypes.c_void_p, ctypes.c_void_p]
     assert lib.sha_select_heads(0x1000, B, H, top_k, 0x2000, None) == code
+
+
+def test_varlen_and_paged_host_checks(lib):
+    P = 0x1000
+    lib.sha_decode_varlen.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 6 + [
+        ctypes.c_float, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
+    # null lengths, unsupported head dim, misaligned lengths
+    assert lib.sha_decode_varlen(P, P, P, P, None, 2, 4, 4, 64, 64, 2, 0.1, P, 0, None) == 1
+    assert lib.sha_decode_varlen(P, P, P, P, P, 2, 4, 4, 64, 96, 2, 0.1, P, 0, None) == 2
+    assert lib.sha_decode_varlen(P, P, P, P, P + 2, 2, 4, 4, 64, 64, 2, 0.1, P, 0, None) == 3
+    lib.sha_decode_paged.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int] * 8 + [
+        ctypes.c_float, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
+    # (B, H_q, H_kv, num_pages, page_size, max_pages, d, top_k)
+    assert lib.sha_decode_paged(P, P, P, P, P, P, 2, 8, 2, 10, 12, 4, 128, 1, 0.1, P, 1,
+                                None) == 2          # GQA needs a power-of-two page size
+    assert lib.sha_decode_paged(P, P, P, P, P, P, 2, 8, 2, 10, 0, 4, 128, 1, 0.1, P, 1,
+                                None) == 1          # page_size 0
+    assert lib.sha_decode_paged(P, P, P, P, None, P, 2, 8, 8, 10, 16, 4, 128, 1, 0.1, P, 0,
+                                None) == 1          # no lengths
+
+
+def test_selective_mlp_host_checks(lib):
+    P = 0x1000
+    lib.sha_selective_mlp.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 5 + [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    lib.sha_selective_mlp_workspace_size.restype = ctypes.c_size_t
+    # batch above 64, d not a multiple of 256, bad activation
+    assert lib.sha_selective_mlp(P, P, P, P, P, 65, 256, 512, 1, 0, P, P, 1 << 30, None) == 2
+    assert lib.sha_selective_mlp(P, P, P, P, P, 4, 300, 512, 1, 0, P, P, 1 << 30, None) == 2
+    assert lib.sha_selective_mlp(P, P, P, P, P, 4, 256, 512, 7, 0, P, P, 1 << 30, None) == 1
+    lib.sha_mlp_union.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int] + [
+        ctypes.c_void_p] * 3 + [ctypes.c_size_t, ctypes.c_void_p]
+    assert lib.sha_mlp_union(P, 0, 100, P, P, P, 1 << 20, None) == 1
+    assert lib.sha_mlp_union(P, 2, 100, P, P, P, 1, None) == 7     # workspace too small

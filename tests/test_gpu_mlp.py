@@ -38,6 +38,8 @@ CASES = [
     M("m3", B=64, d=256, D=1500, density=0.7, dtype="fp16", seed=3),
     M("m4", B=17, d=768, D=3072, density=1.0, dtype="bf16", seed=4),
     M("m5", B=5, d=256, D=4096, density=0.003, dtype="fp16", seed=5),
+    M("m6", B=12, d=512, D=1024, density=0.4, dtype="bf16", seed=6),     # batch tiles of 16
+    M("m7", B=32, d=1024, D=2048, density=0.2, dtype="fp16", seed=7),    # batch tiles of 32
 ]
 
 
