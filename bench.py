@@ -70,6 +70,8 @@ def parse_args():
                    help="run the LLaMA-2-7B-shaped scaling sweep instead (one JSON line)")
     p.add_argument("--mlp", action="store_true",
                    help="run the Selective GEMM (OPT-66B MLP) measurement instead")
+    p.add_argument("--mlp-density", type=float, nargs="*", default=None,
+                   help="union densities for --mlp (default 0.1 0.3 0.5 1.0)")
     return p.parse_args()
 
 
@@ -578,7 +580,8 @@ def run_mlp(args, dev=None):
                      dtype=torch.uint8, device=dev)
     y = torch.empty((base.B, base.d), dtype=x.dtype, device=dev)
     points = []
-    for dens in (0.1, 0.3, 0.5, 1.0):
+    densities = getattr(args, "mlp_density", None) or (0.1, 0.3, 0.5, 1.0)
+    for dens in densities:
         w = base.with_(density=dens)
         _, _, _, active = workloads.make_mlp(w.with_(d=256), device="cpu")   # mask only
         active = active.to(dev)

@@ -141,23 +141,35 @@ __device__ __forceinline__ int neuron_id(const int32_t *S, int t, int D)
 
 constexpr int kUpRows = 16;
 
+// Build-time tuning of the up-projection for batches up to 8.
+#ifndef SHA_MLP_UP8_K
+#define SHA_MLP_UP8_K 2304
+#endif
+#ifndef SHA_MLP_UP8_STAGES
+#define SHA_MLP_UP8_STAGES 2
+#endif
+
 template <int BP>
 struct UpCfg {
     static constexpr int kConsumerWarps = 4;
     static constexpr int kThreads = (kConsumerWarps + 1) * 32;
-    static constexpr int kKMax = BP <= 16 ? 1024 : (BP == 32 ? 512 : 256);  // d per stage
-    static constexpr int kStages = BP == 8 ? 4 : 3;    // small batches: more weight bytes in flight
+    // d per stage and stages: the longest weight-row segments that fit two
+    // (or three) stages next to the matching x rows
+    static constexpr int kKMax =
+        BP == 8 ? SHA_MLP_UP8_K : (BP == 16 ? 1536 : (BP == 32 ? 1024 : 512));
+    static constexpr int kStages = BP == 8 ? SHA_MLP_UP8_STAGES : 2;
     static constexpr int kRow = kKMax * 2 + 16;        // padded row: conflict-free ldmatrix
     static constexpr int kStage = (kUpRows + BP) * kRow;
     static constexpr int kBarOffset = kStages * kStage;
     static constexpr int kSmemBytes = kBarOffset + 2 * kStages * 8;
 };
 
-// d per stage: the largest of 1024/512/256 that divides d and fits the batch.
+// Width of a stage along d (or of an output-column range): the largest
+// multiple of 256 not above kmax that divides d (d is a multiple of 256).
 __host__ __device__ __forceinline__ int stage_width(int d, int kmax)
 {
-    int k = kmax;
-    while (k > 256 && d % k != 0) k >>= 1;
+    int k = kmax / 256 * 256;
+    while (k > 256 && d % k != 0) k -= 256;
     return k;
 }
 
@@ -208,11 +220,18 @@ __global__ void __launch_bounds__(UpCfg<BP>::kThreads, 1)
         int stage = 0;
         uint32_t phase = 0, last_parity = 0, used = 0;
         bool ok = true;
+        // the ids of an item's neurons are loaded one item ahead, so the
+        // pipeline never waits on them at an item boundary
+        auto item_id = [&](int it) {
+            const int t = (it / splits) * kUpRows + lane;
+            return (it < items && lane < kUpRows && t < n_S) ? neuron_id(S, t, D) : -1;
+        };
+        int id_next = item_id(blockIdx.x);
         for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
             const int grp = item / splits, split = item % splits;
             const int kt0 = split * ktiles / splits, kt1 = (split + 1) * ktiles / splits;
-            const int t = grp * kUpRows + lane;
-            const int id = (lane < kUpRows && t < n_S) ? neuron_id(S, t, D) : -1;
+            const int id = id_next;
+            id_next = item_id(item + gridDim.x);
             const int valid = min(kUpRows, n_S - grp * kUpRows);
             for (int kt = kt0; kt < kt1; ++kt) {
                 bool go = true;
@@ -340,22 +359,31 @@ __global__ void mlp_act_kernel(const float *__restrict__ part, const int32_t *__
 //
 // An item is a range of wc output columns (2 KiB of each weight row for
 // batches up to 16) over a range of the union's neurons; stages hold
-// kDownRows weight-row segments and the matching kDownRows x BP block of the
+// kRows weight-row segments and the matching kRows x BP block of the
 // neuron-major activations (one contiguous copy).  Eight consumer warps own
 // wc/8 columns each.  Partial sums over the neuron ranges go to the workspace
 // and mlp_out adds them in a fixed order.
 
-constexpr int kDownRows = 32;
+// Build-time tuning of the down-projection for batches up to 8.
+#ifndef SHA_MLP_DOWN8_W
+#define SHA_MLP_DOWN8_W 1024
+#endif
+#ifndef SHA_MLP_DOWN8_ROWS
+#define SHA_MLP_DOWN8_ROWS 32
+#endif
 
 template <int BP>
 struct DownCfg {
     static constexpr int kConsumerWarps = 8;
     static constexpr int kThreads = (kConsumerWarps + 1) * 32;
-    static constexpr int kWMax = BP <= 16 ? 1024 : (BP == 32 ? 512 : 256);   // columns per item
+    static constexpr int kWMax =                        // columns per item
+        BP == 8 ? SHA_MLP_DOWN8_W : (BP == 16 ? 1024 : (BP == 32 ? 1024 : 512));
+    static constexpr int kRows = BP == 8 ? SHA_MLP_DOWN8_ROWS : 32;   // neurons per stage
     static constexpr int kStages = 3;
     static constexpr int kWRow = kWMax * 2 + 16;       // padded rows
-    static constexpr int kHBytes = kDownRows * BP * 2;
-    static constexpr int kStage = kDownRows * kWRow + kHBytes;
+    static constexpr int kHBytes = kRows * BP * 2;
+    static constexpr int kStage = kRows * kWRow + kHBytes;
+    static_assert(kRows == 16 || kRows == 32, "one or two k-steps per stage");
     static constexpr int kBarOffset = kStages * kStage;
     static constexpr int kSmemBytes = kBarOffset + 2 * kStages * 8;
 };
@@ -384,7 +412,7 @@ __global__ void __launch_bounds__(DownCfg<BP>::kThreads, 1)
 
     const int n_S = union_size(n_S_ptr, D);
     const int wc = stage_width(d, C::kWMax);
-    const int ktiles = (n_S + kDownRows - 1) / kDownRows;
+    const int ktiles = (n_S + C::kRows - 1) / C::kRows;
     const int wchunks = d / wc;
     const int items = wchunks * splits;
 
@@ -393,11 +421,23 @@ __global__ void __launch_bounds__(DownCfg<BP>::kThreads, 1)
         int stage = 0;
         uint32_t phase = 0, last_parity = 0, used = 0;
         bool ok = true;
+        // one weight row per lane and tile; its neuron id is loaded one tile
+        // ahead (rows past the union repeat its last neuron: finite values
+        // times an activation of 0 add nothing, where stale shared memory
+        // could hold NaN)
+        auto tile_id = [&](int kt) {
+            return (kt < ktiles && lane < C::kRows)
+                       ? neuron_id(S, min(kt * C::kRows + lane, n_S - 1), D)
+                       : 0;
+        };
         for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
             const int wcn = item / splits, split = item % splits;
             const int kt0 = split * ktiles / splits, kt1 = (split + 1) * ktiles / splits;
             const size_t c0 = (size_t)wcn * wc;
+            int id_next = tile_id(kt0 < kt1 ? kt0 : ktiles);
             for (int kt = kt0; kt < kt1; ++kt) {
+                const int id = id_next;
+                id_next = tile_id(kt + 1 < kt1 ? kt + 1 : ktiles);
                 bool go = true;
                 if (lane == 0 && !mbar_wait(&empty[stage], phase ^ 1)) {
                     atomicOr(&g_sha_status, kStatusTimeout);
@@ -407,17 +447,14 @@ __global__ void __launch_bounds__(DownCfg<BP>::kThreads, 1)
                 if (!go) { ok = false; break; }
                 if (lane == 0)
                     mbar_arrive_expect_tx(&full[stage],
-                                          (uint32_t)(kDownRows * wc * 2 + C::kHBytes));
+                                          (uint32_t)(C::kRows * wc * 2 + C::kHBytes));
                 __syncwarp();
                 unsigned char *ws = smem + stage * C::kStage;
-                unsigned char *hs = ws + kDownRows * C::kWRow;
-                const int t0 = kt * kDownRows;
-                // rows past the union repeat its last neuron: finite values
-                // times an activation of 0 add nothing (stale shared memory
-                // could be NaN)
-                const int t = min(t0 + lane, n_S - 1);
-                bulk_copy_g2s(ws + lane * C::kWRow, W2t + (size_t)neuron_id(S, t, D) * d + c0,
-                              wc * 2, &full[stage], policy);
+                unsigned char *hs = ws + C::kRows * C::kWRow;
+                const int t0 = kt * C::kRows;
+                if (lane < C::kRows)
+                    bulk_copy_g2s(ws + lane * C::kWRow, W2t + (size_t)id * d + c0, wc * 2,
+                                  &full[stage], policy);
                 if (lane == 0)
                     bulk_copy_g2s(hs, Ht + (size_t)t0 * BP, C::kHBytes, &full[stage], policy);
                 last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -454,9 +491,9 @@ __global__ void __launch_bounds__(DownCfg<BP>::kThreads, 1)
         for (int kt = kt0; kt < kt1; ++kt) {
             const bool live = __all_sync(0xffffffffu, mbar_wait(&full[stage], phase));
             if (live) {
-                const uint32_t ws = base + stage * C::kStage, hs = ws + kDownRows * C::kWRow;
+                const uint32_t ws = base + stage * C::kStage, hs = ws + C::kRows * C::kWRow;
 #pragma unroll
-                for (int k16 = 0; k16 < kDownRows / 16; ++k16) {
+                for (int k16 = 0; k16 < C::kRows / 16; ++k16) {
                     // activations, neuron-major in shared memory: A = Ht^T via ldmatrix.trans
                     uint32_t a[kMT][4];
                     if constexpr (BP == 8) {
@@ -584,8 +621,10 @@ MlpPlan mlp_plan(int B, int d, int D, int sms)
 {
     MlpPlan pl;
     pl.bp = batch_pad(B);
-    const int kmax = pl.bp <= 16 ? 1024 : (pl.bp == 32 ? 512 : 256);
-    pl.h_rows = (int)round_up((size_t)D, (size_t)kDownRows);
+    const int kmax = pl.bp == 8 ? DownCfg<8>::kWMax
+                                : (pl.bp == 16 ? DownCfg<16>::kWMax
+                                               : (pl.bp == 32 ? DownCfg<32>::kWMax : DownCfg<64>::kWMax));
+    pl.h_rows = (int)round_up((size_t)D, (size_t)32);   // whole down-projection stages
     // up partials: splits * 4 warps sums of n_pad neurons; splits * groups <= 4*sms + groups
     const size_t max_groups = (D + kUpRows - 1) / kUpRows;
     pl.up_bytes = round_up((4 * (size_t)sms + max_groups) * 4 * kUpRows * pl.bp * 4, 256);
