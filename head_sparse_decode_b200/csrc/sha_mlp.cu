@@ -31,11 +31,15 @@
 #include <cmath>
 #include <cstdio>
 #include <mutex>
+#include <type_traits>
 #include <utility>
+
+#include <cudaTypedefs.h>
 
 #include "sha_decode.h"
 #include "sha_device.cuh"
 #include "sha_mma.cuh"
+#include "sha_tcgen05.cuh"
 
 namespace {
 
@@ -45,27 +49,60 @@ using namespace sha;
 #define SHA_USE_PDL 1
 #endif
 
+// Up-projection of batches above 8 on tcgen05 (1) or on warp-level MMAs (0).
+#ifndef SHA_MLP_TC_UP
+#define SHA_MLP_TC_UP 1
+#endif
+
 constexpr int kMaxDevicesMlp = 64;
 constexpr int kMlpMaxBatch = 64;        // batch rows per call (MMA tiles cover 64)
-constexpr int kUnionChunk = 1024;       // neurons per block in the union kernels
+constexpr int kUnionChunk = 256;        // neurons per block in the union kernels
 constexpr int kUnionThreads = 256;
+constexpr int kUnionRowGroups = kUnionThreads / (kUnionChunk / 4);   // batch rows split 4 ways
 
 // ---------------------------------------------------------------- union
 
+// flags[j] = 1 if any row of the batch has neuron j active; counts[block] =
+// the number of such neurons in the block's chunk.  A thread ORs four
+// neighbouring neurons over every fourth batch row (one 32-bit load per row
+// when the mask rows are 4-byte aligned).
 __global__ void __launch_bounds__(kUnionThreads)
-    mlp_union_flags_kernel(const uint8_t *__restrict__ active, int B, int D,
+    mlp_union_flags_kernel(const uint8_t *__restrict__ active, int B, int D, int words,
                            uint8_t *__restrict__ flags, int *__restrict__ counts)
 {
     pdl_wait();
     pdl_launch_dependents();
+    __shared__ uint32_t part[kUnionRowGroups][kUnionChunk / 4];
     __shared__ int warp_sum[kUnionThreads / 32];
-    const int j0 = blockIdx.x * kUnionChunk;
+    const int quad = threadIdx.x % (kUnionChunk / 4), rg = threadIdx.x / (kUnionChunk / 4);
+    const int j = blockIdx.x * kUnionChunk + quad * 4;
+    uint32_t any = 0;
+    if (j < D) {
+        if (words) {
+            for (int b = rg; b < B; b += kUnionRowGroups)
+                any |= __ldg(reinterpret_cast<const uint32_t *>(active + (size_t)b * D + j));
+        } else {
+            const int n = min(4, D - j);
+            for (int b = rg; b < B; b += kUnionRowGroups)
+                for (int i = 0; i < n; ++i)
+                    any |= (uint32_t)active[(size_t)b * D + j + i] << (8 * i);
+        }
+    }
+    part[rg][quad] = any;
+    __syncthreads();
     int cnt = 0;
-    for (int j = j0 + threadIdx.x; j < min(D, j0 + kUnionChunk); j += kUnionThreads) {
-        uint8_t any = 0;
-        for (int b = 0; b < B; ++b) any |= active[(size_t)b * D + j];
-        flags[j] = any != 0;
-        cnt += any != 0;
+    if (rg == 0 && j < D) {
+        for (int r = 1; r < kUnionRowGroups; ++r) any |= part[r][quad];
+        uint32_t f = 0;
+        for (int i = 0; i < 4; ++i)
+            if (j + i < D && ((any >> (8 * i)) & 0xffu)) {
+                f |= 1u << (8 * i);
+                ++cnt;
+            }
+        if (words)
+            *reinterpret_cast<uint32_t *>(flags + j) = f;
+        else
+            for (int i = 0; i < min(4, D - j); ++i) flags[j + i] = (f >> (8 * i)) & 1u;
     }
     for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
     if ((threadIdx.x & 31) == 0) warp_sum[threadIdx.x >> 5] = cnt;
@@ -77,38 +114,44 @@ __global__ void __launch_bounds__(kUnionThreads)
     }
 }
 
+// S = the flagged neuron ids in increasing order, n_S = their number.  Each
+// block adds up the counts of the blocks before it, then writes its chunk at
+// that offset in thread order.
 __global__ void __launch_bounds__(kUnionThreads)
     mlp_union_write_kernel(const uint8_t *__restrict__ flags, const int *__restrict__ counts,
                            int D, int32_t *__restrict__ S, int32_t *__restrict__ n_S)
 {
     pdl_wait();
     pdl_launch_dependents();
-    constexpr int kPer = kUnionChunk / kUnionThreads;   // 4 neurons per thread
+    static_assert(kUnionChunk == kUnionThreads, "one neuron per thread");
     __shared__ int warp_sum[kUnionThreads / 32];
-    int base = 0;
-    for (int i = 0; i < (int)blockIdx.x; ++i) base += counts[i];
-    if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) *n_S = base + counts[blockIdx.x];
-    const int j0 = blockIdx.x * kUnionChunk + threadIdx.x * kPer;
-    int f[kPer], mine = 0;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-        f[i] = (j0 + i < D) ? flags[j0 + i] : 0;
-        mine += f[i];
-    }
-    // exclusive prefix of `mine` over the block, in thread order
+    __shared__ int s_base;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int incl = mine;
+    int before = 0;
+    for (int i = threadIdx.x; i < (int)blockIdx.x; i += kUnionThreads) before += counts[i];
+    for (int off = 16; off > 0; off >>= 1) before += __shfl_xor_sync(0xffffffffu, before, off);
+    if (lane == 0) warp_sum[warp] = before;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int base = 0;
+        for (int w = 0; w < kUnionThreads / 32; ++w) base += warp_sum[w];
+        s_base = base;
+        if (blockIdx.x == gridDim.x - 1) *n_S = base + counts[blockIdx.x];
+    }
+    __syncthreads();
+    const int j = blockIdx.x * kUnionChunk + threadIdx.x;
+    const int f = j < D ? flags[j] : 0;
+    // exclusive prefix of the flags over the block, in thread order
+    int incl = f;
     for (int off = 1; off < 32; off <<= 1) {
         const int x = __shfl_up_sync(0xffffffffu, incl, off);
         if (lane >= off) incl += x;
     }
     if (lane == 31) warp_sum[warp] = incl;
     __syncthreads();
-    int pos = base + incl - mine;
+    int pos = s_base + incl - f;
     for (int w = 0; w < warp; ++w) pos += warp_sum[w];
-#pragma unroll
-    for (int i = 0; i < kPer; ++i)
-        if (f[i]) S[pos++] = j0 + i;
+    if (f) S[pos] = j;
 }
 
 // The union size and ids come from device memory (the union kernel or the
@@ -353,6 +396,347 @@ __global__ void mlp_act_kernel(const float *__restrict__ part, const int32_t *__
         if (act == 1) v = fmaxf(v, 0.f);
     }
     Ht[i] = Elem<T>::from_float(v);
+}
+
+// ---------------------------------------------------------------- up-projection on tcgen05
+//
+// For batches of 9 to 64 rows the arithmetic per weight byte (about B flops)
+// is more than warp-level MMAs sustain at HBM speed, so the up-projection of
+// those batches runs on the fifth-generation tensor cores:
+//     D [128 neurons x BP] (fp32, in TMEM) = W1t[S rows] . x^T
+// A = 128 gathered weight rows (TMA four-row gathers) and B = the batch's x
+// rows (one TMA box), both K-major with 128-byte swizzle, four 64-element K
+// atoms (256 elements) per stage.  One thread issues the MMAs; four epilogue
+// warps read the accumulator (double-buffered in TMEM) back.
+//
+// Work units are (group of 128 neurons, 256-element K tile); block b takes the
+// contiguous unit range [b U / NB, (b+1) U / NB) (stream-K), so every block
+// streams the same number of weight bytes at any union size.  A group whose
+// K tiles all fall in one block is finished there: the activation is applied
+// and its Ht rows written.  A group split across blocks leaves fp32 partial
+// sums in slot 0 (the block's first group) or slot 1 (its last group) of the
+// block, and mlp_act_tc adds them up in block order.
+
+// How the gathered weight rows reach shared memory: 0 = TMA four-row gathers
+// issued by one producer warp; 1 = 16-byte cp.async copies from four producer
+// warps (the TMA unit then only loads x).
+#ifndef SHA_MLP_TC_FEED
+#define SHA_MLP_TC_FEED 1
+#endif
+
+namespace uptc {
+constexpr int kM = 128;                    // neurons per group (MMA M)
+constexpr int kAtomK = 64;                 // elements per 128-byte swizzled row
+constexpr int kAtoms = 4;                  // K atoms per stage
+constexpr int kStageK = kAtoms * kAtomK;   // elements of K per stage
+constexpr int kProducerWarps = SHA_MLP_TC_FEED ? 4 : 1;
+constexpr int kMmaWarp = kProducerWarps;   // then four epilogue warps
+constexpr int kThreads = (kProducerWarps + 5) * 32;
+}  // namespace uptc
+
+template <int BP>
+struct UpTcCfg {
+    static constexpr int kAAtom = uptc::kM * 128;             // bytes of one A K atom
+    static constexpr int kABytes = uptc::kAtoms * kAAtom;
+    static constexpr int kBAtom = BP * 128;
+    static constexpr int kBBytes = uptc::kAtoms * kBAtom;
+    static constexpr int kStage = kABytes + kBBytes;
+    static constexpr int kStages = BP == 16 ? 3 : 2;
+    static constexpr int kBarOffset = kStages * kStage;
+    // full[s], empty[s], acc_full[2], acc_empty[2], mma_done; the TMEM address
+    static constexpr int kBarBytes = (2 * kStages + 5) * 8 + 8;
+    static constexpr int kSmemBytes = 1024 + kBarOffset + kBarBytes;   // + alignment slack
+    static constexpr uint32_t kTmemCols = 2 * BP < 32 ? 32 : 2 * BP;   // two accumulators
+    static_assert(BP % 16 == 0 && BP <= 64, "N = BP: a multiple of 16 up to 64");
+    static_assert(kAAtom % 1024 == 0 && kBAtom % 1024 == 0 && kStage % 1024 == 0,
+                  "swizzle atoms stay 1 KiB aligned");
+    static_assert(kSmemBytes <= 232448, "fits the shared-memory opt-in");
+};
+
+// Stream-K split of U units over NB blocks.
+struct UnitSplit {
+    long long U;
+    int NB;
+    __device__ __forceinline__ long long begin(int b) const { return U * b / NB; }
+    // the block whose range holds unit u
+    __device__ __forceinline__ int owner(long long u) const
+    {
+        return (int)(((u + 1) * NB + U - 1) / U - 1);
+    }
+};
+
+__device__ __forceinline__ uint64_t l2_policy_evict_last()
+{
+    uint64_t policy;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(policy));
+    return policy;
+}
+
+template <typename T, int BP>
+__global__ void __launch_bounds__(uptc::kThreads, 1)
+    mlp_up_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+                     const T *__restrict__ W1t, const int32_t *__restrict__ S, const int32_t *__restrict__ n_S_ptr, int B,
+                     int d, int D, int act, float *__restrict__ part, T *__restrict__ Ht)
+{
+    using C = UpTcCfg<BP>;
+    using namespace uptc;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOffset);
+    uint64_t *empty = full + C::kStages;
+    uint64_t *acc_full = empty + C::kStages;
+    uint64_t *acc_empty = acc_full + 2;
+    uint64_t *mma_done = acc_empty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            // the x box's expect-tx arrival, plus one cp.async arrival per producer thread
+            mbar_init(&full[s], SHA_MLP_TC_FEED ? 1 + 32 * kProducerWarps : 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&acc_full[a], 1);
+            mbar_init(&acc_empty[a], 4);
+        }
+        mbar_init(mma_done, 1);
+        mbar_init_fence();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    pdl_wait();
+    pdl_launch_dependents();
+
+    const int n_S = union_size(n_S_ptr, D);
+    const int KT = d / kStageK;
+    const UnitSplit split{(long long)((n_S + kM - 1) / kM) * KT, (int)gridDim.x};
+    const long long u0 = split.begin(blockIdx.x), u1 = split.begin(blockIdx.x + 1);
+    const int g_first = (int)(u0 / KT);
+
+    if (warp < kProducerWarps) {
+        const uint64_t pol_w = l2_policy_evict_first(), pol_x = l2_policy_evict_last();
+        int stage = 0;
+        uint32_t phase = 0, last_parity = 0, used = 0;
+        bool ok = true;
+        for (long long u = u0; u < u1 && ok;) {
+            const int g = (int)(u / KT);
+            const int kt0 = (int)(u - (long long)g * KT);
+            const int kt1 = (int)min((long long)KT, u1 - (long long)g * KT);
+#if SHA_MLP_TC_FEED
+            // warp p copies rows 32p..32p+31: copy i of a k atom moves 128 bytes of
+            // rows 32p+4i .. +3 (eight lanes per row, one 16-byte chunk each) to
+            // their swizzled places (ids past the union repeat its last neuron;
+            // their rows are computed and dropped)
+            const int chunk = lane & 7;
+            int row[8];
+            const T *src[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                row[i] = 32 * warp + 4 * i + (lane >> 3);
+                const int id = neuron_id(S, min(g * kM + row[i], n_S - 1), D);
+                src[i] = W1t + (size_t)id * d + chunk * 8;
+            }
+#else
+            // lane q gathers rows 4q..4q+3 of the group (ids past the union
+            // repeat its last neuron; their rows are computed and dropped)
+            int id[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) id[i] = neuron_id(S, min(g * kM + 4 * lane + i, n_S - 1), D);
+#endif
+            for (int kt = kt0; kt < kt1; ++kt) {
+                bool go = true;
+                if (lane == 0 && !mbar_wait(&empty[stage], phase ^ 1)) {
+                    atomicOr(&g_sha_status, kStatusTimeout);
+                    go = false;
+                }
+                go = __shfl_sync(0xffffffffu, go, 0);
+                if (!go) { ok = false; break; }
+                unsigned char *sa = smem + stage * C::kStage;
+                unsigned char *sb = sa + C::kABytes;
+                const int k0 = kt * kStageK;
+                if (warp == 0) {
+                    if (lane == 0)
+                        mbar_arrive_expect_tx(&full[stage],
+                                              (uint32_t)(SHA_MLP_TC_FEED ? C::kBBytes : C::kStage));
+                    __syncwarp();
+                    if (lane < kAtoms)
+                        tma_load_2d(sb + lane * C::kBAtom, &tm_x, k0 + lane * kAtomK, 0,
+                                    &full[stage], pol_x);
+                }
+#if SHA_MLP_TC_FEED
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+#pragma unroll
+                    for (int j = 0; j < kAtoms; ++j)
+                        cp_async16(sa + j * C::kAAtom + row[i] * 128 + ((chunk ^ (row[i] & 7)) << 4),
+                                   src[i] + k0 + j * kAtomK, pol_w);
+                cp_async_arrive_noinc(&full[stage]);
+#else
+#pragma unroll
+                for (int j = 0; j < kAtoms; ++j)
+                    tma_gather4(sa + j * C::kAAtom + lane * 512, &tm_w, k0 + j * kAtomK, id[0],
+                                id[1], id[2], id[3], &full[stage], pol_w);
+#endif
+                last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+                used |= 1u << stage;
+                if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+            }
+            u = (long long)(g + 1) * KT;
+        }
+        // no copy may be in flight when the block exits
+#if SHA_MLP_TC_FEED
+        cp_async_wait_all();
+#endif
+        if (warp == 0 && lane == 0)
+            for (int s = 0; s < C::kStages; ++s)
+                if (used & (1u << s)) mbar_wait(&full[s], (last_parity >> s) & 1u);
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_f16(sizeof(T) == 2 && !std::is_same<T, __half>::value,
+                                                      kM, BP);
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true;
+            for (long long u = u0; u < u1 && ok;) {
+                const int g = (int)(u / KT);
+                const int kt0 = (int)(u - (long long)g * KT);
+                const int kt1 = (int)min((long long)KT, u1 - (long long)g * KT);
+                if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1)) {
+                    atomicOr(&g_sha_status, kStatusTimeout);
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t dt = tmem + (uint32_t)(acc * BP);
+                for (int kt = kt0; kt < kt1; ++kt) {
+                    if (!mbar_wait(&full[stage], phase)) {
+                        atomicOr(&g_sha_status, kStatusTimeout);
+                        ok = false;
+                        break;
+                    }
+                    fence_proxy_async_shared();    // copied rows -> tensor-core reads
+                    tc_fence_after_sync();
+                    const uint32_t sa = smem_addr(smem + stage * C::kStage);
+                    const uint32_t sb = sa + C::kABytes;
+#pragma unroll
+                    for (int j = 0; j < kAtoms; ++j)
+#pragma unroll
+                        for (int kk = 0; kk < kAtomK / 16; ++kk)
+                            umma_f16(dt, umma_desc_k_sw128(sa + j * C::kAAtom + kk * 32),
+                                     umma_desc_k_sw128(sb + j * C::kBAtom + kk * 32), idesc,
+                                     (kt > kt0 || j > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&empty[stage]);          // stage reusable once read
+                    if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                umma_commit(&acc_full[acc]);
+                if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+                u = (long long)(g + 1) * KT;
+            }
+            // every issued MMA has finished before TMEM is released
+            if (u1 > u0) {
+                umma_commit(mma_done);
+                if (!mbar_wait(mma_done, 0)) atomicOr(&g_sha_status, kStatusTimeout);
+            }
+        }
+        __syncwarp();
+    } else {
+        // epilogue: warp w reads TMEM lanes 32*(w%4)..+31 = neuron rows of the group
+        const int quarter = warp & 3, row = quarter * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (long long u = u0; u < u1;) {
+            const int g = (int)(u / KT);
+            const int kt0 = (int)(u - (long long)g * KT);
+            const int kt1 = (int)min((long long)KT, u1 - (long long)g * KT);
+            const bool live = __all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_phase));
+            if (!live) {
+                if (lane == 0) atomicOr(&g_sha_status, kStatusTimeout);
+                break;
+            }
+            tc_fence_after_sync();
+            float v[BP / 16][16];
+#pragma unroll
+            for (int c = 0; c < BP / 16; ++c)
+                tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BP + c * 16),
+                          v[c]);
+            tmem_ld_wait();
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+            const int t = g * kM + row;
+            if (kt0 == 0 && kt1 == KT) {
+                // whole group here: Ht[t][0..BP) = sigma(D), zero outside the union and batch
+                T *dst = Ht + (size_t)t * BP;
+#pragma unroll
+                for (int c8 = 0; c8 < BP / 8; ++c8) {
+                    __align__(16) T h[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int col = c8 * 8 + e;
+                        float x = v[col / 16][col % 16];
+                        if (act == 1) x = fmaxf(x, 0.f);
+                        h[e] = Elem<T>::from_float((t < n_S && col < B) ? x : 0.f);
+                    }
+                    *reinterpret_cast<uint4 *>(dst + c8 * 8) = *reinterpret_cast<const uint4 *>(h);
+                }
+            } else {
+                const int slot = g == g_first ? 0 : 1;
+                float *dst = part + ((size_t)(blockIdx.x * 2 + slot) * kM + row) * BP;
+#pragma unroll
+                for (int c4 = 0; c4 < BP / 4; ++c4)
+                    *reinterpret_cast<float4 *>(dst + c4 * 4) =
+                        make_float4(v[c4 / 4][(c4 % 4) * 4], v[c4 / 4][(c4 % 4) * 4 + 1],
+                                    v[c4 / 4][(c4 % 4) * 4 + 2], v[c4 / 4][(c4 % 4) * 4 + 3]);
+            }
+            if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+            u = (long long)(g + 1) * KT;
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+// Ht rows of the groups mlp_up_tc split across blocks: the blocks' partial
+// sums added in block order, then sigma; zero outside the union and batch.
+template <typename T, int BP>
+__global__ void mlp_act_tc_kernel(const float *__restrict__ part,
+                                  const int32_t *__restrict__ n_S_ptr, int B, int d, int D,
+                                  int up_blocks, int act, T *__restrict__ Ht)
+{
+    using namespace uptc;
+    pdl_wait();
+    pdl_launch_dependents();
+    const int n_S = union_size(n_S_ptr, D);
+    const int KT = d / kStageK, G = (n_S + kM - 1) / kM;
+    const UnitSplit split{(long long)G * KT, up_blocks};
+    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int t = (int)(i / BP), col = (int)(i % BP), g = t / kM;
+    if (g >= G) return;
+    const int bf = split.owner((long long)g * KT), bl = split.owner((long long)(g + 1) * KT - 1);
+    if (bf == bl) return;                       // finished by the up-projection
+    float v = 0.f;
+    for (int b = bf; b <= bl; ++b) {
+        const long long a = split.begin(b);
+        if (a == split.begin(b + 1)) continue;  // a block with no units
+        const int slot = g == (int)(a / KT) ? 0 : 1;
+        v += part[((size_t)(b * 2 + slot) * kM + t % kM) * BP + col];
+    }
+    if (act == 1) v = fmaxf(v, 0.f);
+    Ht[i] = Elem<T>::from_float((t < n_S && col < B) ? v : 0.f);
 }
 
 // ---------------------------------------------------------------- down-projection
@@ -606,10 +990,55 @@ int device_sms(int *dev)
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// cuTensorMapEncodeTiled from the driver, found through the runtime so the
+// library does not link against libcuda.
+PFN_cuTensorMapEncodeTiled_v12000 mlp_tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 2-D view [rows][d] of a row-major fp16/bf16 matrix, boxes of 64 elements x
+// box_rows rows with 128-byte swizzle; rows past the end read as zero.
+sha_status_t mlp_tensor_map(CUtensorMap *map, const void *base, bool bf16, int d, int rows,
+                            int box_rows)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 encode = mlp_tensor_map_encoder();
+    if (!encode) {
+        std::snprintf(g_mlp_error, sizeof g_mlp_error,
+                      "cuTensorMapEncodeTiled is not available from the driver");
+        return SHA_ERR_LAUNCH;
+    }
+    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    cuuint32_t box[2] = {(cuuint32_t)uptc::kAtomK, (cuuint32_t)box_rows};
+    cuuint32_t elem[2] = {1, 1};
+    CUresult r = encode(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                        2, const_cast<void *>(base), dims, strides, box, elem,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        std::snprintf(g_mlp_error, sizeof g_mlp_error,
+                      "cuTensorMapEncodeTiled failed with CUresult %d", (int)r);
+        return SHA_ERR_LAUNCH;
+    }
+    return SHA_OK;
+}
+
 // Workspace of sha_selective_mlp for these sizes on a device with `sms` SMs.
 struct MlpPlan {
     int bp;                // batch padded to 16, 32 or 64
     int h_rows;            // rows of the neuron-major activations (union padded)
+    bool tc_up;            // up-projection on tcgen05 (batches above 8)
     int down_splits, down_blocks;
     size_t up_bytes, h_bytes, down_bytes;
     size_t total() const { return up_bytes + h_bytes + down_bytes; }
@@ -624,10 +1053,16 @@ MlpPlan mlp_plan(int B, int d, int D, int sms)
     const int kmax = pl.bp == 8 ? DownCfg<8>::kWMax
                                 : (pl.bp == 16 ? DownCfg<16>::kWMax
                                                : (pl.bp == 32 ? DownCfg<32>::kWMax : DownCfg<64>::kWMax));
-    pl.h_rows = (int)round_up((size_t)D, (size_t)32);   // whole down-projection stages
-    // up partials: splits * 4 warps sums of n_pad neurons; splits * groups <= 4*sms + groups
-    const size_t max_groups = (D + kUpRows - 1) / kUpRows;
-    pl.up_bytes = round_up((4 * (size_t)sms + max_groups) * 4 * kUpRows * pl.bp * 4, 256);
+    pl.h_rows = (int)round_up((size_t)D, (size_t)uptc::kM);   // whole neuron groups
+    pl.tc_up = pl.bp >= 16 && SHA_MLP_TC_UP;
+    if (pl.tc_up) {
+        // two partial slots of 128 x BP per block
+        pl.up_bytes = round_up((size_t)sms * 2 * uptc::kM * pl.bp * 4, 256);
+    } else {
+        // splits * 4 warps sums of n_pad neurons; splits * groups <= 4*sms + groups
+        const size_t max_groups = (D + kUpRows - 1) / kUpRows;
+        pl.up_bytes = round_up((4 * (size_t)sms + max_groups) * 4 * kUpRows * pl.bp * 4, 256);
+    }
     pl.h_bytes = round_up((size_t)pl.h_rows * pl.bp * 2, 256);
     const int wc = stage_width(d, kmax);
     const int wchunks = d / wc;
@@ -648,6 +1083,11 @@ sha_status_t run_mlp_bp(const void *x, const void *W1t, const void *W2t, const i
         cudaError_t e = cudaFuncSetAttribute(mlp_up_kernel<T, BP>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              UpCfg<BP>::kSmemBytes);
+        if constexpr (BP >= 16)
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(mlp_up_tc_kernel<T, BP>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         UpTcCfg<BP>::kSmemBytes);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(mlp_down_kernel<T, BP>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -661,14 +1101,33 @@ sha_status_t run_mlp_bp(const void *x, const void *W1t, const void *W2t, const i
     T *Ht = reinterpret_cast<T *>(w + pl.up_bytes);
     float *down_part = reinterpret_cast<float *>(w + pl.up_bytes + pl.h_bytes);
 
-    cudaError_t e = launch_pdl(mlp_up_kernel<T, BP>, dim3(sms), UpCfg<BP>::kThreads,
-                               UpCfg<BP>::kSmemBytes, s, static_cast<const T *>(x),
-                               static_cast<const T *>(W1t), S, n_S, B, d, D, up_part);
-    if (e != cudaSuccess) return mlp_launch_error(e);
     const size_t hn = (size_t)pl.h_rows * BP;
-    e = launch_pdl(mlp_act_kernel<T, BP>, dim3((unsigned)((hn + 255) / 256)), 256, 0, s,
-                   (const float *)up_part, n_S, B, d, D, pl.h_rows, sms, act, Ht);
-    if (e != cudaSuccess) return mlp_launch_error(e);
+    cudaError_t e;
+    if constexpr (BP >= 16) {
+        if (pl.tc_up) {
+            constexpr bool bf16 = !std::is_same<T, __half>::value;
+            CUtensorMap tm_w, tm_x;
+            sha_status_t st = mlp_tensor_map(&tm_w, W1t, bf16, d, D, 1);
+            if (st == SHA_OK) st = mlp_tensor_map(&tm_x, x, bf16, d, B, BP);
+            if (st != SHA_OK) return st;
+            e = launch_pdl(mlp_up_tc_kernel<T, BP>, dim3(sms), uptc::kThreads,
+                           UpTcCfg<BP>::kSmemBytes, s, tm_w, tm_x, static_cast<const T *>(W1t), S,
+                           n_S, B, d, D, act, up_part, Ht);
+            if (e != cudaSuccess) return mlp_launch_error(e);
+            e = launch_pdl(mlp_act_tc_kernel<T, BP>, dim3((unsigned)((hn + 255) / 256)), 256, 0,
+                           s, (const float *)up_part, n_S, B, d, D, sms, act, Ht);
+            if (e != cudaSuccess) return mlp_launch_error(e);
+        }
+    }
+    if (!pl.tc_up) {
+        e = launch_pdl(mlp_up_kernel<T, BP>, dim3(sms), UpCfg<BP>::kThreads,
+                       UpCfg<BP>::kSmemBytes, s, static_cast<const T *>(x),
+                       static_cast<const T *>(W1t), S, n_S, B, d, D, up_part);
+        if (e != cudaSuccess) return mlp_launch_error(e);
+        e = launch_pdl(mlp_act_kernel<T, BP>, dim3((unsigned)((hn + 255) / 256)), 256, 0, s,
+                       (const float *)up_part, n_S, B, d, D, pl.h_rows, sms, act, Ht);
+        if (e != cudaSuccess) return mlp_launch_error(e);
+    }
     e = launch_pdl(mlp_down_kernel<T, BP>, dim3(pl.down_blocks), DownCfg<BP>::kThreads,
                    DownCfg<BP>::kSmemBytes, s, (const T *)Ht, static_cast<const T *>(W2t), S, n_S,
                    B, d, D, pl.down_splits, down_part);
@@ -725,8 +1184,9 @@ sha_status_t sha_mlp_union(const uint8_t *active, int B, int D, int32_t *S, int3
     uint8_t *flags = static_cast<uint8_t *>(workspace);
     int *counts = reinterpret_cast<int *>(static_cast<char *>(workspace) + round_up(D, 256));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int words = (D % 4 == 0 && aligned_to(active, 4)) ? 1 : 0;
     cudaError_t e = launch_pdl(mlp_union_flags_kernel, dim3(blocks), kUnionThreads, 0, s, active,
-                               B, D, flags, counts);
+                               B, D, words, flags, counts);
     if (e != cudaSuccess) return mlp_launch_error(e);
     e = launch_pdl(mlp_union_write_kernel, dim3(blocks), kUnionThreads, 0, s,
                    (const uint8_t *)flags, (const int *)counts, D, S, n_S);

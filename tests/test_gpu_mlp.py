@@ -105,3 +105,27 @@ def test_opt66b_mlp_shape_sampled(sha):
     want = oracle.selective_mlp(x.cpu(), W1t.cpu(), W2t[:, cols].cpu().contiguous(), Sh, w.dtype)
     err = np.abs(y[:, cols].cpu().double().numpy() - want).max()
     assert err <= TOLERANCE[w.dtype], err
+
+
+@pytest.mark.parametrize("B,density", [(64, 1.0), (50, 0.3), (32, 0.05), (16, 0.5), (9, 0.2)])
+def test_opt66b_mlp_large_batch_sampled(sha, B, density):
+    """Batches above 8 (tensor-memory up-projection) at the OPT-66B shape: a dense
+    union leaves some neuron groups whole inside one block and splits others
+    across blocks; sparse unions split every group.  Sampled batch rows and
+    output columns against the oracle (which takes the same union S)."""
+    w = workloads.MLP_CONFIGS["opt66b_mlp"].with_(B=B, density=density, seed=5100 + B)
+    dev = torch.device("cuda")
+    x, W1t, W2t, active = workloads.make_mlp(w, device=dev)
+    S, n_S = sha.sha_mlp_union(active)
+    y = sha.sha_selective_mlp(x, W1t, W2t, S, n_S)
+    torch.cuda.synchronize()
+    assert sha.sha_get_device_status() == sha.SHA_OK
+    n = int(n_S.item())
+    Sh = S[:n].cpu().numpy()
+    assert np.array_equal(Sh, oracle.mlp_union(active.cpu().numpy()))
+    rows = sorted({0, B // 3, (2 * B) // 3, B - 1})
+    cols = np.sort(np.random.default_rng(B).choice(w.d, 192, replace=False))
+    want = oracle.selective_mlp(x[rows].cpu(), W1t.cpu(), W2t[:, cols].cpu().contiguous(), Sh,
+                                w.dtype)
+    err = np.abs(y[rows][:, cols].cpu().double().numpy() - want).max()
+    assert err <= TOLERANCE[w.dtype], err
