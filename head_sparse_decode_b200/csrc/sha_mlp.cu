@@ -49,9 +49,13 @@ using namespace sha;
 #define SHA_USE_PDL 1
 #endif
 
-// Up-projection of batches above 8 on tcgen05 (1) or on warp-level MMAs (0).
-#ifndef SHA_MLP_TC_UP
-#define SHA_MLP_TC_UP 1
+// GEMMs of batches above 8 on tcgen05 (1) or on warp-level MMAs (0); the
+// down-projection joins from padded batch SHA_MLP_TC_DOWN_MIN_BATCH up.
+#ifndef SHA_MLP_TC
+#define SHA_MLP_TC 1
+#endif
+#ifndef SHA_MLP_TC_DOWN_MIN_BATCH
+#define SHA_MLP_TC_DOWN_MIN_BATCH 32
 #endif
 
 constexpr int kMaxDevicesMlp = 64;
@@ -472,11 +476,14 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last()
     return policy;
 }
 
-template <typename T, int BP>
+// kBatchMajor: Ht stored [BP][h_rows] (the tcgen05 down-projection's K-major
+// operand); otherwise [h_rows][BP] (the warp-level down-projection's).
+template <typename T, int BP, bool kBatchMajor>
 __global__ void __launch_bounds__(uptc::kThreads, 1)
     mlp_up_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
-                     const T *__restrict__ W1t, const int32_t *__restrict__ S, const int32_t *__restrict__ n_S_ptr, int B,
-                     int d, int D, int act, float *__restrict__ part, T *__restrict__ Ht)
+                     const T *__restrict__ W1t, const int32_t *__restrict__ S,
+                     const int32_t *__restrict__ n_S_ptr, int B, int d, int D, int act, int h_rows,
+                     float *__restrict__ part, T *__restrict__ Ht)
 {
     using C = UpTcCfg<BP>;
     using namespace uptc;
@@ -674,28 +681,36 @@ __global__ void __launch_bounds__(uptc::kThreads, 1)
             if (lane == 0) mbar_arrive(&acc_empty[acc]);
             const int t = g * kM + row;
             if (kt0 == 0 && kt1 == KT) {
-                // whole group here: Ht[t][0..BP) = sigma(D), zero outside the union and batch
-                T *dst = Ht + (size_t)t * BP;
+                // whole group here: Ht = sigma(D), zero outside the union and batch
+                if constexpr (kBatchMajor) {
 #pragma unroll
-                for (int c8 = 0; c8 < BP / 8; ++c8) {
-                    __align__(16) T h[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int col = c8 * 8 + e;
+                    for (int col = 0; col < BP; ++col) {
                         float x = v[col / 16][col % 16];
                         if (act == 1) x = fmaxf(x, 0.f);
-                        h[e] = Elem<T>::from_float((t < n_S && col < B) ? x : 0.f);
+                        Ht[(size_t)col * h_rows + t] =
+                            Elem<T>::from_float((t < n_S && col < B) ? x : 0.f);
                     }
-                    *reinterpret_cast<uint4 *>(dst + c8 * 8) = *reinterpret_cast<const uint4 *>(h);
+                } else {
+#pragma unroll
+                    for (int c8 = 0; c8 < BP / 8; ++c8) {
+                        __align__(16) T h[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int col = c8 * 8 + e;
+                            float x = v[col / 16][col % 16];
+                            if (act == 1) x = fmaxf(x, 0.f);
+                            h[e] = Elem<T>::from_float((t < n_S && col < B) ? x : 0.f);
+                        }
+                        *reinterpret_cast<uint4 *>(Ht + (size_t)t * BP + c8 * 8) =
+                            *reinterpret_cast<const uint4 *>(h);
+                    }
                 }
             } else {
+                // partial sums, column-major per slot: [slot][col][row]
                 const int slot = g == g_first ? 0 : 1;
-                float *dst = part + ((size_t)(blockIdx.x * 2 + slot) * kM + row) * BP;
+                float *dst = part + (size_t)(blockIdx.x * 2 + slot) * BP * kM + row;
 #pragma unroll
-                for (int c4 = 0; c4 < BP / 4; ++c4)
-                    *reinterpret_cast<float4 *>(dst + c4 * 4) =
-                        make_float4(v[c4 / 4][(c4 % 4) * 4], v[c4 / 4][(c4 % 4) * 4 + 1],
-                                    v[c4 / 4][(c4 % 4) * 4 + 2], v[c4 / 4][(c4 % 4) * 4 + 3]);
+                for (int col = 0; col < BP; ++col) dst[(size_t)col * kM] = v[col / 16][col % 16];
             }
             if (++acc == 2) { acc = 0; acc_phase ^= 1; }
             u = (long long)(g + 1) * KT;
@@ -710,33 +725,378 @@ __global__ void __launch_bounds__(uptc::kThreads, 1)
     }
 }
 
-// Ht rows of the groups mlp_up_tc split across blocks: the blocks' partial
-// sums added in block order, then sigma; zero outside the union and batch.
-template <typename T, int BP>
-__global__ void mlp_act_tc_kernel(const float *__restrict__ part,
-                                  const int32_t *__restrict__ n_S_ptr, int B, int d, int D,
-                                  int up_blocks, int act, T *__restrict__ Ht)
+// Blocks whose unit ranges hold part of unit range [a, e) of a split, and
+// the partial slot each left for it (0 if it is the block's first item, else
+// 1), in block order; returns how many.
+__device__ __forceinline__ int split_contributors(const UnitSplit &split, int item, int per_item,
+                                                  int *blk, int *slot, int max_n)
+{
+    const int bf = split.owner((long long)item * per_item);
+    const int bl = split.owner((long long)(item + 1) * per_item - 1);
+    int n = 0;
+    for (int b = bf; b <= bl && n < max_n; ++b) {
+        const long long a = split.begin(b);
+        if (a == split.begin(b + 1)) continue;  // a block with no units
+        blk[n] = b;
+        slot[n] = item == (int)(a / per_item) ? 0 : 1;
+        ++n;
+    }
+    return n;
+}
+
+constexpr int kMaxContributors = 256;     // >= the blocks of a split (one per SM)
+
+// Ht entries (layout as in mlp_up_tc) of the groups mlp_up_tc split across
+// blocks: the blocks' partial sums added in block order, then sigma; zero
+// outside the union and batch.  Block (g, j) covers columns 2j, 2j+1 of
+// group g, one thread per (column, neuron).
+template <typename T, int BP, bool kBatchMajor>
+__global__ void __launch_bounds__(2 * uptc::kM)
+    mlp_act_tc_kernel(const float *__restrict__ part, const int32_t *__restrict__ n_S_ptr, int B,
+                      int d, int D, int up_blocks, int act, int h_rows, T *__restrict__ Ht)
 {
     using namespace uptc;
+    __shared__ int s_blk[kMaxContributors], s_slot[kMaxContributors], s_n;
     pdl_wait();
     pdl_launch_dependents();
     const int n_S = union_size(n_S_ptr, D);
-    const int KT = d / kStageK, G = (n_S + kM - 1) / kM;
-    const UnitSplit split{(long long)G * KT, up_blocks};
-    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int t = (int)(i / BP), col = (int)(i % BP), g = t / kM;
+    const int KT = d / kStageK, G = (n_S + kM - 1) / kM, g = blockIdx.x;
     if (g >= G) return;
-    const int bf = split.owner((long long)g * KT), bl = split.owner((long long)(g + 1) * KT - 1);
-    if (bf == bl) return;                       // finished by the up-projection
-    float v = 0.f;
-    for (int b = bf; b <= bl; ++b) {
-        const long long a = split.begin(b);
-        if (a == split.begin(b + 1)) continue;  // a block with no units
-        const int slot = g == (int)(a / KT) ? 0 : 1;
-        v += part[((size_t)(b * 2 + slot) * kM + t % kM) * BP + col];
+    if (threadIdx.x == 0) {
+        const UnitSplit split{(long long)G * KT, up_blocks};
+        const bool whole = split.owner((long long)g * KT) == split.owner((long long)(g + 1) * KT - 1);
+        s_n = whole ? 0 : split_contributors(split, g, KT, s_blk, s_slot, kMaxContributors);
     }
+    __syncthreads();
+    const int n = s_n;
+    if (n == 0) return;                         // finished by the up-projection
+    const int col = 2 * blockIdx.y + threadIdx.x / kM, row = threadIdx.x % kM, t = g * kM + row;
+    float v = 0.f;
+    for (int k = 0; k < n; ++k)
+        v += part[((size_t)(s_blk[k] * 2 + s_slot[k]) * BP + col) * kM + row];
     if (act == 1) v = fmaxf(v, 0.f);
-    Ht[i] = Elem<T>::from_float((t < n_S && col < B) ? v : 0.f);
+    Ht[kBatchMajor ? (size_t)col * h_rows + t : (size_t)t * BP + col] =
+        Elem<T>::from_float((t < n_S && col < B) ? v : 0.f);
+}
+
+// ---------------------------------------------------------------- down-projection on tcgen05
+//
+// y[b][c] = sum over the union of Ht[b][t] W2t[S_t][c], for batches of 9 to 64
+// rows, on the fifth-generation tensor cores:
+//     D [128 output columns x BP] (fp32, TMEM) = W2t[S rows][columns]^T . Ht^T
+// An item is 256 output columns (two accumulators, so each selected weight
+// row is read in 512-byte runs) over a range of the union in stages of 64
+// neurons.  A = the stage's weight-row segments, MN-major (output columns
+// contiguous) with 128-byte swizzle, copied by four producer warps with
+// 16-byte cp.async (one 512-byte row segment per warp instruction); B = the
+// stage's 64 x BP block of the batch-major activations (one TMA box, K-major).
+// Units are (256-column block, 64-neuron tile), split over the blocks as in
+// the up-projection: a column block whose tiles all fall in one block is
+// written to y there; a split one leaves fp32 partial sums in the block's
+// slot 0 (first column block) or 1 (last) and mlp_out_tc adds them in block
+// order.
+
+// Output columns per item: 512 (four accumulators, 1 KiB runs of each weight
+// row) when they divide d, else 256.
+#ifndef SHA_MLP_DOWN_TC_WIDE
+#define SHA_MLP_DOWN_TC_WIDE 1
+#endif
+
+// Neurons per stage of the down-projection: 64 (Ht tile one 128-byte swizzle
+// atom) or 32 (64-byte swizzle; twice the stages in the same shared memory).
+#ifndef SHA_MLP_DOWN_TC_ROWS
+#define SHA_MLP_DOWN_TC_ROWS 64
+#endif
+
+namespace downtc {
+constexpr int kM = 128;                    // output columns per accumulator (MMA M)
+constexpr int kR = SHA_MLP_DOWN_TC_ROWS;   // neurons per stage (K steps of 16)
+static_assert(kR == 32 || kR == 64, "a stage's Ht tile is one 64- or 128-byte swizzle row");
+constexpr int kProducerWarps = 4;
+constexpr int kMmaWarp = kProducerWarps;   // then four epilogue warps
+constexpr int kThreads = (kProducerWarps + 5) * 32;
+}  // namespace downtc
+
+template <int BP, int kHalves>
+struct DownTcCfg {
+    static constexpr int kCols = downtc::kM * kHalves;                 // output columns per item
+    static constexpr int kABytes = downtc::kR * kCols * 2;
+    static constexpr int kBBytes = BP * downtc::kR * 2;               // the stage's Ht tile
+    static constexpr int kStage = kABytes + kBBytes;
+    static constexpr int kStages = (200 * 1024) / kStage;
+    static constexpr int kBarOffset = kStages * kStage;
+    static constexpr int kBarBytes = (2 * kStages + 5) * 8 + 8;
+    static constexpr int kSmemBytes = 1024 + kBarOffset + kBarBytes;
+    static constexpr uint32_t kTmemCols = 2 * kHalves * BP;   // two items in flight
+    static_assert(kABytes % 1024 == 0 && kStage % 1024 == 0, "swizzle atoms stay 1 KiB aligned");
+    static_assert(kTmemCols >= 32 && (kTmemCols & (kTmemCols - 1)) == 0, "TMEM allocation size");
+    static_assert(kSmemBytes <= 232448, "fits the shared-memory opt-in");
+};
+
+template <typename T, int BP, int kHalves>
+__global__ void __launch_bounds__(downtc::kThreads, 1)
+    mlp_down_tc_kernel(const __grid_constant__ CUtensorMap tm_h, const T *__restrict__ W2t,
+                       const int32_t *__restrict__ S, const int32_t *__restrict__ n_S_ptr, int B,
+                       int d, int D, float *__restrict__ part, T *__restrict__ y)
+{
+    using C = DownTcCfg<BP, kHalves>;
+    using namespace downtc;
+    constexpr int kCols = C::kCols;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOffset);
+    uint64_t *empty = full + C::kStages;
+    uint64_t *acc_full = empty + C::kStages;
+    uint64_t *acc_empty = acc_full + 2;
+    uint64_t *mma_done = acc_empty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            // the Ht box's expect-tx arrival, plus one cp.async arrival per producer thread
+            mbar_init(&full[s], 1 + 32 * kProducerWarps);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&acc_full[a], 1);
+            mbar_init(&acc_empty[a], 4);
+        }
+        mbar_init(mma_done, 1);
+        mbar_init_fence();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    pdl_wait();
+    pdl_launch_dependents();
+
+    const int n_S = union_size(n_S_ptr, D);
+    const int KT = (n_S + uptc::kM - 1) / uptc::kM * (uptc::kM / kR);   // tiles of the padded union
+    const UnitSplit split{(long long)(d / kCols) * KT, (int)gridDim.x};
+    const long long u0 = split.begin(blockIdx.x), u1 = split.begin(blockIdx.x + 1);
+    const int cb_first = KT > 0 ? (int)(u0 / KT) : 0;
+
+    if (warp < kProducerWarps) {
+        // warp p copies neurons (kR/4)p .. +kR/4 of each stage.  An instruction
+        // moves 64 output columns (128 bytes) of four neurons: lane l takes
+        // neuron 4j + l/8 of the warp's quad j and 16-byte chunk l%8, so the
+        // four rows land as four consecutive 128-byte K rows of one swizzle atom
+        // (512 contiguous bytes of shared memory); the 2*kHalves pieces of the
+        // same four rows follow back to back.
+        const uint64_t pol_w = l2_policy_evict_first(), pol_h = l2_policy_evict_last();
+        constexpr int kQuads = kR / 16;                    // neuron quads per warp and stage
+        const int rsub = lane >> 3, cc = lane & 7;
+        int stage = 0;
+        uint32_t phase = 0, last_parity = 0, used = 0;
+        bool ok = true;
+        // this lane's neuron ids of a stage (rows past the union repeat its last
+        // neuron: their activations are zero)
+        auto stage_ids = [&](int kt, int (&ids)[kQuads]) {
+#pragma unroll
+            for (int j = 0; j < kQuads; ++j)
+                ids[j] = neuron_id(S, min(kt * kR + (kR / 4) * warp + 4 * j + rsub, n_S - 1), D);
+        };
+        for (long long u = u0; u < u1 && ok;) {
+            const int cb = (int)(u / KT);
+            const int kt0 = (int)(u - (long long)cb * KT);
+            const int kt1 = (int)min((long long)KT, u1 - (long long)cb * KT);
+            const T *col_src = W2t + (size_t)cb * kCols + cc * 8;
+            int ids_next[kQuads];
+            stage_ids(kt0, ids_next);
+            for (int kt = kt0; kt < kt1; ++kt) {
+                int ids[kQuads];
+#pragma unroll
+                for (int j = 0; j < kQuads; ++j) ids[j] = ids_next[j];
+                if (kt + 1 < kt1) stage_ids(kt + 1, ids_next);
+                bool go = true;
+                if (lane == 0 && !mbar_wait(&empty[stage], phase ^ 1)) {
+                    atomicOr(&g_sha_status, kStatusTimeout);
+                    go = false;
+                }
+                go = __shfl_sync(0xffffffffu, go, 0);
+                if (!go) { ok = false; break; }
+                unsigned char *sa = smem + stage * C::kStage;
+                unsigned char *sb = sa + C::kABytes;
+                if (warp == 0) {
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&full[stage], (uint32_t)C::kBBytes);
+                        tma_load_2d(sb, &tm_h, kt * kR, 0, &full[stage], pol_h);
+                    }
+                    __syncwarp();
+                }
+#pragma unroll
+                for (int j = 0; j < kQuads; ++j) {
+                    const int t = (kR / 4) * warp + 4 * j + rsub, kb = t >> 3, kr = t & 7;
+                    const T *src = col_src + (size_t)ids[j] * d;
+                    unsigned char *dst = sa + kb * 2048 + kr * 128 + ((cc ^ kr) << 4);
+#pragma unroll
+                    for (int pc = 0; pc < 2 * kHalves; ++pc)     // accumulator pc/2, 64-column block pc%2
+                        cp_async16(dst + ((pc >> 1) * (kR / 8) * 2 + (pc & 1)) * 1024,
+                                   src + pc * 64, pol_w);
+                }
+                cp_async_arrive_noinc(&full[stage]);
+                last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+                used |= 1u << stage;
+                if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+            }
+            u = (long long)(cb + 1) * KT;
+        }
+        // no copy may be in flight when the block exits
+        cp_async_wait_all();
+        if (warp == 0 && lane == 0)
+            for (int s = 0; s < C::kStages; ++s)
+                if (used & (1u << s)) mbar_wait(&full[s], (last_parity >> s) & 1u);
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) {
+            constexpr uint32_t idesc =
+                umma_idesc_f16(!std::is_same<T, __half>::value, kM, BP, /*a_mn=*/true);
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true;
+            for (long long u = u0; u < u1 && ok;) {
+                const int cb = (int)(u / KT);
+                const int kt0 = (int)(u - (long long)cb * KT);
+                const int kt1 = (int)min((long long)KT, u1 - (long long)cb * KT);
+                if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1)) {
+                    atomicOr(&g_sha_status, kStatusTimeout);
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t dt = tmem + (uint32_t)(acc * kHalves * BP);
+                for (int kt = kt0; kt < kt1; ++kt) {
+                    if (!mbar_wait(&full[stage], phase)) {
+                        atomicOr(&g_sha_status, kStatusTimeout);
+                        ok = false;
+                        break;
+                    }
+                    fence_proxy_async_shared();    // copied rows -> tensor-core reads
+                    tc_fence_after_sync();
+                    const uint32_t sa = smem_addr(smem + stage * C::kStage);
+                    const uint32_t sb = sa + C::kABytes;
+#pragma unroll
+                    for (int ks = 0; ks < kR / 16; ++ks) {
+                        const uint64_t bdesc = kR == 64 ? umma_desc_k_sw128(sb + ks * 32)
+                                                        : umma_desc_k_sw64(sb + ks * 32);
+#pragma unroll
+                        for (int h = 0; h < kHalves; ++h)
+                            umma_f16(dt + (uint32_t)(h * BP),
+                                     umma_desc_mn_sw128(sa + (h * (kR / 8) + 2 * ks) * 2 * 1024, 1024,
+                                                        2048),
+                                     bdesc, idesc, (kt > kt0 || ks > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&empty[stage]);
+                    if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                umma_commit(&acc_full[acc]);
+                if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+                u = (long long)(cb + 1) * KT;
+            }
+            if (u1 > u0) {
+                umma_commit(mma_done);
+                if (!mbar_wait(mma_done, 0)) atomicOr(&g_sha_status, kStatusTimeout);
+            }
+        }
+        __syncwarp();
+    } else {
+        // epilogue: warp w reads TMEM lanes 32*(w%4)..+31 = output columns of each half
+        const int quarter = warp & 3, row = quarter * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (long long u = u0; u < u1;) {
+            const int cb = (int)(u / KT);
+            const int kt0 = (int)(u - (long long)cb * KT);
+            const int kt1 = (int)min((long long)KT, u1 - (long long)cb * KT);
+            const bool live = __all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_phase));
+            if (!live) {
+                if (lane == 0) atomicOr(&g_sha_status, kStatusTimeout);
+                break;
+            }
+            tc_fence_after_sync();
+            const bool whole = kt0 == 0 && kt1 == KT;
+            const int slot = cb == cb_first ? 0 : 1;
+#pragma unroll 1
+            for (int h = 0; h < kHalves; ++h) {
+                float v[BP / 16][16];
+#pragma unroll
+                for (int c = 0; c < BP / 16; ++c)
+                    tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) +
+                                  (uint32_t)(acc * kHalves * BP + h * BP + c * 16),
+                              v[c]);
+                tmem_ld_wait();
+                const int col = h * kM + row;             // within the item
+                if (whole) {
+                    T *dst = y + (size_t)cb * kCols + col;
+#pragma unroll
+                    for (int b = 0; b < BP; ++b)
+                        if (b < B) dst[(size_t)b * d] = Elem<T>::from_float(v[b / 16][b % 16]);
+                } else {
+                    float *dst = part + (size_t)(blockIdx.x * 2 + slot) * BP * kCols + col;
+#pragma unroll
+                    for (int b = 0; b < BP; ++b) dst[(size_t)b * kCols] = v[b / 16][b % 16];
+                }
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+            if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+            u = (long long)(cb + 1) * KT;
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+// y entries of the column blocks mlp_down_tc split across blocks: the blocks'
+// partial sums added in block order; all of y when the union is empty.  Block
+// (cb, j) covers batch rows 8j..8j+7 of column block cb, one thread per column.
+constexpr int kOutRows = 8;
+
+template <typename T, int BP, int kCols>
+__global__ void __launch_bounds__(kCols)
+    mlp_out_tc_kernel(const float *__restrict__ part, const int32_t *__restrict__ n_S_ptr, int B,
+                      int d, int D, int down_blocks, T *__restrict__ y)
+{
+    using namespace downtc;
+    __shared__ int s_blk[kMaxContributors], s_slot[kMaxContributors], s_n;
+    pdl_wait();
+    pdl_launch_dependents();
+    const int cb = blockIdx.x, c = cb * kCols + threadIdx.x;
+    const int b0 = blockIdx.y * kOutRows, b1 = min(B, b0 + kOutRows);
+    const int n_S = union_size(n_S_ptr, D);
+    const int KT = (n_S + uptc::kM - 1) / uptc::kM * (uptc::kM / kR);
+    if (KT == 0) {
+        for (int b = b0; b < b1; ++b) y[(size_t)b * d + c] = Elem<T>::from_float(0.f);
+        return;
+    }
+    if (threadIdx.x == 0) {
+        const UnitSplit split{(long long)(d / kCols) * KT, down_blocks};
+        const bool whole =
+            split.owner((long long)cb * KT) == split.owner((long long)(cb + 1) * KT - 1);
+        s_n = whole ? 0 : split_contributors(split, cb, KT, s_blk, s_slot, kMaxContributors);
+    }
+    __syncthreads();
+    const int n = s_n;
+    if (n == 0) return;                         // written by the down-projection
+    for (int b = b0; b < b1; ++b) {
+        float v = 0.f;
+        for (int k = 0; k < n; ++k)
+            v += part[((size_t)(s_blk[k] * 2 + s_slot[k]) * BP + b) * kCols + threadIdx.x];
+        y[(size_t)b * d + c] = Elem<T>::from_float(v);
+    }
 }
 
 // ---------------------------------------------------------------- down-projection
@@ -1007,10 +1367,11 @@ PFN_cuTensorMapEncodeTiled_v12000 mlp_tensor_map_encoder()
     return fn;
 }
 
-// 2-D view [rows][d] of a row-major fp16/bf16 matrix, boxes of 64 elements x
-// box_rows rows with 128-byte swizzle; rows past the end read as zero.
+// 2-D view [rows][d] of a row-major fp16/bf16 matrix, boxes of box_cols (64
+// or 32) elements x box_rows rows with 128- (or 64-) byte swizzle; rows past
+// the end read as zero.
 sha_status_t mlp_tensor_map(CUtensorMap *map, const void *base, bool bf16, int d, int rows,
-                            int box_rows)
+                            int box_rows, int box_cols = uptc::kAtomK)
 {
     PFN_cuTensorMapEncodeTiled_v12000 encode = mlp_tensor_map_encoder();
     if (!encode) {
@@ -1020,11 +1381,12 @@ sha_status_t mlp_tensor_map(CUtensorMap *map, const void *base, bool bf16, int d
     }
     cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    cuuint32_t box[2] = {(cuuint32_t)uptc::kAtomK, (cuuint32_t)box_rows};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
     cuuint32_t elem[2] = {1, 1};
     CUresult r = encode(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
                         2, const_cast<void *>(base), dims, strides, box, elem,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         std::snprintf(g_mlp_error, sizeof g_mlp_error,
@@ -1039,6 +1401,7 @@ struct MlpPlan {
     int bp;                // batch padded to 16, 32 or 64
     int h_rows;            // rows of the neuron-major activations (union padded)
     bool tc_up;            // up-projection on tcgen05 (batches above 8)
+    bool tc;               // down-projection on tcgen05 as well
     int down_splits, down_blocks;
     size_t up_bytes, h_bytes, down_bytes;
     size_t total() const { return up_bytes + h_bytes + down_bytes; }
@@ -1054,7 +1417,8 @@ MlpPlan mlp_plan(int B, int d, int D, int sms)
                                 : (pl.bp == 16 ? DownCfg<16>::kWMax
                                                : (pl.bp == 32 ? DownCfg<32>::kWMax : DownCfg<64>::kWMax));
     pl.h_rows = (int)round_up((size_t)D, (size_t)uptc::kM);   // whole neuron groups
-    pl.tc_up = pl.bp >= 16 && SHA_MLP_TC_UP;
+    pl.tc_up = pl.bp >= 16 && SHA_MLP_TC && sms <= kMaxContributors;
+    pl.tc = pl.tc_up && pl.bp >= SHA_MLP_TC_DOWN_MIN_BATCH;
     if (pl.tc_up) {
         // two partial slots of 128 x BP per block
         pl.up_bytes = round_up((size_t)sms * 2 * uptc::kM * pl.bp * 4, 256);
@@ -1070,6 +1434,8 @@ MlpPlan mlp_plan(int B, int d, int D, int sms)
     const int items = wchunks * pl.down_splits;
     pl.down_blocks = items < sms ? items : sms;
     pl.down_bytes = round_up((size_t)pl.down_splits * kMlpMaxBatch * d * 4, 256);
+    if (pl.tc)   // two partial slots of BP x (up to 512) columns per block
+        pl.down_bytes = round_up((size_t)sms * 2 * pl.bp * 512 * 4, 256);
     return pl;
 }
 
@@ -1083,11 +1449,24 @@ sha_status_t run_mlp_bp(const void *x, const void *W1t, const void *W2t, const i
         cudaError_t e = cudaFuncSetAttribute(mlp_up_kernel<T, BP>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              UpCfg<BP>::kSmemBytes);
-        if constexpr (BP >= 16)
+        if constexpr (BP >= 16) {
             if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(mlp_up_tc_kernel<T, BP>,
+                e = cudaFuncSetAttribute(mlp_up_tc_kernel<T, BP, true>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          UpTcCfg<BP>::kSmemBytes);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(mlp_up_tc_kernel<T, BP, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         UpTcCfg<BP>::kSmemBytes);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(mlp_down_tc_kernel<T, BP, 2>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         DownTcCfg<BP, 2>::kSmemBytes);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(mlp_down_tc_kernel<T, BP, 4>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         DownTcCfg<BP, 4>::kSmemBytes);
+        }
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(mlp_down_kernel<T, BP>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1102,24 +1481,62 @@ sha_status_t run_mlp_bp(const void *x, const void *W1t, const void *W2t, const i
     float *down_part = reinterpret_cast<float *>(w + pl.up_bytes + pl.h_bytes);
 
     const size_t hn = (size_t)pl.h_rows * BP;
+    const size_t n = (size_t)B * d;
     cudaError_t e;
+    bool up_done = false;
     if constexpr (BP >= 16) {
         if (pl.tc_up) {
             constexpr bool bf16 = !std::is_same<T, __half>::value;
-            CUtensorMap tm_w, tm_x;
+            CUtensorMap tm_w, tm_x, tm_h;
             sha_status_t st = mlp_tensor_map(&tm_w, W1t, bf16, d, D, 1);
             if (st == SHA_OK) st = mlp_tensor_map(&tm_x, x, bf16, d, B, BP);
+            if (st == SHA_OK && pl.tc)
+                st = mlp_tensor_map(&tm_h, Ht, bf16, pl.h_rows, BP, BP, downtc::kR);
             if (st != SHA_OK) return st;
-            e = launch_pdl(mlp_up_tc_kernel<T, BP>, dim3(sms), uptc::kThreads,
+            const dim3 act_grid((unsigned)(pl.h_rows / uptc::kM), BP / 2);
+            if (pl.tc) {
+                e = launch_pdl(mlp_up_tc_kernel<T, BP, true>, dim3(sms), uptc::kThreads,
+                               UpTcCfg<BP>::kSmemBytes, s, tm_w, tm_x, static_cast<const T *>(W1t),
+                               S, n_S, B, d, D, act, pl.h_rows, up_part, Ht);
+                if (e != cudaSuccess) return mlp_launch_error(e);
+                e = launch_pdl(mlp_act_tc_kernel<T, BP, true>, act_grid, 2 * uptc::kM, 0, s,
+                               (const float *)up_part, n_S, B, d, D, sms, act, pl.h_rows, Ht);
+                if (e != cudaSuccess) return mlp_launch_error(e);
+                if (SHA_MLP_DOWN_TC_WIDE && d % 512 == 0) {
+                    e = launch_pdl(mlp_down_tc_kernel<T, BP, 4>, dim3(sms), downtc::kThreads,
+                                   DownTcCfg<BP, 4>::kSmemBytes, s, tm_h,
+                                   static_cast<const T *>(W2t), S, n_S, B, d, D, down_part,
+                                   static_cast<T *>(y));
+                    if (e != cudaSuccess) return mlp_launch_error(e);
+                    e = launch_pdl(mlp_out_tc_kernel<T, BP, 512>,
+                                   dim3((unsigned)(d / 512), (B + kOutRows - 1) / kOutRows), 512, 0,
+                                   s, (const float *)down_part, n_S, B, d, D, sms,
+                                   static_cast<T *>(y));
+                } else {
+                    e = launch_pdl(mlp_down_tc_kernel<T, BP, 2>, dim3(sms), downtc::kThreads,
+                                   DownTcCfg<BP, 2>::kSmemBytes, s, tm_h,
+                                   static_cast<const T *>(W2t), S, n_S, B, d, D, down_part,
+                                   static_cast<T *>(y));
+                    if (e != cudaSuccess) return mlp_launch_error(e);
+                    e = launch_pdl(mlp_out_tc_kernel<T, BP, 256>,
+                                   dim3((unsigned)(d / 256), (B + kOutRows - 1) / kOutRows), 256, 0,
+                                   s, (const float *)down_part, n_S, B, d, D, sms,
+                                   static_cast<T *>(y));
+                }
+                if (e != cudaSuccess) return mlp_launch_error(e);
+                return SHA_OK;
+            }
+            e = launch_pdl(mlp_up_tc_kernel<T, BP, false>, dim3(sms), uptc::kThreads,
                            UpTcCfg<BP>::kSmemBytes, s, tm_w, tm_x, static_cast<const T *>(W1t), S,
-                           n_S, B, d, D, act, up_part, Ht);
+                           n_S, B, d, D, act, pl.h_rows, up_part, Ht);
             if (e != cudaSuccess) return mlp_launch_error(e);
-            e = launch_pdl(mlp_act_tc_kernel<T, BP>, dim3((unsigned)((hn + 255) / 256)), 256, 0,
-                           s, (const float *)up_part, n_S, B, d, D, sms, act, Ht);
+            e = launch_pdl(mlp_act_tc_kernel<T, BP, false>, act_grid, 2 * uptc::kM, 0, s,
+                           (const float *)up_part, n_S, B, d, D, sms, act, pl.h_rows, Ht);
             if (e != cudaSuccess) return mlp_launch_error(e);
+            up_done = true;
         }
     }
-    if (!pl.tc_up) {
+    if (!up_done) {
         e = launch_pdl(mlp_up_kernel<T, BP>, dim3(sms), UpCfg<BP>::kThreads,
                        UpCfg<BP>::kSmemBytes, s, static_cast<const T *>(x),
                        static_cast<const T *>(W1t), S, n_S, B, d, D, up_part);
@@ -1132,7 +1549,6 @@ sha_status_t run_mlp_bp(const void *x, const void *W1t, const void *W2t, const i
                    DownCfg<BP>::kSmemBytes, s, (const T *)Ht, static_cast<const T *>(W2t), S, n_S,
                    B, d, D, pl.down_splits, down_part);
     if (e != cudaSuccess) return mlp_launch_error(e);
-    const size_t n = (size_t)B * d;
     e = launch_pdl(mlp_out_kernel<T>, dim3((unsigned)((n + 255) / 256)), 256, 0, s,
                    (const float *)down_part, B, d, pl.down_splits, static_cast<T *>(y));
     if (e != cudaSuccess) return mlp_launch_error(e);

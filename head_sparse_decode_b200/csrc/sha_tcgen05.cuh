@@ -73,13 +73,45 @@ __device__ __forceinline__ uint64_t umma_desc_k_sw128(uint32_t addr)
     return d;
 }
 
+// The same for a 64-byte swizzle: 64-byte rows (32 elements), 8-row groups
+// 512 bytes apart, layout type 4.
+__device__ __forceinline__ uint64_t umma_desc_k_sw64(uint32_t addr)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1u << 16;
+    d |= (uint64_t)(512u >> 4) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)4u << 61;
+    return d;
+}
+
+// Shared-memory matrix descriptor of an MN-major, 128-byte-swizzled operand:
+// 64-element MN blocks `lbo` bytes apart (leading byte offset), 8-row K groups
+// `sbo` bytes apart (stride byte offset); each 1024-byte atom holds 8 K rows of
+// 64 MN elements, chunks XOR-swizzled by the K row.
+__device__ __forceinline__ uint64_t umma_desc_mn_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)2u << 61;
+    return d;
+}
+
 // Instruction descriptor of kind::f16 with fp32 accumulation, both operands
-// K-major and of the same type (fp16, or bf16 when `bf16`), M x N.
-__host__ __device__ constexpr uint32_t umma_idesc_f16(bool bf16, int M, int N)
+// of the same type (fp16, or bf16 when `bf16`), M x N; A and B K-major unless
+// `a_mn` / `b_mn` (MN-major).
+__host__ __device__ constexpr uint32_t umma_idesc_f16(bool bf16, int M, int N, bool a_mn = false,
+                                                      bool b_mn = false)
 {
     return (1u << 4)                                  // accumulator format: f32
            | ((bf16 ? 1u : 0u) << 7)                  // A format
            | ((bf16 ? 1u : 0u) << 10)                 // B format
+           | ((a_mn ? 1u : 0u) << 15)                 // A major-ness
+           | ((b_mn ? 1u : 0u) << 16)                 // B major-ness
            | ((uint32_t)(N >> 3) << 17)               // N / 8
            | ((uint32_t)(M >> 4) << 24);              // M / 16
 }

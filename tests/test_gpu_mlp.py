@@ -68,8 +68,9 @@ def test_selective_mlp_identity_activation(sha):
     assert err <= TOLERANCE["bf16"], err
 
 
-def test_empty_union_gives_zero(sha):
-    w = CASES[0]
+@pytest.mark.parametrize("case", [0, 6], ids=["batch1", "batch32"])
+def test_empty_union_gives_zero(sha, case):
+    w = CASES[case]
     x, W1t, W2t, _ = workloads.make_mlp(w)
     dev = torch.device("cuda")
     S = torch.zeros(w.D, dtype=torch.int32, device=dev)
@@ -79,8 +80,9 @@ def test_empty_union_gives_zero(sha):
     assert (y == 0).all()
 
 
-def test_out_of_range_ids_are_flagged_not_read(sha):
-    w = CASES[0]
+@pytest.mark.parametrize("case", [0, 6], ids=["batch1", "batch32"])
+def test_out_of_range_ids_are_flagged_not_read(sha, case):
+    w = CASES[case]
     x, W1t, W2t, _ = workloads.make_mlp(w)
     dev = torch.device("cuda")
     S = torch.tensor([3, 10**6, 7], dtype=torch.int32, device=dev)
@@ -107,13 +109,16 @@ def test_opt66b_mlp_shape_sampled(sha):
     assert err <= TOLERANCE[w.dtype], err
 
 
-@pytest.mark.parametrize("B,density", [(64, 1.0), (50, 0.3), (32, 0.05), (16, 0.5), (9, 0.2)])
-def test_opt66b_mlp_large_batch_sampled(sha, B, density):
+@pytest.mark.parametrize("B,density,dtype", [(64, 1.0, "fp16"), (50, 0.3, "fp16"),
+                                             (32, 0.05, "fp16"), (16, 0.5, "fp16"),
+                                             (9, 0.2, "fp16"), (40, 0.3, "bf16")])
+def test_opt66b_mlp_large_batch_sampled(sha, B, density, dtype):
     """Batches above 8 (tensor-memory up-projection) at the OPT-66B shape: a dense
     union leaves some neuron groups whole inside one block and splits others
     across blocks; sparse unions split every group.  Sampled batch rows and
     output columns against the oracle (which takes the same union S)."""
-    w = workloads.MLP_CONFIGS["opt66b_mlp"].with_(B=B, density=density, seed=5100 + B)
+    w = workloads.MLP_CONFIGS["opt66b_mlp"].with_(B=B, density=density, dtype=dtype,
+                                                  seed=5100 + B)
     dev = torch.device("cuda")
     x, W1t, W2t, active = workloads.make_mlp(w, device=dev)
     S, n_S = sha.sha_mlp_union(active)
