@@ -462,11 +462,6 @@ struct UnitSplit {
     long long U;
     int NB;
     __device__ __forceinline__ long long begin(int b) const { return U * b / NB; }
-    // the block whose range holds unit u
-    __device__ __forceinline__ int owner(long long u) const
-    {
-        return (int)(((u + 1) * NB + U - 1) / U - 1);
-    }
 };
 
 __device__ __forceinline__ uint64_t l2_policy_evict_last()
@@ -725,22 +720,39 @@ __global__ void __launch_bounds__(uptc::kThreads, 1)
     }
 }
 
-// Blocks whose unit ranges hold part of unit range [a, e) of a split, and
-// the partial slot each left for it (0 if it is the block's first item, else
-// 1), in block order; returns how many.
-__device__ __forceinline__ int split_contributors(const UnitSplit &split, int item, int per_item,
-                                                  int *blk, int *slot, int max_n)
-{
-    const int bf = split.owner((long long)item * per_item);
-    const int bl = split.owner((long long)(item + 1) * per_item - 1);
-    int n = 0;
-    for (int b = bf; b <= bl && n < max_n; ++b) {
-        const long long a = split.begin(b);
-        if (a == split.begin(b + 1)) continue;  // a block with no units
-        blk[n] = b;
-        slot[n] = item == (int)(a / per_item) ? 0 : 1;
-        ++n;
+// The split as the fix-up kernels compute it: 32-bit arithmetic (the host
+// keeps U * NB below 2^32), so the per-block setup stays cheap.
+struct UnitSplit32 {
+    uint32_t U, NB;
+    __device__ __forceinline__ uint32_t begin(uint32_t b) const { return U * b / NB; }
+    __device__ __forceinline__ uint32_t owner(uint32_t u) const
+    {
+        return ((u + 1) * NB + U - 1) / U - 1;
     }
+};
+
+// Fills, for item `item` (units item*per_item .. +per_item) of a split, the
+// blocks that hold part of it in block order -- blk[k] = bf + k, slot[k] = 0
+// if the item is that block's first, 1 if not, -1 for a block with no units
+// -- one entry per thread of the calling block, and returns how many (0 when
+// one block holds the whole item).  Ends with a block barrier.
+__device__ __forceinline__ int split_contributors(const UnitSplit32 &split, uint32_t item,
+                                                  uint32_t per_item, int *slot, int *s_bf,
+                                                  int *s_n)
+{
+    if (threadIdx.x == 0) {
+        const uint32_t bf = split.owner(item * per_item);
+        const uint32_t bl = split.owner((item + 1) * per_item - 1);
+        *s_bf = (int)bf;
+        *s_n = bf == bl ? 0 : (int)(bl - bf + 1);
+    }
+    __syncthreads();
+    const int n = *s_n;
+    for (int k = threadIdx.x; k < n; k += blockDim.x) {
+        const uint32_t b = (uint32_t)(*s_bf + k), a = split.begin(b);
+        slot[k] = a == split.begin(b + 1) ? -1 : (item == a / per_item ? 0 : 1);
+    }
+    __syncthreads();
     return n;
 }
 
@@ -748,35 +760,36 @@ constexpr int kMaxContributors = 256;     // >= the blocks of a split (one per S
 
 // Ht entries (layout as in mlp_up_tc) of the groups mlp_up_tc split across
 // blocks: the blocks' partial sums added in block order, then sigma; zero
-// outside the union and batch.  Block (g, j) covers columns 2j, 2j+1 of
-// group g, one thread per (column, neuron).
+// outside the union and batch.  Block (g, j) covers columns kActCols*j ..
+// +kActCols of group g, two columns at a time, one thread per (column, neuron).
+constexpr int kActCols = 8;
+
 template <typename T, int BP, bool kBatchMajor>
 __global__ void __launch_bounds__(2 * uptc::kM)
     mlp_act_tc_kernel(const float *__restrict__ part, const int32_t *__restrict__ n_S_ptr, int B,
                       int d, int D, int up_blocks, int act, int h_rows, T *__restrict__ Ht)
 {
     using namespace uptc;
-    __shared__ int s_blk[kMaxContributors], s_slot[kMaxContributors], s_n;
+    __shared__ int s_slot[kMaxContributors], s_bf, s_n;
     pdl_wait();
     pdl_launch_dependents();
     const int n_S = union_size(n_S_ptr, D);
     const int KT = d / kStageK, G = (n_S + kM - 1) / kM, g = blockIdx.x;
     if (g >= G) return;
-    if (threadIdx.x == 0) {
-        const UnitSplit split{(long long)G * KT, up_blocks};
-        const bool whole = split.owner((long long)g * KT) == split.owner((long long)(g + 1) * KT - 1);
-        s_n = whole ? 0 : split_contributors(split, g, KT, s_blk, s_slot, kMaxContributors);
-    }
-    __syncthreads();
-    const int n = s_n;
+    const UnitSplit32 split{(uint32_t)(G * KT), (uint32_t)up_blocks};
+    const int n = split_contributors(split, (uint32_t)g, (uint32_t)KT, s_slot, &s_bf, &s_n);
     if (n == 0) return;                         // finished by the up-projection
-    const int col = 2 * blockIdx.y + threadIdx.x / kM, row = threadIdx.x % kM, t = g * kM + row;
-    float v = 0.f;
-    for (int k = 0; k < n; ++k)
-        v += part[((size_t)(s_blk[k] * 2 + s_slot[k]) * BP + col) * kM + row];
-    if (act == 1) v = fmaxf(v, 0.f);
-    Ht[kBatchMajor ? (size_t)col * h_rows + t : (size_t)t * BP + col] =
-        Elem<T>::from_float((t < n_S && col < B) ? v : 0.f);
+    const int row = threadIdx.x % kM, t = g * kM + row;
+    for (int col = blockIdx.y * kActCols + threadIdx.x / kM; col < (int)(blockIdx.y + 1) * kActCols;
+         col += blockDim.x / kM) {
+        float v = 0.f;
+        for (int k = 0; k < n; ++k)
+            if (s_slot[k] >= 0)
+                v += part[((size_t)((s_bf + k) * 2 + s_slot[k]) * BP + col) * kM + row];
+        if (act == 1) v = fmaxf(v, 0.f);
+        Ht[kBatchMajor ? (size_t)col * h_rows + t : (size_t)t * BP + col] =
+            Elem<T>::from_float((t < n_S && col < B) ? v : 0.f);
+    }
 }
 
 // ---------------------------------------------------------------- down-projection on tcgen05
@@ -1071,7 +1084,7 @@ __global__ void __launch_bounds__(kCols)
                       int d, int D, int down_blocks, T *__restrict__ y)
 {
     using namespace downtc;
-    __shared__ int s_blk[kMaxContributors], s_slot[kMaxContributors], s_n;
+    __shared__ int s_slot[kMaxContributors], s_bf, s_n;
     pdl_wait();
     pdl_launch_dependents();
     const int cb = blockIdx.x, c = cb * kCols + threadIdx.x;
@@ -1082,19 +1095,14 @@ __global__ void __launch_bounds__(kCols)
         for (int b = b0; b < b1; ++b) y[(size_t)b * d + c] = Elem<T>::from_float(0.f);
         return;
     }
-    if (threadIdx.x == 0) {
-        const UnitSplit split{(long long)(d / kCols) * KT, down_blocks};
-        const bool whole =
-            split.owner((long long)cb * KT) == split.owner((long long)(cb + 1) * KT - 1);
-        s_n = whole ? 0 : split_contributors(split, cb, KT, s_blk, s_slot, kMaxContributors);
-    }
-    __syncthreads();
-    const int n = s_n;
+    const UnitSplit32 split{(uint32_t)((d / kCols) * KT), (uint32_t)down_blocks};
+    const int n = split_contributors(split, (uint32_t)cb, (uint32_t)KT, s_slot, &s_bf, &s_n);
     if (n == 0) return;                         // written by the down-projection
     for (int b = b0; b < b1; ++b) {
         float v = 0.f;
         for (int k = 0; k < n; ++k)
-            v += part[((size_t)(s_blk[k] * 2 + s_slot[k]) * BP + b) * kCols + threadIdx.x];
+            if (s_slot[k] >= 0)
+                v += part[((size_t)((s_bf + k) * 2 + s_slot[k]) * BP + b) * kCols + threadIdx.x];
         y[(size_t)b * d + c] = Elem<T>::from_float(v);
     }
 }
@@ -1417,7 +1425,10 @@ MlpPlan mlp_plan(int B, int d, int D, int sms)
                                 : (pl.bp == 16 ? DownCfg<16>::kWMax
                                                : (pl.bp == 32 ? DownCfg<32>::kWMax : DownCfg<64>::kWMax));
     pl.h_rows = (int)round_up((size_t)D, (size_t)uptc::kM);   // whole neuron groups
-    pl.tc_up = pl.bp >= 16 && SHA_MLP_TC && sms <= kMaxContributors;
+    // split sizes the fix-up kernels compute in 32 bits: U * NB < 2^32
+    const size_t max_units = ((size_t)D + uptc::kM - 1) / uptc::kM * ((size_t)d / 128);
+    pl.tc_up = pl.bp >= 16 && SHA_MLP_TC && sms <= kMaxContributors &&
+               max_units * (size_t)(sms + 1) < (1ull << 32);
     pl.tc = pl.tc_up && pl.bp >= SHA_MLP_TC_DOWN_MIN_BATCH;
     if (pl.tc_up) {
         // two partial slots of 128 x BP per block
@@ -1493,7 +1504,7 @@ sha_status_t run_mlp_bp(const void *x, const void *W1t, const void *W2t, const i
             if (st == SHA_OK && pl.tc)
                 st = mlp_tensor_map(&tm_h, Ht, bf16, pl.h_rows, BP, BP, downtc::kR);
             if (st != SHA_OK) return st;
-            const dim3 act_grid((unsigned)(pl.h_rows / uptc::kM), BP / 2);
+            const dim3 act_grid((unsigned)(pl.h_rows / uptc::kM), BP / kActCols);
             if (pl.tc) {
                 e = launch_pdl(mlp_up_tc_kernel<T, BP, true>, dim3(sms), uptc::kThreads,
                                UpTcCfg<BP>::kSmemBytes, s, tm_w, tm_x, static_cast<const T *>(W1t),
