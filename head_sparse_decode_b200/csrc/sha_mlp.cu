@@ -13,20 +13,30 @@
 //
 // Kernels (each launched with programmatic stream serialization):
 //   mlp_union_flags / mlp_union_write -- S_B as sorted neuron ids + n_S
+// Batches up to 8 (and the down-projection of batches up to 16), on
+// warp-level tensor-core MMAs (mma.sync m16n8k16, fp32 accumulate):
 //   mlp_up    -- partial x . W1t[S]^T (fp32): M = 16 gathered neurons, N =
-//                batch, K = d streamed in 2 KiB row segments
+//                batch, K = d streamed in long row segments
 //   mlp_act   -- Ht = sigma(sum of the partials), rounded to the input dtype,
 //                neuron-major
 //   mlp_down  -- partial Ht^T . W2t[S] over a range of neurons (fp32): M =
 //                batch, N = up to 1024 output columns, K = neurons
 //   mlp_out   -- y = sum of the partials, in a fixed order
-// The GEMMs stream weight-row segments with 1-D bulk copies (one per row)
-// into shared-memory rows padded by 16 bytes, so ldmatrix reads are free of
-// bank conflicts, and run on the tensor cores (mma.sync m16n8k16, fp32
-// accumulate).  Segments are long (2 KiB for batches up to 16) so DRAM sees
-// contiguous runs of each selected row.
-// They are bound by HBM: every selected weight byte is read once, and the
-// arithmetic intensity is about B flops per weight byte.
+// These stream weight-row segments with 1-D bulk copies (one per row and
+// stage, up to 4.5 KiB) into shared-memory rows padded by 16 bytes, so
+// ldmatrix reads are free of bank conflicts.
+// Batches of 9 to 64, on tcgen05 with fp32 accumulators in tensor memory:
+//   mlp_up_tc   -- D[128 neurons x batch] = W1t[S] . x^T, stream-K over
+//                  (neuron group, K tile); whole groups write Ht directly
+//   mlp_act_tc  -- Ht of the groups split across blocks
+//   mlp_down_tc -- D[128 output columns x batch] = W2t[S]^T . Ht^T (from batch
+//                  32), stream-K over (512-column block, 64-neuron tile)
+//   mlp_out_tc  -- y of the column blocks split across blocks
+// Their gathered weight rows are copied by 16-byte cp.async into 128-byte
+// swizzled operand tiles (a TMA gather moves too little per operation), the
+// dense operand (x, Ht) by one TMA box per stage.
+// All of them are bound by HBM: every selected weight byte is read once, and
+// the arithmetic intensity is about B flops per weight byte.
 #include <atomic>
 #include <cmath>
 #include <cstdio>
