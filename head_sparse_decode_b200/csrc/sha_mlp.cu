@@ -789,16 +789,26 @@ __global__ void __launch_bounds__(2 * uptc::kM)
     const UnitSplit32 split{(uint32_t)(G * KT), (uint32_t)up_blocks};
     const int n = split_contributors(split, (uint32_t)g, (uint32_t)KT, s_slot, &s_bf, &s_n);
     if (n == 0) return;                         // finished by the up-projection
+    // this thread: neuron `row`, columns col0, col0 + 2, ... (kActCols / 2 of
+    // them, summed side by side so their loads are in flight together)
+    constexpr int kPer = kActCols / 2;
     const int row = threadIdx.x % kM, t = g * kM + row;
-    for (int col = blockIdx.y * kActCols + threadIdx.x / kM; col < (int)(blockIdx.y + 1) * kActCols;
-         col += blockDim.x / kM) {
-        float v = 0.f;
-        for (int k = 0; k < n; ++k)
-            if (s_slot[k] >= 0)
-                v += part[((size_t)((s_bf + k) * 2 + s_slot[k]) * BP + col) * kM + row];
-        if (act == 1) v = fmaxf(v, 0.f);
+    const int col0 = blockIdx.y * kActCols + threadIdx.x / kM;
+    float v[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) v[j] = 0.f;
+    for (int k = 0; k < n; ++k) {
+        if (s_slot[k] < 0) continue;
+        const float *src = part + (size_t)((s_bf + k) * 2 + s_slot[k]) * BP * kM + row;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) v[j] += src[(size_t)(col0 + 2 * j) * kM];
+    }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        const int col = col0 + 2 * j;
+        const float x = act == 1 ? fmaxf(v[j], 0.f) : v[j];
         Ht[kBatchMajor ? (size_t)col * h_rows + t : (size_t)t * BP + col] =
-            Elem<T>::from_float((t < n_S && col < B) ? v : 0.f);
+            Elem<T>::from_float((t < n_S && col < B) ? x : 0.f);
     }
 }
 
@@ -1108,13 +1118,20 @@ __global__ void __launch_bounds__(kCols)
     const UnitSplit32 split{(uint32_t)((d / kCols) * KT), (uint32_t)down_blocks};
     const int n = split_contributors(split, (uint32_t)cb, (uint32_t)KT, s_slot, &s_bf, &s_n);
     if (n == 0) return;                         // written by the down-projection
-    for (int b = b0; b < b1; ++b) {
-        float v = 0.f;
-        for (int k = 0; k < n; ++k)
-            if (s_slot[k] >= 0)
-                v += part[((size_t)((s_bf + k) * 2 + s_slot[k]) * BP + b) * kCols + threadIdx.x];
-        y[(size_t)b * d + c] = Elem<T>::from_float(v);
+    // the block's batch rows summed side by side, so their loads are in flight together
+    float v[kOutRows];
+#pragma unroll
+    for (int r = 0; r < kOutRows; ++r) v[r] = 0.f;
+    for (int k = 0; k < n; ++k) {
+        if (s_slot[k] < 0) continue;
+        const float *src = part + ((size_t)((s_bf + k) * 2 + s_slot[k]) * BP + b0) * kCols + threadIdx.x;
+#pragma unroll
+        for (int r = 0; r < kOutRows; ++r)
+            if (b0 + r < b1) v[r] += src[(size_t)r * kCols];
     }
+#pragma unroll
+    for (int r = 0; r < kOutRows; ++r)
+        if (b0 + r < b1) y[(size_t)(b0 + r) * d + c] = Elem<T>::from_float(v[r]);
 }
 
 // ---------------------------------------------------------------- down-projection

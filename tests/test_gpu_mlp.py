@@ -63,9 +63,11 @@ def test_selective_mlp_parity(sha, w):
     assert err <= TOLERANCE[w.dtype], err
 
 
-def test_selective_mlp_identity_activation(sha):
-    err, _ = _run(sha, CASES[1].with_(seed=21), act="identity")
-    assert err <= TOLERANCE["bf16"], err
+@pytest.mark.parametrize("case", [1, 6, 2], ids=["batch8", "batch32", "batch64"])
+def test_selective_mlp_identity_activation(sha, case):
+    w = CASES[case].with_(seed=21)
+    err, _ = _run(sha, w, act="identity")
+    assert err <= TOLERANCE[w.dtype], err
 
 
 @pytest.mark.parametrize("case", [0, 6], ids=["batch1", "batch32"])
