@@ -866,6 +866,49 @@ struct DownTcCfg {
     static_assert(kSmemBytes <= 232448, "fits the shared-memory opt-in");
 };
 
+// Work of the down-projection's blocks.  With no more column blocks (CB) than
+// blocks (NB), each column block gets its own NB/CB or NB/CB + 1 blocks (the
+// first NB % CB column blocks one more), which split its K tiles evenly: a
+// block then leaves at most one partial slot.  Otherwise the units are split
+// evenly over the blocks (stream-K).  Returns block b's unit range [u0, u1),
+// a unit being (column block, tile) = cb * KT + tile.
+struct ColumnSplit {
+    int CB, KT, NB;
+    __host__ __device__ bool aligned() const { return CB <= NB; }
+    __host__ __device__ int blocks_of(int cb) const
+    {
+        return NB / CB + (cb < NB % CB ? 1 : 0);
+    }
+    __host__ __device__ int first_block(int cb) const
+    {
+        const int per = NB / CB, extra = NB % CB;
+        return cb * per + (cb < extra ? cb : extra);
+    }
+    __device__ void range(int b, long long &u0, long long &u1) const
+    {
+        if (!aligned()) {
+            const UnitSplit split{(long long)CB * KT, NB};
+            u0 = split.begin(b);
+            u1 = split.begin(b + 1);
+            return;
+        }
+        const int per = NB / CB, extra = NB % CB;
+        int cb, sp, nsp;
+        if (b < extra * (per + 1)) {
+            cb = b / (per + 1);
+            sp = b % (per + 1);
+            nsp = per + 1;
+        } else {
+            const int bb = b - extra * (per + 1);
+            cb = extra + bb / per;
+            sp = bb % per;
+            nsp = per;
+        }
+        u0 = (long long)cb * KT + (long long)sp * KT / nsp;
+        u1 = (long long)cb * KT + (long long)(sp + 1) * KT / nsp;
+    }
+};
+
 template <typename T, int BP, int kHalves>
 __global__ void __launch_bounds__(downtc::kThreads, 1)
     mlp_down_tc_kernel(const __grid_constant__ CUtensorMap tm_h, const T *__restrict__ W2t,
@@ -912,8 +955,8 @@ __global__ void __launch_bounds__(downtc::kThreads, 1)
 
     const int n_S = union_size(n_S_ptr, D);
     const int KT = (n_S + uptc::kM - 1) / uptc::kM * (uptc::kM / kR);   // tiles of the padded union
-    const UnitSplit split{(long long)(d / kCols) * KT, (int)gridDim.x};
-    const long long u0 = split.begin(blockIdx.x), u1 = split.begin(blockIdx.x + 1);
+    long long u0 = 0, u1 = 0;
+    if (KT > 0) ColumnSplit{d / kCols, KT, (int)gridDim.x}.range(blockIdx.x, u0, u1);
     const int cb_first = KT > 0 ? (int)(u0 / KT) : 0;
 
     if (warp < kProducerWarps) {
@@ -1115,8 +1158,23 @@ __global__ void __launch_bounds__(kCols)
         for (int b = b0; b < b1; ++b) y[(size_t)b * d + c] = Elem<T>::from_float(0.f);
         return;
     }
-    const UnitSplit32 split{(uint32_t)((d / kCols) * KT), (uint32_t)down_blocks};
-    const int n = split_contributors(split, (uint32_t)cb, (uint32_t)KT, s_slot, &s_bf, &s_n);
+    const ColumnSplit cs{d / kCols, KT, down_blocks};
+    int n;
+    if (cs.aligned()) {
+        // this column block's own blocks, one partial slot each (none for an
+        // empty K range).  An even split of KT tiles over nsp blocks leaves
+        // min(nsp, KT) of them non-empty; when that is one, its block covered
+        // the whole column block and wrote y itself.
+        const int nsp = cs.blocks_of(cb);
+        if (threadIdx.x == 0) s_bf = cs.first_block(cb);
+        for (int k = threadIdx.x; k < nsp; k += blockDim.x)
+            s_slot[k] = (long long)(k + 1) * KT / nsp > (long long)k * KT / nsp ? 0 : -1;
+        n = min(nsp, KT) == 1 ? 0 : nsp;
+        __syncthreads();
+    } else {
+        const UnitSplit32 split{(uint32_t)((d / kCols) * KT), (uint32_t)down_blocks};
+        n = split_contributors(split, (uint32_t)cb, (uint32_t)KT, s_slot, &s_bf, &s_n);
+    }
     if (n == 0) return;                         // written by the down-projection
     // the block's batch rows summed side by side, so their loads are in flight together
     float v[kOutRows];
