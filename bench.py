@@ -401,7 +401,7 @@ def density_sweep(sha, w, q, k, v, dev, stream, peak):
 def other_configs(sha, w_main, dev, stream, peak, rank):
     """The other full-size workloads, timed the same way (fewer steps)."""
     res = []
-    for name in ("llama2_7b", "llama31_70b_gqa"):
+    for name in ("llama2_7b", "llama31_70b_gqa", "llama2_7b_ctx16k", "llama31_70b_gqa_ctx16k"):
         if name == w_main.name:
             continue
         w = workloads.CONFIGS[name]

@@ -190,7 +190,7 @@ def test_rows_of_other_tensors_are_not_read(sha):
 
 # ---------------------------------------------------------------- full-size configs
 
-@pytest.mark.parametrize("name", ["opt66b", "opt66b_dense", "llama2_7b"])
+@pytest.mark.parametrize("name", ["opt66b", "opt66b_dense", "llama2_7b", "llama2_7b_ctx16k"])
 def test_full_size_config_sampled(sha, name):
     w = workloads.CONFIGS[name]
     q, k, v = workloads.make_qkv(w, device="cuda")
@@ -269,8 +269,9 @@ def test_gqa_out_of_range_group_ids(sha):
     check_against_oracle(w, q, k, v, idx, out)
 
 
-def test_gqa_full_size_config_sampled(sha):
-    w = workloads.CONFIGS["llama31_70b_gqa"]
+@pytest.mark.parametrize("name", ["llama31_70b_gqa", "llama31_70b_gqa_ctx16k"])
+def test_gqa_full_size_config_sampled(sha, name):
+    w = workloads.CONFIGS[name]
     q, k, v = workloads.make_qkv(w, device="cuda")
     idx = workloads.make_index(w).cuda()
     out = workloads.make_out(w, "cuda")
@@ -278,7 +279,7 @@ def test_gqa_full_size_config_sampled(sha):
     torch.cuda.synchronize()
     assert sha.sha_get_device_status() == sha.SHA_OK
     err, n = check_sampled_units(w, q, k, v, idx, out, n_random=48)
-    assert n >= 48
+    assert n >= min(48, w.units)
 
 
 # ---------------------------------------------------------------- scaling-sweep points

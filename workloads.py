@@ -86,6 +86,13 @@ CONFIGS = {
     # LLaMA-3.1-70B-shaped GQA decode: 5 of 8 KV groups, 8 query heads each
     "llama31_70b_gqa": Workload("llama31_70b_gqa", B=32, H_q=64, H_kv=8, N_kv=4096,
                                 d=128, top_k=5, dtype="bf16", index="perm", seed=3000),
+    # the longest context the pages evaluate (16K tokens), LLaMA-2-7B and
+    # LLaMA-3.1-70B shapes
+    "llama2_7b_ctx16k": Workload("llama2_7b_ctx16k", B=16, H_q=32, H_kv=32, N_kv=16384, d=128,
+                                 top_k=16, dtype="fp16", index="zipf", seed=2600),
+    "llama31_70b_gqa_ctx16k": Workload("llama31_70b_gqa_ctx16k", B=8, H_q=64, H_kv=8,
+                                       N_kv=16384, d=128, top_k=5, dtype="bf16", index="perm",
+                                       seed=3100),
 }
 
 
