@@ -418,10 +418,12 @@ __global__ void mlp_act_kernel(const float *__restrict__ part, const int32_t *__
 // is more than warp-level MMAs sustain at HBM speed, so the up-projection of
 // those batches runs on the fifth-generation tensor cores:
 //     D [128 neurons x BP] (fp32, in TMEM) = W1t[S rows] . x^T
-// A = 128 gathered weight rows (TMA four-row gathers) and B = the batch's x
-// rows (one TMA box), both K-major with 128-byte swizzle, four 64-element K
-// atoms (256 elements) per stage.  One thread issues the MMAs; four epilogue
-// warps read the accumulator (double-buffered in TMEM) back.
+// A = 128 gathered weight rows and B = the batch's x rows, both K-major with
+// 128-byte swizzle, four 64-element K atoms (256 elements) per stage.  Four
+// producer warps copy the rows with 16-byte cp.async (a TMA four-row gather
+// moves at most 512 bytes per operation, too little to keep HBM busy); x is
+// one TMA box per atom.  One thread issues the MMAs; four epilogue warps read
+// the accumulator (double-buffered in TMEM) back.
 //
 // Work units are (group of 128 neurons, 256-element K tile); block b takes the
 // contiguous unit range [b U / NB, (b+1) U / NB) (stream-K), so every block
@@ -431,19 +433,12 @@ __global__ void mlp_act_kernel(const float *__restrict__ part, const int32_t *__
 // sums in slot 0 (the block's first group) or slot 1 (its last group) of the
 // block, and mlp_act_tc adds them up in block order.
 
-// How the gathered weight rows reach shared memory: 0 = TMA four-row gathers
-// issued by one producer warp; 1 = 16-byte cp.async copies from four producer
-// warps (the TMA unit then only loads x).
-#ifndef SHA_MLP_TC_FEED
-#define SHA_MLP_TC_FEED 1
-#endif
-
 namespace uptc {
 constexpr int kM = 128;                    // neurons per group (MMA M)
 constexpr int kAtomK = 64;                 // elements per 128-byte swizzled row
 constexpr int kAtoms = 4;                  // K atoms per stage
 constexpr int kStageK = kAtoms * kAtomK;   // elements of K per stage
-constexpr int kProducerWarps = SHA_MLP_TC_FEED ? 4 : 1;
+constexpr int kProducerWarps = 4;        // cp.async copies of the gathered rows
 constexpr int kMmaWarp = kProducerWarps;   // then four epilogue warps
 constexpr int kThreads = (kProducerWarps + 5) * 32;
 }  // namespace uptc
@@ -485,7 +480,7 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last()
 // operand); otherwise [h_rows][BP] (the warp-level down-projection's).
 template <typename T, int BP, bool kBatchMajor>
 __global__ void __launch_bounds__(uptc::kThreads, 1)
-    mlp_up_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+    mlp_up_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                      const T *__restrict__ W1t, const int32_t *__restrict__ S,
                      const int32_t *__restrict__ n_S_ptr, int B, int d, int D, int act, int h_rows,
                      float *__restrict__ part, T *__restrict__ Ht)
@@ -505,7 +500,7 @@ __global__ void __launch_bounds__(uptc::kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
             // the x box's expect-tx arrival, plus one cp.async arrival per producer thread
-            mbar_init(&full[s], SHA_MLP_TC_FEED ? 1 + 32 * kProducerWarps : 1);
+            mbar_init(&full[s], 1 + 32 * kProducerWarps);
             mbar_init(&empty[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
@@ -542,7 +537,6 @@ __global__ void __launch_bounds__(uptc::kThreads, 1)
             const int g = (int)(u / KT);
             const int kt0 = (int)(u - (long long)g * KT);
             const int kt1 = (int)min((long long)KT, u1 - (long long)g * KT);
-#if SHA_MLP_TC_FEED
             // warp p copies rows 32p..32p+31: copy i of a k atom moves 128 bytes of
             // rows 32p+4i .. +3 (eight lanes per row, one 16-byte chunk each) to
             // their swizzled places (ids past the union repeat its last neuron;
@@ -556,13 +550,6 @@ __global__ void __launch_bounds__(uptc::kThreads, 1)
                 const int id = neuron_id(S, min(g * kM + row[i], n_S - 1), D);
                 src[i] = W1t + (size_t)id * d + chunk * 8;
             }
-#else
-            // lane q gathers rows 4q..4q+3 of the group (ids past the union
-            // repeat its last neuron; their rows are computed and dropped)
-            int id[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) id[i] = neuron_id(S, min(g * kM + 4 * lane + i, n_S - 1), D);
-#endif
             for (int kt = kt0; kt < kt1; ++kt) {
                 bool go = true;
                 if (lane == 0 && !mbar_wait(&empty[stage], phase ^ 1)) {
@@ -575,15 +562,12 @@ __global__ void __launch_bounds__(uptc::kThreads, 1)
                 unsigned char *sb = sa + C::kABytes;
                 const int k0 = kt * kStageK;
                 if (warp == 0) {
-                    if (lane == 0)
-                        mbar_arrive_expect_tx(&full[stage],
-                                              (uint32_t)(SHA_MLP_TC_FEED ? C::kBBytes : C::kStage));
+                    if (lane == 0) mbar_arrive_expect_tx(&full[stage], (uint32_t)C::kBBytes);
                     __syncwarp();
                     if (lane < kAtoms)
                         tma_load_2d(sb + lane * C::kBAtom, &tm_x, k0 + lane * kAtomK, 0,
                                     &full[stage], pol_x);
                 }
-#if SHA_MLP_TC_FEED
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
 #pragma unroll
@@ -591,12 +575,6 @@ __global__ void __launch_bounds__(uptc::kThreads, 1)
                         cp_async16(sa + j * C::kAAtom + row[i] * 128 + ((chunk ^ (row[i] & 7)) << 4),
                                    src[i] + k0 + j * kAtomK, pol_w);
                 cp_async_arrive_noinc(&full[stage]);
-#else
-#pragma unroll
-                for (int j = 0; j < kAtoms; ++j)
-                    tma_gather4(sa + j * C::kAAtom + lane * 512, &tm_w, k0 + j * kAtomK, id[0],
-                                id[1], id[2], id[3], &full[stage], pol_w);
-#endif
                 last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
                 used |= 1u << stage;
                 if (++stage == C::kStages) { stage = 0; phase ^= 1; }
@@ -604,17 +582,14 @@ __global__ void __launch_bounds__(uptc::kThreads, 1)
             u = (long long)(g + 1) * KT;
         }
         // no copy may be in flight when the block exits
-#if SHA_MLP_TC_FEED
         cp_async_wait_all();
-#endif
         if (warp == 0 && lane == 0)
             for (int s = 0; s < C::kStages; ++s)
                 if (used & (1u << s)) mbar_wait(&full[s], (last_parity >> s) & 1u);
         __syncwarp();
     } else if (warp == kMmaWarp) {
         if (lane == 0) {
-            constexpr uint32_t idesc = umma_idesc_f16(sizeof(T) == 2 && !std::is_same<T, __half>::value,
-                                                      kM, BP);
+            constexpr uint32_t idesc = umma_idesc_f16(!std::is_same<T, __half>::value, kM, BP);
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
@@ -1583,16 +1558,15 @@ sha_status_t run_mlp_bp(const void *x, const void *W1t, const void *W2t, const i
     if constexpr (BP >= 16) {
         if (pl.tc_up) {
             constexpr bool bf16 = !std::is_same<T, __half>::value;
-            CUtensorMap tm_w, tm_x, tm_h;
-            sha_status_t st = mlp_tensor_map(&tm_w, W1t, bf16, d, D, 1);
-            if (st == SHA_OK) st = mlp_tensor_map(&tm_x, x, bf16, d, B, BP);
+            CUtensorMap tm_x, tm_h;
+            sha_status_t st = mlp_tensor_map(&tm_x, x, bf16, d, B, BP);
             if (st == SHA_OK && pl.tc)
                 st = mlp_tensor_map(&tm_h, Ht, bf16, pl.h_rows, BP, BP, downtc::kR);
             if (st != SHA_OK) return st;
             const dim3 act_grid((unsigned)(pl.h_rows / uptc::kM), BP / kActCols);
             if (pl.tc) {
                 e = launch_pdl(mlp_up_tc_kernel<T, BP, true>, dim3(sms), uptc::kThreads,
-                               UpTcCfg<BP>::kSmemBytes, s, tm_w, tm_x, static_cast<const T *>(W1t),
+                               UpTcCfg<BP>::kSmemBytes, s, tm_x, static_cast<const T *>(W1t),
                                S, n_S, B, d, D, act, pl.h_rows, up_part, Ht);
                 if (e != cudaSuccess) return mlp_launch_error(e);
                 e = launch_pdl(mlp_act_tc_kernel<T, BP, true>, act_grid, 2 * uptc::kM, 0, s,
@@ -1623,7 +1597,7 @@ sha_status_t run_mlp_bp(const void *x, const void *W1t, const void *W2t, const i
                 return SHA_OK;
             }
             e = launch_pdl(mlp_up_tc_kernel<T, BP, false>, dim3(sms), uptc::kThreads,
-                           UpTcCfg<BP>::kSmemBytes, s, tm_w, tm_x, static_cast<const T *>(W1t), S,
+                           UpTcCfg<BP>::kSmemBytes, s, tm_x, static_cast<const T *>(W1t), S,
                            n_S, B, d, D, act, pl.h_rows, up_part, Ht);
             if (e != cudaSuccess) return mlp_launch_error(e);
             e = launch_pdl(mlp_act_tc_kernel<T, BP, false>, act_grid, 2 * uptc::kM, 0, s,

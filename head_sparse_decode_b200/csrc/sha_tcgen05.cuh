@@ -2,7 +2,7 @@
 // tensor-memory (TMEM) allocation, shared-memory matrix descriptors for
 // 128-byte-swizzled K-major operands, the kind::f16 MMA with an fp32
 // accumulator in TMEM, commit-to-mbarrier, TMEM -> register loads, and the
-// TMA loads (tiled, and the four-row gather) that fill the operands.
+// copies that fill the operands (TMA tiled loads, 16-byte cp.async).
 //
 // Operand layout used throughout: a K-major tile of R rows x 64 elements
 // (128 bytes per row) is one "K atom"; 8-row groups of an atom are 1024
@@ -174,20 +174,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
         ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(policy)
-        : "memory");
-}
-
-// Four rows r0..r3 of a 2-D tensor map (box one row high), elements x .. x+box
-// of each, stored as four consecutive box rows at `dst`.
-__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, int x, int r0,
-                                            int r1, int r2, int r3, uint64_t *bar,
-                                            uint64_t policy)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(smem_addr(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
-        "r"(smem_addr(bar)), "l"(policy)
         : "memory");
 }
 
