@@ -86,7 +86,8 @@ struct Plan {
     size_t workspace_bytes() const { return counter_bytes + slot_bytes; }
 };
 
-constexpr int kBlocksPerSm = 1;
+// resident blocks per SM each kernel is planned for
+int blocks_per_sm(int G) { return G == 1 ? SHA_MHA_BLOCKS_PER_SM : 1; }
 
 // keys per tile of the kernel that serves G query heads per KV head
 int tile_keys(int G) { return G == 1 ? sha::MhaConfig<128>::kTile : sha::GqaConfig<128>::kTile; }
@@ -100,7 +101,7 @@ Plan make_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int num_spl
     const int tile = tile_keys(G);
     pl.sched.tiles_per_unit = (N_kv + tile - 1) / tile;
     pl.sched.total_tiles = units * pl.sched.tiles_per_unit;
-    long long ctas = num_splits > 0 ? num_splits : (long long)num_sms * kBlocksPerSm;
+    long long ctas = num_splits > 0 ? num_splits : (long long)num_sms * blocks_per_sm(G);
     if (ctas > sha::kMaxBlocks) ctas = sha::kMaxBlocks;
     if (ctas > pl.sched.total_tiles) ctas = pl.sched.total_tiles;
     // every block gets at least ceil((Tu-1)/(kMaxMergeParts-1)) tiles, so a
@@ -205,7 +206,7 @@ Plan make_varlen_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int 
                       int num_sms)
 {
     Plan pl = make_plan(B, H_q, H_kv, N_kv, d, top_k, 0, num_sms);
-    long long ctas = num_splits > 0 ? num_splits : (long long)num_sms * kBlocksPerSm;
+    long long ctas = num_splits > 0 ? num_splits : (long long)num_sms * blocks_per_sm(H_q / H_kv);
     if (ctas > sha::kMaxBlocks) ctas = sha::kMaxBlocks;
     if (ctas > pl.sched.total_tiles) ctas = pl.sched.total_tiles;
     if (ctas < 1) ctas = 1;

@@ -67,6 +67,10 @@ enum : int { kLayoutFixed = 0, kLayoutVarlen = 1, kLayoutPaged = 2 };
 #ifndef SHA_MHA_STAGES
 #define SHA_MHA_STAGES 3
 #endif
+// Blocks per SM the multi-head kernel is planned and compiled for.
+#ifndef SHA_MHA_BLOCKS_PER_SM
+#define SHA_MHA_BLOCKS_PER_SM 1
+#endif
 
 template <int D>
 struct MhaConfig {
@@ -99,7 +103,7 @@ struct MhaConfig {
 };
 
 template <typename T, int D, int kLayout>
-__global__ void __launch_bounds__(MhaConfig<D>::kThreads, 1)
+__global__ void __launch_bounds__(MhaConfig<D>::kThreads, SHA_MHA_BLOCKS_PER_SM)
     sha_mha_decode_kernel(const DecodeParams p)
 {
     constexpr bool kVarlen = kLayout != kLayoutFixed;
