@@ -1475,7 +1475,17 @@ struct MlpPlan {
     size_t total() const { return up_bytes + h_bytes + down_bytes; }
 };
 
-int batch_pad(int B) { return B <= 8 ? 8 : (B <= 16 ? 16 : (B <= 32 ? 32 : 64)); }
+// Batches up to 8 run padded to 8 on warp-level MMAs (1) or padded to 16 on the
+// tcgen05 path (0).
+#ifndef SHA_MLP_PAD8
+#define SHA_MLP_PAD8 1
+#endif
+
+int batch_pad(int B)
+{
+    if (B <= 8) return SHA_MLP_PAD8 ? 8 : 16;
+    return B <= 16 ? 16 : (B <= 32 ? 32 : 64);
+}
 
 MlpPlan mlp_plan(int B, int d, int D, int sms)
 {
