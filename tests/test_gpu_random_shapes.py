@@ -1,0 +1,89 @@
+"""Seeded random shapes against the float64 oracle: decode (G = 1..16, d = 64 /
+128, ragged key counts, top_k from 0 to H_kv, automatic and forced splits) and
+the Selective GEMM (batch 1..64 on both GEMM paths, ragged neuron counts,
+unions from almost empty to full, both activations)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from parity import check_against_oracle, mlp_excess
+
+pytestmark = pytest.mark.gpu
+W = workloads.Workload
+M = workloads.MlpWorkload
+
+
+def _decode_cases(n, seed):
+    rng = np.random.default_rng(seed)
+    cases = []
+    for i in range(n):
+        G = int(rng.choice([1, 1, 2, 4, 8, 16]))
+        H_kv = int(rng.integers(1, 17)) if G < 16 else int(rng.integers(1, 5))
+        d = int(rng.choice([64, 128]))
+        N_kv = int(rng.integers(1, 3001))
+        top_k = int(rng.integers(1, H_kv + 1)) if rng.random() > 0.1 else 0
+        B = int(rng.integers(1, 13))
+        dtype = str(rng.choice(["fp16", "bf16"]))
+        splits = int(rng.choice([0, 0, int(rng.integers(1, 400))]))
+        cases.append((W(f"rand{i}_B{B}_G{G}_Hkv{H_kv}_N{N_kv}_d{d}_k{top_k}_{dtype}", B=B,
+                        H_q=G * H_kv, H_kv=H_kv, N_kv=N_kv, d=d, top_k=top_k, dtype=dtype,
+                        seed=9000 + i), splits))
+    return cases
+
+
+def _mlp_cases(n, seed):
+    rng = np.random.default_rng(seed)
+    cases = []
+    for i in range(n):
+        B = int(rng.choice([1, 3, 8, 9, 16, 23, 32, 47, 64]))
+        d = int(rng.choice([256, 512, 768, 1024, 1536]))
+        D = int(rng.integers(1, 3001))
+        density = float(rng.choice([0.005, 0.05, 0.2, 0.5, 1.0]))
+        dtype = str(rng.choice(["fp16", "bf16"]))
+        act = str(rng.choice(["relu", "identity"]))
+        cases.append((M(f"mrand{i}_B{B}_d{d}_D{D}_p{density}_{dtype}", B=B, d=d, D=D,
+                        density=density, dtype=dtype, seed=9500 + i), act))
+    return cases
+
+
+@pytest.fixture(scope="module")
+def sha():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import head_sparse_decode_b200 as h
+    return h
+
+
+@pytest.mark.parametrize("w,splits", _decode_cases(24, 1234), ids=lambda c: getattr(c, "name", str(c)))
+def test_random_decode_shape(sha, w, splits):
+    q, k, v = workloads.make_qkv(w)
+    idx = workloads.make_index(w)
+    dev = torch.device("cuda")
+    q, k, v, idx = q.to(dev), k.to(dev), v.to(dev), idx.to(dev)
+    out = workloads.make_out(w, "cuda")
+    if splits == 0:
+        sha.decode(q, k, v, idx, w.scale, out)
+    else:
+        ws = sha.alloc_workspace(q, k, idx, splits)
+        sha.sha_decode_ex(q, k, v, idx, w.scale, out, ws, splits)
+    torch.cuda.synchronize()
+    assert sha.sha_get_device_status() == sha.SHA_OK
+    check_against_oracle(w, q, k, v, idx, out)
+
+
+@pytest.mark.parametrize("w,act", _mlp_cases(16, 4321), ids=lambda c: getattr(c, "name", str(c)))
+def test_random_selective_mlp_shape(sha, w, act):
+    x, W1t, W2t, active = workloads.make_mlp(w)
+    dev = torch.device("cuda")
+    S, n_S = sha.sha_mlp_union(active.to(dev))
+    y = sha.sha_selective_mlp(x.to(dev), W1t.to(dev), W2t.to(dev), S, n_S, activation=act)
+    torch.cuda.synchronize()
+    assert sha.sha_get_device_status() == sha.SHA_OK
+    want_S = oracle.mlp_union(active.numpy())
+    n = int(n_S.item())
+    assert n == len(want_S) and np.array_equal(S[:n].cpu().numpy(), want_S)
+    want = oracle.selective_mlp(x, W1t, W2t, want_S, w.dtype, act=act)
+    excess, err = mlp_excess(y.cpu().double().numpy(), want, w.dtype)
+    assert excess <= 0, err
