@@ -1177,6 +1177,9 @@ __global__ void __launch_bounds__(kCols)
 // and mlp_out adds them in a fixed order.
 
 // Build-time tuning of the down-projection for batches up to 8.
+#ifndef SHA_MLP_DOWN_CPASYNC
+#define SHA_MLP_DOWN_CPASYNC 1
+#endif
 #ifndef SHA_MLP_DOWN8_W
 #define SHA_MLP_DOWN8_W 1024
 #endif
@@ -1187,7 +1190,10 @@ __global__ void __launch_bounds__(kCols)
 template <int BP>
 struct DownCfg {
     static constexpr int kConsumerWarps = 8;
-    static constexpr int kThreads = (kConsumerWarps + 1) * 32;
+    // weight rows: one bulk copy per row segment from one producer warp, or
+    // 16-byte cp.async copies (128 bytes of four rows per instruction) from four
+    static constexpr int kProducerWarps = SHA_MLP_DOWN_CPASYNC ? 4 : 1;
+    static constexpr int kThreads = (kConsumerWarps + kProducerWarps) * 32;
     static constexpr int kWMax =                        // columns per item
         BP == 8 ? SHA_MLP_DOWN8_W : (BP == 16 ? 1024 : (BP == 32 ? 1024 : 512));
     static constexpr int kRows = BP == 8 ? SHA_MLP_DOWN8_ROWS : 32;   // neurons per stage
@@ -1213,7 +1219,8 @@ __global__ void __launch_bounds__(DownCfg<BP>::kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(&full[s], 1);
+            // the Ht tile's expect-tx arrival (+ one cp.async arrival per producer thread)
+            mbar_init(&full[s], SHA_MLP_DOWN_CPASYNC ? 1 + 32 * C::kProducerWarps : 1);
             mbar_init(&empty[s], C::kConsumerWarps);
         }
         mbar_init_fence();
@@ -1228,6 +1235,73 @@ __global__ void __launch_bounds__(DownCfg<BP>::kThreads, 1)
     const int wchunks = d / wc;
     const int items = wchunks * splits;
 
+#if SHA_MLP_DOWN_CPASYNC
+    if (warp >= C::kConsumerWarps) {
+        // producer warp p (of 4) copies row quads p, p+4, ... of each stage: an
+        // instruction moves 128 bytes (64 columns) of four rows, lane l taking
+        // row 4q + l/8 and 16-byte chunk l%8; the stage's Ht tile is one bulk
+        // copy.  Rows past the union repeat its last neuron (finite values times
+        // an activation of 0 add nothing, where stale shared memory could hold NaN).
+        constexpr int kQuads = C::kRows / 4 / C::kProducerWarps;   // row quads per warp
+        const int pw = warp - C::kConsumerWarps, chunk = lane & 7;
+        const uint64_t policy = l2_policy_evict_first();
+        int stage = 0;
+        uint32_t phase = 0, last_parity = 0, used = 0;
+        bool ok = true;
+        auto stage_ids = [&](int kt, int (&ids)[kQuads]) {
+#pragma unroll
+            for (int j = 0; j < kQuads; ++j)
+                ids[j] = neuron_id(
+                    S, min(kt * C::kRows + 4 * (pw + C::kProducerWarps * j) + (lane >> 3), n_S - 1), D);
+        };
+        for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
+            const int wcn = item / splits, split = item % splits;
+            const int kt0 = split * ktiles / splits, kt1 = (split + 1) * ktiles / splits;
+            const size_t c0 = (size_t)wcn * wc;
+            int ids_next[kQuads];
+            if (kt0 < kt1) stage_ids(kt0, ids_next);
+            for (int kt = kt0; kt < kt1; ++kt) {
+                int ids[kQuads];
+#pragma unroll
+                for (int j = 0; j < kQuads; ++j) ids[j] = ids_next[j];
+                if (kt + 1 < kt1) stage_ids(kt + 1, ids_next);
+                bool go = true;
+                if (lane == 0 && !mbar_wait(&empty[stage], phase ^ 1)) {
+                    atomicOr(&g_sha_status, kStatusTimeout);
+                    go = false;
+                }
+                go = __shfl_sync(0xffffffffu, go, 0);
+                if (!go) { ok = false; break; }
+                unsigned char *ws = smem + stage * C::kStage;
+                unsigned char *hs = ws + C::kRows * C::kWRow;
+                if (pw == 0 && lane == 0) {
+                    mbar_arrive_expect_tx(&full[stage], (uint32_t)C::kHBytes);
+                    bulk_copy_g2s(hs, Ht + (size_t)kt * C::kRows * BP, C::kHBytes, &full[stage],
+                                  policy);
+                }
+#pragma unroll
+                for (int j = 0; j < kQuads; ++j) {
+                    const int row = 4 * (pw + C::kProducerWarps * j) + (lane >> 3);
+                    const T *src = W2t + (size_t)ids[j] * d + c0 + chunk * 8;
+                    unsigned char *dst = ws + row * C::kWRow + chunk * 16;
+                    for (int piece = 0; piece < wc / 64; ++piece)
+                        cp_async16(dst + piece * 128, src + piece * 64, policy);
+                }
+                cp_async_arrive_noinc(&full[stage]);
+                last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+                used |= 1u << stage;
+                if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+            }
+        }
+        // no copy may be in flight when the block exits
+        cp_async_wait_all();
+        if (pw == 0 && lane == 0)
+            for (int s = 0; s < C::kStages; ++s)
+                if (used & (1u << s)) mbar_wait(&full[s], (last_parity >> s) & 1u);
+        __syncwarp();
+        return;
+    }
+#else
     if (warp == C::kConsumerWarps) {
         const uint64_t policy = l2_policy_evict_first();
         int stage = 0;
@@ -1280,6 +1354,8 @@ __global__ void __launch_bounds__(DownCfg<BP>::kThreads, 1)
         __syncwarp();
         return;
     }
+
+#endif
 
     // consumers: warp w owns output columns [w*wc/8, (w+1)*wc/8) x the batch
     const int g = lane >> 2, qd = lane & 3, mi = lane >> 3;
