@@ -228,10 +228,18 @@ size_t sha_selective_mlp_workspace_size(int B, int d, int D);
  *   x, y      : device, [B, d], fp16 or bf16 (dtype); W1t, W2t: [D, d]
  *   1 <= B <= 64, d a multiple of 256 (SHA_ERR_UNSUPPORTED otherwise)
  *   activation: 1 = ReLU (OPT's MLP), 0 = identity
- *   workspace : device, 256-byte aligned, >= sha_selective_mlp_workspace_size
+ *   workspace : device, 256-byte aligned, >= sha_selective_mlp_workspace_size;
+ *               scratch only (no contents carried between calls), owned by the
+ *               caller; calls that share it must not overlap on the device
+ *   x, W1t, W2t, y 16-byte aligned; S, n_S 4-byte aligned (SHA_ERR_MISALIGNED)
  * The hidden activations are rounded to the input dtype before the second
- * product (tensor-core operands); all sums are fp32.  Ids outside [0, D) are
- * bad input: the flag is raised, no memory outside the weights is read.
+ * product (tensor-core operands); all sums are fp32, and y is rounded to the
+ * input dtype.  Partial sums of neuron ranges split across thread blocks are
+ * added in a fixed order, so results do not depend on timing.  Batches up to
+ * 8 run on warp-level MMAs; larger batches run the up-projection (and from 17
+ * rows the down-projection) on tcgen05 with tensor-memory accumulators.  Ids
+ * outside [0, D) are bad input: the flag is raised (SHA_ERR_BAD_INDEX from
+ * sha_get_device_status), no memory outside the weights is read.
  */
 sha_status_t sha_selective_mlp(const void *x, const void *W1t, const void *W2t,
                                const int32_t *S, const int32_t *n_S, int B, int d, int D,
