@@ -135,3 +135,17 @@ def test_opt66b_mlp_large_batch_sampled(sha, B, density, dtype):
                                 w.dtype)
     excess, err = mlp_excess(y[rows][:, cols].cpu().double().numpy(), want, w.dtype)
     assert excess <= 0, err
+
+
+@pytest.mark.parametrize("case", [1, 3, 6, 2], ids=["batch8", "batch17", "batch32", "batch64"])
+def test_repeat_calls_are_bit_identical(sha, case):
+    """Split partial sums are added in a fixed order: no dependence on timing."""
+    w = CASES[case]
+    x, W1t, W2t, active = workloads.make_mlp(w)
+    dev = torch.device("cuda")
+    x, W1t, W2t = x.to(dev), W1t.to(dev), W2t.to(dev)
+    S, n_S = sha.sha_mlp_union(active.to(dev))
+    ys = [sha.sha_selective_mlp(x, W1t, W2t, S, n_S) for _ in range(3)]
+    torch.cuda.synchronize()
+    for y in ys[1:]:
+        assert torch.equal(y.view(torch.int16), ys[0].view(torch.int16))
