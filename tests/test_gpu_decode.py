@@ -76,6 +76,26 @@ def test_forced_splits_match_oracle(sha, splits):
     check_against_oracle(w, q, k, v, idx, out, expected)
 
 
+def test_block_cap_and_many_part_merges(sha):
+    """Limits of the split: a forced 10 000 blocks over 8192 tiles is clamped to
+    4096 (each head's 64 tiles then merge from 32 blocks), and one 64K-key head
+    is spread over as many blocks as the 64-part merge cap allows."""
+    for w, splits in ((W("cap4096", B=16, H_q=8, H_kv=8, N_kv=8192, d=64, top_k=8,
+                         dtype="fp16", seed=23), 10_000),
+                      (W("ctx64k", B=1, H_q=2, H_kv=2, N_kv=65536, d=128, top_k=1,
+                         dtype="bf16", seed=24), 10_000),
+                      (W("ctx64k_auto", B=1, H_q=2, H_kv=2, N_kv=65536, d=128, top_k=1,
+                         dtype="bf16", seed=25), None),
+                      (W("ctx64k_gqa", B=1, H_q=16, H_kv=2, N_kv=65536, d=128, top_k=1,
+                         dtype="bf16", seed=26), None)):
+        q, k, v, idx = _on_gpu(w)
+        if splits is not None:
+            plan = sha.sha_decode_plan(w.B, w.H_q, w.H_kv, w.N_kv, w.d, w.top_k, splits)
+            assert plan["blocks"] <= 4096
+        out = _run(sha, w, q, k, v, idx, num_splits=splits)
+        check_against_oracle(w, q, k, v, idx, out)
+
+
 def test_workspace_counters_return_to_zero(sha):
     w = W("ws", B=2, H_q=4, H_kv=4, N_kv=300, d=64, top_k=3, dtype="bf16", seed=22)
     q, k, v, idx = _on_gpu(w)
