@@ -339,6 +339,7 @@ def run_ours(args, rank, world, local):
         extras["other_configs"] = other_configs(sha, w, dev, stream, peak, rank)
         extras["other_configs"].append(varlen_config(sha, dev, stream, peak, rank))
         extras["other_configs"].append(paged_config(sha, dev, stream, peak, rank))
+        extras["other_configs"].extend(strided_configs(sha, dev, stream, peak, rank))
         mlp = run_mlp(argparse.Namespace(batch=None), dev)
         extras["selective_mlp"] = {"config": mlp["config"], "cublas_dense_us": mlp["cublas_dense_us"],
                                    "points": mlp["points"]}
@@ -417,6 +418,36 @@ def other_configs(sha, w_main, dev, stream, peak, rank):
         res.append({"workload": name, "us_per_step": round(t / steps * 1e6, 2),
                     "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
                     "steps_per_s": round(steps / t, 1), "G": w.G, "dtype": w.dtype,
+                    "bytes_per_step": w.algorithmic_bytes()})
+        del q, k, v, idx, out
+        torch.cuda.empty_cache()
+    return res
+
+
+def strided_configs(sha, dev, stream, peak, rank):
+    """OPT-66B and LLaMA-3.1-70B shapes with the cache stored token-major,
+    [B, N_kv, H_kv, d] (sha_decode_strided): each key row of a head is H_kv*d
+    elements from the next."""
+    res = []
+    for name in ("opt66b", "llama31_70b_gqa"):
+        w = workloads.CONFIGS[name].with_(seed=workloads.CONFIGS[name].seed + 100 * rank + 7)
+        q, k, v = workloads.make_qkv(w, device=dev)
+        k = k.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+        v = v.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+        torch.cuda.empty_cache()
+        idx = workloads.make_index(w).to(dev)
+        out = workloads.make_out(w, dev)
+
+        def call():
+            sha.sha_decode_strided(q, k, v, idx, w.scale, out)
+        for _ in range(20):
+            call()
+        steps = 500
+        t = timed_graphs(call, steps, dev, stream)
+        gbs = w.algorithmic_bytes() * steps / t / 1e9
+        res.append({"workload": name + "_token_major", "layout": "[B, N_kv, H_kv, d]",
+                    "us_per_step": round(t / steps * 1e6, 2), "gbs": round(gbs, 1),
+                    "frac": round(gbs / peak, 4), "steps_per_s": round(steps / t, 1),
                     "bytes_per_step": w.algorithmic_bytes()})
         del q, k, v, idx, out
         torch.cuda.empty_cache()

@@ -209,6 +209,46 @@ def sha_decode_paged(q, k_pages, v_pages, batch_head_index, seqlens, block_table
     return out
 
 
+_lib.sha_decode_strided.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_float,
+                                    _vp, ctypes.POINTER(ctypes.c_int64),
+                                    ctypes.POINTER(ctypes.c_int64), _i, _vp]
+_lib.sha_decode_strided.restype = _i
+
+
+def sha_decode_strided(q, k, v, batch_head_index, scale, out, stream=None):
+    """Selective head decode where k and v are [B, H_kv, N_kv, d] views with any
+    strides and d contiguous (e.g. a token-major [B, N_kv, H_kv, d] cache viewed
+    with .permute(0, 2, 1, 3), or a padded cache sliced to N_kv keys)."""
+    if k.dim() != 4 or v.shape != k.shape:
+        raise ValueError("k and v must both be [B, H_kv, N_kv, d] views")
+    if k.stride(3) != 1 or v.stride(3) != 1:
+        raise ValueError("k and v must have d contiguous")
+    B, H_kv, N_kv, d = k.shape
+    for name, t in (("q", q), ("out", out), ("batch_head_index", batch_head_index)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    for name, t in (("q", q), ("v", v), ("out", out), ("batch_head_index", batch_head_index)):
+        if not t.is_cuda or t.device != k.device:
+            raise ValueError(f"{name} must be a CUDA tensor on {k.device}")
+    for name, t in (("q", q), ("v", v), ("out", out)):
+        if t.dtype != k.dtype:
+            raise TypeError(f"{name} has dtype {t.dtype}, k has {k.dtype}")
+    if batch_head_index.dtype != torch.int32 or batch_head_index.dim() != 2 \
+            or batch_head_index.shape[0] != B:
+        raise ValueError("batch_head_index must be int32 [B, top_k]")
+    H_q = q.shape[1]
+    if q.shape[0] != B or q.shape[-1] != d or out.numel() != B * H_q * d:
+        raise ValueError("inconsistent shapes")
+    ks = (ctypes.c_int64 * 3)(k.stride(0), k.stride(1), k.stride(2))
+    vs = (ctypes.c_int64 * 3)(v.stride(0), v.stride(1), v.stride(2))
+    with torch.cuda.device(k.device):
+        _check(_lib.sha_decode_strided(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), batch_head_index.data_ptr(), B, H_q, H_kv,
+            N_kv, d, batch_head_index.shape[1], _default_scale(scale, d), out.data_ptr(), ks, vs,
+            _dtype_code(k.dtype), _stream_handle(stream, k.device)))
+    return out
+
+
 def _dtype_code(dtype):
     if dtype == torch.float16:
         return SHA_FP16

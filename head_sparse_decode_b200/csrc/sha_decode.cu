@@ -200,6 +200,72 @@ sha_status_t kv_tensor_map(CUtensorMap *map, const void *base, sha_dtype_t dtype
     return SHA_OK;
 }
 
+// 4-D view [d, o1, o2, o3] of a strided K or V cache: d contiguous, the outer
+// dimensions (token, head, batch in the order of increasing stride) with the
+// given sizes and byte strides, boxes of box_d x box_rows tokens (1 along the
+// other dimensions), 128-byte swizzled (64-element boxes of the grouped-query
+// kernel) or not (whole rows for the multi-head kernel).  Tokens past the end
+// read as zero.
+sha_status_t kv_tensor_map_4d(CUtensorMap *map, const void *base, sha_dtype_t dtype, int d,
+                              const long long (&size)[3], const long long (&stride_bytes)[3],
+                              int tok_dim, int box_d, int box_rows, bool swizzle128)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+    if (!encode) {
+        std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error,
+                      "cuTensorMapEncodeTiled is not available from the driver");
+        return SHA_ERR_LAUNCH;
+    }
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)size[0], (cuuint64_t)size[1],
+                          (cuuint64_t)size[2]};
+    cuuint64_t strides[3] = {(cuuint64_t)stride_bytes[0], (cuuint64_t)stride_bytes[1],
+                             (cuuint64_t)stride_bytes[2]};
+    cuuint32_t box[4] = {(cuuint32_t)box_d, 1, 1, 1};
+    box[1 + tok_dim] = (cuuint32_t)box_rows;
+    cuuint32_t elem[4] = {1, 1, 1, 1};
+    CUresult r = encode(map,
+                        dtype == SHA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                          : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                        4, const_cast<void *>(base), dims, strides, box, elem,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error,
+                      "cuTensorMapEncodeTiled failed with CUresult %d", (int)r);
+        return SHA_ERR_LAUNCH;
+    }
+    return SHA_OK;
+}
+
+// Strides of a strided K or V cache in elements: batch, head, token.
+struct KvStrides {
+    long long batch, head, token;
+};
+
+// Sizes and byte strides of the outer dimensions in the order of increasing
+// stride (ties keep token, head, batch order) and each dimension's position.
+void order_outer_dims(const KvStrides &st, int B, int H_kv, int N_kv, long long (&size)[3],
+                      long long (&stride_bytes)[3], int &tok_dim, int &head_dim,
+                      int &batch_dim)
+{
+    long long sv[3] = {st.token, st.head, st.batch};
+    long long nv[3] = {N_kv, H_kv, B};
+    int order[3] = {0, 1, 2};
+    for (int i = 1; i < 3; ++i)
+        for (int j = i; j > 0 && sv[order[j]] < sv[order[j - 1]]; --j)
+            std::swap(order[j], order[j - 1]);
+    int pos[3];
+    for (int i = 0; i < 3; ++i) {
+        size[i] = nv[order[i]];
+        stride_bytes[i] = sv[order[i]] * 2;
+        pos[order[i]] = i;
+    }
+    tok_dim = pos[0];
+    head_dim = pos[1];
+    batch_dim = pos[2];
+}
+
 // Per-row lengths: the kernel plans its own split from the lengths on the
 // device, using at most this many blocks; the workspace covers any split.
 Plan make_varlen_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int num_splits,
@@ -216,9 +282,14 @@ Plan make_varlen_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int 
     return pl;
 }
 
+// Tensor-map shapes of a strided cache (outer dimensions ordered by stride).
+struct StridedMaps {
+    long long k_size[3], k_stride[3], v_size[3], v_stride[3];
+};
+
 template <typename T, int D, int kLayout>
 sha_status_t launch_gqa(const sha::DecodeParams &prm, sha_dtype_t dtype, int dev,
-                        cudaStream_t stream)
+                        cudaStream_t stream, const StridedMaps *kv)
 {
     using C = sha::GqaConfig<D>;
     static std::atomic<bool> configured[kMaxDevices];
@@ -230,6 +301,19 @@ sha_status_t launch_gqa(const sha::DecodeParams &prm, sha_dtype_t dtype, int dev
         configured[dev].store(true, std::memory_order_release);
     }
     CUtensorMap tm_k, tm_v;
+    if constexpr (kLayout == sha::kLayoutStrided) {
+        sha_status_t st = kv_tensor_map_4d(&tm_k, prm.k, dtype, D, kv->k_size, kv->k_stride,
+                                           prm.tok_dim, 64, C::kTile, true);
+        if (st == SHA_OK)
+            st = kv_tensor_map_4d(&tm_v, prm.v, dtype, D, kv->v_size, kv->v_stride, prm.tok_dim,
+                                  64, C::kTile, true);
+        if (st != SHA_OK) return st;
+        cudaError_t e = launch_kernel(sha::sha_gqa_decode_kernel<T, D, kLayout>,
+                                      prm.sched.num_ctas, C::kThreads, C::kSmemBytes, stream, prm,
+                                      tm_k, tm_v);
+        if (e != cudaSuccess) return launch_error(e);
+        return SHA_OK;
+    }
     // a padded cache: [B*H_kv][N_kv][d]; a page pool: [num_pages*H_kv][page_size][d]
     const bool paged = kLayout == sha::kLayoutPaged;
     const long long planes = paged ? (long long)prm.num_pages * prm.H_kv : (long long)prm.B * prm.H_kv;
@@ -246,7 +330,8 @@ sha_status_t launch_gqa(const sha::DecodeParams &prm, sha_dtype_t dtype, int dev
 }
 
 template <typename T, int D, int kLayout>
-sha_status_t launch_mha(const sha::DecodeParams &prm, int dev, cudaStream_t stream)
+sha_status_t launch_mha(const sha::DecodeParams &prm, sha_dtype_t dtype, int dev,
+                        cudaStream_t stream, const StridedMaps *kv)
 {
     using C = sha::MhaConfig<D>;
     static std::atomic<bool> configured[kMaxDevices];
@@ -257,28 +342,40 @@ sha_status_t launch_mha(const sha::DecodeParams &prm, int dev, cudaStream_t stre
         if (e != cudaSuccess) return launch_error(e);
         configured[dev].store(true, std::memory_order_release);
     }
+    CUtensorMap tm_k, tm_v;                 // used by the strided layout only
+    std::memset(&tm_k, 0, sizeof tm_k);
+    std::memset(&tm_v, 0, sizeof tm_v);
+    if constexpr (kLayout == sha::kLayoutStrided) {
+        // whole [kTile][d] rows, unswizzled: the same tile layout as a bulk copy
+        sha_status_t st = kv_tensor_map_4d(&tm_k, prm.k, dtype, D, kv->k_size, kv->k_stride,
+                                           prm.tok_dim, D, C::kTile, false);
+        if (st == SHA_OK)
+            st = kv_tensor_map_4d(&tm_v, prm.v, dtype, D, kv->v_size, kv->v_stride, prm.tok_dim,
+                                  D, C::kTile, false);
+        if (st != SHA_OK) return st;
+    }
     cudaError_t e = launch_kernel(sha::sha_mha_decode_kernel<T, D, kLayout>, prm.sched.num_ctas,
-                                  C::kThreads, C::kSmemBytes, stream, prm);
+                                  C::kThreads, C::kSmemBytes, stream, prm, tm_k, tm_v);
     if (e != cudaSuccess) return launch_error(e);
     return SHA_OK;
 }
 
 template <int kLayout>
 sha_status_t launch_decode(const sha::DecodeParams &prm, sha_dtype_t dtype, int d, int G,
-                           int dev, cudaStream_t s)
+                           int dev, cudaStream_t s, const StridedMaps *kv = nullptr)
 {
     if (G > 1) {
         if (dtype == SHA_FP16)
-            return d == 128 ? launch_gqa<__half, 128, kLayout>(prm, dtype, dev, s)
-                            : launch_gqa<__half, 64, kLayout>(prm, dtype, dev, s);
-        return d == 128 ? launch_gqa<__nv_bfloat16, 128, kLayout>(prm, dtype, dev, s)
-                        : launch_gqa<__nv_bfloat16, 64, kLayout>(prm, dtype, dev, s);
+            return d == 128 ? launch_gqa<__half, 128, kLayout>(prm, dtype, dev, s, kv)
+                            : launch_gqa<__half, 64, kLayout>(prm, dtype, dev, s, kv);
+        return d == 128 ? launch_gqa<__nv_bfloat16, 128, kLayout>(prm, dtype, dev, s, kv)
+                        : launch_gqa<__nv_bfloat16, 64, kLayout>(prm, dtype, dev, s, kv);
     }
     if (dtype == SHA_FP16)
-        return d == 128 ? launch_mha<__half, 128, kLayout>(prm, dev, s)
-                        : launch_mha<__half, 64, kLayout>(prm, dev, s);
-    return d == 128 ? launch_mha<__nv_bfloat16, 128, kLayout>(prm, dev, s)
-                    : launch_mha<__nv_bfloat16, 64, kLayout>(prm, dev, s);
+        return d == 128 ? launch_mha<__half, 128, kLayout>(prm, dtype, dev, s, kv)
+                        : launch_mha<__half, 64, kLayout>(prm, dtype, dev, s, kv);
+    return d == 128 ? launch_mha<__nv_bfloat16, 128, kLayout>(prm, dtype, dev, s, kv)
+                    : launch_mha<__nv_bfloat16, 64, kLayout>(prm, dtype, dev, s, kv);
 }
 
 // Where the keys of a call live beyond the plain [B, H_kv, N_kv, d] cache.
@@ -286,6 +383,8 @@ struct KvLayout {
     const int32_t *seqlens = nullptr;       // per-row lengths (device), or null
     const int32_t *block_table = nullptr;   // paged pool: [B, max_pages] (device), or null
     int page_size = 0, max_pages = 0, num_pages = 0;
+    bool strided = false;                   // K, V with the strides below (elements)
+    KvStrides k_strides{}, v_strides{};
 };
 
 // N_kv is the padded length (per-row lengths) or max_pages * page_size (paged).
@@ -365,6 +464,20 @@ sha_status_t decode_impl(const void *q, const void *k, const void *v, const int3
     prm.page_size = lay.page_size;
     prm.max_pages = lay.max_pages;
     prm.num_pages = lay.num_pages;
+    prm.tok_dim = 0;
+    prm.head_dim = 1;
+    prm.batch_dim = 2;
+    if (lay.strided) {
+        StridedMaps kv;
+        int vt, vh, vb;
+        order_outer_dims(lay.k_strides, B, H_kv, N_kv, kv.k_size, kv.k_stride, prm.tok_dim,
+                         prm.head_dim, prm.batch_dim);
+        order_outer_dims(lay.v_strides, B, H_kv, N_kv, kv.v_size, kv.v_stride, vt, vh, vb);
+        // one set of coordinates serves both maps
+        if (vt != prm.tok_dim || vh != prm.head_dim || vb != prm.batch_dim)
+            return SHA_ERR_UNSUPPORTED;
+        return launch_decode<sha::kLayoutStrided>(prm, dtype, d, G, dev, s, &kv);
+    }
     if (lay.block_table) return launch_decode<sha::kLayoutPaged>(prm, dtype, d, G, dev, s);
     if (seqlens) return launch_decode<sha::kLayoutVarlen>(prm, dtype, d, G, dev, s);
     return launch_decode<sha::kLayoutFixed>(prm, dtype, d, G, dev, s);
@@ -451,6 +564,27 @@ sha_status_t sha_decode_paged(const void *q, const void *k_pages, const void *v_
     return decode_impl(q, k_pages, v_pages, batch_head_index, B, H_q, H_kv,
                        max_pages * page_size, d, top_k, scale, out, dtype, nullptr, 0, 0,
                        stream, true, lay);
+}
+
+sha_status_t sha_decode_strided(const void *q, const void *k, const void *v,
+                                const int32_t *batch_head_index, int B, int H_q, int H_kv,
+                                int N_kv, int d, int top_k, float scale, void *out,
+                                const int64_t k_strides[3], const int64_t v_strides[3],
+                                sha_dtype_t dtype, void *stream)
+{
+    if (!k_strides || !v_strides) return SHA_ERR_INVALID_ARG;
+    KvLayout lay;
+    lay.strided = true;
+    lay.k_strides = {k_strides[0], k_strides[1], k_strides[2]};
+    lay.v_strides = {v_strides[0], v_strides[1], v_strides[2]};
+    for (int i = 0; i < 3; ++i) {
+        if (k_strides[i] < 1 || v_strides[i] < 1) return SHA_ERR_INVALID_ARG;
+        // TMA: every stride a multiple of 16 bytes, below 2^40 bytes
+        if (k_strides[i] % 8 || v_strides[i] % 8) return SHA_ERR_MISALIGNED;
+        if (k_strides[i] >= (1ll << 39) || v_strides[i] >= (1ll << 39)) return SHA_ERR_INVALID_ARG;
+    }
+    return decode_impl(q, k, v, batch_head_index, B, H_q, H_kv, N_kv, d, top_k, scale, out,
+                       dtype, nullptr, 0, 0, stream, true, lay);
 }
 
 size_t sha_decode_workspace_size(int B, int H_q, int H_kv, int N_kv, int d, int top_k,

@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
     sha_gqa_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v)
 {
-    constexpr bool kVarlen = kLayout != kLayoutFixed;
+    constexpr bool kVarlen = kLayout == kLayoutVarlen || kLayout == kLayoutPaged;
     using Walk = typename std::conditional<kVarlen, VarlenWalk, UniformWalk>::type;
     using C = GqaConfig<D>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -215,6 +215,18 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
                                             c * box_rows * 128,
                                         &tm_v, bx * 64, off, pplane, &full[stage], policy);
                         }
+                    }
+                } else if constexpr (kLayout == kLayoutStrided) {
+                    // boxes of a 4-D map whose outer dimensions follow the caller's strides
+                    int c[3];
+                    strided_coords(p, j * C::kTile, h, b, c);
+                    mbar_arrive_expect_tx(&full[stage], 2 * C::kTileBytes);
+#pragma unroll
+                    for (int bx = 0; bx < C::kBoxes; ++bx) {
+                        tma_load_4d(k_ring + stage * C::kTileBytes + bx * C::kBoxBytes, &tm_k,
+                                    bx * 64, c[0], c[1], c[2], &full[stage], policy);
+                        tma_load_4d(v_ring + stage * C::kTileBytes + bx * C::kBoxBytes, &tm_v,
+                                    bx * 64, c[0], c[1], c[2], &full[stage], policy);
                     }
                 } else {
                     mbar_arrive_expect_tx(&full[stage], 2 * C::kTileBytes);

@@ -28,6 +28,7 @@
 // O unnormalised and divides once at the end, which is the same quantity.
 #pragma once
 
+#include <cuda.h>
 #include <type_traits>
 
 #include "sha_device.cuh"
@@ -54,11 +55,37 @@ struct DecodeParams {
     // of row b sits in page block_table[b, n / page_size]
     const int32_t *block_table;
     int page_size, max_pages, num_pages;
+    // strided cache: K and V are read through 4-D tensor maps [d, ., ., .] whose
+    // three outer dimensions are the token, head and batch dimensions in the
+    // order of increasing stride; these give each one's position (0..2)
+    int tok_dim, head_dim, batch_dim;
 };
 
 // How K/V of a unit are found: one padded [N_kv] block per (b, h) with every
-// row N_kv long or with per-row lengths, or pages of a shared pool.
-enum : int { kLayoutFixed = 0, kLayoutVarlen = 1, kLayoutPaged = 2 };
+// row N_kv long or with per-row lengths, pages of a shared pool, or any
+// (batch, head, token) strides with d contiguous (every row N_kv long).
+enum : int { kLayoutFixed = 0, kLayoutVarlen = 1, kLayoutPaged = 2, kLayoutStrided = 3 };
+
+// TMA tiled load of one box of a 4-D tensor map into shared memory.
+__device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, int x, int c1,
+                                            int c2, int c3, uint64_t *bar, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(c1), "r"(c2), "r"(c3),
+        "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+// Tile (keys n0.., head h, row b) of a strided cache: the box's outer coordinates.
+__device__ __forceinline__ void strided_coords(const DecodeParams &p, int n0, int h, int b,
+                                               int (&c)[3])
+{
+    c[p.tok_dim] = n0;
+    c[p.head_dim] = h;
+    c[p.batch_dim] = b;
+}
 
 // Build-time tuning of the multi-head kernel (defaults measured best on B200).
 #ifndef SHA_MHA_TILE_KEYS
@@ -104,9 +131,10 @@ struct MhaConfig {
 
 template <typename T, int D, int kLayout>
 __global__ void __launch_bounds__(MhaConfig<D>::kThreads, SHA_MHA_BLOCKS_PER_SM)
-    sha_mha_decode_kernel(const DecodeParams p)
+    sha_mha_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v)
 {
-    constexpr bool kVarlen = kLayout != kLayoutFixed;
+    constexpr bool kVarlen = kLayout == kLayoutVarlen || kLayout == kLayoutPaged;
     using Walk = typename std::conditional<kVarlen, VarlenWalk, UniformWalk>::type;
     using C = MhaConfig<D>;
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -185,6 +213,16 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, SHA_MHA_BLOCKS_PER_SM)
                 const int n0 = j * C::kTile;
                 const int rows = min(C::kTile, seg.n_keys - n0);
                 const uint32_t bytes = (uint32_t)rows * C::kRowBytes;
+                if constexpr (kLayout == kLayoutStrided) {
+                    // one [kTile][d] box per tensor (rows past N_kv arrive as zeros)
+                    int c[3];
+                    strided_coords(p, n0, h, b, c);
+                    mbar_arrive_expect_tx(&full[stage], 2 * C::kTileBytes);
+                    tma_load_4d(k_ring + stage * C::kTileBytes, &tm_k, 0, c[0], c[1], c[2],
+                                &full[stage], policy);
+                    tma_load_4d(v_ring + stage * C::kTileBytes, &tm_v, 0, c[0], c[1], c[2],
+                                &full[stage], policy);
+                } else {
                 if (lane == 0) mbar_arrive_expect_tx(&full[stage], 2 * bytes);
                 if constexpr (kLayout == kLayoutPaged) {
                     // one copy per run of keys that lie in one page, a run per lane
@@ -215,6 +253,7 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, SHA_MHA_BLOCKS_PER_SM)
                                   bytes, &full[stage], policy);
                     bulk_copy_g2s(v_ring + stage * C::kTileBytes, vbase + (size_t)n0 * D,
                                   bytes, &full[stage], policy);
+                }
                 }
                 last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
                 used |= 1u << stage;

@@ -136,6 +136,29 @@ sha_status_t sha_decode_varlen(const void *q, const void *k, const void *v,
                                float scale, void *out, sha_dtype_t dtype, void *stream);
 
 /*
+ * sha_decode_strided -- the same operation over K and V caches laid out with
+ * any strides, d contiguous: element (b, h, n, c) of K is at
+ *   k + b*k_strides[0] + h*k_strides[1] + n*k_strides[2] + c
+ * (strides in elements; likewise for V).  This covers a token-major cache
+ * [B, N, H_kv, d] (strides N*H_kv*d, d, H_kv*d), a head-major cache padded
+ * to N_max > N_kv (strides H_kv*N_max*d, N_max*d, d), and the K and V views
+ * of one fused buffer.  Each key tile is one TMA tensor box.
+ *   k_strides, v_strides : host arrays of 3 int64 (batch, head, token), each
+ *                          >= 1 and a multiple of 8 elements (16 bytes;
+ *                          SHA_ERR_MISALIGNED otherwise); K and V strides must
+ *                          rank their dimensions in the same order
+ *                          (SHA_ERR_UNSUPPORTED otherwise)
+ *   dtype                : SHA_FP16 or SHA_BF16; other arguments as for sha_decode.
+ * The caller guarantees that the addressed elements lie inside its buffers.
+ * Uses the library-owned per-device workspace, like sha_decode.
+ */
+sha_status_t sha_decode_strided(const void *q, const void *k, const void *v,
+                                const int32_t *batch_head_index, int B, int H_q, int H_kv,
+                                int N_kv, int d, int top_k, float scale, void *out,
+                                const int64_t k_strides[3], const int64_t v_strides[3],
+                                sha_dtype_t dtype, void *stream);
+
+/*
  * sha_decode_paged -- the same operation over a paged KV cache, the serving
  * layout in which each sequence's keys live in fixed-size pages of a pool:
  *   k_pages, v_pages : [num_pages, H_kv, page_size, d]
