@@ -209,16 +209,17 @@ def sha_decode_paged(q, k_pages, v_pages, batch_head_index, seqlens, block_table
     return out
 
 
-_lib.sha_decode_strided.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_float,
+_lib.sha_decode_strided.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_float,
                                     _vp, ctypes.POINTER(ctypes.c_int64),
                                     ctypes.POINTER(ctypes.c_int64), _i, _vp]
 _lib.sha_decode_strided.restype = _i
 
 
-def sha_decode_strided(q, k, v, batch_head_index, scale, out, stream=None):
+def sha_decode_strided(q, k, v, batch_head_index, scale, out, seqlens=None, stream=None):
     """Selective head decode where k and v are [B, H_kv, N_kv, d] views with any
     strides and d contiguous (e.g. a token-major [B, N_kv, H_kv, d] cache viewed
-    with .permute(0, 2, 1, 3), or a padded cache sliced to N_kv keys)."""
+    with .permute(0, 2, 1, 3), or a padded cache sliced to N_kv keys); with
+    seqlens (int32 [B] on the device) row b uses its first seqlens[b] keys."""
     if k.dim() != 4 or v.shape != k.shape:
         raise ValueError("k and v must both be [B, H_kv, N_kv, d] views")
     if k.stride(3) != 1 or v.stride(3) != 1:
@@ -239,11 +240,16 @@ def sha_decode_strided(q, k, v, batch_head_index, scale, out, stream=None):
     H_q = q.shape[1]
     if q.shape[0] != B or q.shape[-1] != d or out.numel() != B * H_q * d:
         raise ValueError("inconsistent shapes")
+    if seqlens is not None and (seqlens.dim() != 1 or seqlens.shape[0] != B
+                                or seqlens.dtype != torch.int32 or not seqlens.is_contiguous()
+                                or seqlens.device != k.device):
+        raise ValueError("seqlens must be a contiguous int32 [B] tensor on k's device")
     ks = (ctypes.c_int64 * 3)(k.stride(0), k.stride(1), k.stride(2))
     vs = (ctypes.c_int64 * 3)(v.stride(0), v.stride(1), v.stride(2))
     with torch.cuda.device(k.device):
         _check(_lib.sha_decode_strided(
-            q.data_ptr(), k.data_ptr(), v.data_ptr(), batch_head_index.data_ptr(), B, H_q, H_kv,
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), batch_head_index.data_ptr(),
+            None if seqlens is None else seqlens.data_ptr(), B, H_q, H_kv,
             N_kv, d, batch_head_index.shape[1], _default_scale(scale, d), out.data_ptr(), ks, vs,
             _dtype_code(k.dtype), _stream_handle(stream, k.device)))
     return out

@@ -301,7 +301,7 @@ sha_status_t launch_gqa(const sha::DecodeParams &prm, sha_dtype_t dtype, int dev
         configured[dev].store(true, std::memory_order_release);
     }
     CUtensorMap tm_k, tm_v;
-    if constexpr (kLayout == sha::kLayoutStrided) {
+    if constexpr (sha::layout_strided(kLayout)) {
         sha_status_t st = kv_tensor_map_4d(&tm_k, prm.k, dtype, D, kv->k_size, kv->k_stride,
                                            prm.tok_dim, 64, C::kTile, true);
         if (st == SHA_OK)
@@ -345,7 +345,7 @@ sha_status_t launch_mha(const sha::DecodeParams &prm, sha_dtype_t dtype, int dev
     CUtensorMap tm_k, tm_v;                 // used by the strided layout only
     std::memset(&tm_k, 0, sizeof tm_k);
     std::memset(&tm_v, 0, sizeof tm_v);
-    if constexpr (kLayout == sha::kLayoutStrided) {
+    if constexpr (sha::layout_strided(kLayout)) {
         // whole [kTile][d] rows, unswizzled: the same tile layout as a bulk copy
         sha_status_t st = kv_tensor_map_4d(&tm_k, prm.k, dtype, D, kv->k_size, kv->k_stride,
                                            prm.tok_dim, D, C::kTile, false);
@@ -476,6 +476,7 @@ sha_status_t decode_impl(const void *q, const void *k, const void *v, const int3
         // one set of coordinates serves both maps
         if (vt != prm.tok_dim || vh != prm.head_dim || vb != prm.batch_dim)
             return SHA_ERR_UNSUPPORTED;
+        if (seqlens) return launch_decode<sha::kLayoutStridedVarlen>(prm, dtype, d, G, dev, s, &kv);
         return launch_decode<sha::kLayoutStrided>(prm, dtype, d, G, dev, s, &kv);
     }
     if (lay.block_table) return launch_decode<sha::kLayoutPaged>(prm, dtype, d, G, dev, s);
@@ -567,14 +568,15 @@ sha_status_t sha_decode_paged(const void *q, const void *k_pages, const void *v_
 }
 
 sha_status_t sha_decode_strided(const void *q, const void *k, const void *v,
-                                const int32_t *batch_head_index, int B, int H_q, int H_kv,
-                                int N_kv, int d, int top_k, float scale, void *out,
-                                const int64_t k_strides[3], const int64_t v_strides[3],
+                                const int32_t *batch_head_index, const int32_t *seqlens, int B,
+                                int H_q, int H_kv, int N_kv, int d, int top_k, float scale,
+                                void *out, const int64_t k_strides[3], const int64_t v_strides[3],
                                 sha_dtype_t dtype, void *stream)
 {
     if (!k_strides || !v_strides) return SHA_ERR_INVALID_ARG;
     KvLayout lay;
     lay.strided = true;
+    lay.seqlens = seqlens;
     lay.k_strides = {k_strides[0], k_strides[1], k_strides[2]};
     lay.v_strides = {v_strides[0], v_strides[1], v_strides[2]};
     for (int i = 0; i < 3; ++i) {

@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
     sha_gqa_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v)
 {
-    constexpr bool kVarlen = kLayout == kLayoutVarlen || kLayout == kLayoutPaged;
+    constexpr bool kVarlen = layout_varlen(kLayout);
     using Walk = typename std::conditional<kVarlen, VarlenWalk, UniformWalk>::type;
     using C = GqaConfig<D>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -216,7 +216,7 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
                                         &tm_v, bx * 64, off, pplane, &full[stage], policy);
                         }
                     }
-                } else if constexpr (kLayout == kLayoutStrided) {
+                } else if constexpr (layout_strided(kLayout)) {
                     // boxes of a 4-D map whose outer dimensions follow the caller's strides
                     int c[3];
                     strided_coords(p, j * C::kTile, h, b, c);

@@ -63,8 +63,26 @@ struct DecodeParams {
 
 // How K/V of a unit are found: one padded [N_kv] block per (b, h) with every
 // row N_kv long or with per-row lengths, pages of a shared pool, or any
-// (batch, head, token) strides with d contiguous (every row N_kv long).
-enum : int { kLayoutFixed = 0, kLayoutVarlen = 1, kLayoutPaged = 2, kLayoutStrided = 3 };
+// (batch, head, token) strides with d contiguous (every row N_kv long, or
+// per-row lengths within N_kv).
+enum : int {
+    kLayoutFixed = 0,
+    kLayoutVarlen = 1,
+    kLayoutPaged = 2,
+    kLayoutStrided = 3,
+    kLayoutStridedVarlen = 4
+};
+
+// Layouts whose rows have their own lengths (planned on the device) and that
+// read K/V through strided 4-D tensor maps.
+constexpr bool layout_varlen(int layout)
+{
+    return layout == kLayoutVarlen || layout == kLayoutPaged || layout == kLayoutStridedVarlen;
+}
+constexpr bool layout_strided(int layout)
+{
+    return layout == kLayoutStrided || layout == kLayoutStridedVarlen;
+}
 
 // TMA tiled load of one box of a 4-D tensor map into shared memory.
 __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, int x, int c1,
@@ -134,7 +152,7 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, SHA_MHA_BLOCKS_PER_SM)
     sha_mha_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v)
 {
-    constexpr bool kVarlen = kLayout == kLayoutVarlen || kLayout == kLayoutPaged;
+    constexpr bool kVarlen = layout_varlen(kLayout);
     using Walk = typename std::conditional<kVarlen, VarlenWalk, UniformWalk>::type;
     using C = MhaConfig<D>;
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -213,7 +231,7 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, SHA_MHA_BLOCKS_PER_SM)
                 const int n0 = j * C::kTile;
                 const int rows = min(C::kTile, seg.n_keys - n0);
                 const uint32_t bytes = (uint32_t)rows * C::kRowBytes;
-                if constexpr (kLayout == kLayoutStrided) {
+                if constexpr (layout_strided(kLayout)) {
                     // one [kTile][d] box per tensor (rows past N_kv arrive as zeros)
                     int c[3];
                     strided_coords(p, n0, h, b, c);

@@ -143,6 +143,9 @@ sha_status_t sha_decode_varlen(const void *q, const void *k, const void *v,
  * [B, N, H_kv, d] (strides N*H_kv*d, d, H_kv*d), a head-major cache padded
  * to N_max > N_kv (strides H_kv*N_max*d, N_max*d, d), and the K and V views
  * of one fused buffer.  Each key tile is one TMA tensor box.
+ *   seqlens              : NULL (every row N_kv keys long) or a device pointer,
+ *                          int32 [B], each in [1, N_kv]: row b attends to its
+ *                          first seqlens[b] keys, as in sha_decode_varlen
  *   k_strides, v_strides : host arrays of 3 int64 (batch, head, token), each
  *                          >= 1 and a multiple of 8 elements (16 bytes;
  *                          SHA_ERR_MISALIGNED otherwise); K and V strides must
@@ -153,9 +156,9 @@ sha_status_t sha_decode_varlen(const void *q, const void *k, const void *v,
  * Uses the library-owned per-device workspace, like sha_decode.
  */
 sha_status_t sha_decode_strided(const void *q, const void *k, const void *v,
-                                const int32_t *batch_head_index, int B, int H_q, int H_kv,
-                                int N_kv, int d, int top_k, float scale, void *out,
-                                const int64_t k_strides[3], const int64_t v_strides[3],
+                                const int32_t *batch_head_index, const int32_t *seqlens, int B,
+                                int H_q, int H_kv, int N_kv, int d, int top_k, float scale,
+                                void *out, const int64_t k_strides[3], const int64_t v_strides[3],
                                 sha_dtype_t dtype, void *stream);
 
 /*

@@ -126,7 +126,7 @@ def test_varlen_and_paged_host_checks(lib):
 
 def test_strided_host_checks(lib):
     P = 0x1000
-    lib.sha_decode_strided.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 6 + [
+    lib.sha_decode_strided.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 6 + [
         ctypes.c_float, ctypes.c_void_p, ctypes.POINTER(ctypes.c_int64),
         ctypes.POINTER(ctypes.c_int64), ctypes.c_int, ctypes.c_void_p]
     good = (ctypes.c_int64 * 3)(4 * 64 * 128, 128, 4 * 128)    # token-major [B, N, H, d]
@@ -134,7 +134,8 @@ def test_strided_host_checks(lib):
     zero = (ctypes.c_int64 * 3)(4 * 64 * 128, 0, 4 * 128)
 
     def call(ks, vs, d=128):
-        return lib.sha_decode_strided(P, P, P, P, 2, 4, 4, 64, d, 2, 0.1, P, ks, vs, 0, None)
+        return lib.sha_decode_strided(P, P, P, P, None, 2, 4, 4, 64, d, 2, 0.1, P, ks, vs, 0,
+                                      None)
     assert call(None, good) == 1
     assert call(good, zero) == 1
     assert call(good, odd) == 3

@@ -103,3 +103,38 @@ def test_k_and_v_strides_must_rank_alike(sha):
     assert e.value.status == sha.SHA_ERR_UNSUPPORTED
     bits = out.cpu().view(torch.int16).numpy().view(np.uint16)
     assert (bits == workloads.SENTINEL[w.dtype]).all()
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_token_major_cache_with_row_lengths(sha, w):
+    """Token-major cache, row b using its first seqlens[b] keys; keys at or past a
+    row's length hold NaN and must never reach the result."""
+    import oracle
+    from parity import TOLERANCE, out_bits
+
+    q, k, v = workloads.make_qkv(w)
+    idx = workloads.make_index(w)
+    g = torch.Generator().manual_seed(w.seed + 5)
+    lens = torch.randint(1, w.N_kv + 1, (w.B,), generator=g, dtype=torch.int32)
+    lens[0] = 1
+    lens[-1] = w.N_kv
+    k_poison, v_poison = k.clone(), v.clone()
+    for b in range(w.B):
+        k_poison[b, :, int(lens[b]):] = float("nan")
+        v_poison[b, :, int(lens[b]):] = float("nan")
+    dev = torch.device("cuda")
+    k_tok = k_poison.permute(0, 2, 1, 3).contiguous().to(dev).permute(0, 2, 1, 3)
+    v_tok = v_poison.permute(0, 2, 1, 3).contiguous().to(dev).permute(0, 2, 1, 3)
+    out = workloads.make_out(w, "cuda")
+    sha.sha_decode_strided(q.to(dev), k_tok, v_tok, idx.to(dev), w.scale, out,
+                           seqlens=lens.to(dev))
+    torch.cuda.synchronize()
+    assert sha.sha_get_device_status() == sha.SHA_OK
+    want, bad = oracle.sha_decode_varlen(q, k, v, idx.numpy(), lens.numpy(), w.scale, w.dtype)
+    assert bad == 0
+    written = ~np.isnan(want[..., 0])
+    bits = out_bits(out).reshape(w.B, w.H_q, w.d)
+    assert (bits[~written] == np.uint16(workloads.SENTINEL[w.dtype])).all()
+    got = out.cpu().double().numpy()
+    assert np.isfinite(got[written]).all()
+    assert np.abs(got[written] - want[written]).max() <= TOLERANCE[w.dtype]
