@@ -61,6 +61,9 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=100)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--config", default="opt66b", choices=sorted(workloads.CONFIGS))
+    p.add_argument("--layout", default="head_major", choices=["head_major", "token_major"],
+                   help="K/V cache layout of the timed step: [B, H_kv, N_kv, d] (sha_decode) "
+                        "or [B, N_kv, H_kv, d] (sha_decode_strided; implies --no-extras)")
     p.add_argument("--batch", type=int, default=None,
                    help="override the workload's batch size (small ncu captures)")
     p.add_argument("--no-extras", action="store_true",
@@ -299,8 +302,18 @@ def run_ours(args, rank, world, local):
     out = workloads.make_out(w, dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        sha.decode(q, k, v, idx, w.scale, out)
+    if args.layout == "token_major":
+        # the same values stored [B, N_kv, H_kv, d], read through strided views
+        k = k.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+        v = v.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+        torch.cuda.empty_cache()
+        args.no_extras = True
+
+        def step():
+            sha.sha_decode_strided(q, k, v, idx, w.scale, out)
+    else:
+        def step():
+            sha.decode(q, k, v, idx, w.scale, out)
 
     # same-run HBM copy probe (1 GiB read + 1 GiB written)
     src = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
@@ -355,6 +368,8 @@ def run_ours(args, rank, world, local):
                    "accumulation": "fp32", "l2": "no flush: active K/V per step "
                    f"{w.units * 2 * w.N_kv * w.d * 2 / 1e9:.2f} GB > 126 MB L2",
                    "blocks": plan["blocks"], "tile_keys": plan["tile_keys"],
+                   "kv_layout": "[B, H_kv, N_kv, d]" if args.layout == "head_major"
+                   else "[B, N_kv, H_kv, d] (strided views)",
                    "launch": "CUDA graph replay, 100 steps per graph"},
         "steps_per_s": round(args.steps / t_max, 2),
         "tokens_per_s": round(world * w.B * args.steps / t_max, 1),
@@ -364,7 +379,8 @@ def run_ours(args, rank, world, local):
         "gpu_launches": args.steps,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "traffic": profiled_traffic(w.name), "peak_source": peak_src,
+                     "traffic": profiled_traffic(w.name) if args.layout == "head_major" else None,
+                     "peak_source": peak_src,
                      "kernel": "sha_mha_decode_kernel" if w.G == 1 else "sha_gqa_decode_kernel",
                      "launch_us": round(launch_s * 1e6, 3),
                      "bytes_per_launch": bytes_step},
