@@ -1172,11 +1172,13 @@ __global__ void __launch_bounds__(kCols)
 // An item is a range of wc output columns (2 KiB of each weight row for
 // batches up to 16) over a range of the union's neurons; stages hold
 // kRows weight-row segments and the matching kRows x BP block of the
-// neuron-major activations (one contiguous copy).  Eight consumer warps own
-// wc/8 columns each.  Partial sums over the neuron ranges go to the workspace
-// and mlp_out adds them in a fixed order.
+// neuron-major activations (one contiguous copy).  The weight rows arrive by
+// 16-byte cp.async from four producer warps (or, with SHA_MLP_DOWN_CPASYNC=0,
+// by one bulk copy per row segment).  Eight consumer warps own wc/8 columns
+// each.  Partial sums over the neuron ranges go to the workspace and mlp_out
+// adds them in a fixed order.
 
-// Build-time tuning of the down-projection for batches up to 8.
+// Build-time tuning of the down-projection (the feed; widths for batches up to 8).
 #ifndef SHA_MLP_DOWN_CPASYNC
 #define SHA_MLP_DOWN_CPASYNC 1
 #endif
