@@ -22,9 +22,10 @@
 //   mlp_down  -- partial Ht^T . W2t[S] over a range of neurons (fp32): M =
 //                batch, N = up to 1024 output columns, K = neurons
 //   mlp_out   -- y = sum of the partials, in a fixed order
-// These stream weight-row segments with 1-D bulk copies (one per row and
-// stage, up to 4.5 KiB) into shared-memory rows padded by 16 bytes, so
-// ldmatrix reads are free of bank conflicts.
+// These stream weight-row segments into shared-memory rows padded by 16
+// bytes, so ldmatrix reads are free of bank conflicts: 1-D bulk copies (one
+// per row and stage, up to 4.5 KiB) for the up-projection, 16-byte cp.async
+// copies from four producer warps for the down-projection.
 // Batches of 9 to 64, on tcgen05 with fp32 accumulators in tensor memory:
 //   mlp_up_tc   -- D[128 neurons x batch] = W1t[S] . x^T, stream-K over
 //                  (neuron group, K tile); whole groups write Ht directly
