@@ -86,6 +86,16 @@ struct Plan {
     size_t workspace_bytes() const { return counter_bytes + slot_bytes; }
 };
 
+// Whether the host may cut a call at unit boundaries (see make_plan), and
+// what a split unit's merge is taken to cost, in key tiles of streaming.
+#ifndef SHA_ALIGN_UNITS
+#define SHA_ALIGN_UNITS 1
+#endif
+#ifndef SHA_MERGE_COST_TILES
+#define SHA_MERGE_COST_TILES 2
+#endif
+constexpr long long kMergeCostTiles = SHA_MERGE_COST_TILES;
+
 // resident blocks per SM each kernel is planned for
 int blocks_per_sm(int G) { return G == 1 ? SHA_MHA_BLOCKS_PER_SM : 1; }
 
@@ -101,6 +111,7 @@ Plan make_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int num_spl
     const int tile = tile_keys(G);
     pl.sched.tiles_per_unit = (N_kv + tile - 1) / tile;
     pl.sched.total_tiles = units * pl.sched.tiles_per_unit;
+    pl.sched.pieces = 0;
     long long ctas = num_splits > 0 ? num_splits : (long long)num_sms * blocks_per_sm(G);
     if (ctas > sha::kMaxBlocks) ctas = sha::kMaxBlocks;
     if (ctas > pl.sched.total_tiles) ctas = pl.sched.total_tiles;
@@ -111,15 +122,42 @@ Plan make_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int num_spl
     if (min_tiles > 1 && ctas > pl.sched.total_tiles / min_tiles)
         ctas = pl.sched.total_tiles / min_tiles;
     if (ctas < 1) ctas = 1;
-    if (ctas < 1) ctas = 1;
+    if (num_splits == 0 && SHA_ALIGN_UNITS) {
+        // Cut at unit boundaries when the busiest block then streams no more
+        // tiles than under the even cut plus what the merges of split units
+        // cost (kMergeCostTiles): whole units per block when there are at
+        // least as many units as blocks, else each unit in p equal pieces.
+        // (the merges sit on the critical path at the end of a short call; in a
+        // long one the other blocks' streaming hides all but about a tile)
+        const long long tpu = pl.sched.tiles_per_unit;
+        const long long even_tiles = (pl.sched.total_tiles + ctas - 1) / ctas;
+        const long long even = even_tiles + (even_tiles < 32 ? kMergeCostTiles : 1);
+        const long long blocks = (long long)num_sms * blocks_per_sm(G);
+        if (units >= blocks) {
+            if ((units + blocks - 1) / blocks * tpu <= even && blocks <= sha::kMaxBlocks) {
+                pl.sched.pieces = 1;
+                ctas = blocks;
+            }
+        } else {
+            long long p = blocks / units;
+            if (p > tpu) p = tpu;
+            if (p > sha::kMaxMergeParts) p = sha::kMaxMergeParts;
+            // pieces of one or two tiles merge as often as the even cut does
+            if ((p == 1 || tpu >= 3 * p) && (tpu + p - 1) / p <= even) {
+                pl.sched.pieces = (int)p;
+                ctas = units * p;
+            }
+        }
+    }
     pl.sched.num_ctas = (int)ctas;
     // one partial state: G rows of (O[d], m, l), padded to 128 bytes
     pl.slot_floats = ((G * (d + 2)) + 31) / 32 * 32;
     pl.counter_bytes = sha::kCounterBytes;
     pl.slot_bytes = (size_t)2 * pl.sched.num_ctas * pl.slot_floats * sizeof(float);
     // every unit held whole by one block: no partial state is needed
-    if (pl.sched.total_tiles % pl.sched.num_ctas == 0 &&
-        (pl.sched.total_tiles / pl.sched.num_ctas) % pl.sched.tiles_per_unit == 0) {
+    if (pl.sched.pieces == 1 ||
+        (pl.sched.total_tiles % pl.sched.num_ctas == 0 &&
+         (pl.sched.total_tiles / pl.sched.num_ctas) % pl.sched.tiles_per_unit == 0)) {
         pl.counter_bytes = 0;
         pl.slot_bytes = 0;
     }
@@ -272,6 +310,7 @@ Plan make_varlen_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int 
                       int num_sms)
 {
     Plan pl = make_plan(B, H_q, H_kv, N_kv, d, top_k, 0, num_sms);
+    pl.sched.pieces = 0;                    // the device plans an even cut
     long long ctas = num_splits > 0 ? num_splits : (long long)num_sms * blocks_per_sm(H_q / H_kv);
     if (ctas > sha::kMaxBlocks) ctas = sha::kMaxBlocks;
     if (ctas > pl.sched.total_tiles) ctas = pl.sched.total_tiles;

@@ -9,7 +9,9 @@
 // one per thread block.  Every block therefore streams the same number of
 // K/V bytes whatever B, top_k and N_kv are.  A unit whose tiles fall in more
 // than one piece is finished by a log-sum-exp merge of the pieces' partial
-// (m, l, O) states (see the kernels).
+// (m, l, O) states (see the kernels).  When units are only a few tiles long
+// the merges cost more than an uneven cut, and the host may instead cut at
+// unit boundaries: whole units per block, or each unit in p equal pieces.
 //
 // A unit split across blocks c_first..c_last is merged by whichever of them
 // finishes last, found with an arrival counter.  Counter c_first belongs to
@@ -34,16 +36,35 @@ struct Schedule {
     int tiles_per_unit;      // ceil(N_kv / kTile)
     long long total_tiles;   // units * tiles_per_unit
     int num_ctas;            // 1 <= num_ctas <= total_tiles
+    // 0: the tiles are cut evenly across the blocks, whatever the unit
+    // boundaries.  p >= 1: each unit is cut into p equal pieces (by tiles) and
+    // block c takes the whole pieces [c P / num_ctas, (c+1) P / num_ctas) of
+    // the P = units * p pieces, so no block starts or ends inside a piece.
+    int pieces;
 
+    // First tile of piece i of the unit-aligned cut (pieces >= 1).
+    __host__ __device__ __forceinline__ long long piece_start(long long i) const
+    {
+        const long long u = i / pieces;
+        const long long k = i - u * pieces;
+        return u * tiles_per_unit + k * tiles_per_unit / pieces;
+    }
     // First tile of block c (c in [0, num_ctas]); begin(num_ctas) == total_tiles.
     __host__ __device__ __forceinline__ long long begin(int c) const
     {
-        return (long long)c * total_tiles / num_ctas;
+        if (pieces == 0) return (long long)c * total_tiles / num_ctas;
+        const long long P = total_tiles / tiles_per_unit * pieces;
+        return piece_start((long long)c * P / num_ctas);
     }
     // The block whose range holds tile t: the largest c with begin(c) <= t.
     __host__ __device__ __forceinline__ int cta_of(long long t) const
     {
-        return (int)(((t + 1) * (long long)num_ctas - 1) / total_tiles);
+        if (pieces == 0) return (int)(((t + 1) * (long long)num_ctas - 1) / total_tiles);
+        const long long P = total_tiles / tiles_per_unit * pieces;
+        const long long u = t / tiles_per_unit, j = t - u * tiles_per_unit;
+        // the last piece of the unit that starts at or before tile j
+        const long long i = u * pieces + ((j + 1) * pieces - 1) / tiles_per_unit;
+        return (int)(((i + 1) * (long long)num_ctas - 1) / P);
     }
     __host__ __device__ __forceinline__ long long unit_of(long long t) const
     {

@@ -156,6 +156,7 @@ __device__ bool varlen_plan(const int32_t *seqlens, int B, int top_k, int n_max,
     S.tiles_per_unit = 0;                  // units differ; the walk carries their size
     S.total_tiles = total;
     S.num_ctas = (int)ctas;
+    S.pieces = 0;                          // tiles cut evenly
     if ((int)blockIdx.x >= S.num_ctas) return false;
     const long long t0 = S.begin(blockIdx.x);
 
