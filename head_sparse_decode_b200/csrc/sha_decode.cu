@@ -142,8 +142,13 @@ Plan make_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int num_spl
             long long p = blocks / units;
             if (p > tpu) p = tpu;
             if (p > sha::kMaxMergeParts) p = sha::kMaxMergeParts;
-            // pieces of one or two tiles merge as often as the even cut does
-            if ((p == 1 || tpu >= 3 * p) && (tpu + p - 1) / p <= even) {
+            // pieces of one or two tiles merge as often as the even cut does:
+            // take fewer, longer pieces
+            while (p > 1 && tpu < 3 * p) --p;
+            // pieces still merge, so they must keep most blocks streaming to
+            // beat the even cut; whole units (p = 1) merge nothing
+            if (p > 1 && 5 * units * p < 4 * blocks) p = 1;
+            if ((tpu + p - 1) / p <= even) {
                 pl.sched.pieces = (int)p;
                 ctas = units * p;
             }
