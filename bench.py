@@ -97,8 +97,9 @@ def measured_peak():
 
 # the sources the selective-head decode kernels are built from (kernels, their
 # helpers and the launch path); a change to any of them voids a stored capture
-DECODE_SOURCES = ("sha_decode.cu", "sha_device.cuh", "sha_gqa_kernel.cuh", "sha_merge.cuh",
-                  "sha_mha_kernel.cuh", "sha_mma.cuh", "sha_schedule.cuh", "sha_walk.cuh")
+DECODE_SOURCES = ("sha_decode.cu", "sha_device.cuh", "sha_gqa_kernel.cuh", "sha_lookahead.cuh",
+                  "sha_merge.cuh", "sha_mha_kernel.cuh", "sha_mma.cuh", "sha_schedule.cuh",
+                  "sha_walk.cuh")
 
 
 def kernel_source_hash():

@@ -331,14 +331,14 @@ struct StridedMaps {
     long long k_size[3], k_stride[3], v_size[3], v_stride[3];
 };
 
-template <typename T, int D, int kLayout>
+template <typename T, int D, int kLayout, bool kLook>
 sha_status_t launch_gqa(const sha::DecodeParams &prm, sha_dtype_t dtype, int dev,
                         cudaStream_t stream, const StridedMaps *kv)
 {
     using C = sha::GqaConfig<D>;
     static std::atomic<bool> configured[kMaxDevices];
     if (!configured[dev].load(std::memory_order_acquire)) {
-        cudaError_t e = cudaFuncSetAttribute(sha::sha_gqa_decode_kernel<T, D, kLayout>,
+        cudaError_t e = cudaFuncSetAttribute(sha::sha_gqa_decode_kernel<T, D, kLayout, kLook>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::kSmemBytes);
         if (e != cudaSuccess) return launch_error(e);
@@ -352,9 +352,9 @@ sha_status_t launch_gqa(const sha::DecodeParams &prm, sha_dtype_t dtype, int dev
             st = kv_tensor_map_4d(&tm_v, prm.v, dtype, D, kv->v_size, kv->v_stride, prm.tok_dim,
                                   64, C::kTile, true);
         if (st != SHA_OK) return st;
-        cudaError_t e = launch_kernel(sha::sha_gqa_decode_kernel<T, D, kLayout>,
-                                      prm.sched.num_ctas, C::kThreads, C::kSmemBytes, stream, prm,
-                                      tm_k, tm_v);
+        cudaError_t e = launch_kernel(sha::sha_gqa_decode_kernel<T, D, kLayout, kLook>,
+                                      prm.sched.num_ctas, C::threads(kLook), C::kSmemBytes, stream,
+                                      prm, tm_k, tm_v);
         if (e != cudaSuccess) return launch_error(e);
         return SHA_OK;
     }
@@ -367,20 +367,20 @@ sha_status_t launch_gqa(const sha::DecodeParams &prm, sha_dtype_t dtype, int dev
     if (st != SHA_OK) return st;
     st = kv_tensor_map(&tm_v, prm.v, dtype, D, rows, planes, box_rows);
     if (st != SHA_OK) return st;
-    cudaError_t e = launch_kernel(sha::sha_gqa_decode_kernel<T, D, kLayout>, prm.sched.num_ctas,
-                                  C::kThreads, C::kSmemBytes, stream, prm, tm_k, tm_v);
+    cudaError_t e = launch_kernel(sha::sha_gqa_decode_kernel<T, D, kLayout, kLook>, prm.sched.num_ctas,
+                                  C::threads(kLook), C::kSmemBytes, stream, prm, tm_k, tm_v);
     if (e != cudaSuccess) return launch_error(e);
     return SHA_OK;
 }
 
-template <typename T, int D, int kLayout>
+template <typename T, int D, int kLayout, bool kLook>
 sha_status_t launch_mha(const sha::DecodeParams &prm, sha_dtype_t dtype, int dev,
                         cudaStream_t stream, const StridedMaps *kv)
 {
     using C = sha::MhaConfig<D>;
     static std::atomic<bool> configured[kMaxDevices];
     if (!configured[dev].load(std::memory_order_acquire)) {
-        cudaError_t e = cudaFuncSetAttribute(sha::sha_mha_decode_kernel<T, D, kLayout>,
+        cudaError_t e = cudaFuncSetAttribute(sha::sha_mha_decode_kernel<T, D, kLayout, kLook>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::kSmemBytes);
         if (e != cudaSuccess) return launch_error(e);
@@ -398,28 +398,59 @@ sha_status_t launch_mha(const sha::DecodeParams &prm, sha_dtype_t dtype, int dev
                                   D, C::kTile, false);
         if (st != SHA_OK) return st;
     }
-    cudaError_t e = launch_kernel(sha::sha_mha_decode_kernel<T, D, kLayout>, prm.sched.num_ctas,
-                                  C::kThreads, C::kSmemBytes, stream, prm, tm_k, tm_v);
+    cudaError_t e = launch_kernel(sha::sha_mha_decode_kernel<T, D, kLayout, kLook>, prm.sched.num_ctas,
+                                  C::threads(kLook), C::kSmemBytes, stream, prm, tm_k, tm_v);
     if (e != cudaSuccess) return launch_error(e);
     return SHA_OK;
 }
 
+template <typename T, int D, int kLayout, bool kLook>
+sha_status_t launch_one(const sha::DecodeParams &prm, sha_dtype_t dtype, int G, int dev,
+                        cudaStream_t s, const StridedMaps *kv)
+{
+    return G > 1 ? launch_gqa<T, D, kLayout, kLook>(prm, dtype, dev, s, kv)
+                 : launch_mha<T, D, kLayout, kLook>(prm, dtype, dev, s, kv);
+}
+
+template <typename T, int D, int kLayout>
+sha_status_t launch_look(const sha::DecodeParams &prm, sha_dtype_t dtype, int G, bool look,
+                         int dev, cudaStream_t s, const StridedMaps *kv)
+{
+    return look ? launch_one<T, D, kLayout, true>(prm, dtype, G, dev, s, kv)
+                : launch_one<T, D, kLayout, false>(prm, dtype, G, dev, s, kv);
+}
+
 template <int kLayout>
 sha_status_t launch_decode(const sha::DecodeParams &prm, sha_dtype_t dtype, int d, int G,
-                           int dev, cudaStream_t s, const StridedMaps *kv = nullptr)
+                           bool look, int dev, cudaStream_t s, const StridedMaps *kv = nullptr)
 {
-    if (G > 1) {
-        if (dtype == SHA_FP16)
-            return d == 128 ? launch_gqa<__half, 128, kLayout>(prm, dtype, dev, s, kv)
-                            : launch_gqa<__half, 64, kLayout>(prm, dtype, dev, s, kv);
-        return d == 128 ? launch_gqa<__nv_bfloat16, 128, kLayout>(prm, dtype, dev, s, kv)
-                        : launch_gqa<__nv_bfloat16, 64, kLayout>(prm, dtype, dev, s, kv);
-    }
     if (dtype == SHA_FP16)
-        return d == 128 ? launch_mha<__half, 128, kLayout>(prm, dtype, dev, s, kv)
-                        : launch_mha<__half, 64, kLayout>(prm, dtype, dev, s, kv);
-    return d == 128 ? launch_mha<__nv_bfloat16, 128, kLayout>(prm, dtype, dev, s, kv)
-                    : launch_mha<__nv_bfloat16, 64, kLayout>(prm, dtype, dev, s, kv);
+        return d == 128 ? launch_look<__half, 128, kLayout>(prm, dtype, G, look, dev, s, kv)
+                        : launch_look<__half, 64, kLayout>(prm, dtype, G, look, dev, s, kv);
+    return d == 128 ? launch_look<__nv_bfloat16, 128, kLayout>(prm, dtype, G, look, dev, s, kv)
+                    : launch_look<__nv_bfloat16, 64, kLayout>(prm, dtype, G, look, dev, s, kv);
+}
+
+// Whether to launch the build with a scout warp (sha_lookahead.cuh): it pays
+// when blocks end with the head of a split unit whose other parts were done
+// early, as under the even cut when a unit meets at most 1 + max_partners
+// blocks.  Pieces of the unit-aligned cut all finish together, so they do
+// not qualify.  Calls with per-row lengths are planned on the device and
+// take it whenever the kernel can hold a partner's state.
+bool lookahead_pays(const Plan &pl, int G, bool device_planned)
+{
+    if (!SHA_LOOKAHEAD) return false;
+    const int max_partners = G == 1 ? sha::MhaConfig<128>::kMaxPartners
+                           : G <= sha::GqaConfig<128>::kMaxPartRows
+                               ? sha::GqaConfig<128>::kConsumerWarps - 2
+                               : 0;
+    if (max_partners == 0) return false;
+    if (device_planned) return true;
+    if (pl.sched.pieces != 0) return false;
+    const long long per_block = pl.sched.total_tiles / pl.sched.num_ctas;
+    if (per_block < 1) return false;
+    const long long parts = (pl.sched.tiles_per_unit - 1 + per_block - 1) / per_block + 1;
+    return parts >= 2 && parts - 1 <= max_partners;
 }
 
 // Where the keys of a call live beyond the plain [B, H_kv, N_kv, d] cache.
@@ -462,6 +493,7 @@ sha_status_t decode_impl(const void *q, const void *k, const void *v, const int3
                                                info->num_sms)
                             : make_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits, info->num_sms);
     const size_t need = pl.workspace_bytes();
+    const bool look = lookahead_pays(pl, G, seqlens != nullptr);
 
     if (library_workspace && need > 0) {
         OwnedWorkspace *owned = g_owned;
@@ -520,12 +552,13 @@ sha_status_t decode_impl(const void *q, const void *k, const void *v, const int3
         // one set of coordinates serves both maps
         if (vt != prm.tok_dim || vh != prm.head_dim || vb != prm.batch_dim)
             return SHA_ERR_UNSUPPORTED;
-        if (seqlens) return launch_decode<sha::kLayoutStridedVarlen>(prm, dtype, d, G, dev, s, &kv);
-        return launch_decode<sha::kLayoutStrided>(prm, dtype, d, G, dev, s, &kv);
+        if (seqlens)
+            return launch_decode<sha::kLayoutStridedVarlen>(prm, dtype, d, G, look, dev, s, &kv);
+        return launch_decode<sha::kLayoutStrided>(prm, dtype, d, G, look, dev, s, &kv);
     }
-    if (lay.block_table) return launch_decode<sha::kLayoutPaged>(prm, dtype, d, G, dev, s);
-    if (seqlens) return launch_decode<sha::kLayoutVarlen>(prm, dtype, d, G, dev, s);
-    return launch_decode<sha::kLayoutFixed>(prm, dtype, d, G, dev, s);
+    if (lay.block_table) return launch_decode<sha::kLayoutPaged>(prm, dtype, d, G, look, dev, s);
+    if (seqlens) return launch_decode<sha::kLayoutVarlen>(prm, dtype, d, G, look, dev, s);
+    return launch_decode<sha::kLayoutFixed>(prm, dtype, d, G, look, dev, s);
 }
 
 __global__ void copy_probe_kernel(uint4 *__restrict__ dst, const uint4 *__restrict__ src,

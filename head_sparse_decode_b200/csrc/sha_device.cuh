@@ -157,6 +157,19 @@ template <> struct Elem<__nv_bfloat16> {
     }
 };
 
+// Two fp32 values rounded to T and packed low/high into one 32-bit register.
+template <typename T> __device__ __forceinline__ uint32_t pack2(float lo, float hi);
+template <> __device__ __forceinline__ uint32_t pack2<__half>(float lo, float hi)
+{
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+template <> __device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float lo, float hi)
+{
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
 // Eight 16-bit elements (one 16-byte vector) widened to fp32.
 template <typename T>
 __device__ __forceinline__ void widen8(const uint4 &v, float (&f)[8])

@@ -22,7 +22,9 @@
 //   * P V: the S accumulators, exponentiated, are reused in registers as the
 //     A operand (16 keys = one k-step); V fragments come from ldmatrix.trans;
 //   * warps merge once per unit; units split across blocks merge in the
-//     workspace exactly as in the multi-head kernel.
+//     workspace exactly as in the multi-head kernel, and with G <= 8 the block
+//     finishes the split unit it ends with on chip (sha_lookahead.cuh), its
+//     parts kept in the rows G..15 that the warps' state areas leave free.
 #pragma once
 
 #include <cuda.h>
@@ -30,6 +32,7 @@
 #include <type_traits>
 
 #include "sha_device.cuh"
+#include "sha_lookahead.cuh"
 #include "sha_merge.cuh"
 #include "sha_mha_kernel.cuh"
 #include "sha_mma.cuh"
@@ -50,7 +53,9 @@ template <int D>
 struct GqaConfig {
     static constexpr int kConsumerWarps = 4;
     static constexpr int kConsumers = kConsumerWarps * 32;
-    static constexpr int kThreads = kConsumers + 32;
+    static constexpr int kThreads = kConsumers + 32;   // + one producer warp
+    // ... and a scout warp in the builds that finish a block's last unit on chip
+    static constexpr int threads(bool look) { return kThreads + (look ? 32 : 0); }
     static constexpr int kTile = SHA_GQA_TILE_KEYS;    // keys per tile (one pipeline stage)
     static constexpr int kSlices = kTile / 64;         // 64-key slices per tile
     static constexpr int kKeysPerWarp = 64 / kConsumerWarps;      // 16 per slice: one m16n8k16 k-step
@@ -66,17 +71,30 @@ struct GqaConfig {
     static constexpr int kKOffset = 0;
     static constexpr int kVOffset = kStages * kTileBytes;
     static constexpr int kBarOffset = 2 * kStages * kTileBytes;
-    static constexpr int kFlagOffset = kBarOffset + 2 * kStages * 8;
+    // ring barriers (full, empty), then the copy barrier of the on-chip merge
+    static constexpr int kFlagOffset = kBarOffset + 2 * kStages * 8 + 16;
     static constexpr int kPlanOffset = kFlagOffset + 16;       // 32 longs: per-row-length plan
     static constexpr int kStateOffset = kPlanOffset + 256;
-    static constexpr int kSmemBytes =
-        kAlignPad + kStateOffset + kConsumerWarps * kStateFloats * 4;
-    static_assert(2 * (kThreads / 32) + 8 <= 32, "plan scratch fits");
+    // on-chip merge (G <= 8): part i (0 = this block's) in rows 8..15 of warp
+    // i+1's state area, so at most 2 other parts
+    static constexpr int kMaxPartRows = 8;
+    static constexpr int kPartFloats = kStateFloats;
+    static constexpr int kPartRowOffset = kMaxPartRows * (D + 2);
+    // per query row: the warps' weights 2^(m_w - M), then M and L
+    static constexpr int kCombineFloats = kConsumerWarps + 2;
+    static constexpr int kCombineOffset = kStateOffset + kConsumerWarps * kStateFloats * 4;
+    static constexpr int kSmemBytes = kAlignPad + kCombineOffset + kRows * kCombineFloats * 4;
+    static_assert(2 * (threads(true) / 32) + 8 <= 32, "plan scratch fits");
     static_assert(kKeysPerWarp == 16, "one k-step of 16 keys per warp and slice");
     static_assert(kTile % 64 == 0 && kTile <= 256, "whole 64-key slices, TMA box <= 256 rows");
     static_assert(kBoxBytes % 1024 == 0, "boxes stay 1 KiB aligned");
     static_assert(kConsumerWarps * kStateFloats >= 3 * kMaxMergeParts * kRows,
                   "merge staging fits");
+    static_assert(kStateOffset % 16 == 0 && (kStateFloats * 4) % 16 == 0 &&
+                      (kPartRowOffset * 4) % 16 == 0,
+                  "bulk-copy alignment");
+    static_assert(3 * kMaxMergeParts * kMaxPartRows <= kStateFloats + kPartRowOffset,
+                  "merge staging for G <= 8 ends before the first part's rows");
 };
 
 // TMA tiled load of one box of a 3-D tensor map into shared memory.
@@ -101,8 +119,8 @@ __device__ __forceinline__ uint32_t swizzled(uint32_t tile, int key, int chunk)
     return tile + box * C::kBoxBytes + key * 128 + ((c ^ (key & 7)) << 4);
 }
 
-template <typename T, int D, int kLayout>
-__global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
+template <typename T, int D, int kLayout, bool kLook>
+__global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
     sha_gqa_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v)
 {
@@ -116,20 +134,29 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
     unsigned char *v_ring = smem + C::kVOffset;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOffset);
     uint64_t *empty = full + C::kStages;
+    uint64_t *part_bar = empty + C::kStages;
     volatile int *flags = reinterpret_cast<volatile int *>(smem + C::kFlagOffset);
     float *wstate = reinterpret_cast<float *>(smem + C::kStateOffset);
+    float *own_part = wstate + C::kStateFloats + C::kPartRowOffset;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int G = p.H_q / p.H_kv;
+    const int max_partners = G <= C::kMaxPartRows ? C::kConsumerWarps - 2 : 0;
+    // a part's bytes rounded up to 16: within the slot (padded to 32 floats) and
+    // within rows 8..15 (G <= 7 whenever G * (D + 2) is not a multiple of 4)
+    const uint32_t part_bytes = (uint32_t)((G * (D + 2) * 4 + 15) & ~15);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], C::kConsumerWarps);
         }
+        mbar_init(part_bar, 1);
         flags[0] = 0;
         flags[1] = 0;
+        flags[kFlagClaim] = 0;
+        flags[kFlagOnChip] = 0;
         mbar_init_fence();
     }
     __syncthreads();
@@ -140,7 +167,7 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
     Schedule S = p.sched;
     Walk walk;
     if constexpr (kVarlen) {
-        if (!varlen_plan<C::kThreads>(p.seqlens, p.B, p.top_k, p.N_kv, C::kTile, gridDim.x,
+        if (!varlen_plan<C::threads(kLook)>(p.seqlens, p.B, p.top_k, p.N_kv, C::kTile, gridDim.x,
                                       reinterpret_cast<long long *>(smem + C::kPlanOffset), S,
                                       walk))
             return;
@@ -149,6 +176,16 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
         walk.t = S.begin(blockIdx.x);
         walk.t_end = S.begin(blockIdx.x + 1);
         walk.n_keys = p.N_kv;
+    }
+
+    // ------------------------------------------------------------ scout
+    if constexpr (kLook) {
+        if (warp == C::kConsumerWarps + 1) {
+            if (lane == 0)
+                lookahead_scout(walk, S, max_partners, p.counters, p.slots, p.slot_floats,
+                                part_bytes, own_part, C::kPartFloats, flags, part_bar);
+            return;
+        }
     }
 
     // ------------------------------------------------------------ producer
@@ -429,47 +466,87 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
                 }
             }
         }
+        // blocks first..last share a split unit; the one the block ends with may
+        // be finished on chip
+        int first = 0, last = 0, first_slot = 0;
+        if (!seg.whole) unit_parts(S, seg, first, last, first_slot);
+        const int la_parts =
+            kLook && wk.t >= wk.t_end ? lookahead_parts(seg, first, last, max_partners) : 0;
+        if (la_parts && tid == 0) flags[kFlagOnChip] = lookahead_claim(flags);
+        named_barrier(1, C::kConsumers);
+        const bool on_chip = la_parts && flags[kFlagOnChip];
+
+        // the warps' weights of each query row, once: c_w = 2^(m_w - M), L = sum_w c_w l_w
+        float *cw = reinterpret_cast<float *>(smem + C::kCombineOffset);
+        if (tid < G) {
+            const float *st = wstate + tid * (D + 2);
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < C::kConsumerWarps; ++w) M = fmaxf(M, st[w * C::kStateFloats + D]);
+            const float M_ref = (M == -INFINITY) ? 0.f : M;
+            float L = 0.f;
+#pragma unroll
+            for (int w = 0; w < C::kConsumerWarps; ++w) {
+                const float c = exp2f(st[w * C::kStateFloats + D] - M_ref);
+                cw[tid * C::kCombineFloats + w] = c;
+                L = fmaf(c, st[w * C::kStateFloats + D + 1], L);
+            }
+            cw[tid * C::kCombineFloats + C::kConsumerWarps] = M;
+            cw[tid * C::kCombineFloats + C::kConsumerWarps + 1] = L;
+        }
         named_barrier(1, C::kConsumers);
 
         T *out_g = static_cast<T *>(p.out) + ((size_t)b * p.H_q + (size_t)h * G) * D;
         const bool aborted = flags[0] != 0;
-        // this block's first unit goes to slot 2c, any later partial one to 2c+1
-        float *slot = p.slots ? p.slots + (size_t)(2 * blockIdx.x + (first_seg ? 0 : 1)) *
+        // this block's first unit goes to slot 2c, any later partial one to 2c+1;
+        // on chip it is part 0, beside the copies of the others
+        float *slot = on_chip ? own_part
+                    : p.slots ? p.slots + (size_t)(2 * blockIdx.x + (first_seg ? 0 : 1)) *
                                               p.slot_floats
                               : nullptr;
         if (!aborted) {
-            for (int e = tid; e < G * D; e += C::kConsumers) {
+            // two neighbouring elements of a row per thread (D is even)
+            for (int e = 2 * tid; e < G * D; e += 2 * C::kConsumers) {
                 const int row = e / D, c = e - row * D;
-                float M = -INFINITY;
-#pragma unroll
-                for (int w = 0; w < C::kConsumerWarps; ++w)
-                    M = fmaxf(M, wstate[w * C::kStateFloats + row * (D + 2) + D]);
-                const float M_ref = (M == -INFINITY) ? 0.f : M;
-                float L = 0.f, O = 0.f;
+                const float *cr = cw + row * C::kCombineFloats;
+                float2 O = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int w = 0; w < C::kConsumerWarps; ++w) {
-                    const float *st = wstate + w * C::kStateFloats + row * (D + 2);
-                    const float cw = exp2f(st[D] - M_ref);
-                    L = fmaf(cw, st[D + 1], L);
-                    O = fmaf(cw, st[c], O);
+                    const float2 x = *reinterpret_cast<const float2 *>(
+                        wstate + w * C::kStateFloats + row * (D + 2) + c);
+                    O.x = fmaf(cr[w], x.x, O.x);
+                    O.y = fmaf(cr[w], x.y, O.y);
                 }
+                const float L = cr[C::kConsumerWarps + 1];
                 if (seg.whole) {
-                    out_g[e] = Elem<T>::from_float(O / L);
+                    *reinterpret_cast<uint32_t *>(out_g + e) = pack2<T>(O.x / L, O.y / L);
                 } else {
-                    slot[e] = O;
+                    *reinterpret_cast<float2 *>(slot + e) = O;
                     if (c == 0) {
-                        slot[G * D + row] = M;
+                        slot[G * D + row] = cr[C::kConsumerWarps];
                         slot[G * D + G + row] = L;
                     }
                 }
             }
-            if (!seg.whole) __threadfence();
+            if (!seg.whole && !on_chip) __threadfence();
         }
         named_barrier(1, C::kConsumers);
 
-        if (!seg.whole) {
-            int first, last, first_slot;
-            unit_parts(S, seg, first, last, first_slot);
+        if (on_chip) {
+            // every other part has arrived and none merged: this block merges
+            if (!mbar_wait(part_bar, 0)) {
+                atomicOr(&g_sha_status, kStatusTimeout);
+                flags[0] = 1;
+            }
+            named_barrier(1, C::kConsumers);
+            if (tid == 0) flags[1] = !flags[0];
+            named_barrier(1, C::kConsumers);
+            if (flags[1]) {
+                merge_parts<T, D, C::kConsumers>(SharedParts{own_part, C::kPartFloats}, la_parts,
+                                                  G, out_g, wstate, tid);
+                if (tid == 0) p.counters[first] = 0;
+            }
+        } else if (!seg.whole) {
             if (tid == 0) {
                 int merge = 0;
                 if (!flags[0]) {
@@ -481,12 +558,14 @@ __global__ void __launch_bounds__(GqaConfig<D>::kThreads, 1)
             named_barrier(1, C::kConsumers);
             if (flags[1]) {
                 __threadfence();
-                merge_parts<T, D, C::kConsumers>(p.slots, p.slot_floats, first, first_slot,
-                                                  last - first + 1, G, out_g, wstate, tid);
+                merge_parts<T, D, C::kConsumers>(
+                    GlobalParts{p.slots, p.slot_floats, first, first_slot}, last - first + 1, G,
+                    out_g, wstate, tid);
                 if (tid == 0) p.counters[first] = 0;
             }
         }
     }
+    if (kLook && tid == 0) lookahead_claim(flags);   // the scout stops looking
 }
 
 }  // namespace sha

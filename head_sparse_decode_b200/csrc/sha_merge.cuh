@@ -9,7 +9,8 @@
 // visiting the parts in block order so the result does not depend on which
 // block came last.  Loads are issued so that their latencies overlap: all
 // (m_s, l_s) first, staged in shared memory, then the O rows as independent
-// 16-byte loads.
+// 16-byte loads.  The parts are read from the slots, or from copies that a
+// block brought into its own shared memory ahead of time (sha_lookahead.cuh).
 #pragma once
 
 #include "sha_device.cuh"
@@ -28,11 +29,45 @@ __device__ __forceinline__ int merge_slot(int first, int first_slot, int i)
     return i == 0 ? first_slot : 2 * (first + i);
 }
 
-// All NT consumer threads of the merging block call this together.
+// Where the parts of a unit are read from.  GlobalParts: the blocks' slots
+// in the workspace (read through L2, never a stale L1 line).  SharedParts:
+// copies in this block's shared memory, part i at base + i * stride.
+struct GlobalParts {
+    const float *slots;
+    int slot_floats, first, first_slot;
+    static constexpr bool kShared = false;
+    __device__ __forceinline__ const float *operator()(int i) const
+    {
+        return slots + (size_t)merge_slot(first, first_slot, i) * slot_floats;
+    }
+};
+struct SharedParts {
+    const float *base;
+    int stride;
+    static constexpr bool kShared = true;
+    __device__ __forceinline__ const float *operator()(int i) const { return base + i * stride; }
+};
+
+template <bool kShared>
+__device__ __forceinline__ float load_part(const float *p)
+{
+    if constexpr (kShared) return *p;
+    else return __ldcg(p);
+}
+template <bool kShared>
+__device__ __forceinline__ float4 load_part4(const float *p)
+{
+    if constexpr (kShared) return *reinterpret_cast<const float4 *>(p);
+    else return __ldcg(reinterpret_cast<const float4 *>(p));
+}
+
+// All NT consumer threads of the merging block call this together.  Part i
+// holds O (G rows x D), then m (G), then l (G).  The arithmetic, and its
+// order, is the same wherever the parts are read from, so a unit merged from
+// shared-memory copies is bit-identical to one merged from the slots.
 // stage: shared scratch of at least 3 * kMaxMergeParts * G floats, free for use.
-template <typename T, int D, int NT>
-__device__ __forceinline__ void merge_parts(const float *__restrict__ slots, int slot_floats,
-                                            int first, int first_slot, int parts, int G,
+template <typename T, int D, int NT, typename Parts>
+__device__ __forceinline__ void merge_parts(const Parts &part, int parts, int G,
                                             T *__restrict__ out_rows, float *stage, int tid)
 {
     float *s_m = stage;
@@ -40,9 +75,9 @@ __device__ __forceinline__ void merge_parts(const float *__restrict__ slots, int
     float *s_w = stage + 2 * parts * G;
     for (int t = tid; t < parts * G; t += NT) {
         const int i = t / G, row = t - i * G;
-        const float *sl = slots + (size_t)merge_slot(first, first_slot, i) * slot_floats;
-        s_m[t] = __ldcg(sl + G * D + row);
-        s_l[t] = __ldcg(sl + G * D + G + row);
+        const float *sl = part(i);
+        s_m[t] = load_part<Parts::kShared>(sl + G * D + row);
+        s_l[t] = load_part<Parts::kShared>(sl + G * D + G + row);
     }
     named_barrier(1, NT);
     for (int row = tid; row < G; row += NT) {
@@ -59,18 +94,16 @@ __device__ __forceinline__ void merge_parts(const float *__restrict__ slots, int
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
         for (int i = 0; i < parts; ++i) {
-            const float *sl = slots + (size_t)merge_slot(first, first_slot, i) * slot_floats;
-            const float4 x = __ldcg(reinterpret_cast<const float4 *>(sl + e));
+            const float4 x = load_part4<Parts::kShared>(part(i) + e);
             const float w = s_w[i * G + row];
             acc.x = fmaf(w, x.x, acc.x);
             acc.y = fmaf(w, x.y, acc.y);
             acc.z = fmaf(w, x.z, acc.z);
             acc.w = fmaf(w, x.w, acc.w);
         }
-        out_rows[e + 0] = Elem<T>::from_float(acc.x);
-        out_rows[e + 1] = Elem<T>::from_float(acc.y);
-        out_rows[e + 2] = Elem<T>::from_float(acc.z);
-        out_rows[e + 3] = Elem<T>::from_float(acc.w);
+        // four elements in one 8-byte store (rows of D 16-bit elements, D % 4 == 0)
+        *reinterpret_cast<uint2 *>(out_rows + e) =
+            make_uint2(pack2<T>(acc.x, acc.y), pack2<T>(acc.z, acc.w));
     }
     named_barrier(1, NT);   // the staging area is reused by the caller's next unit
 }

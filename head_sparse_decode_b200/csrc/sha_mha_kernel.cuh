@@ -23,7 +23,9 @@
 //     q in registers, reduced with 3 shuffles; the 16-byte shared loads of 8
 //     lanes cover 128 consecutive bytes, so they are free of bank conflicts;
 //   * P.V: d/8 lanes per row, one 16-byte vector each, fp32 accumulators;
-//   * q is pre-multiplied by scale*log2(e) so every weight is one exp2f.
+//   * q is pre-multiplied by scale*log2(e) so every weight is one exp2f;
+//   * the block finishes the split unit it ends with on chip when the other
+//     parts are done in time (sha_lookahead.cuh).
 // The pages' Algorithm 1 renormalises O after every tile; this kernel keeps
 // O unnormalised and divides once at the end, which is the same quantity.
 #pragma once
@@ -32,6 +34,7 @@
 #include <type_traits>
 
 #include "sha_device.cuh"
+#include "sha_lookahead.cuh"
 #include "sha_merge.cuh"
 #include "sha_schedule.cuh"
 #include "sha_walk.cuh"
@@ -122,6 +125,8 @@ struct MhaConfig {
     static constexpr int kConsumerWarps = 8;
     static constexpr int kConsumers = kConsumerWarps * 32;
     static constexpr int kThreads = kConsumers + 32;   // + one producer warp
+    // ... and a scout warp in the builds that finish a block's last unit on chip
+    static constexpr int threads(bool look) { return kThreads + (look ? 32 : 0); }
     static constexpr int kTile = SHA_MHA_TILE_KEYS;    // keys per tile
     static constexpr int kStages = SHA_MHA_STAGES;
     static constexpr int kRowsPerWarp = kTile / kConsumerWarps;
@@ -136,19 +141,26 @@ struct MhaConfig {
     static constexpr int kKOffset = 0;
     static constexpr int kVOffset = kStages * kTileBytes;
     static constexpr int kBarOffset = 2 * kStages * kTileBytes;
-    static constexpr int kFlagOffset = kBarOffset + 2 * kStages * 8;
+    // ring barriers (full, empty), then the copy barrier of the on-chip merge
+    static constexpr int kFlagOffset = kBarOffset + 2 * kStages * 8 + 16;
     static constexpr int kPlanOffset = kFlagOffset + 16;       // 32 longs: per-row-length plan
     static constexpr int kStateOffset = kPlanOffset + 256;
-    static constexpr int kSmemBytes = kStateOffset + kConsumerWarps * kStateFloats * 4;
-    static_assert(2 * (kThreads / 32) + 8 <= 32, "plan scratch fits");
+    // the block's own part and up to kMaxPartners others, for an on-chip merge
+    static constexpr int kMaxPartners = 3;
+    static constexpr int kPartFloats = (kStateFloats + 3) / 4 * 4;
+    static constexpr uint32_t kPartBytes = kPartFloats * 4;
+    static constexpr int kPartOffset = kStateOffset + kConsumerWarps * kStateFloats * 4;
+    static constexpr int kSmemBytes = kPartOffset + (1 + kMaxPartners) * kPartBytes;
+    static_assert(kStateOffset % 16 == 0 && kPartOffset % 16 == 0, "bulk-copy alignment");
+    static_assert(2 * (threads(true) / 32) + 8 <= 32, "plan scratch fits");
     static_assert(kRowsPerWarp % 4 == 0, "score passes cover 4 rows");
     static_assert(kRowsPerWarp % kPvRowsPerIter == 0, "P.V iterations");
     static_assert(kConsumers >= D, "one consumer thread per output element");
     static_assert(kConsumerWarps * kStateFloats >= 3 * kMaxMergeParts, "merge staging fits");
 };
 
-template <typename T, int D, int kLayout>
-__global__ void __launch_bounds__(MhaConfig<D>::kThreads, SHA_MHA_BLOCKS_PER_SM)
+template <typename T, int D, int kLayout, bool kLook>
+__global__ void __launch_bounds__(MhaConfig<D>::threads(kLook), SHA_MHA_BLOCKS_PER_SM)
     sha_mha_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v)
 {
@@ -160,8 +172,10 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, SHA_MHA_BLOCKS_PER_SM)
     unsigned char *v_ring = smem + C::kVOffset;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOffset);
     uint64_t *empty = full + C::kStages;
+    uint64_t *part_bar = empty + C::kStages;
     volatile int *flags = reinterpret_cast<volatile int *>(smem + C::kFlagOffset);
     float *wstate = reinterpret_cast<float *>(smem + C::kStateOffset);
+    float *own_part = reinterpret_cast<float *>(smem + C::kPartOffset);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -171,8 +185,11 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, SHA_MHA_BLOCKS_PER_SM)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], C::kConsumerWarps);
         }
+        mbar_init(part_bar, 1);
         flags[0] = 0;   // abort: a wait gave up
         flags[1] = 0;   // this block merges the current unit
+        flags[kFlagClaim] = 0;
+        flags[kFlagOnChip] = 0;
         mbar_init_fence();
     }
     __syncthreads();
@@ -183,7 +200,7 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, SHA_MHA_BLOCKS_PER_SM)
     Schedule S = p.sched;
     Walk walk;
     if constexpr (kVarlen) {
-        if (!varlen_plan<C::kThreads>(p.seqlens, p.B, p.top_k, p.N_kv, C::kTile, gridDim.x,
+        if (!varlen_plan<C::threads(kLook)>(p.seqlens, p.B, p.top_k, p.N_kv, C::kTile, gridDim.x,
                                       reinterpret_cast<long long *>(smem + C::kPlanOffset), S,
                                       walk))
             return;
@@ -192,6 +209,16 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, SHA_MHA_BLOCKS_PER_SM)
         walk.t = S.begin(blockIdx.x);
         walk.t_end = S.begin(blockIdx.x + 1);
         walk.n_keys = p.N_kv;
+    }
+
+    // ------------------------------------------------------------ scout
+    if constexpr (kLook) {
+        if (warp == C::kConsumerWarps + 1) {
+            if (lane == 0)
+                lookahead_scout(walk, S, C::kMaxPartners, p.counters, p.slots, p.slot_floats,
+                                C::kPartBytes, own_part, C::kPartFloats, flags, part_bar);
+            return;
+        }
     }
 
     // ------------------------------------------------------------ producer
@@ -422,7 +449,15 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, SHA_MHA_BLOCKS_PER_SM)
             ws[D] = m_run;
             ws[D + 1] = l_run;
         }
+        // blocks first..last share a split unit; the one the block ends with may
+        // be finished on chip
+        int first = 0, last = 0, first_slot = 0;
+        if (!seg.whole) unit_parts(S, seg, first, last, first_slot);
+        const int la_parts =
+            kLook && wk.t >= wk.t_end ? lookahead_parts(seg, first, last, C::kMaxPartners) : 0;
+        if (la_parts && tid == 0) flags[kFlagOnChip] = lookahead_claim(flags);
         named_barrier(1, C::kConsumers);
+        const bool on_chip = la_parts && flags[kFlagOnChip];
 
         const bool aborted = flags[0] != 0;
         if (tid < D && !aborted) {
@@ -440,6 +475,13 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, SHA_MHA_BLOCKS_PER_SM)
             if (seg.whole) {
                 T *orow = static_cast<T *>(p.out) + ((size_t)b * p.H_q + h) * D;
                 orow[tid] = Elem<T>::from_float(O / L);
+            } else if (on_chip) {
+                // part 0 of the unit, beside the copies of the others
+                own_part[tid] = O;
+                if (tid == 0) {
+                    own_part[D] = M;
+                    own_part[D + 1] = L;
+                }
             } else {
                 // this block's first unit goes to slot 2c, any later partial one to 2c+1
                 float *slot = p.slots + (size_t)(2 * blockIdx.x + (first_seg ? 0 : 1)) *
@@ -454,9 +496,22 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, SHA_MHA_BLOCKS_PER_SM)
         }
         named_barrier(1, C::kConsumers);
 
-        if (!seg.whole) {
-            int first, last, first_slot;
-            unit_parts(S, seg, first, last, first_slot);
+        if (on_chip) {
+            // every other part has arrived and none merged: this block merges
+            if (!mbar_wait(part_bar, 0)) {
+                atomicOr(&g_sha_status, kStatusTimeout);
+                flags[0] = 1;
+            }
+            named_barrier(1, C::kConsumers);
+            if (tid == 0) flags[1] = !flags[0];
+            named_barrier(1, C::kConsumers);
+            if (flags[1]) {
+                T *orow = static_cast<T *>(p.out) + ((size_t)b * p.H_q + h) * D;
+                merge_parts<T, D, C::kConsumers>(SharedParts{own_part, C::kPartFloats}, la_parts,
+                                                  1, orow, wstate, tid);
+                if (tid == 0) p.counters[first] = 0;
+            }
+        } else if (!seg.whole) {
             if (tid == 0) {
                 int merge = 0;
                 if (!flags[0]) {
@@ -471,12 +526,14 @@ __global__ void __launch_bounds__(MhaConfig<D>::kThreads, SHA_MHA_BLOCKS_PER_SM)
                 // Last block to finish its piece: merge all pieces in block order.
                 __threadfence();
                 T *orow = static_cast<T *>(p.out) + ((size_t)b * p.H_q + h) * D;
-                merge_parts<T, D, C::kConsumers>(p.slots, p.slot_floats, first, first_slot,
-                                                  last - first + 1, 1, orow, wstate, tid);
+                merge_parts<T, D, C::kConsumers>(
+                    GlobalParts{p.slots, p.slot_floats, first, first_slot}, last - first + 1, 1,
+                    orow, wstate, tid);
                 if (tid == 0) p.counters[first] = 0;
             }
         }
     }
+    if (kLook && tid == 0) lookahead_claim(flags);   // the scout stops looking
 }
 
 }  // namespace sha
