@@ -267,10 +267,9 @@ __global__ void __launch_bounds__(MhaConfig<D>::threads(kLook), SHA_MHA_BLOCKS_P
                                 &full[stage], policy);
                     tma_load_4d(v_ring + stage * C::kTileBytes, &tm_v, 0, c[0], c[1], c[2],
                                 &full[stage], policy);
-                } else {
-                if (lane == 0) mbar_arrive_expect_tx(&full[stage], 2 * bytes);
-                if constexpr (kLayout == kLayoutPaged) {
+                } else if constexpr (kLayout == kLayoutPaged) {
                     // one copy per run of keys that lie in one page, a run per lane
+                    if (lane == 0) mbar_arrive_expect_tx(&full[stage], 2 * bytes);
                     __syncwarp();
                     const int32_t *bt = p.block_table + (size_t)b * p.max_pages;
                     const int ps = p.page_size;
@@ -294,11 +293,11 @@ __global__ void __launch_bounds__(MhaConfig<D>::threads(kLook), SHA_MHA_BLOCKS_P
                                       (uint32_t)(k1 - k0) * C::kRowBytes, &full[stage], policy);
                     }
                 } else {
+                    mbar_arrive_expect_tx(&full[stage], 2 * bytes);
                     bulk_copy_g2s(k_ring + stage * C::kTileBytes, kbase + (size_t)n0 * D,
                                   bytes, &full[stage], policy);
                     bulk_copy_g2s(v_ring + stage * C::kTileBytes, vbase + (size_t)n0 * D,
                                   bytes, &full[stage], policy);
-                }
                 }
                 last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
                 used |= 1u << stage;

@@ -138,6 +138,35 @@ def test_repeat_calls_are_bit_identical(sha):
     assert np.array_equal(a, b)
 
 
+@pytest.mark.parametrize("w", [
+    # even tile cut, units split between two blocks: the block holding a unit's head
+    # merges it on chip when the other part is in, through the slots otherwise
+    W("det_split_mha", B=32, H_q=32, H_kv=32, N_kv=1920, d=128, top_k=16, dtype="fp16",
+      seed=27),
+    W("det_split_gqa", B=32, H_q=64, H_kv=8, N_kv=2048, d=128, top_k=5, dtype="bf16", seed=28),
+], ids=lambda w: w.name)
+def test_split_unit_merges_are_bit_identical_under_contention(sha, w):
+    """Which path merges a split unit depends on timing; the result must not.
+    Repeats run while a large copy on another stream perturbs the blocks'
+    progress, and every repeat must give the same bits (and match the oracle)."""
+    q, k, v, idx = _on_gpu(w)
+    ref = _run(sha, w, q, k, v, idx)
+    check_sampled_units(w, q, k, v, idx, ref, n_random=48)
+    ref_bits = out_bits(ref)
+    src = torch.empty(1 << 28, dtype=torch.uint8, device="cuda")
+    dst = torch.empty_like(src)
+    side = torch.cuda.Stream()
+    for i in range(12):
+        if i % 3:
+            with torch.cuda.stream(side):
+                dst.copy_(src)
+        out = workloads.make_out(w, "cuda")
+        sha.decode(q, k, v, idx, w.scale, out)
+        torch.cuda.synchronize()
+        assert sha.sha_get_device_status() == sha.SHA_OK
+        assert np.array_equal(out_bits(out), ref_bits), i
+
+
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
 def test_single_key_returns_value_rows_exactly(sha, dtype):
     w = W("n1", B=3, H_q=8, H_kv=8, N_kv=1, d=128, top_k=4, dtype=dtype, seed=24)
