@@ -434,9 +434,10 @@ sha_status_t launch_decode(const sha::DecodeParams &prm, sha_dtype_t dtype, int 
 // Whether to launch the build with a scout warp (sha_lookahead.cuh): it pays
 // when blocks end with the head of a split unit whose other parts were done
 // early, as under the even cut when a unit meets at most 1 + max_partners
-// blocks.  Pieces of the unit-aligned cut all finish together, so they do
-// not qualify.  Calls with per-row lengths are planned on the device and
-// take it whenever the kernel can hold a partner's state.
+// blocks and each block streams a few tiles (with one or two, every part
+// finishes at the same moment).  Pieces of the unit-aligned cut all finish
+// together, so they do not qualify.  Calls with per-row lengths are planned
+// on the device and take it whenever the kernel can hold a partner's state.
 bool lookahead_pays(const Plan &pl, int G, bool device_planned)
 {
     if (!SHA_LOOKAHEAD) return false;
@@ -448,7 +449,7 @@ bool lookahead_pays(const Plan &pl, int G, bool device_planned)
     if (device_planned) return true;
     if (pl.sched.pieces != 0) return false;
     const long long per_block = pl.sched.total_tiles / pl.sched.num_ctas;
-    if (per_block < 1) return false;
+    if (per_block < 4) return false;
     const long long parts = (pl.sched.tiles_per_unit - 1 + per_block - 1) / per_block + 1;
     return parts >= 2 && parts - 1 <= max_partners;
 }
