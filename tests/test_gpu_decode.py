@@ -271,6 +271,24 @@ def test_gqa_parity(sha, w):
     check_against_oracle(w, q, k, v, idx, out)
 
 
+# Odd group sizes under the even tile cut, where a block ends with the head of a unit
+# split in two and merges it on chip: a part's G * (d + 2) floats are copied rounded
+# up to 16 bytes.
+@pytest.mark.parametrize("w", [
+    W("gqa_G3_d128", B=16, H_q=24, H_kv=8, N_kv=3000, d=128, top_k=5, dtype="bf16", seed=81),
+    W("gqa_G3_d64", B=16, H_q=24, H_kv=8, N_kv=3000, d=64, top_k=5, dtype="fp16", seed=82),
+    W("gqa_G5_d64", B=40, H_q=40, H_kv=8, N_kv=2600, d=64, top_k=4, dtype="bf16", seed=83),
+    W("gqa_G7_d128", B=32, H_q=56, H_kv=8, N_kv=2200, d=128, top_k=5, dtype="fp16", seed=84),
+    W("gqa_G7_d64", B=40, H_q=28, H_kv=4, N_kv=1700, d=64, top_k=4, dtype="bf16", seed=85),
+], ids=lambda w: w.name)
+def test_gqa_odd_group_sizes_with_split_units(sha, w):
+    q, k, v, idx = _on_gpu(w)
+    out = _run(sha, w, q, k, v, idx)
+    check_sampled_units(w, q, k, v, idx, out, n_random=64)
+    again = _run(sha, w, q, k, v, idx)
+    assert np.array_equal(out_bits(out), out_bits(again))
+
+
 @pytest.mark.parametrize("splits", [1, 3, 7, 64, 10_000])
 def test_gqa_forced_splits(sha, splits):
     w = W("gqa_splits", B=2, H_q=32, H_kv=4, N_kv=900, d=128, top_k=3, dtype="bf16", seed=47)
