@@ -8,7 +8,7 @@ import torch
 
 import oracle
 import workloads
-from parity import check_against_oracle, mlp_excess
+from parity import check_against_oracle, check_sampled_units, mlp_excess
 
 pytestmark = pytest.mark.gpu
 W = workloads.Workload
@@ -30,6 +30,25 @@ def _decode_cases(n, seed):
         cases.append((W(f"rand{i}_B{B}_G{G}_Hkv{H_kv}_N{N_kv}_d{d}_k{top_k}_{dtype}", B=B,
                         H_q=G * H_kv, H_kv=H_kv, N_kv=N_kv, d=d, top_k=top_k, dtype=dtype,
                         seed=9000 + i), splits))
+    return cases
+
+
+def _split_regime_cases(n, seed):
+    """More units than blocks and units a few tiles long: the even tile cut, with
+    most blocks ending on the head of a unit split in two (merged on chip)."""
+    rng = np.random.default_rng(seed)
+    cases = []
+    for i in range(n):
+        G = int(rng.integers(1, 9))
+        H_kv = int(rng.choice([4, 8, 16]))
+        d = int(rng.choice([64, 128]))
+        N_kv = int(rng.integers(600, 3001))
+        top_k = int(rng.integers(max(1, H_kv // 2), H_kv + 1))
+        B = int(rng.integers(16, 49))
+        dtype = str(rng.choice(["fp16", "bf16"]))
+        cases.append(W(f"split{i}_B{B}_G{G}_Hkv{H_kv}_N{N_kv}_d{d}_k{top_k}_{dtype}", B=B,
+                       H_q=G * H_kv, H_kv=H_kv, N_kv=N_kv, d=d, top_k=top_k, dtype=dtype,
+                       seed=9700 + i))
     return cases
 
 
@@ -71,6 +90,23 @@ def test_random_decode_shape(sha, w, splits):
     torch.cuda.synchronize()
     assert sha.sha_get_device_status() == sha.SHA_OK
     check_against_oracle(w, q, k, v, idx, out)
+
+
+@pytest.mark.parametrize("w", _split_regime_cases(16, 2468), ids=lambda w: w.name)
+def test_random_split_regime_shape(sha, w):
+    q, k, v = workloads.make_qkv(w)
+    idx = workloads.make_index(w)
+    dev = torch.device("cuda")
+    q, k, v, idx = q.to(dev), k.to(dev), v.to(dev), idx.to(dev)
+    outs = []
+    for _ in range(2):
+        out = workloads.make_out(w, "cuda")
+        sha.decode(q, k, v, idx, w.scale, out)
+        torch.cuda.synchronize()
+        assert sha.sha_get_device_status() == sha.SHA_OK
+        outs.append(out)
+    check_sampled_units(w, q, k, v, idx, outs[0], n_random=32)
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
 
 
 @pytest.mark.parametrize("w,act", _mlp_cases(16, 4321), ids=lambda c: getattr(c, "name", str(c)))
