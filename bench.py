@@ -382,7 +382,9 @@ def run_ours(args, rank, world, local):
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": profiled_traffic(w.name) if args.layout == "head_major" else None,
                      "peak_source": peak_src,
-                     "kernel": "sha_mha_decode_kernel" if w.G == 1 else "sha_gqa_decode_kernel",
+                     # multi-head calls with d = 128 run on the grouped kernel's tensor cores
+                     "kernel": "sha_mha_decode_kernel" if w.G == 1 and w.d != 128
+                               else "sha_gqa_decode_kernel",
                      "launch_us": round(launch_s * 1e6, 3),
                      "bytes_per_launch": bytes_step},
     }

@@ -96,23 +96,50 @@ struct Plan {
 #endif
 constexpr long long kMergeCostTiles = SHA_MERGE_COST_TILES;
 
-// resident blocks per SM each kernel is planned for
-int blocks_per_sm(int G) { return G == 1 ? SHA_MHA_BLOCKS_PER_SM : 1; }
+// Multi-head calls (G = 1) with d = 128 and one length for every row run on
+// the grouped kernel's tensor-core path, one query row of the 16 an MMA
+// covers.  Under the power cap that a sustained decode load holds the GPU at,
+// it is 3-6 % faster than the FMA kernel (fewer instructions per byte).  The
+// FMA kernel keeps d = 64 and per-row lengths (paged caches included), where
+// it is faster.
+#ifndef SHA_MHA_TENSOR_CORES
+#define SHA_MHA_TENSOR_CORES 1
+#endif
 
-// keys per tile of the kernel that serves G query heads per KV head
-int tile_keys(int G) { return G == 1 ? sha::MhaConfig<128>::kTile : sha::GqaConfig<128>::kTile; }
+// whether a call runs on the multi-head FMA kernel
+bool fma_path(int G, int d, bool per_row_lengths)
+{
+    return G == 1 && !(SHA_MHA_TENSOR_CORES && d == 128 && !per_row_lengths);
+}
+
+// pages the grouped kernel loads as whole TMA boxes: powers of two from 8 keys
+bool boxable_pages(int page_size) { return page_size >= 8 && (page_size & (page_size - 1)) == 0; }
+
+// resident blocks per SM each kernel is planned for
+int blocks_per_sm(int G, int d, bool per_row_lengths)
+{
+    return fma_path(G, d, per_row_lengths) ? SHA_MHA_BLOCKS_PER_SM : 1;
+}
+
+// keys per tile of the kernel that serves the call
+int tile_keys(int G, int d, bool per_row_lengths)
+{
+    return fma_path(G, d, per_row_lengths) ? sha::MhaConfig<128>::kTile
+                                           : sha::GqaConfig<128>::kTile;
+}
 
 Plan make_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int num_splits,
-               int num_sms)
+               int num_sms, bool per_row_lengths = false)
 {
     Plan pl;
     const int G = H_q / H_kv;
     const long long units = (long long)B * top_k;
-    const int tile = tile_keys(G);
+    const int tile = tile_keys(G, d, per_row_lengths);
     pl.sched.tiles_per_unit = (N_kv + tile - 1) / tile;
     pl.sched.total_tiles = units * pl.sched.tiles_per_unit;
     pl.sched.pieces = 0;
-    long long ctas = num_splits > 0 ? num_splits : (long long)num_sms * blocks_per_sm(G);
+    long long ctas =
+        num_splits > 0 ? num_splits : (long long)num_sms * blocks_per_sm(G, d, per_row_lengths);
     if (ctas > sha::kMaxBlocks) ctas = sha::kMaxBlocks;
     if (ctas > pl.sched.total_tiles) ctas = pl.sched.total_tiles;
     // every block gets at least ceil((Tu-1)/(kMaxMergeParts-1)) tiles, so a
@@ -132,7 +159,7 @@ Plan make_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int num_spl
         const long long tpu = pl.sched.tiles_per_unit;
         const long long even_tiles = (pl.sched.total_tiles + ctas - 1) / ctas;
         const long long even = even_tiles + (even_tiles < 32 ? kMergeCostTiles : 1);
-        const long long blocks = (long long)num_sms * blocks_per_sm(G);
+        const long long blocks = (long long)num_sms * blocks_per_sm(G, d, per_row_lengths);
         if (units >= blocks) {
             if ((units + blocks - 1) / blocks * tpu <= even && blocks <= sha::kMaxBlocks) {
                 pl.sched.pieces = 1;
@@ -314,9 +341,10 @@ void order_outer_dims(const KvStrides &st, int B, int H_kv, int N_kv, long long 
 Plan make_varlen_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int num_splits,
                       int num_sms)
 {
-    Plan pl = make_plan(B, H_q, H_kv, N_kv, d, top_k, 0, num_sms);
+    Plan pl = make_plan(B, H_q, H_kv, N_kv, d, top_k, 0, num_sms, true);
     pl.sched.pieces = 0;                    // the device plans an even cut
-    long long ctas = num_splits > 0 ? num_splits : (long long)num_sms * blocks_per_sm(H_q / H_kv);
+    long long ctas = num_splits > 0 ? num_splits
+                                    : (long long)num_sms * blocks_per_sm(H_q / H_kv, d, true);
     if (ctas > sha::kMaxBlocks) ctas = sha::kMaxBlocks;
     if (ctas > pl.sched.total_tiles) ctas = pl.sched.total_tiles;
     if (ctas < 1) ctas = 1;
@@ -405,30 +433,31 @@ sha_status_t launch_mha(const sha::DecodeParams &prm, sha_dtype_t dtype, int dev
 }
 
 template <typename T, int D, int kLayout, bool kLook>
-sha_status_t launch_one(const sha::DecodeParams &prm, sha_dtype_t dtype, int G, int dev,
+sha_status_t launch_one(const sha::DecodeParams &prm, sha_dtype_t dtype, bool fma, int dev,
                         cudaStream_t s, const StridedMaps *kv)
 {
-    return G > 1 ? launch_gqa<T, D, kLayout, kLook>(prm, dtype, dev, s, kv)
-                 : launch_mha<T, D, kLayout, kLook>(prm, dtype, dev, s, kv);
+    return fma ? launch_mha<T, D, kLayout, kLook>(prm, dtype, dev, s, kv)
+               : launch_gqa<T, D, kLayout, kLook>(prm, dtype, dev, s, kv);
 }
 
 template <typename T, int D, int kLayout>
-sha_status_t launch_look(const sha::DecodeParams &prm, sha_dtype_t dtype, int G, bool look,
+sha_status_t launch_look(const sha::DecodeParams &prm, sha_dtype_t dtype, bool fma, bool look,
                          int dev, cudaStream_t s, const StridedMaps *kv)
 {
-    return look ? launch_one<T, D, kLayout, true>(prm, dtype, G, dev, s, kv)
-                : launch_one<T, D, kLayout, false>(prm, dtype, G, dev, s, kv);
+    return look ? launch_one<T, D, kLayout, true>(prm, dtype, fma, dev, s, kv)
+                : launch_one<T, D, kLayout, false>(prm, dtype, fma, dev, s, kv);
 }
 
+// fma: the multi-head FMA kernel, else the grouped kernel; look: its scout build
 template <int kLayout>
-sha_status_t launch_decode(const sha::DecodeParams &prm, sha_dtype_t dtype, int d, int G,
+sha_status_t launch_decode(const sha::DecodeParams &prm, sha_dtype_t dtype, int d, bool fma,
                            bool look, int dev, cudaStream_t s, const StridedMaps *kv = nullptr)
 {
     if (dtype == SHA_FP16)
-        return d == 128 ? launch_look<__half, 128, kLayout>(prm, dtype, G, look, dev, s, kv)
-                        : launch_look<__half, 64, kLayout>(prm, dtype, G, look, dev, s, kv);
-    return d == 128 ? launch_look<__nv_bfloat16, 128, kLayout>(prm, dtype, G, look, dev, s, kv)
-                    : launch_look<__nv_bfloat16, 64, kLayout>(prm, dtype, G, look, dev, s, kv);
+        return d == 128 ? launch_look<__half, 128, kLayout>(prm, dtype, fma, look, dev, s, kv)
+                        : launch_look<__half, 64, kLayout>(prm, dtype, fma, look, dev, s, kv);
+    return d == 128 ? launch_look<__nv_bfloat16, 128, kLayout>(prm, dtype, fma, look, dev, s, kv)
+                    : launch_look<__nv_bfloat16, 64, kLayout>(prm, dtype, fma, look, dev, s, kv);
 }
 
 // Whether to launch the build with a scout warp (sha_lookahead.cuh): it pays
@@ -438,10 +467,10 @@ sha_status_t launch_decode(const sha::DecodeParams &prm, sha_dtype_t dtype, int 
 // finishes at the same moment).  Pieces of the unit-aligned cut all finish
 // together, so they do not qualify.  Calls with per-row lengths are planned
 // on the device and take it whenever the kernel can hold a partner's state.
-bool lookahead_pays(const Plan &pl, int G, bool device_planned)
+bool lookahead_pays(const Plan &pl, int G, bool fma, bool device_planned)
 {
     if (!SHA_LOOKAHEAD) return false;
-    const int max_partners = G == 1 ? sha::MhaConfig<128>::kMaxPartners
+    const int max_partners = fma ? sha::MhaConfig<128>::kMaxPartners
                            : G <= sha::GqaConfig<128>::kMaxPartRows
                                ? sha::GqaConfig<128>::kConsumerWarps - 2
                                : 0;
@@ -494,7 +523,8 @@ sha_status_t decode_impl(const void *q, const void *k, const void *v, const int3
                                                info->num_sms)
                             : make_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits, info->num_sms);
     const size_t need = pl.workspace_bytes();
-    const bool look = lookahead_pays(pl, G, seqlens != nullptr);
+    const bool fma = fma_path(G, d, seqlens != nullptr);   // paged calls carry lengths too
+    const bool look = lookahead_pays(pl, G, fma, seqlens != nullptr);
 
     if (library_workspace && need > 0) {
         OwnedWorkspace *owned = g_owned;
@@ -554,12 +584,12 @@ sha_status_t decode_impl(const void *q, const void *k, const void *v, const int3
         if (vt != prm.tok_dim || vh != prm.head_dim || vb != prm.batch_dim)
             return SHA_ERR_UNSUPPORTED;
         if (seqlens)
-            return launch_decode<sha::kLayoutStridedVarlen>(prm, dtype, d, G, look, dev, s, &kv);
-        return launch_decode<sha::kLayoutStrided>(prm, dtype, d, G, look, dev, s, &kv);
+            return launch_decode<sha::kLayoutStridedVarlen>(prm, dtype, d, fma, look, dev, s, &kv);
+        return launch_decode<sha::kLayoutStrided>(prm, dtype, d, fma, look, dev, s, &kv);
     }
-    if (lay.block_table) return launch_decode<sha::kLayoutPaged>(prm, dtype, d, G, look, dev, s);
-    if (seqlens) return launch_decode<sha::kLayoutVarlen>(prm, dtype, d, G, look, dev, s);
-    return launch_decode<sha::kLayoutFixed>(prm, dtype, d, G, look, dev, s);
+    if (lay.block_table) return launch_decode<sha::kLayoutPaged>(prm, dtype, d, fma, look, dev, s);
+    if (seqlens) return launch_decode<sha::kLayoutVarlen>(prm, dtype, d, fma, look, dev, s);
+    return launch_decode<sha::kLayoutFixed>(prm, dtype, d, fma, look, dev, s);
 }
 
 __global__ void copy_probe_kernel(uint4 *__restrict__ dst, const uint4 *__restrict__ src,
@@ -630,8 +660,7 @@ sha_status_t sha_decode_paged(const void *q, const void *k_pages, const void *v_
 {
     if (num_pages < 1 || page_size < 1 || max_pages < 1) return SHA_ERR_INVALID_ARG;
     if ((long long)max_pages * page_size > (1 << 30)) return SHA_ERR_INVALID_ARG;
-    if (H_kv >= 1 && H_q % H_kv == 0 && H_q / H_kv > 1 &&
-        (page_size < 8 || (page_size & (page_size - 1)) != 0))
+    if (H_kv >= 1 && H_q % H_kv == 0 && H_q / H_kv > 1 && !boxable_pages(page_size))
         return SHA_ERR_UNSUPPORTED;   // TMA boxes of whole pages: powers of two >= 8
     if (B > 0 && top_k > 0 && (!seqlens || !block_table)) return SHA_ERR_INVALID_ARG;
     KvLayout lay;
@@ -685,7 +714,7 @@ sha_status_t sha_decode_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_
     sha_status_t st = check_shape(B, H_q, H_kv, N_kv, d, top_k, 1.0f);
     if (st != SHA_OK) return st;
     if (num_splits < 0 || num_sms < 1 || !plan) return SHA_ERR_INVALID_ARG;
-    const int tile = tile_keys(H_q / H_kv);
+    const int tile = tile_keys(H_q / H_kv, d, false);
     if (B == 0 || top_k == 0) {
         plan[0] = (N_kv + tile - 1) / tile;
         plan[1] = plan[2] = plan[3] = 0;
