@@ -1,4 +1,5 @@
-// sha_gqa_kernel.cuh -- selective decode for grouped-query attention (G > 1).
+// sha_gqa_kernel.cuh -- selective decode for grouped-query attention (G > 1),
+// and for multi-head attention (G = 1) at d = 128 with one length per row.
 //
 // What one thread block does.  As in the multi-head kernel, it walks a
 // contiguous range of key tiles (sha_schedule.cuh).  Here a unit is a batch
@@ -21,6 +22,10 @@
 //     swizzled tile (conflict-free);
 //   * P V: the S accumulators, exponentiated, are reused in registers as the
 //     A operand (16 keys = one k-step); V fragments come from ldmatrix.trans;
+//   * with G = 1, fifteen of the sixteen MMA rows are padding, yet the path
+//     issues far fewer instructions per byte than the multi-head FMA kernel
+//     and holds its speed under the power cap of a sustained load, so the host
+//     sends multi-head calls with d = 128 and one length per row here;
 //   * warps merge once per unit; units split across blocks merge in the
 //     workspace exactly as in the multi-head kernel, and with G <= 8 the block
 //     finishes the split unit it ends with on chip (sha_lookahead.cuh), its

@@ -1,4 +1,6 @@
-// sha_mha_kernel.cuh -- selective head decode for multi-head attention (G = 1).
+// sha_mha_kernel.cuh -- selective head decode for multi-head attention (G = 1)
+// with d = 64, per-row lengths or a paged cache (the host sends d = 128 calls
+// with one length per row to the grouped kernel's tensor cores, sha_gqa_kernel.cuh).
 //
 // What one thread block does.  It owns a contiguous range of key tiles (see
 // sha_schedule.cuh) and walks it one unit (batch row b, selected head h) at a
