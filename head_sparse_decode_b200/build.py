@@ -19,7 +19,6 @@ NVCC_FLAGS = [
     "-O3", "-lineinfo", "-std=c++17",
     "--expt-relaxed-constexpr",
     "-Xcompiler", "-fPIC,-O2,-Wall",
-    "-shared",
 ]
 
 
@@ -38,11 +37,24 @@ def build(force: bool = False, verbose: bool = False, defines=(), output=None) -
         newest = max(os.path.getmtime(p) for p in _sources())
         if os.path.getmtime(library) >= newest:
             return library
+    # each .cu is its own translation unit (its kernels are launched from it),
+    # so the objects compile side by side and link without relocatable device code
     cmd = [NVCC, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, *[f"-D{d}" for d in defines]]
     if verbose:
         cmd += ["-Xptxas", "-v"]
-    cmd += ["-o", library + ".tmp", *sorted(glob.glob(os.path.join(CSRC, "*.cu")))]
-    subprocess.run(cmd, check=True)
+    sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    objects = [f"{library}.{os.path.basename(src)}.o" for src in sources]
+    procs = [subprocess.Popen(cmd + ["-c", "-o", obj, src]) for src, obj in zip(sources, objects)]
+    failed = [src for src, proc in zip(sources, procs) if proc.wait() != 0]
+    try:
+        if failed:
+            raise subprocess.CalledProcessError(1, failed)
+        subprocess.run([NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared",
+                        "-o", library + ".tmp", *objects], check=True)
+    finally:
+        for obj in objects:
+            if os.path.exists(obj):
+                os.remove(obj)
     os.replace(library + ".tmp", library)
     return library
 
