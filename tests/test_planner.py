@@ -1,0 +1,59 @@
+"""The decode planner's choices, on the host (no GPU): which cut a call gets on
+a 148-SM part, and invariants of every plan.  The expected cuts are the ones
+measured fastest on B200 (even tile cut for long calls, whole units or equal
+pieces of units for short ones)."""
+import math
+
+import pytest
+
+import head_sparse_decode_b200 as sha
+
+# (B, H_q, H_kv, N_kv, d, top_k) -> (blocks, whole units: no workspace)
+CUTS = {
+    # long calls: the even tile cut, units split across neighbouring blocks
+    "opt66b": ((64, 72, 72, 1920, 128, 22), 148, False),
+    "llama2_7b": ((128, 32, 32, 2048, 128, 16), 148, False),
+    "llama31_70b_gqa": ((32, 64, 8, 4096, 128, 5), 148, False),
+    "llama31_70b_gqa_16k": ((8, 64, 8, 16384, 128, 5), 148, False),
+    # whole units per block: no split, no merge, no workspace
+    "b8_n512_k8": ((8, 32, 32, 512, 128, 8), 64, True),      # 64 blocks of 4 tiles
+    "b8_n512_k16": ((8, 32, 32, 512, 128, 16), 128, True),
+    "b64_n512_k8": ((64, 32, 32, 512, 128, 8), 148, True),   # 3 or 4 units per block
+    # each unit in p equal pieces of at least 3 tiles
+    "b1_n1920_k24": ((1, 32, 32, 1920, 128, 24), 120, False),  # p = 5
+    "b1_n8192_k32": ((1, 32, 32, 8192, 128, 32), 128, False),  # p = 4
+    # pieces would leave too many SMs idle or be too short: the even cut
+    "b1_n1920_k16": ((1, 32, 32, 1920, 128, 16), 148, False),
+    "b1_n512_k32": ((1, 32, 32, 512, 128, 32), 128, False),    # one tile per block
+}
+
+
+@pytest.mark.parametrize("name", sorted(CUTS))
+def test_cut_of_measured_shapes(name):
+    args, blocks, whole = CUTS[name]
+    p = sha.sha_decode_plan(*args, num_sms=148)
+    assert p["blocks"] == blocks
+    assert (p["workspace_bytes"] == 0) == whole
+
+
+def test_forced_split_count_is_kept():
+    p = sha.sha_decode_plan(4, 8, 8, 640, 128, 2, num_splits=7, num_sms=148)
+    assert p["blocks"] == 7 and p["workspace_bytes"] > 0
+
+
+@pytest.mark.parametrize("G", [1, 8])
+@pytest.mark.parametrize("d", [64, 128])
+def test_plan_invariants(G, d):
+    for B in (1, 3, 8, 32, 64, 256):
+        for N in (1, 100, 512, 1920, 4096, 16384):
+            for k in (1, 4, 8):
+                H_kv = 8
+                p = sha.sha_decode_plan(B, G * H_kv, H_kv, N, d, k, num_sms=148)
+                tiles = math.ceil(N / 128)
+                assert p["tiles_per_head"] == tiles and p["tile_keys"] == 128
+                assert p["total_tiles"] == B * k * tiles
+                assert 1 <= p["blocks"] <= min(4096, p["total_tiles"])
+                # a workspace, when needed, holds the counters and two slots per block
+                ws = p["workspace_bytes"]
+                slot_bytes = math.ceil(G * (d + 2) / 32) * 32 * 4
+                assert ws == 0 or ws >= 4096 * 4 + 2 * p["blocks"] * slot_bytes
