@@ -77,6 +77,12 @@ sha_status_t current_device(int *dev, DeviceInfo **info)
     return SHA_OK;
 }
 
+// Co-resident thread-block clusters of each size of the clustered grouped
+// kernel (index = blocks per cluster, 2..kClusterMax; 0 where none fit).
+struct ClusterCaps {
+    int n[sha::GqaConfig<128>::kClusterMax + 1];
+};
+
 // The call's plan: tile schedule and workspace layout.
 struct Plan {
     sha::Schedule sched;
@@ -95,6 +101,49 @@ struct Plan {
 #define SHA_MERGE_COST_TILES 2
 #endif
 constexpr long long kMergeCostTiles = SHA_MERGE_COST_TILES;
+
+// The clustered cut (Schedule::cluster): 1 lets the planner choose it for the
+// grouped kernel's fixed-length calls where it is estimated faster, 0 never.
+#ifndef SHA_CLUSTER_CUT
+#define SHA_CLUSTER_CUT 1
+#endif
+
+// Cost model of a call's cuts (ns), measured on B200 with per-block timer
+// stamps and CUDA-graph timings: a block streams a 64 KiB K+V tile in about
+// kBlockTileNs at best (80 blocks of a GQA call at 16K context streamed at
+// 64 GB/s each); all blocks together share the HBM rate; a unit split across
+// blocks and merged through the workspace adds kSlotMergeNs at the end of the
+// call (partial write, fence, arrival atomic, reading the parts back), and a
+// unit merged in a cluster's shared memory adds kClusterMergeNs.
+constexpr double kBlockTileNs = 1000.0;
+constexpr double kHbmBytesPerNs = 6500.0;
+#ifndef SHA_SLOT_MERGE_NS
+#define SHA_SLOT_MERGE_NS 3500
+#endif
+#ifndef SHA_CLUSTER_MERGE_NS
+#define SHA_CLUSTER_MERGE_NS 2000
+#endif
+
+// Whether the clustered kernel can stage a unit's parts for clusters of c
+// blocks: each block receives every part's slice of its share of the G x d
+// outputs (plus m and l), two units' worth, in the rows 8..15 of its four
+// warps' state areas (two per unit, the first (c+1)/2 parts in one).
+bool cluster_stage_fits(int G, int d, int c)
+{
+    const int groups = G * d / 4;
+    const int stride = 4 * ((groups + c - 1) / c) + 4 * ((2 * G + 3) / 4);
+    const int region = sha::GqaConfig<128>::kMaxPartRows * (d + 2);
+    return G <= sha::GqaConfig<128>::kMaxPartRows && (c + 1) / 2 * stride <= region;
+}
+
+// Streaming time of a cut whose busiest of `active` blocks streams max_tiles
+// tiles of tile_bytes each.
+double stream_ns(long long max_tiles, long long active, double tile_bytes)
+{
+    const double per_tile = std::fmax(kBlockTileNs * tile_bytes / 65536.0,
+                                      (double)active * tile_bytes / kHbmBytesPerNs);
+    return (double)max_tiles * per_tile;
+}
 
 // Multi-head calls (G = 1) with d = 128 and one length for every row run on
 // the grouped kernel's tensor-core path, one query row of the 16 an MMA
@@ -129,7 +178,7 @@ int tile_keys(int G, int d, bool per_row_lengths)
 }
 
 Plan make_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int num_splits,
-               int num_sms, bool per_row_lengths = false)
+               int num_sms, bool per_row_lengths = false, const ClusterCaps *caps = nullptr)
 {
     Plan pl;
     const int G = H_q / H_kv;
@@ -138,6 +187,8 @@ Plan make_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int num_spl
     pl.sched.tiles_per_unit = (N_kv + tile - 1) / tile;
     pl.sched.total_tiles = units * pl.sched.tiles_per_unit;
     pl.sched.pieces = 0;
+    pl.sched.cluster = 0;
+    pl.sched.units_per_cluster = 0;
     long long ctas =
         num_splits > 0 ? num_splits : (long long)num_sms * blocks_per_sm(G, d, per_row_lengths);
     if (ctas > sha::kMaxBlocks) ctas = sha::kMaxBlocks;
@@ -182,18 +233,69 @@ Plan make_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int num_spl
         }
     }
     pl.sched.num_ctas = (int)ctas;
+    // The clustered cut, for calls with fewer units than blocks (whole units
+    // per block would leave SMs idle; pieces merged through the workspace pay
+    // a merge tail that grows with the parts): one unit per cluster of c
+    // blocks, all clusters in one wave, each block streaming one piece, the
+    // pieces merged in the cluster's shared memory.  Taken where the cost
+    // model rates it faster than whole units per block.
+    const long long blocks_avail = (long long)num_sms * blocks_per_sm(G, d, per_row_lengths);
+    if (num_splits == 0 && SHA_CLUSTER_CUT && caps && units < blocks_avail &&
+        !fma_path(G, d, per_row_lengths)) {
+        const long long tpu = pl.sched.tiles_per_unit;
+        const double tile_bytes = 2.0 * tile * d * 2;
+        double best = stream_ns(tpu, units, tile_bytes);      // whole units, no merge
+        for (int c = 2; c <= sha::GqaConfig<128>::kClusterMax && c <= tpu; ++c) {
+            if (caps->n[c] < units || !cluster_stage_fits(G, d, c)) continue;
+            const double est =
+                stream_ns((tpu + c - 1) / c, units * c, tile_bytes) + SHA_CLUSTER_MERGE_NS;
+            if (est < best) {
+                best = est;
+                pl.sched.cluster = c;
+                pl.sched.units_per_cluster = 1;
+                pl.sched.num_ctas = (int)(units * c);
+                pl.sched.pieces = 0;
+            }
+        }
+    }
     // one partial state: G rows of (O[d], m, l), padded to 128 bytes
     pl.slot_floats = ((G * (d + 2)) + 31) / 32 * 32;
     pl.counter_bytes = sha::kCounterBytes;
     pl.slot_bytes = (size_t)2 * pl.sched.num_ctas * pl.slot_floats * sizeof(float);
-    // every unit held whole by one block: no partial state is needed
-    if (pl.sched.pieces == 1 ||
+    // every unit held whole by one block, or merged on chip: no workspace
+    if (pl.sched.pieces == 1 || pl.sched.cluster >= 2 ||
         (pl.sched.total_tiles % pl.sched.num_ctas == 0 &&
          (pl.sched.total_tiles / pl.sched.num_ctas) % pl.sched.tiles_per_unit == 0)) {
         pl.counter_bytes = 0;
         pl.slot_bytes = 0;
     }
     return pl;
+}
+
+// A clustered cut chosen by the caller: clusters of `cluster` blocks, each
+// taking `units_per_cluster` whole units.  SHA_ERR_UNSUPPORTED where the
+// clustered kernel cannot serve the call, SHA_ERR_INVALID_ARG for sizes out
+// of range.
+sha_status_t forced_cluster_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k,
+                                 int cluster, int units_per_cluster, Plan &pl)
+{
+    const int G = H_q / H_kv;
+    if (G > sha::GqaConfig<128>::kMaxPartRows || fma_path(G, d, false)) return SHA_ERR_UNSUPPORTED;
+    pl = make_plan(B, H_q, H_kv, N_kv, d, top_k, 0, 1);
+    const long long units = (long long)B * top_k;
+    if (cluster < 2 || cluster > sha::GqaConfig<128>::kClusterMax ||
+        cluster > pl.sched.tiles_per_unit || units_per_cluster < 1)
+        return SHA_ERR_INVALID_ARG;
+    if (!cluster_stage_fits(G, d, cluster)) return SHA_ERR_UNSUPPORTED;
+    const long long clusters = (units + units_per_cluster - 1) / units_per_cluster;
+    if (clusters * cluster > sha::kMaxBlocks) return SHA_ERR_INVALID_ARG;
+    pl.sched.cluster = cluster;
+    pl.sched.units_per_cluster = units_per_cluster;
+    pl.sched.num_ctas = (int)(clusters * cluster);
+    pl.sched.pieces = 0;
+    pl.counter_bytes = 0;
+    pl.slot_bytes = 0;
+    return SHA_OK;
 }
 
 static_assert(sha::MhaConfig<128>::kTile == sha::MhaConfig<64>::kTile &&
@@ -207,21 +309,37 @@ static_assert(sha::MhaConfig<128>::kTile == sha::MhaConfig<64>::kTile &&
 // Launch with programmatic stream serialization: the kernel may be scheduled
 // while the previous kernel in the stream finishes, and waits for it on the
 // device (griddepcontrol.wait) before reading any input.
+// cluster > 1: the grid is launched as thread-block clusters of that many blocks.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_kernel(void (*kernel)(KArgs...), int grid, int block, size_t smem,
-                          cudaStream_t stream, Args &&...args)
+cudaError_t launch_kernel_cluster(void (*kernel)(KArgs...), int grid, int block, size_t smem,
+                                  cudaStream_t stream, int cluster, Args &&...args)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(block);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = SHA_USE_PDL;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (cluster > 1) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = cluster;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
+    }
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), int grid, int block, size_t smem,
+                          cudaStream_t stream, Args &&...args)
+{
+    return launch_kernel_cluster(kernel, grid, block, smem, stream, 0,
+                                 std::forward<Args>(args)...);
 }
 
 // cuTensorMapEncodeTiled from the driver, found through the runtime so the
@@ -395,8 +513,10 @@ sha_status_t launch_gqa(const sha::DecodeParams &prm, sha_dtype_t dtype, int dev
     if (st != SHA_OK) return st;
     st = kv_tensor_map(&tm_v, prm.v, dtype, D, rows, planes, box_rows);
     if (st != SHA_OK) return st;
-    cudaError_t e = launch_kernel(sha::sha_gqa_decode_kernel<T, D, kLayout, kLook>, prm.sched.num_ctas,
-                                  C::threads(kLook), C::kSmemBytes, stream, prm, tm_k, tm_v);
+    cudaError_t e = launch_kernel_cluster(
+        sha::sha_gqa_decode_kernel<T, D, kLayout, kLook>, prm.sched.num_ctas, C::threads(kLook),
+        C::kSmemBytes, stream, kLayout == sha::kLayoutCluster ? prm.sched.cluster : 0, prm, tm_k,
+        tm_v);
     if (e != cudaSuccess) return launch_error(e);
     return SHA_OK;
 }
@@ -448,6 +568,15 @@ sha_status_t launch_look(const sha::DecodeParams &prm, sha_dtype_t dtype, bool f
                 : launch_one<T, D, kLayout, false>(prm, dtype, fma, dev, s, kv);
 }
 
+// The clustered cut: the grouped kernel only, no scout.
+template <typename T>
+sha_status_t launch_cluster(const sha::DecodeParams &prm, sha_dtype_t dtype, int d, int dev,
+                            cudaStream_t s)
+{
+    return d == 128 ? launch_gqa<T, 128, sha::kLayoutCluster, false>(prm, dtype, dev, s, nullptr)
+                    : launch_gqa<T, 64, sha::kLayoutCluster, false>(prm, dtype, dev, s, nullptr);
+}
+
 // fma: the multi-head FMA kernel, else the grouped kernel; look: its scout build
 template <int kLayout>
 sha_status_t launch_decode(const sha::DecodeParams &prm, sha_dtype_t dtype, int d, bool fma,
@@ -458,6 +587,57 @@ sha_status_t launch_decode(const sha::DecodeParams &prm, sha_dtype_t dtype, int 
                         : launch_look<__half, 64, kLayout>(prm, dtype, fma, look, dev, s, kv);
     return d == 128 ? launch_look<__nv_bfloat16, 128, kLayout>(prm, dtype, fma, look, dev, s, kv)
                     : launch_look<__nv_bfloat16, 64, kLayout>(prm, dtype, fma, look, dev, s, kv);
+}
+
+// Co-resident clusters of the clustered grouped kernel at head dim D, from the
+// occupancy calculator (the same for both element types).
+template <int D>
+void query_cluster_caps(ClusterCaps &caps)
+{
+    using C = sha::GqaConfig<D>;
+    auto kernel = sha::sha_gqa_decode_kernel<__half, D, sha::kLayoutCluster, false>;
+    for (int c = 0; c <= C::kClusterMax; ++c) caps.n[c] = 0;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return;                               // no clustered cut on this device
+    }
+    for (int c = 2; c <= C::kClusterMax; ++c) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(c * 64);
+        cfg.blockDim = dim3(C::threads(false));
+        cfg.dynamicSmemBytes = C::kSmemBytes;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = c;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
+            (void)cudaGetLastError();
+            n = 0;
+        }
+        caps.n[c] = n;
+    }
+}
+
+// The cluster capacities of device `dev` (looked up once), or null where the
+// clustered cut does not apply: per-row lengths, paged or strided caches.
+const ClusterCaps *cluster_caps(int dev, int d, bool fixed_layout)
+{
+    if (!SHA_CLUSTER_CUT || !fixed_layout) return nullptr;
+    static ClusterCaps caps[kMaxDevices][2];
+    static bool known[kMaxDevices][2];
+    const int i = d == 128 ? 1 : 0;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!known[dev][i]) {
+        if (d == 128) query_cluster_caps<128>(caps[dev][i]);
+        else query_cluster_caps<64>(caps[dev][i]);
+        known[dev][i] = true;
+    }
+    return &caps[dev][i];
 }
 
 // Whether to launch the build with a scout warp (sha_lookahead.cuh): it pays
@@ -493,11 +673,17 @@ struct KvLayout {
 };
 
 // N_kv is the padded length (per-row lengths) or max_pages * page_size (paged).
+// A caller's choice of the clustered cut (sha_decode_clustered); 0: the planner's.
+struct ForcedCluster {
+    int cluster = 0, units_per_cluster = 0;
+};
+
 sha_status_t decode_impl(const void *q, const void *k, const void *v, const int32_t *idx,
                          int B, int H_q, int H_kv, int N_kv, int d, int top_k, float scale,
                          void *out, sha_dtype_t dtype, void *workspace,
                          size_t workspace_bytes, int num_splits, void *stream,
-                         bool library_workspace, const KvLayout &lay = KvLayout())
+                         bool library_workspace, const KvLayout &lay = KvLayout(),
+                         ForcedCluster force = ForcedCluster())
 {
     const int32_t *seqlens = lay.seqlens;
     if (dtype != SHA_FP16 && dtype != SHA_BF16) return SHA_ERR_UNSUPPORTED;
@@ -519,12 +705,21 @@ sha_status_t decode_impl(const void *q, const void *k, const void *v, const int3
     st = current_device(&dev, &info);
     if (st != SHA_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const Plan pl = seqlens ? make_varlen_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits,
-                                               info->num_sms)
-                            : make_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits, info->num_sms);
+    const ClusterCaps *caps =
+        cluster_caps(dev, d, !seqlens && !lay.strided && !lay.block_table);
+    Plan pl;
+    if (force.cluster) {
+        st = forced_cluster_plan(B, H_q, H_kv, N_kv, d, top_k, force.cluster,
+                                 force.units_per_cluster, pl);
+        if (st != SHA_OK) return st;
+    } else {
+        pl = seqlens ? make_varlen_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits, info->num_sms)
+                     : make_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits, info->num_sms, false,
+                                 caps);
+    }
     const size_t need = pl.workspace_bytes();
     const bool fma = fma_path(G, d, seqlens != nullptr);   // paged calls carry lengths too
-    const bool look = lookahead_pays(pl, G, fma, seqlens != nullptr);
+    const bool look = pl.sched.cluster < 2 && lookahead_pays(pl, G, fma, seqlens != nullptr);
 
     if (library_workspace && need > 0) {
         OwnedWorkspace *owned = g_owned;
@@ -587,6 +782,9 @@ sha_status_t decode_impl(const void *q, const void *k, const void *v, const int3
             return launch_decode<sha::kLayoutStridedVarlen>(prm, dtype, d, fma, look, dev, s, &kv);
         return launch_decode<sha::kLayoutStrided>(prm, dtype, d, fma, look, dev, s, &kv);
     }
+    if (pl.sched.cluster >= 2)
+        return dtype == SHA_FP16 ? launch_cluster<__half>(prm, dtype, d, dev, s)
+                                 : launch_cluster<__nv_bfloat16>(prm, dtype, d, dev, s);
     if (lay.block_table) return launch_decode<sha::kLayoutPaged>(prm, dtype, d, fma, look, dev, s);
     if (seqlens) return launch_decode<sha::kLayoutVarlen>(prm, dtype, d, fma, look, dev, s);
     return launch_decode<sha::kLayoutFixed>(prm, dtype, d, fma, look, dev, s);
@@ -730,6 +928,63 @@ sha_status_t sha_decode_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_
     return SHA_OK;
 }
 
+sha_status_t sha_decode_plan_ex(int B, int H_q, int H_kv, int N_kv, int d, int top_k,
+                                int num_splits, int num_sms, const int32_t cluster_capacity[9],
+                                int64_t plan[8])
+{
+    sha_status_t st = check_shape(B, H_q, H_kv, N_kv, d, top_k, 1.0f);
+    if (st != SHA_OK) return st;
+    if (num_splits < 0 || num_sms < 1 || !plan) return SHA_ERR_INVALID_ARG;
+    const int tile = tile_keys(H_q / H_kv, d, false);
+    for (int i = 0; i < 8; ++i) plan[i] = 0;
+    plan[4] = tile;
+    if (B == 0 || top_k == 0) {
+        plan[0] = (N_kv + tile - 1) / tile;
+        return SHA_OK;
+    }
+    ClusterCaps caps;
+    for (int c = 0; c <= sha::GqaConfig<128>::kClusterMax; ++c)
+        caps.n[c] = cluster_capacity && c >= 2 ? cluster_capacity[c] : 0;
+    const Plan pl = make_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits, num_sms, false,
+                              cluster_capacity ? &caps : nullptr);
+    plan[0] = pl.sched.tiles_per_unit;
+    plan[1] = pl.sched.total_tiles;
+    plan[2] = pl.sched.num_ctas;
+    plan[3] = (int64_t)pl.workspace_bytes();
+    plan[5] = pl.sched.cluster;
+    plan[6] = pl.sched.units_per_cluster;
+    plan[7] = pl.sched.pieces;
+    return SHA_OK;
+}
+
+sha_status_t sha_decode_cluster_capacity(int d, int32_t cluster_capacity[9])
+{
+    if (!cluster_capacity) return SHA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return SHA_ERR_UNSUPPORTED;
+    int dev;
+    DeviceInfo *info;
+    sha_status_t st = current_device(&dev, &info);
+    if (st != SHA_OK) return st;
+    const ClusterCaps *caps = cluster_caps(dev, d, true);
+    for (int c = 0; c < 9; ++c)
+        cluster_capacity[c] = caps && c <= sha::GqaConfig<128>::kClusterMax ? caps->n[c] : 0;
+    return SHA_OK;
+}
+
+sha_status_t sha_decode_clustered(const void *q, const void *k, const void *v,
+                                  const int32_t *batch_head_index, int B, int H_q, int H_kv,
+                                  int N_kv, int d, int top_k, float scale, void *out,
+                                  sha_dtype_t dtype, int cluster, int units_per_cluster,
+                                  void *stream)
+{
+    if (cluster < 2) return SHA_ERR_INVALID_ARG;
+    ForcedCluster force;
+    force.cluster = cluster;
+    force.units_per_cluster = units_per_cluster;
+    return decode_impl(q, k, v, batch_head_index, B, H_q, H_kv, N_kv, d, top_k, scale, out,
+                       dtype, nullptr, 0, 0, stream, false, KvLayout(), force);
+}
+
 sha_status_t sha_select_heads(const float *scores, int B, int H, int top_k,
                               int32_t *batch_head_index, void *stream)
 {
@@ -860,7 +1115,8 @@ extern "C" sha_status_t sha_decode_noalloc(const void *q, const void *k, const v
     DeviceInfo *info;
     st = current_device(&dev, &info);
     if (st != SHA_OK) return st;
-    const Plan pl = make_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits, info->num_sms);
+    const Plan pl = make_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits, info->num_sms, false,
+                              cluster_caps(dev, d, true));
     const size_t need = pl.workspace_bytes();
     if (need > (size_t)SHA_NOALLOC_SCRATCH_BYTES) return SHA_ERR_WORKSPACE;
     void *scratch = nullptr;

@@ -82,6 +82,91 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
     return true;
 }
 
+// ---- thread-block clusters --------------------------------------------------
+// A unit split across the blocks of one cluster is merged through distributed
+// shared memory: each block stores its part of the unit straight into the
+// shared memory of the blocks that finish it (asynchronous stores counted on
+// their mbarriers), so no block reads another's memory.
+
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Hardware cluster barrier, split into its two halves.  Every thread of every
+// block arrives once; a thread waits before its first access to another
+// block's shared memory (its mbarriers must be initialised by then).
+__device__ __forceinline__ void cluster_arrive()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait()
+{
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Asynchronous stores into the shared memory of block `rank` of this cluster,
+// at the same offset as `local` has in this block; the bytes are counted
+// (complete_tx) on the mbarrier at `bar`'s offset in that block, so a thread
+// there that waits on it sees them.
+__device__ __forceinline__ void st_async_f32x2(const float *local, uint32_t rank, float a, float b,
+                                               uint64_t *bar)
+{
+    asm volatile(
+        "{\n\t.reg .b32 ra, rb;\n\t"
+        "mapa.shared::cluster.u32 ra, %0, %4;\n\t"
+        "mapa.shared::cluster.u32 rb, %1, %4;\n\t"
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [ra], {%2, %3}, [rb];\n\t}"
+        ::"r"(smem_addr(local)), "r"(smem_addr(bar)), "f"(a), "f"(b), "r"(rank)
+        : "memory");
+}
+__device__ __forceinline__ void st_async_f32(const float *local, uint32_t rank, float a,
+                                             uint64_t *bar)
+{
+    asm volatile(
+        "{\n\t.reg .b32 ra, rb;\n\t"
+        "mapa.shared::cluster.u32 ra, %0, %3;\n\t"
+        "mapa.shared::cluster.u32 rb, %1, %3;\n\t"
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [ra], %2, [rb];\n\t}"
+        ::"r"(smem_addr(local)), "r"(smem_addr(bar)), "f"(a), "r"(rank)
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// mbar_wait with acquire at cluster scope: what other blocks of the cluster
+// stored into this block before the phase completed is visible afterwards.
+// Bounded like mbar_wait.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity)
+{
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const unsigned long long t0 = global_timer_ns();
+    while (!mbar_try_wait_cluster(bar, parity)) {
+        if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    }
+    return true;
+}
+
+// The hardware cluster barrier for threads that may be diverged within their
+// warp (the kernels' last step under the clustered cut).
+__device__ __forceinline__ void cluster_sync_unaligned()
+{
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
 // L2 policy for data read exactly once per call (the selected K/V rows).
 __device__ __forceinline__ uint64_t l2_policy_evict_first()
 {

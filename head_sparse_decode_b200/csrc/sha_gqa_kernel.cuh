@@ -76,8 +76,10 @@ struct GqaConfig {
     static constexpr int kKOffset = 0;
     static constexpr int kVOffset = kStages * kTileBytes;
     static constexpr int kBarOffset = 2 * kStages * kTileBytes;
-    // ring barriers (full, empty), then the copy barrier of the on-chip merge
-    static constexpr int kFlagOffset = kBarOffset + 2 * kStages * 8 + 16;
+    // ring barriers (full, empty), then the copy barrier of the on-chip merge,
+    // then the clustered cut's barriers (parts ready x2, parts read x2)
+    static constexpr int kClusterBarOffset = kBarOffset + 2 * kStages * 8 + 16;
+    static constexpr int kFlagOffset = kClusterBarOffset + 32;
     static constexpr int kPlanOffset = kFlagOffset + 16;       // 32 longs: per-row-length plan
     static constexpr int kStateOffset = kPlanOffset + 256;
     // on-chip merge (G <= 8): part i (0 = this block's) in rows 8..15 of warp
@@ -85,10 +87,19 @@ struct GqaConfig {
     static constexpr int kMaxPartRows = 8;
     static constexpr int kPartFloats = kStateFloats;
     static constexpr int kPartRowOffset = kMaxPartRows * (D + 2);
+    // clustered cut (G <= 8): the slices of a unit's parts that the cluster's
+    // blocks store into this block, double-buffered by unit, in rows 8..15 of
+    // the warps' state areas (warps 0, 1 for even units, 2, 3 for odd ones)
+    static constexpr int kClusterMax = 8;                 // blocks per cluster (portable)
+    static constexpr int kRegionFloats = kPartRowOffset;  // rows 8..15 of one warp
     // per query row: the warps' weights 2^(m_w - M), then M and L
     static constexpr int kCombineFloats = kConsumerWarps + 2;
     static constexpr int kCombineOffset = kStateOffset + kConsumerWarps * kStateFloats * 4;
-    static constexpr int kSmemBytes = kAlignPad + kCombineOffset + kRows * kCombineFloats * 4;
+    // clustered cut: per 4-element group of a unit's outputs, the block that
+    // finishes it and the group's offset in that block's slice
+    static constexpr int kOwnerOffset = kCombineOffset + kRows * kCombineFloats * 4;
+    static constexpr int kOwnerGroups = kMaxPartRows * D / 4;
+    static constexpr int kSmemBytes = kAlignPad + kOwnerOffset + kOwnerGroups * 2;
     static_assert(2 * (threads(true) / 32) + 8 <= 32, "plan scratch fits");
     static_assert(kKeysPerWarp == 16, "one k-step of 16 keys per warp and slice");
     static_assert(kTile % 64 == 0 && kTile <= 256, "whole 64-key slices, TMA box <= 256 rows");
@@ -130,7 +141,10 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
                           const __grid_constant__ CUtensorMap tm_v)
 {
     constexpr bool kVarlen = layout_varlen(kLayout);
-    using Walk = typename std::conditional<kVarlen, VarlenWalk, UniformWalk>::type;
+    constexpr bool kCluster = kLayout == kLayoutCluster;
+    using Walk = typename std::conditional<
+        kVarlen, VarlenWalk,
+        typename std::conditional<kCluster, ClusterWalk, UniformWalk>::type>::type;
     using C = GqaConfig<D>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = reinterpret_cast<unsigned char *>(
@@ -143,6 +157,9 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
     volatile int *flags = reinterpret_cast<volatile int *>(smem + C::kFlagOffset);
     float *wstate = reinterpret_cast<float *>(smem + C::kStateOffset);
     float *own_part = wstate + C::kStateFloats + C::kPartRowOffset;
+    // clustered cut: one barrier per unit buffer; it completes when all the
+    // cluster's slices of the unit have landed here
+    uint64_t *cbar = reinterpret_cast<uint64_t *>(smem + C::kClusterBarOffset);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -158,6 +175,8 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
             mbar_init(&empty[s], C::kConsumerWarps);
         }
         mbar_init(part_bar, 1);
+        if constexpr (kCluster)
+            for (int i = 0; i < 2; ++i) mbar_init(&cbar[i], 1);
         flags[0] = 0;
         flags[1] = 0;
         flags[kFlagClaim] = 0;
@@ -165,9 +184,20 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
         mbar_init_fence();
     }
     __syncthreads();
+    // the cluster's barriers are initialised before any block signals another's
+    if constexpr (kCluster) cluster_arrive();
+    // the tensor maps are kernel parameters: fetch them while the previous
+    // kernel finishes
+    if (warp == C::kConsumerWarps && lane == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k))
+                     : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v))
+                     : "memory");
+    }
     // inputs, workspace and the output may come from the previous kernel
     pdl_wait();
     pdl_launch_dependents();
+    if constexpr (kCluster) cluster_wait();
 
     Schedule S = p.sched;
     Walk walk;
@@ -176,6 +206,8 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
                                       reinterpret_cast<long long *>(smem + C::kPlanOffset), S,
                                       walk))
             return;
+    } else if constexpr (kCluster) {
+        walk.start(S, (long long)p.B * p.top_k, p.N_kv);
     } else {
         walk.S = S;
         walk.t = S.begin(blockIdx.x);
@@ -198,11 +230,10 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
         // A paged cache needs several page ids per tile: the whole warp gathers
         // them (one page box per lane).  Otherwise one lane drives the pipeline.
         constexpr bool kWarpProducer = kLayout == kLayoutPaged;
-        if (!kWarpProducer && lane != 0) return;
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k))
-                     : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v))
-                     : "memory");
+        if (!kWarpProducer && lane != 0) {
+            if constexpr (kCluster) cluster_sync_unaligned();
+            return;
+        }
         const uint64_t policy = l2_policy_evict_first();
         int stage = 0;
         uint32_t phase = 0;
@@ -289,6 +320,7 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
             for (int s = 0; s < C::kStages; ++s)
                 if (used & (1u << s)) mbar_wait(&full[s], (last_parity >> s) & 1u);
         if constexpr (kWarpProducer) __syncwarp();
+        if constexpr (kCluster) cluster_sync_unaligned();
         return;
     }
 
@@ -306,8 +338,40 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
     int stage = 0;
     uint32_t phase = 0;
 
+    // Clustered cut: block r of the P-block cluster finishes the 4-element
+    // groups [r*groups/P, (r+1)*groups/P) of a unit's G x D outputs, and every
+    // block stores each part's slices (and its m, l) where their finishers
+    // stage them: part i of a unit at cstage(buf, i) in every block, the
+    // first (P+1)/2 parts in one warp's rows 8..15, the others in the next's.
+    // All of it is fixed for the kernel: worked out here once.
+    const int P = kCluster ? S.cluster : 1;
+    const int groups = G * D / 4;
+    const int slice_max = 4 * ((groups + P - 1) / P);
+    const int part_stride = slice_max + 4 * ((2 * G + 3) / 4);
+    const int half = (P + 1) / 2;
+    auto cstage = [=](int buf, int i) {
+        const bool hi = i >= half;
+        return wstate + (2 * buf + (hi ? 1 : 0)) * C::kStateFloats + C::kPartRowOffset +
+               (hi ? i - half : i) * part_stride;
+    };
+    uint16_t *owner_tab = reinterpret_cast<uint16_t *>(smem + C::kOwnerOffset);
+    int e0 = 0, e1 = 0;
+    uint32_t cluster_bytes = 0;
+    if constexpr (kCluster) {
+        e0 = 4 * (walk.rank * groups / P);
+        e1 = 4 * ((walk.rank + 1) * groups / P);
+        cluster_bytes = (uint32_t)(P * (e1 - e0 + 2 * G) * 4);
+        // owner (high 4 bits) and offset within its slice (floats) per group;
+        // read after the consumers' first named barrier
+        for (int g4 = tid; g4 < groups; g4 += C::kConsumers) {
+            const int r = ((g4 + 1) * P - 1) / groups;
+            owner_tab[g4] = (uint16_t)((r << 12) | (4 * g4 - 4 * (r * groups / P)));
+        }
+    }
+
     Walk wk = walk;
     Seg seg;
+    int n_done = 0;   // clustered cut: units this block has finished (its buffers' parity)
     for (bool first_seg = true; wk.next(seg); first_seg = false) {
         const long long u = seg.unit;
         const int b = (int)(u / p.top_k);
@@ -474,9 +538,10 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
         // blocks first..last share a split unit; the one the block ends with may
         // be finished on chip
         int first = 0, last = 0, first_slot = 0;
-        if (!seg.whole) unit_parts(S, seg, first, last, first_slot);
-        const int la_parts =
-            kLook && wk.t >= wk.t_end ? lookahead_parts(seg, first, last, max_partners) : 0;
+        if (!kCluster && !seg.whole) unit_parts(S, seg, first, last, first_slot);
+        int la_parts = 0;
+        if constexpr (kLook)
+            if (wk.t >= wk.t_end) la_parts = lookahead_parts(seg, first, last, max_partners);
         if (la_parts && tid == 0) flags[kFlagOnChip] = lookahead_claim(flags);
         named_barrier(1, C::kConsumers);
         const bool on_chip = la_parts && flags[kFlagOnChip];
@@ -505,11 +570,38 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
         const bool aborted = flags[0] != 0;
         // this block's first unit goes to slot 2c, any later partial one to 2c+1;
         // on chip it is part 0, beside the copies of the others
-        float *slot = on_chip ? own_part
+        float *slot = on_chip   ? own_part
                     : p.slots ? p.slots + (size_t)(2 * blockIdx.x + (first_seg ? 0 : 1)) *
                                               p.slot_floats
                               : nullptr;
-        if (!aborted) {
+        if constexpr (kCluster) {
+            // this block's part of the unit, slice by slice, to the blocks that
+            // finish them (always, so that every block's byte count completes)
+            const int buf = n_done & 1;
+            float *mine = cstage(buf, wk.rank);
+            for (int e = 2 * tid; e < G * D; e += 2 * C::kConsumers) {
+                const uint32_t code = owner_tab[e >> 2];
+                const int row = e / D, c = e - row * D;
+                const float *cr = cw + row * C::kCombineFloats;
+                float2 O = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int w = 0; w < C::kConsumerWarps; ++w) {
+                    const float2 x = *reinterpret_cast<const float2 *>(
+                        wstate + w * C::kStateFloats + row * (D + 2) + c);
+                    O.x = fmaf(cr[w], x.x, O.x);
+                    O.y = fmaf(cr[w], x.y, O.y);
+                }
+                st_async_f32x2(mine + (code & 0xfff) + (e & 3), code >> 12, O.x, O.y,
+                               &cbar[buf]);
+            }
+            // every row's (m, l) to every block: one pair per thread
+            if (tid < P * G) {
+                const int r = tid / G, row = tid - r * G;
+                const float *cr = cw + row * C::kCombineFloats;
+                st_async_f32x2(mine + slice_max + 2 * row, (uint32_t)r, cr[C::kConsumerWarps],
+                               cr[C::kConsumerWarps + 1], &cbar[buf]);
+            }
+        } else if (!aborted) {
             // two neighbouring elements of a row per thread (D is even)
             for (int e = 2 * tid; e < G * D; e += 2 * C::kConsumers) {
                 const int row = e / D, c = e - row * D;
@@ -533,11 +625,30 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
                     }
                 }
             }
-            if (!seg.whole && !on_chip) __threadfence();
+            if (!kCluster && !seg.whole && !on_chip) __threadfence();
         }
         named_barrier(1, C::kConsumers);
 
-        if (on_chip) {
+        if constexpr (kCluster) {
+            // wait for this block's slices of every part (its own included), then
+            // write them out merged in block order
+            const int buf = n_done & 1;
+            if (tid == 0) mbar_arrive_expect_tx(&cbar[buf], cluster_bytes);
+            if (!mbar_wait_cluster(&cbar[buf], (n_done >> 1) & 1)) {
+                atomicOr(&g_sha_status, kStatusTimeout);
+                flags[0] = 1;
+            }
+            named_barrier(1, C::kConsumers);
+            if (tid == 0) flags[1] = !flags[0];
+            named_barrier(1, C::kConsumers);
+            if (flags[1]) {
+                auto part_at = [=](int i) { return cstage(buf, i); };
+                merge_parts<T, D, C::kConsumers>(
+                    StagedParts<decltype(part_at)>{part_at, e0, slice_max}, P, G, out_g, wstate,
+                    tid, e0, e1);
+            }
+            ++n_done;
+        } else if (on_chip) {
             // every other part has arrived and none merged: this block merges
             if (!mbar_wait(part_bar, 0)) {
                 atomicOr(&g_sha_status, kStatusTimeout);
@@ -547,7 +658,7 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
             if (tid == 0) flags[1] = !flags[0];
             named_barrier(1, C::kConsumers);
             if (flags[1]) {
-                merge_parts<T, D, C::kConsumers>(SharedParts{own_part, C::kPartFloats}, la_parts,
+                merge_parts<T, D, C::kConsumers>(SharedParts{own_part, C::kPartFloats, G * D}, la_parts,
                                                   G, out_g, wstate, tid);
                 if (tid == 0) p.counters[first] = 0;
             }
@@ -564,13 +675,15 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
             if (flags[1]) {
                 __threadfence();
                 merge_parts<T, D, C::kConsumers>(
-                    GlobalParts{p.slots, p.slot_floats, first, first_slot}, last - first + 1, G,
+                    GlobalParts{p.slots, p.slot_floats, first, first_slot, G * D}, last - first + 1, G,
                     out_g, wstate, tid);
                 if (tid == 0) p.counters[first] = 0;
             }
         }
     }
     if (kLook && tid == 0) lookahead_claim(flags);   // the scout stops looking
+    // no block of a cluster leaves while another may still store into it
+    if constexpr (kCluster) cluster_sync_unaligned();
 }
 
 }  // namespace sha

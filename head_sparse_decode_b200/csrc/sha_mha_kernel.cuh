@@ -75,7 +75,10 @@ enum : int {
     kLayoutVarlen = 1,
     kLayoutPaged = 2,
     kLayoutStrided = 3,
-    kLayoutStridedVarlen = 4
+    kLayoutStridedVarlen = 4,
+    // the padded layout of kLayoutFixed under the clustered cut (grouped kernel
+    // only): thread-block clusters, split units merged in distributed shared memory
+    kLayoutCluster = 5
 };
 
 // Layouts whose rows have their own lengths (planned on the device) and that
@@ -508,7 +511,7 @@ __global__ void __launch_bounds__(MhaConfig<D>::threads(kLook), SHA_MHA_BLOCKS_P
             named_barrier(1, C::kConsumers);
             if (flags[1]) {
                 T *orow = static_cast<T *>(p.out) + ((size_t)b * p.H_q + h) * D;
-                merge_parts<T, D, C::kConsumers>(SharedParts{own_part, C::kPartFloats}, la_parts,
+                merge_parts<T, D, C::kConsumers>(SharedParts{own_part, C::kPartFloats, D}, la_parts,
                                                   1, orow, wstate, tid);
                 if (tid == 0) p.counters[first] = 0;
             }
@@ -528,7 +531,7 @@ __global__ void __launch_bounds__(MhaConfig<D>::threads(kLook), SHA_MHA_BLOCKS_P
                 __threadfence();
                 T *orow = static_cast<T *>(p.out) + ((size_t)b * p.H_q + h) * D;
                 merge_parts<T, D, C::kConsumers>(
-                    GlobalParts{p.slots, p.slot_floats, first, first_slot}, last - first + 1, 1,
+                    GlobalParts{p.slots, p.slot_floats, first, first_slot, D}, last - first + 1, 1,
                     orow, wstate, tid);
                 if (tid == 0) p.counters[first] = 0;
             }

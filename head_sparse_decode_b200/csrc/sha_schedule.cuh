@@ -11,7 +11,9 @@
 // than one piece is finished by a log-sum-exp merge of the pieces' partial
 // (m, l, O) states (see the kernels).  When units are only a few tiles long
 // the merges cost more than an uneven cut, and the host may instead cut at
-// unit boundaries: whole units per block, or each unit in p equal pieces.
+// unit boundaries: whole units per block, or each unit in p equal pieces,
+// or (the clustered cut) each unit in p pieces held by the p blocks of one
+// thread-block cluster, which merge them in distributed shared memory.
 //
 // A unit split across blocks c_first..c_last is merged by whichever of them
 // finishes last, found with an arrival counter.  Counter c_first belongs to
@@ -41,6 +43,13 @@ struct Schedule {
     // block c takes the whole pieces [c P / num_ctas, (c+1) P / num_ctas) of
     // the P = units * p pieces, so no block starts or ends inside a piece.
     int pieces;
+    // >= 2: the clustered cut.  Blocks form thread-block clusters of this many;
+    // cluster k takes whole units [k * units_per_cluster, (k+1) * units_per_cluster)
+    // and its block of rank r streams piece r of each of them (tiles
+    // [r * tiles_per_unit / cluster, (r+1) * tiles_per_unit / cluster)).  The
+    // parts of a unit meet in the cluster's shared memory, not in the workspace.
+    int cluster;
+    int units_per_cluster;
 
     // First tile of piece i of the unit-aligned cut (pieces >= 1).
     __host__ __device__ __forceinline__ long long piece_start(long long i) const

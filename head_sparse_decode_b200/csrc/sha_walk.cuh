@@ -63,6 +63,39 @@ struct UniformWalk {
     }
 };
 
+// Clustered cut (Schedule::cluster >= 2): this block's piece of each unit of
+// its cluster's range; every block of the cluster visits the same units.
+struct ClusterWalk {
+    int tiles_per_unit, cluster, rank;
+    long long u, u_end;
+    int n_keys;
+
+    __device__ __forceinline__ void start(const Schedule &S, long long units, int keys)
+    {
+        tiles_per_unit = S.tiles_per_unit;
+        cluster = S.cluster;
+        rank = (int)cluster_ctarank();
+        u = (long long)(blockIdx.x / S.cluster) * S.units_per_cluster;
+        u_end = u + S.units_per_cluster < units ? u + S.units_per_cluster : units;
+        n_keys = keys;
+    }
+    __device__ __forceinline__ bool next(Seg &s)
+    {
+        if (u >= u_end) return false;
+        const int j0 = rank * tiles_per_unit / cluster;
+        const int j1 = (rank + 1) * tiles_per_unit / cluster;
+        s.unit = u;
+        s.first_tile = j0;
+        s.num_tiles = j1 - j0;
+        s.whole = false;
+        s.unit_start = u * tiles_per_unit;
+        s.unit_tiles = tiles_per_unit;
+        s.n_keys = n_keys;
+        ++u;
+        return true;
+    }
+};
+
 __device__ __forceinline__ int varlen_tiles(int len, int n_max, int tile)
 {
     return (len >= 1 && len <= n_max) ? (len + tile - 1) / tile : 0;

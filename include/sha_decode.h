@@ -207,6 +207,64 @@ sha_status_t sha_decode_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_
                              int num_splits, int num_sms, int64_t plan[5]);
 
 /*
+ * The clustered cut.  A short call -- few (batch row, head) units, or few key
+ * tiles per unit -- keeps most SMs idle if every unit stays in one thread
+ * block, and if a unit's tiles are spread over several blocks, merging the
+ * parts through global memory (write, fence, arrival counter, read back) adds
+ * microseconds at the end of the call.  Under the clustered cut the blocks
+ * form thread-block clusters of c blocks (2 <= c <= 8); each cluster takes
+ * units_per_cluster whole units, block r of the cluster streams piece r of
+ * each of them (its tiles [r*T/c, (r+1)*T/c) of T = ceil(N_kv/tile)), and the
+ * c parts of a unit are merged in the cluster's distributed shared memory,
+ * each block writing 1/c of the unit's output.  It serves the grouped kernel:
+ * G = H_q/H_kv <= 8 with d = 128 (G = 1 included) or G >= 2 with d = 64, one
+ * length per row, the contiguous [B, H_kv, N_kv, d] layout.  With
+ * num_splits = 0 the planner of sha_decode, sha_decode_bf16, sha_decode_ex
+ * and sha_decode_noalloc takes it where a cost model of the call's streaming
+ * time and merge tail, with the device's cluster capacities, rates it faster
+ * than the other cuts; it needs no workspace.
+ *
+ * sha_decode_plan_ex -- sha_decode_plan with the clustered cut: the planner's
+ * choice on a device with num_sms SMs that holds cluster_capacity[c] clusters
+ * of c blocks at once (c = 2..8; entries 0 and 1 ignored; NULL = no clustered
+ * cut, as in sha_decode_plan).  Host only, no CUDA call.  Writes plan[0..4]
+ * as sha_decode_plan, and
+ *   plan[5] = blocks per cluster (0: not the clustered cut)
+ *   plan[6] = units per cluster
+ *   plan[7] = 0 (tiles cut evenly), 1 (whole units per block),
+ *             p >= 2 (each unit in p equal pieces) -- 0 under the clustered cut
+ */
+sha_status_t sha_decode_plan_ex(int B, int H_q, int H_kv, int N_kv, int d, int top_k,
+                                int num_splits, int num_sms, const int32_t cluster_capacity[9],
+                                int64_t plan[8]);
+
+/*
+ * sha_decode_cluster_capacity -- the current device's cluster capacities for
+ * head dim d (64 or 128), as the planner uses them: cluster_capacity[c] =
+ * clusters of c blocks of the clustered kernel that fit on the device at once
+ * (from cudaOccupancyMaxActiveClusters), c = 2..8; [0] = [1] = 0.  Queried
+ * once per device and cached.
+ */
+sha_status_t sha_decode_cluster_capacity(int d, int32_t cluster_capacity[9]);
+
+/*
+ * sha_decode_clustered -- sha_decode_ex with the clustered cut chosen by the
+ * caller (for tests and measurements): clusters of `cluster` blocks, each
+ * taking `units_per_cluster` whole units (the last cluster the rest).
+ *   2 <= cluster <= min(8, ceil(N_kv / tile)), units_per_cluster >= 1, at most
+ *   4096 blocks in all (SHA_ERR_INVALID_ARG otherwise); calls the clustered
+ *   kernel cannot serve (above) return SHA_ERR_UNSUPPORTED.
+ * Clusters beyond the device's capacity run in further waves.  The result is
+ * the same as sha_decode_ex's to within rounding (the parts are merged in
+ * block order by the same log-sum-exp arithmetic).  Allocates nothing.
+ */
+sha_status_t sha_decode_clustered(const void *q, const void *k, const void *v,
+                                  const int32_t *batch_head_index, int B, int H_q, int H_kv,
+                                  int N_kv, int d, int top_k, float scale, void *out,
+                                  sha_dtype_t dtype, int cluster, int units_per_cluster,
+                                  void *stream);
+
+/*
  * sha_select_heads -- router scores to batch_head_index on the device.
  * Polar Sparsity (papernotes.org summary, "Router 训练"; atlas.scime.ai
  * summary): an attention router scores the heads (or GQA groups) of each
