@@ -295,13 +295,16 @@ def sha_decode_ex(q, k, v, batch_head_index, scale, out, workspace=None, num_spl
 _lib.sha_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_float,
                                     _vp, _i, _i, _vp]
 _lib.sha_decode_noalloc.restype = _i
-NOALLOC_SCRATCH_BYTES = 512 * 1024
+_lib.sha_noalloc_scratch_bytes.argtypes = []
+_lib.sha_noalloc_scratch_bytes.restype = ctypes.c_size_t
+# size of the library's fixed scratch array, as the library was built
+NOALLOC_SCRATCH_BYTES = int(_lib.sha_noalloc_scratch_bytes())
 
 
 def sha_decode_noalloc(q, k, v, batch_head_index, scale, out, num_splits=0, stream=None):
     """Multi-head decode for callers that cannot allocate device memory: the
-    library keeps the split-merge scratch in a fixed 512 KiB device array
-    instead of a workspace, so the call allocates nothing.  Calls on one device
+    library keeps the split-merge scratch in a fixed device array
+    (NOALLOC_SCRATCH_BYTES) instead of a workspace, so the call allocates nothing.  Calls on one device
     share that array: do not let them overlap on the GPU."""
     args, s = _decode_args(q, k, v, batch_head_index, scale, out, stream)
     with torch.cuda.device(k.device):

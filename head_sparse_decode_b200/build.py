@@ -27,11 +27,13 @@ def _sources():
                   + [os.path.join(INCLUDE, "sha_decode.h")])
 
 
-def build(force: bool = False, verbose: bool = False, defines=(), output=None) -> str:
+def build(force: bool = False, verbose: bool = False, defines=(), output=None,
+          sources=None) -> str:
     """Compile the library unless it is newer than every source file.
 
     defines: extra -D settings (the kernels' build-time tuning knobs);
-    output:  another path for the library (builds with non-default knobs)."""
+    output:  another path for the library (builds with non-default knobs);
+    sources: the .cu files of csrc/ to compile (default all of them)."""
     library = output or LIBRARY
     if not force and os.path.exists(library):
         newest = max(os.path.getmtime(p) for p in _sources())
@@ -42,7 +44,8 @@ def build(force: bool = False, verbose: bool = False, defines=(), output=None) -
     cmd = [NVCC, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, *[f"-D{d}" for d in defines]]
     if verbose:
         cmd += ["-Xptxas", "-v"]
-    sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")) if sources is None
+                     else [os.path.join(CSRC, name) for name in sources])
     objects = [f"{library}.{os.path.basename(src)}.o" for src in sources]
     procs = [subprocess.Popen(cmd + ["-c", "-o", obj, src]) for src, obj in zip(sources, objects)]
     failed = [src for src, proc in zip(sources, procs) if proc.wait() != 0]
@@ -59,5 +62,15 @@ def build(force: bool = False, verbose: bool = False, defines=(), output=None) -
     return library
 
 
+# The decode library with test hooks (a pipeline wait limit the tests can
+# lower, see sha_test_set_wait_limit); only the tests load it.
+TEST_HOOKS_LIBRARY = os.path.join(PKG, "libsha_decode_test_hooks.so")
+
+
+def build_test_hooks(force: bool = False) -> str:
+    return build(force=force, defines=("SHA_TEST_HOOKS=1",), output=TEST_HOOKS_LIBRARY)
+
+
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))
+    print(build_test_hooks(force="--force" in sys.argv))

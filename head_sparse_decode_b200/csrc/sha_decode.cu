@@ -1016,11 +1016,16 @@ sha_status_t sha_get_device_status(void *stream)
     if (e != cudaSuccess) return launch_error(e);
     flags |= sha_mlp_take_status();
     if (flags & sha::kStatusTimeout) {
-        // an abandoned merge can leave arrival counters raised: clear them
+        // an abandoned merge can leave arrival counters raised: clear the
+        // library workspace's, in order on `stream`
         int dev;
         if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices) {
             std::lock_guard<std::mutex> lock(g_mutex);
-            if (g_owned[dev].ptr) cudaMemset(g_owned[dev].ptr, 0, sha::kCounterBytes);
+            if (g_owned[dev].ptr) {
+                e = cudaMemsetAsync(g_owned[dev].ptr, 0, sha::kCounterBytes, s);
+                if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+                if (e != cudaSuccess) return launch_error(e);
+            }
         }
         return SHA_ERR_TIMEOUT;
     }
@@ -1044,6 +1049,19 @@ const char *sha_status_string(sha_status_t status)
 }
 
 const char *sha_last_cuda_error(void) { return g_last_cuda_error; }
+
+#ifdef SHA_TEST_HOOKS
+// Test builds only (not part of the ABI): lower the pipeline wait limit of
+// the current device, so that a test can make waits give up on purpose.
+sha_status_t sha_test_set_wait_limit(unsigned long long ns)
+{
+    cudaError_t e = cudaMemcpyToSymbol(sha::g_wait_limit_ns, &ns, sizeof ns);
+    if (e != cudaSuccess) return launch_error(e);
+    e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return launch_error(e);
+    return SHA_OK;
+}
+#endif
 
 sha_status_t sha_copy_bandwidth_probe(void *dst, const void *src, size_t bytes, void *stream)
 {
@@ -1093,6 +1111,8 @@ sha_status_t noalloc_scratch_address(int dev, void **ptr)
 
 }  // namespace
 
+extern "C" size_t sha_noalloc_scratch_bytes(void) { return SHA_NOALLOC_SCRATCH_BYTES; }
+
 extern "C" sha_status_t sha_decode_noalloc(const void *q, const void *k, const void *v,
                                            const int32_t *batch_head_index, int B, int H_q,
                                            int H_kv, int N_kv, int d, int top_k, float scale,
@@ -1104,7 +1124,7 @@ extern "C" sha_status_t sha_decode_noalloc(const void *q, const void *k, const v
     sha_status_t st = check_shape(B, H_q, H_kv, N_kv, d, top_k, scale);
     if (st != SHA_OK) return st;
     if (num_splits < 0) return SHA_ERR_INVALID_ARG;
-    if (H_q != H_kv) return SHA_ERR_UNSUPPORTED;   // the multi-head kernel only
+    if (H_q != H_kv) return SHA_ERR_UNSUPPORTED;   // multi-head calls (G = 1) only
     if (B == 0 || top_k == 0) return SHA_OK;
     if (!q || !k || !v || !batch_head_index || !out) return SHA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||

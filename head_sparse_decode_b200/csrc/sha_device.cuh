@@ -20,6 +20,20 @@ static __device__ unsigned int g_sha_status;
 // A pipeline wait that has not completed after this long gives up, raises
 // kStatusTimeout and lets the kernel unwind.  Healthy waits last microseconds.
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;
+// A thread waiting for its own asynchronous copies to land before its block
+// exits (or before tensor memory is released) gives up only after this long:
+// the copies write into the block's memory, so it waits for them even after
+// a pipeline wait has given up.
+constexpr unsigned long long kDrainLimitNs = 4000000000ull;
+
+#ifdef SHA_TEST_HOOKS
+// Test builds only: the pipeline wait limit is a device variable the tests
+// can lower (sha_test_set_wait_limit) to make waits give up on purpose.
+static __device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
+__device__ __forceinline__ unsigned long long wait_limit_ns() { return g_wait_limit_ns; }
+#else
+__device__ __forceinline__ unsigned long long wait_limit_ns() { return kWaitLimitNs; }
+#endif
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p)
 {
@@ -57,9 +71,22 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  : "memory");
 }
 
+// A try_wait may suspend the thread until the phase completes (or a limit of
+// the hardware's choosing), so a short wait never reaches the code that gives
+// up.  Test builds poll with the non-blocking test_wait instead, so that a
+// lowered wait limit makes waits give up; the unwinding is the same code.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 {
     uint32_t done;
+#ifdef SHA_TEST_HOOKS
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+#else
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -67,17 +94,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
         : "=r"(done)
         : "r"(smem_addr(bar)), "r"(parity)
         : "memory");
+#endif
     return done != 0;
 }
 
 // Wait for the phase of `bar` with the given parity to complete.  Returns
-// false (and the caller must unwind) if it has not after kWaitLimitNs.
+// false (and the caller must unwind) if it has not after wait_limit_ns().
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_timer_ns();
+    const unsigned long long limit = wait_limit_ns();
     while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+        if (global_timer_ns() - t0 > limit) return false;
+    }
+    return true;
+}
+
+// mbar_wait for a phase completed by this block's own asynchronous copies
+// (or tensor-core work), before their destination is given up: bounded by
+// kDrainLimitNs whatever the pipeline limit.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > kDrainLimitNs) return false;
     }
     return true;
 }
@@ -147,15 +189,16 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
     return done != 0;
 }
 
-// mbar_wait with acquire at cluster scope: what other blocks of the cluster
-// stored into this block before the phase completed is visible afterwards.
-// Bounded like mbar_wait.
+// Wait, with acquire at cluster scope, for a phase completed by other blocks'
+// asynchronous stores into this block: what they stored is visible
+// afterwards.  The stores write into this block's memory, so the wait is
+// bounded by kDrainLimitNs, like a wait for the block's own copies.
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity)
 {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     const unsigned long long t0 = global_timer_ns();
     while (!mbar_try_wait_cluster(bar, parity)) {
-        if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+        if (global_timer_ns() - t0 > kDrainLimitNs) return false;
     }
     return true;
 }

@@ -255,6 +255,10 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
                         atomicOr(&g_sha_status, kStatusTimeout);
                         flags[0] = 1;
                         go = false;
+                    } else if (flags[0]) {
+                        // a consumer that gave up raised the flag before releasing
+                        // this stage: its last copy may still be landing
+                        go = false;
                     }
                 }
                 if constexpr (kWarpProducer) go = __shfl_sync(0xffffffffu, go, 0);
@@ -318,7 +322,7 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
         }
         if (lane == 0)
             for (int s = 0; s < C::kStages; ++s)
-                if (used & (1u << s)) mbar_wait(&full[s], (last_parity >> s) & 1u);
+                if (used & (1u << s)) mbar_wait_drain(&full[s], (last_parity >> s) & 1u);
         if constexpr (kWarpProducer) __syncwarp();
         if constexpr (kCluster) cluster_sync_unaligned();
         return;

@@ -104,7 +104,7 @@ __device__ void lookahead_scout(Walk wk, const Schedule &S, int max_partners,
     bool copied = false;
     const unsigned long long t0 = global_timer_ns();
     // the consumers always take the claim by the time they leave
-    while (flags[kFlagClaim] == 0 && global_timer_ns() - t0 <= kWaitLimitNs) {
+    while (flags[kFlagClaim] == 0 && global_timer_ns() - t0 <= wait_limit_ns()) {
         if (load_relaxed_gpu(counters + first) == parts - 1) {
             if (atomicCAS(claim, 0, 1) == 0) {
                 fence_acquire_gpu();          // the other parts' slots, as they arrived
@@ -121,7 +121,7 @@ __device__ void lookahead_scout(Walk wk, const Schedule &S, int max_partners,
         }
         __nanosleep(500);
     }
-    if (copied && !mbar_wait(bar, 0)) atomicOr(&g_sha_status, kStatusTimeout);
+    if (copied && !mbar_wait_drain(bar, 0)) atomicOr(&g_sha_status, kStatusTimeout);
 }
 
 // The consumers' side (one thread).  At the end of the block's last segment:

@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(UpCfg<BP>::kThreads, 1)
         }
         if (lane == 0)
             for (int s = 0; s < C::kStages; ++s)
-                if (used & (1u << s)) mbar_wait(&full[s], (last_parity >> s) & 1u);
+                if (used & (1u << s)) mbar_wait_drain(&full[s], (last_parity >> s) & 1u);
         __syncwarp();
         return;
     }
@@ -586,7 +586,7 @@ __global__ void __launch_bounds__(uptc::kThreads, 1)
         cp_async_wait_all();
         if (warp == 0 && lane == 0)
             for (int s = 0; s < C::kStages; ++s)
-                if (used & (1u << s)) mbar_wait(&full[s], (last_parity >> s) & 1u);
+                if (used & (1u << s)) mbar_wait_drain(&full[s], (last_parity >> s) & 1u);
         __syncwarp();
     } else if (warp == kMmaWarp) {
         if (lane == 0) {
@@ -632,7 +632,7 @@ __global__ void __launch_bounds__(uptc::kThreads, 1)
             // every issued MMA has finished before TMEM is released
             if (u1 > u0) {
                 umma_commit(mma_done);
-                if (!mbar_wait(mma_done, 0)) atomicOr(&g_sha_status, kStatusTimeout);
+                if (!mbar_wait_drain(mma_done, 0)) atomicOr(&g_sha_status, kStatusTimeout);
             }
         }
         __syncwarp();
@@ -1004,7 +1004,7 @@ __global__ void __launch_bounds__(downtc::kThreads, 1)
         cp_async_wait_all();
         if (warp == 0 && lane == 0)
             for (int s = 0; s < C::kStages; ++s)
-                if (used & (1u << s)) mbar_wait(&full[s], (last_parity >> s) & 1u);
+                if (used & (1u << s)) mbar_wait_drain(&full[s], (last_parity >> s) & 1u);
         __syncwarp();
     } else if (warp == kMmaWarp) {
         if (lane == 0) {
@@ -1054,7 +1054,7 @@ __global__ void __launch_bounds__(downtc::kThreads, 1)
             }
             if (u1 > u0) {
                 umma_commit(mma_done);
-                if (!mbar_wait(mma_done, 0)) atomicOr(&g_sha_status, kStatusTimeout);
+                if (!mbar_wait_drain(mma_done, 0)) atomicOr(&g_sha_status, kStatusTimeout);
             }
         }
         __syncwarp();
@@ -1300,7 +1300,7 @@ __global__ void __launch_bounds__(DownCfg<BP>::kThreads, 1)
         cp_async_wait_all();
         if (pw == 0 && lane == 0)
             for (int s = 0; s < C::kStages; ++s)
-                if (used & (1u << s)) mbar_wait(&full[s], (last_parity >> s) & 1u);
+                if (used & (1u << s)) mbar_wait_drain(&full[s], (last_parity >> s) & 1u);
         __syncwarp();
         return;
     }
@@ -1353,7 +1353,7 @@ __global__ void __launch_bounds__(DownCfg<BP>::kThreads, 1)
         }
         if (lane == 0)
             for (int s = 0; s < C::kStages; ++s)
-                if (used & (1u << s)) mbar_wait(&full[s], (last_parity >> s) & 1u);
+                if (used & (1u << s)) mbar_wait_drain(&full[s], (last_parity >> s) & 1u);
         __syncwarp();
         return;
     }

@@ -35,6 +35,16 @@
  * Head ids out of [0, H_kv) are a device-side condition: that (b, k) slot is
  * skipped (nothing read, nothing written) and a sticky flag is raised, which
  * sha_get_device_status() reports.  No kernel traps.
+ *
+ * Determinism.  Repeated calls with the same arguments on the same device
+ * give bit-identical outputs: a head split across thread blocks is merged in
+ * a fixed block order, never in arrival order.  The result does depend, at
+ * the level of rounding, on where a head's id sits in its row of
+ * batch_head_index: the key tiles of a call are cut in slot order, so
+ * permuting a row can move a head's tiles to other blocks and change the
+ * order of its fp32 sums.  A caller that reorders the ids of a row between
+ * steps gets outputs equal within the fp32-accumulation tolerance, not bit
+ * for bit.
  */
 #ifndef SHA_DECODE_H
 #define SHA_DECODE_H
@@ -334,7 +344,12 @@ sha_status_t sha_selective_mlp(const void *x, const void *W1t, const void *W2t,
  * sha_get_device_status -- synchronises `stream`, then reads and clears the
  * current device's sticky flags: SHA_ERR_BAD_INDEX if any call since the last
  * read met an out-of-range head id, SHA_ERR_TIMEOUT if a pipeline wait gave
- * up, SHA_OK otherwise (SHA_ERR_LAUNCH if the read itself failed).
+ * up, SHA_OK otherwise (SHA_ERR_LAUNCH if the read itself failed).  After a
+ * timeout it also zeroes the arrival counters of the library-owned workspace
+ * (sha_decode, _bf16, _varlen, _paged, _strided), enqueued on `stream` and
+ * waited for: no call that uses that workspace may then be running on
+ * another stream.  A caller-owned workspace (sha_decode_ex) must be zeroed by
+ * its owner.
  */
 sha_status_t sha_get_device_status(void *stream);
 
@@ -376,8 +391,10 @@ sha_status_t sha_copy_bandwidth_probe(void *dst, const void *src, size_t bytes,
  *     SHA_ERR_WORKSPACE before anything is enqueued; with num_splits = 0 this
  *     happens only on GPUs with more than 396 SMs (d = 128);
  *   - the first call on a device looks the array's address up once
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture;
+ *     (cudaGetSymbolAddress) with that device current and keeps it for the
+ *     life of the process; make that first call before any stream capture.
+ *     The kept address does not survive cudaDeviceReset: do not call this
+ *     entry point on a device after resetting it;
  *   - every call on a device shares the one array, which keeps whatever the
  *     last call left in it.  Each call clears the arrival counters it uses
  *     (a cudaMemsetAsync on `stream`) before its kernel; partial states need
@@ -385,6 +402,8 @@ sha_status_t sha_copy_bandwidth_probe(void *dst, const void *src, size_t bytes,
  *     threads) race on the array and give wrong results: serialise them.
  */
 #define SHA_NOALLOC_SCRATCH_BYTES (512 * 1024)
+/* The size of that array in the library as built (SHA_NOALLOC_SCRATCH_BYTES). */
+size_t sha_noalloc_scratch_bytes(void);
 sha_status_t sha_decode_noalloc(const void *q, const void *k, const void *v,
                                 const int32_t *batch_head_index, int B, int H_q,
                                 int H_kv, int N_kv, int d, int top_k, float scale,
