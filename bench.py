@@ -61,9 +61,14 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=100)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--config", default="opt66b", choices=sorted(workloads.CONFIGS))
-    p.add_argument("--layout", default="head_major", choices=["head_major", "token_major"],
-                   help="K/V cache layout of the timed step: [B, H_kv, N_kv, d] (sha_decode) "
-                        "or [B, N_kv, H_kv, d] (sha_decode_strided; implies --no-extras)")
+    p.add_argument("--layout", default="head_major",
+                   choices=["head_major", "token_major", "varlen", "paged16"],
+                   help="K/V cache of the timed step: [B, H_kv, N_kv, d] (sha_decode), "
+                        "[B, N_kv, H_kv, d] (sha_decode_strided), per-row lengths uniform in "
+                        "[1, N_kv] (sha_decode_varlen) or 16-key pages in random pool order "
+                        "(sha_decode_paged); all but head_major imply --no-extras")
+    p.add_argument("--sustained-s", type=float, default=1.5,
+                   help="seconds of graph-replayed steps in the sustained leg (0 skips it)")
     p.add_argument("--batch", type=int, default=None,
                    help="override the workload's batch size (small ncu captures)")
     p.add_argument("--no-extras", action="store_true",
@@ -320,6 +325,54 @@ def aggregate(bytes_per_step, steps, elapsed_s, world, device="cuda"):
 
 # ---------------------------------------------------------------- arms
 
+KV_LAYOUTS = {"head_major": "[B, H_kv, N_kv, d]",
+              "token_major": "[B, N_kv, H_kv, d] (strided views)",
+              "varlen": "[B, H_kv, N_kv, d], per-row lengths uniform in [1, N_kv]",
+              "paged16": "pool [pages, H_kv, 16, d] + block table, random page order"}
+
+
+def paged_cache(k, v, w, page_size, dev):
+    """k, v [B, H_kv, N_kv, d] moved into a page pool in random page order:
+    (k_pages, v_pages, block_table, lengths), all on dev."""
+    P = -(-w.N_kv // page_size)
+    n_pages = w.B * P
+    gc = torch.Generator().manual_seed(w.seed + 3)
+    table = torch.randperm(n_pages, generator=gc).to(torch.int32).view(w.B, P).to(dev)
+    kp = torch.zeros((n_pages, w.H_kv, page_size, w.d), dtype=k.dtype, device=dev)
+    vp = torch.zeros_like(kp)
+    pad = P * page_size - w.N_kv
+    for b in range(w.B):
+        kb = torch.nn.functional.pad(k[b], (0, 0, 0, pad)).view(w.H_kv, P, page_size, w.d)
+        vb = torch.nn.functional.pad(v[b], (0, 0, 0, pad)).view(w.H_kv, P, page_size, w.d)
+        kp[table[b].long()] = kb.permute(1, 0, 2, 3)
+        vp[table[b].long()] = vb.permute(1, 0, 2, 3)
+    lens = torch.full((w.B,), w.N_kv, dtype=torch.int32, device=dev)
+    return kp, vp, table, lens
+
+
+def sustained_leg(sha, step, bytes_step, launch_s, seconds, dev, stream, world, local, peak):
+    """The same step replayed for about `seconds` (graphs of 100 steps), with its
+    own clock record: the rate a decode server sees under the power cap, beside
+    the short burst of the main timing."""
+    steps = max(100, int(math.ceil(seconds / max(launch_s, 1e-7) / 100.0)) * 100)
+    sampler = ClockSampler(dev)
+    time.sleep(0.3)                       # first samples before the load starts
+    sync_all(world, local)
+    t0 = time.time()
+    elapsed = timed_graphs(step, steps, dev, stream)
+    t1 = time.time()
+    sync_all(world, local)
+    clocks = sampler.stop(t0, t1)
+    status = sha.sha_get_device_status()
+    if status != sha.SHA_OK:
+        raise RuntimeError(f"device status after the sustained leg: {sha.sha_status_string(status)}")
+    value, t_max = aggregate(bytes_step, steps, elapsed, world)
+    return {"value": round(value, 2), "unit": "GB/s", "steps": steps,
+            "seconds": round(t_max, 3), "ms_per_step": round(t_max / steps * 1e3, 5),
+            "frac_of_measured": round(bytes_step * steps / t_max / 1e9 / peak, 4),
+            "gpu_launches": steps, "clocks": clocks}
+
+
 def run_ours(args, rank, world, local):
     import head_sparse_decode_b200 as sha
 
@@ -331,6 +384,7 @@ def run_ours(args, rank, world, local):
     out = workloads.make_out(w, dev)
     stream = torch.cuda.current_stream(dev)
 
+    bytes_step = w.algorithmic_bytes()
     if args.layout == "token_major":
         # the same values stored [B, N_kv, H_kv, d], read through strided views
         k = k.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
@@ -340,6 +394,27 @@ def run_ours(args, rank, world, local):
 
         def step():
             sha.sha_decode_strided(q, k, v, idx, w.scale, out)
+    elif args.layout == "varlen":
+        # row b attends to its first lens[b] keys, lengths uniform in [1, N_kv]
+        args.no_extras = True
+        g = torch.Generator().manual_seed(w.seed + 11)
+        lens = torch.randint(1, w.N_kv + 1, (w.B,), generator=g, dtype=torch.int32)
+        lens_d = lens.to(dev)
+        bytes_step = (sum(2 * int(L) * w.d * 2 * w.top_k for L in lens.tolist())
+                      + 2 * w.units * w.G * w.d * 2 + 4 * w.units + 4 * w.B)
+
+        def step():
+            sha.sha_decode_varlen(q, k, v, idx, lens_d, w.scale, out)
+    elif args.layout == "paged16":
+        # the cache in 16-key pages scattered over a pool in random order
+        args.no_extras = True
+        kp, vp, table, lens_d = paged_cache(k, v, w, 16, dev)
+        del k, v
+        torch.cuda.empty_cache()
+        bytes_step = w.algorithmic_bytes() + 4 * w.B + 4 * table.numel()
+
+        def step():
+            sha.sha_decode_paged(q, kp, vp, idx, lens_d, table, w.scale, out)
     else:
         def step():
             sha.decode(q, k, v, idx, w.scale, out)
@@ -368,11 +443,14 @@ def run_ours(args, rank, world, local):
     if status != sha.SHA_OK:
         raise RuntimeError(f"device status after timing: {sha.sha_status_string(status)}")
 
-    bytes_step = w.algorithmic_bytes()
     value, t_max = aggregate(bytes_step, args.steps, elapsed, world)
     launch_s = elapsed / args.steps
     achieved = bytes_step / launch_s / 1e9
     peak, peak_src = measured_peak()
+    sustained = None
+    if args.sustained_s > 0:
+        sustained = sustained_leg(sha, step, bytes_step, launch_s, args.sustained_s, dev,
+                                  stream, world, local, peak)
 
     extras = {}
     if not args.no_extras:
@@ -385,8 +463,10 @@ def run_ours(args, rank, world, local):
         mlp = run_mlp(argparse.Namespace(batch=None), dev)
         extras["selective_mlp"] = {"config": mlp["config"], "cublas_dense_us": mlp["cublas_dense_us"],
                                    "points": mlp["points"]}
-    plan = sha.sha_decode_plan(w.B, w.H_q, w.H_kv, w.N_kv, w.d, w.top_k,
-                               num_sms=torch.cuda.get_device_properties(dev).multi_processor_count)
+    plan = sha.sha_decode_plan_ex(
+        w.B, w.H_q, w.H_kv, w.N_kv, w.d, w.top_k,
+        num_sms=torch.cuda.get_device_properties(dev).multi_processor_count,
+        cluster_capacity=sha.sha_decode_cluster_capacity(w.d, dev))
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
@@ -397,21 +477,23 @@ def run_ours(args, rank, world, local):
                    "accumulation": "fp32", "l2": "no flush: active K/V per step "
                    f"{w.units * 2 * w.N_kv * w.d * 2 / 1e9:.2f} GB > 126 MB L2",
                    "blocks": plan["blocks"], "tile_keys": plan["tile_keys"],
-                   "kv_layout": "[B, H_kv, N_kv, d]" if args.layout == "head_major"
-                   else "[B, N_kv, H_kv, d] (strided views)",
+                   "cluster": plan["cluster"],
+                   "kv_layout": KV_LAYOUTS[args.layout],
                    "launch": "CUDA graph replay, 100 steps per graph"},
         "steps_per_s": round(args.steps / t_max, 2),
         "tokens_per_s": round(world * w.B * args.steps / t_max, 1),
         "hbm_frac_of_measured": round(achieved / peak, 4),
         "copy_probe_gbs": round(copy_gbs, 1),
         "clocks": clocks,
+        "sustained": sustained,
         "gpu_launches": args.steps,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": profiled_traffic(w.name) if args.layout == "head_major" else None,
                      "peak_source": peak_src,
                      # multi-head calls with d = 128 run on the grouped kernel's tensor cores
-                     "kernel": "sha_mha_decode_kernel" if w.G == 1 and w.d != 128
+                     "kernel": "sha_mha_decode_kernel"
+                               if w.G == 1 and (w.d != 128 or args.layout in ("varlen", "paged16"))
                                else "sha_gqa_decode_kernel",
                      "launch_us": round(launch_s * 1e6, 3),
                      "bytes_per_launch": bytes_step},

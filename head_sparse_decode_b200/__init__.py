@@ -22,7 +22,10 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIBRARY_PATH = os.path.join(_PKG, "libsha_decode.so")
+# SHA_DECODE_LIBRARY names another build of the same library, e.g. one made with
+# non-default tuning knobs (python head_sparse_decode_b200/build.py --define
+# SHA_MHA_TENSOR_CORES=0 --output /tmp/libsha_fma.so), for measurements.
+LIBRARY_PATH = os.environ.get("SHA_DECODE_LIBRARY") or os.path.join(_PKG, "libsha_decode.so")
 
 if not os.path.exists(LIBRARY_PATH):
     raise ImportError(

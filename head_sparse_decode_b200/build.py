@@ -1,6 +1,11 @@
 """Build libsha_decode.so (the C-ABI CUDA library) in-tree for sm_100a.
 
     python head_sparse_decode_b200/build.py [--force] [--verbose]
+    python head_sparse_decode_b200/build.py --define KNOB=VALUE [...] --output PATH
+
+The second form builds the library with non-default build-time knobs (for
+example SHA_MHA_TENSOR_CORES=0) at another path; the binding loads it when
+SHA_DECODE_LIBRARY names that path.
 """
 import glob
 import os
@@ -72,5 +77,15 @@ def build_test_hooks(force: bool = False) -> str:
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))
-    print(build_test_hooks(force="--force" in sys.argv))
+    import argparse
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--define", action="append", default=[])
+    ap.add_argument("--output")
+    a = ap.parse_args()
+    if a.define or a.output:
+        print(build(force=True, verbose=a.verbose, defines=a.define, output=a.output))
+    else:
+        print(build(force=a.force, verbose=a.verbose))
+        print(build_test_hooks(force=a.force))
