@@ -340,7 +340,7 @@ _lib.sha_decode_plan_ex.restype = _i
 _lib.sha_decode_cluster_capacity.argtypes = [_i, ctypes.POINTER(ctypes.c_int32)]
 _lib.sha_decode_cluster_capacity.restype = _i
 _lib.sha_decode_clustered.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_float,
-                                      _vp, _i, _i, _i, _vp]
+                                      _vp, _i, _i, _i, _i, _vp]
 _lib.sha_decode_clustered.restype = _i
 
 
@@ -348,15 +348,15 @@ def sha_decode_plan_ex(B, H_q, H_kv, N_kv, d, top_k, num_splits=0, num_sms=148,
                        cluster_capacity=None):
     """sha_decode_plan with the clustered cut: ``cluster_capacity`` maps a cluster
     size c (2..8) to the clusters of c blocks the device holds at once (None: no
-    clustered cut).  Adds cluster, units_per_cluster and pieces to the dict."""
-    plan = (ctypes.c_int64 * 8)()
+    clustered cut).  Adds cluster, units_per_cluster, whole_per_block and pieces."""
+    plan = (ctypes.c_int64 * 9)()
     caps = None
     if cluster_capacity is not None:
         caps = (ctypes.c_int32 * 9)(*[int(cluster_capacity.get(c, 0)) for c in range(9)])
     _check(_lib.sha_decode_plan_ex(B, H_q, H_kv, N_kv, d, top_k, num_splits, num_sms, caps, plan))
     return {"tiles_per_head": plan[0], "total_tiles": plan[1], "blocks": plan[2],
             "workspace_bytes": plan[3], "tile_keys": plan[4], "cluster": plan[5],
-            "units_per_cluster": plan[6], "pieces": plan[7]}
+            "units_per_cluster": plan[6], "pieces": plan[7], "whole_per_block": plan[8]}
 
 
 def sha_decode_cluster_capacity(d=128, device=None):
@@ -368,14 +368,15 @@ def sha_decode_cluster_capacity(d=128, device=None):
 
 
 def sha_decode_clustered(q, k, v, batch_head_index, scale, out, cluster, units_per_cluster=1,
-                         stream=None):
+                         whole_per_block=0, stream=None):
     """Selective head decode under a clustered cut chosen by the caller: clusters of
-    ``cluster`` blocks, each taking ``units_per_cluster`` whole (row, head) units
-    and merging their pieces in distributed shared memory."""
+    ``cluster`` blocks, each taking ``units_per_cluster`` (row, head) units, of which
+    ``whole_per_block`` go whole to each block and the rest are split into pieces
+    merged in distributed shared memory."""
     args, s = _decode_args(q, k, v, batch_head_index, scale, out, stream)
     with torch.cuda.device(k.device):
         _check(_lib.sha_decode_clustered(*args, _dtype_code(k.dtype), int(cluster),
-                                         int(units_per_cluster), s))
+                                         int(units_per_cluster), int(whole_per_block), s))
     return out
 
 

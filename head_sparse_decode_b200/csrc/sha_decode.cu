@@ -189,6 +189,7 @@ Plan make_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int num_spl
     pl.sched.pieces = 0;
     pl.sched.cluster = 0;
     pl.sched.units_per_cluster = 0;
+    pl.sched.whole_per_block = 0;
     long long ctas =
         num_splits > 0 ? num_splits : (long long)num_sms * blocks_per_sm(G, d, per_row_lengths);
     if (ctas > sha::kMaxBlocks) ctas = sha::kMaxBlocks;
@@ -233,28 +234,63 @@ Plan make_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int num_spl
         }
     }
     pl.sched.num_ctas = (int)ctas;
-    // The clustered cut, for calls with fewer units than blocks (whole units
-    // per block would leave SMs idle; pieces merged through the workspace pay
-    // a merge tail that grows with the parts): one unit per cluster of c
-    // blocks, all clusters in one wave, each block streaming one piece, the
-    // pieces merged in the cluster's shared memory.  Taken where the cost
-    // model rates it faster than whole units per block.
+    // The clustered cut.  Clusters of c blocks take upc units each: w whole
+    // units per block, and s = upc - c*w units split into c pieces whose parts
+    // merge in the cluster's shared memory, with every cluster in one wave.
+    // It pays where whole units per block would leave SMs idle (fewer units
+    // than blocks: w = 0, one unit per cluster) or stream unevenly in a short
+    // call (a few units per block: the leftover units shared), and is taken
+    // where the cost model rates it faster than the cut chosen so far.
     const long long blocks_avail = (long long)num_sms * blocks_per_sm(G, d, per_row_lengths);
-    if (num_splits == 0 && SHA_CLUSTER_CUT && caps && units < blocks_avail &&
+    if (num_splits == 0 && SHA_CLUSTER_CUT && caps && G <= sha::GqaConfig<128>::kMaxPartRows &&
         !fma_path(G, d, per_row_lengths)) {
         const long long tpu = pl.sched.tiles_per_unit;
         const double tile_bytes = 2.0 * tile * d * 2;
-        double best = stream_ns(tpu, units, tile_bytes);      // whole units, no merge
-        for (int c = 2; c <= sha::GqaConfig<128>::kClusterMax && c <= tpu; ++c) {
-            if (caps->n[c] < units || !cluster_stage_fits(G, d, c)) continue;
-            const double est =
-                stream_ns((tpu + c - 1) / c, units * c, tile_bytes) + SHA_CLUSTER_MERGE_NS;
-            if (est < best) {
-                best = est;
-                pl.sched.cluster = c;
-                pl.sched.units_per_cluster = 1;
-                pl.sched.num_ctas = (int)(units * c);
-                pl.sched.pieces = 0;
+        const long long n = pl.sched.num_ctas;
+        long long busiest;
+        bool merges;
+        if (pl.sched.pieces >= 1) {
+            const long long P = units * pl.sched.pieces;
+            busiest = 0;
+            for (long long c = 0; c < n; ++c) {
+                const long long t =
+                    pl.sched.piece_start((c + 1) * P / n) - pl.sched.piece_start(c * P / n);
+                busiest = t > busiest ? t : busiest;
+            }
+            merges = pl.sched.pieces > 1;
+        } else {
+            busiest = (pl.sched.total_tiles + n - 1) / n;
+            merges = !(pl.sched.total_tiles % n == 0 && (pl.sched.total_tiles / n) % tpu == 0);
+        }
+        // with fewer units than blocks the cluster cut is weighed against whole
+        // units per block (the merges of pieces through the workspace cost more
+        // than the model can say); otherwise against the cut chosen so far
+        const bool few_units = units < blocks_avail;
+        double best = few_units ? stream_ns(tpu, units, tile_bytes)
+                                : stream_ns(busiest, n, tile_bytes) + (merges ? SHA_SLOT_MERGE_NS : 0);
+        if (few_units || busiest < 32) {
+            for (int c = 2; c <= sha::GqaConfig<128>::kClusterMax && c <= tpu; ++c) {
+                if (caps->n[c] < 1 || !cluster_stage_fits(G, d, c)) continue;
+                const long long upc_min = (units + caps->n[c] - 1) / caps->n[c];
+                for (long long upc = upc_min; upc <= upc_min + 1; ++upc) {
+                    const long long w = upc / c, shared = upc - c * w;
+                    if (shared == 0) continue;              // whole units: not clustered
+                    const long long clusters = (units + upc - 1) / upc;
+                    if (clusters > caps->n[c] || clusters * c > sha::kMaxBlocks) continue;
+                    const long long tiles = w * tpu + shared * ((tpu + c - 1) / c);
+                    const double est = stream_ns(tiles, clusters * c, tile_bytes) +
+                                       (double)shared * SHA_CLUSTER_MERGE_NS;
+                    // a cut that also holds whole units must win clearly: the
+                    // model's error is about a tenth of a short call
+                    if (est < (w > 0 ? 0.9 : 1.0) * best) {
+                        best = est;
+                        pl.sched.cluster = c;
+                        pl.sched.units_per_cluster = (int)upc;
+                        pl.sched.whole_per_block = (int)w;
+                        pl.sched.num_ctas = (int)(clusters * c);
+                        pl.sched.pieces = 0;
+                    }
+                }
             }
         }
     }
@@ -277,20 +313,25 @@ Plan make_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k, int num_spl
 // clustered kernel cannot serve the call, SHA_ERR_INVALID_ARG for sizes out
 // of range.
 sha_status_t forced_cluster_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_k,
-                                 int cluster, int units_per_cluster, Plan &pl)
+                                 int cluster, int units_per_cluster, int whole_per_block,
+                                 Plan &pl)
 {
     const int G = H_q / H_kv;
     if (G > sha::GqaConfig<128>::kMaxPartRows || fma_path(G, d, false)) return SHA_ERR_UNSUPPORTED;
     pl = make_plan(B, H_q, H_kv, N_kv, d, top_k, 0, 1);
     const long long units = (long long)B * top_k;
-    if (cluster < 2 || cluster > sha::GqaConfig<128>::kClusterMax ||
-        cluster > pl.sched.tiles_per_unit || units_per_cluster < 1)
+    if (cluster < 2 || cluster > sha::GqaConfig<128>::kClusterMax || units_per_cluster < 1 ||
+        whole_per_block < 0 || (long long)cluster * whole_per_block > units_per_cluster)
+        return SHA_ERR_INVALID_ARG;
+    // units split into pieces need a tile per piece
+    if ((long long)cluster * whole_per_block < units_per_cluster && cluster > pl.sched.tiles_per_unit)
         return SHA_ERR_INVALID_ARG;
     if (!cluster_stage_fits(G, d, cluster)) return SHA_ERR_UNSUPPORTED;
     const long long clusters = (units + units_per_cluster - 1) / units_per_cluster;
     if (clusters * cluster > sha::kMaxBlocks) return SHA_ERR_INVALID_ARG;
     pl.sched.cluster = cluster;
     pl.sched.units_per_cluster = units_per_cluster;
+    pl.sched.whole_per_block = whole_per_block;
     pl.sched.num_ctas = (int)(clusters * cluster);
     pl.sched.pieces = 0;
     pl.counter_bytes = 0;
@@ -675,7 +716,7 @@ struct KvLayout {
 // N_kv is the padded length (per-row lengths) or max_pages * page_size (paged).
 // A caller's choice of the clustered cut (sha_decode_clustered); 0: the planner's.
 struct ForcedCluster {
-    int cluster = 0, units_per_cluster = 0;
+    int cluster = 0, units_per_cluster = 0, whole_per_block = 0;
 };
 
 sha_status_t decode_impl(const void *q, const void *k, const void *v, const int32_t *idx,
@@ -710,7 +751,7 @@ sha_status_t decode_impl(const void *q, const void *k, const void *v, const int3
     Plan pl;
     if (force.cluster) {
         st = forced_cluster_plan(B, H_q, H_kv, N_kv, d, top_k, force.cluster,
-                                 force.units_per_cluster, pl);
+                                 force.units_per_cluster, force.whole_per_block, pl);
         if (st != SHA_OK) return st;
     } else {
         pl = seqlens ? make_varlen_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits, info->num_sms)
@@ -930,13 +971,13 @@ sha_status_t sha_decode_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_
 
 sha_status_t sha_decode_plan_ex(int B, int H_q, int H_kv, int N_kv, int d, int top_k,
                                 int num_splits, int num_sms, const int32_t cluster_capacity[9],
-                                int64_t plan[8])
+                                int64_t plan[9])
 {
     sha_status_t st = check_shape(B, H_q, H_kv, N_kv, d, top_k, 1.0f);
     if (st != SHA_OK) return st;
     if (num_splits < 0 || num_sms < 1 || !plan) return SHA_ERR_INVALID_ARG;
     const int tile = tile_keys(H_q / H_kv, d, false);
-    for (int i = 0; i < 8; ++i) plan[i] = 0;
+    for (int i = 0; i < 9; ++i) plan[i] = 0;
     plan[4] = tile;
     if (B == 0 || top_k == 0) {
         plan[0] = (N_kv + tile - 1) / tile;
@@ -954,6 +995,7 @@ sha_status_t sha_decode_plan_ex(int B, int H_q, int H_kv, int N_kv, int d, int t
     plan[5] = pl.sched.cluster;
     plan[6] = pl.sched.units_per_cluster;
     plan[7] = pl.sched.pieces;
+    plan[8] = pl.sched.whole_per_block;
     return SHA_OK;
 }
 
@@ -975,12 +1017,13 @@ sha_status_t sha_decode_clustered(const void *q, const void *k, const void *v,
                                   const int32_t *batch_head_index, int B, int H_q, int H_kv,
                                   int N_kv, int d, int top_k, float scale, void *out,
                                   sha_dtype_t dtype, int cluster, int units_per_cluster,
-                                  void *stream)
+                                  int whole_per_block, void *stream)
 {
     if (cluster < 2) return SHA_ERR_INVALID_ARG;
     ForcedCluster force;
     force.cluster = cluster;
     force.units_per_cluster = units_per_cluster;
+    force.whole_per_block = whole_per_block;
     return decode_impl(q, k, v, batch_head_index, B, H_q, H_kv, N_kv, d, top_k, scale, out,
                        dtype, nullptr, 0, 0, stream, false, KvLayout(), force);
 }

@@ -359,11 +359,12 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
                (hi ? i - half : i) * part_stride;
     };
     uint16_t *owner_tab = reinterpret_cast<uint16_t *>(smem + C::kOwnerOffset);
-    int e0 = 0, e1 = 0;
+    int crank = 0, e0 = 0, e1 = 0;
     uint32_t cluster_bytes = 0;
     if constexpr (kCluster) {
-        e0 = 4 * (walk.rank * groups / P);
-        e1 = 4 * ((walk.rank + 1) * groups / P);
+        crank = walk.rank;
+        e0 = 4 * (crank * groups / P);
+        e1 = 4 * ((crank + 1) * groups / P);
         cluster_bytes = (uint32_t)(P * (e1 - e0 + 2 * G) * 4);
         // owner (high 4 bits) and offset within its slice (floats) per group;
         // read after the consumers' first named barrier
@@ -578,11 +579,15 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
                     : p.slots ? p.slots + (size_t)(2 * blockIdx.x + (first_seg ? 0 : 1)) *
                                               p.slot_floats
                               : nullptr;
-        if constexpr (kCluster) {
+        // under the clustered cut, a unit that is not whole here is shared by
+        // the cluster's blocks
+        bool shared = false;
+        if constexpr (kCluster) shared = !seg.whole;
+        if (shared) {
             // this block's part of the unit, slice by slice, to the blocks that
             // finish them (always, so that every block's byte count completes)
             const int buf = n_done & 1;
-            float *mine = cstage(buf, wk.rank);
+            float *mine = cstage(buf, crank);
             for (int e = 2 * tid; e < G * D; e += 2 * C::kConsumers) {
                 const uint32_t code = owner_tab[e >> 2];
                 const int row = e / D, c = e - row * D;
@@ -633,7 +638,7 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
         }
         named_barrier(1, C::kConsumers);
 
-        if constexpr (kCluster) {
+        if (shared) {
             // wait for this block's slices of every part (its own included), then
             // write them out merged in block order
             const int buf = n_done & 1;

@@ -44,12 +44,15 @@ struct Schedule {
     // the P = units * p pieces, so no block starts or ends inside a piece.
     int pieces;
     // >= 2: the clustered cut.  Blocks form thread-block clusters of this many;
-    // cluster k takes whole units [k * units_per_cluster, (k+1) * units_per_cluster)
-    // and its block of rank r streams piece r of each of them (tiles
-    // [r * tiles_per_unit / cluster, (r+1) * tiles_per_unit / cluster)).  The
-    // parts of a unit meet in the cluster's shared memory, not in the workspace.
+    // cluster k takes the units [k * units_per_cluster, (k+1) * units_per_cluster).
+    // The first cluster * whole_per_block of them go whole, whole_per_block to
+    // each block in rank order; the block of rank r streams piece r of each of
+    // the others (tiles [r * tiles_per_unit / cluster, (r+1) * tiles_per_unit /
+    // cluster)), before its whole units, and the pieces meet in the cluster's
+    // shared memory, not in the workspace.
     int cluster;
     int units_per_cluster;
+    int whole_per_block;
 
     // First tile of piece i of the unit-aligned cut (pieces >= 1).
     __host__ __device__ __forceinline__ long long piece_start(long long i) const

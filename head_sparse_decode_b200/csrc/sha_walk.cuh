@@ -63,11 +63,14 @@ struct UniformWalk {
     }
 };
 
-// Clustered cut (Schedule::cluster >= 2): this block's piece of each unit of
-// its cluster's range; every block of the cluster visits the same units.
+// Clustered cut (Schedule::cluster >= 2): this block's piece of each unit the
+// cluster shares, then its whole units.  Every block of a cluster visits the
+// same shared units in the same order; taking them first lets their merges
+// overlap the streaming of the whole units.
 struct ClusterWalk {
     int tiles_per_unit, cluster, rank;
-    long long u, u_end;
+    long long s, s_end;           // the cluster's shared units
+    long long u, u_end;           // this block's whole units
     int n_keys;
 
     __device__ __forceinline__ void start(const Schedule &S, long long units, int keys)
@@ -75,22 +78,38 @@ struct ClusterWalk {
         tiles_per_unit = S.tiles_per_unit;
         cluster = S.cluster;
         rank = (int)cluster_ctarank();
-        u = (long long)(blockIdx.x / S.cluster) * S.units_per_cluster;
-        u_end = u + S.units_per_cluster < units ? u + S.units_per_cluster : units;
+        const long long base = (long long)(blockIdx.x / S.cluster) * S.units_per_cluster;
+        const long long end =
+            base + S.units_per_cluster < units ? base + S.units_per_cluster : units;
+        const long long shared0 = base + (long long)S.cluster * S.whole_per_block;
+        u = base + (long long)rank * S.whole_per_block;
+        u_end = u + S.whole_per_block;
+        if (u_end > end) u_end = end;
+        s = shared0 < end ? shared0 : end;
+        s_end = end;
         n_keys = keys;
     }
-    __device__ __forceinline__ bool next(Seg &s)
+    __device__ __forceinline__ bool next(Seg &g)
     {
+        g.unit_tiles = tiles_per_unit;
+        g.n_keys = n_keys;
+        if (s < s_end) {
+            const int j0 = rank * tiles_per_unit / cluster;
+            const int j1 = (rank + 1) * tiles_per_unit / cluster;
+            g.unit = s;
+            g.first_tile = j0;
+            g.num_tiles = j1 - j0;
+            g.whole = false;
+            g.unit_start = s * tiles_per_unit;
+            ++s;
+            return true;
+        }
         if (u >= u_end) return false;
-        const int j0 = rank * tiles_per_unit / cluster;
-        const int j1 = (rank + 1) * tiles_per_unit / cluster;
-        s.unit = u;
-        s.first_tile = j0;
-        s.num_tiles = j1 - j0;
-        s.whole = false;
-        s.unit_start = u * tiles_per_unit;
-        s.unit_tiles = tiles_per_unit;
-        s.n_keys = n_keys;
+        g.unit = u;
+        g.first_tile = 0;
+        g.num_tiles = tiles_per_unit;
+        g.whole = true;
+        g.unit_start = u * tiles_per_unit;
         ++u;
         return true;
     }

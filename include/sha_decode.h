@@ -223,10 +223,11 @@ sha_status_t sha_decode_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_
  * parts through global memory (write, fence, arrival counter, read back) adds
  * microseconds at the end of the call.  Under the clustered cut the blocks
  * form thread-block clusters of c blocks (2 <= c <= 8); each cluster takes
- * units_per_cluster whole units, block r of the cluster streams piece r of
- * each of them (its tiles [r*T/c, (r+1)*T/c) of T = ceil(N_kv/tile)), and the
- * c parts of a unit are merged in the cluster's distributed shared memory,
- * each block writing 1/c of the unit's output.  It serves the grouped kernel:
+ * units_per_cluster units.  The first c * w of them go whole, w to each
+ * block; block r of the cluster streams piece r of each of the others (its
+ * tiles [r*T/c, (r+1)*T/c) of T = ceil(N_kv/tile)), and the c parts of such a
+ * unit are merged in the cluster's distributed shared memory, each block
+ * writing 1/c of the unit's output.  It serves the grouped kernel:
  * G = H_q/H_kv <= 8 with d = 128 (G = 1 included) or G >= 2 with d = 64, one
  * length per row, the contiguous [B, H_kv, N_kv, d] layout.  With
  * num_splits = 0 the planner of sha_decode, sha_decode_bf16, sha_decode_ex
@@ -243,10 +244,11 @@ sha_status_t sha_decode_plan(int B, int H_q, int H_kv, int N_kv, int d, int top_
  *   plan[6] = units per cluster
  *   plan[7] = 0 (tiles cut evenly), 1 (whole units per block),
  *             p >= 2 (each unit in p equal pieces) -- 0 under the clustered cut
+ *   plan[8] = whole units per block of a cluster (the clustered cut's w)
  */
 sha_status_t sha_decode_plan_ex(int B, int H_q, int H_kv, int N_kv, int d, int top_k,
                                 int num_splits, int num_sms, const int32_t cluster_capacity[9],
-                                int64_t plan[8]);
+                                int64_t plan[9]);
 
 /*
  * sha_decode_cluster_capacity -- the current device's cluster capacities for
@@ -260,10 +262,13 @@ sha_status_t sha_decode_cluster_capacity(int d, int32_t cluster_capacity[9]);
 /*
  * sha_decode_clustered -- sha_decode_ex with the clustered cut chosen by the
  * caller (for tests and measurements): clusters of `cluster` blocks, each
- * taking `units_per_cluster` whole units (the last cluster the rest).
- *   2 <= cluster <= min(8, ceil(N_kv / tile)), units_per_cluster >= 1, at most
- *   4096 blocks in all (SHA_ERR_INVALID_ARG otherwise); calls the clustered
- *   kernel cannot serve (above) return SHA_ERR_UNSUPPORTED.
+ * taking `units_per_cluster` units (the last cluster the rest), of which
+ * `whole_per_block` go whole to each block and the rest are split into
+ * `cluster` pieces.
+ *   2 <= cluster <= 8, units_per_cluster >= 1, 0 <= cluster * whole_per_block
+ *   <= units_per_cluster, cluster <= ceil(N_kv / tile) when any unit is split,
+ *   at most 4096 blocks in all (SHA_ERR_INVALID_ARG otherwise); calls the
+ *   clustered kernel cannot serve (above) return SHA_ERR_UNSUPPORTED.
  * Clusters beyond the device's capacity run in further waves.  The result is
  * the same as sha_decode_ex's to within rounding (the parts are merged in
  * block order by the same log-sum-exp arithmetic).  Allocates nothing.
@@ -272,7 +277,7 @@ sha_status_t sha_decode_clustered(const void *q, const void *k, const void *v,
                                   const int32_t *batch_head_index, int B, int H_q, int H_kv,
                                   int N_kv, int d, int top_k, float scale, void *out,
                                   sha_dtype_t dtype, int cluster, int units_per_cluster,
-                                  void *stream);
+                                  int whole_per_block, void *stream);
 
 /*
  * sha_select_heads -- router scores to batch_head_index on the device.

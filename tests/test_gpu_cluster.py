@@ -28,9 +28,9 @@ def _on_gpu(w):
     return q.to(dev), k.to(dev), v.to(dev), idx.to(dev)
 
 
-def _clustered(sha, w, q, k, v, idx, cluster, upc):
+def _clustered(sha, w, q, k, v, idx, cluster, upc, whole=0):
     out = workloads.make_out(w, "cuda")
-    sha.sha_decode_clustered(q, k, v, idx, w.scale, out, cluster, upc)
+    sha.sha_decode_clustered(q, k, v, idx, w.scale, out, cluster, upc, whole)
     torch.cuda.synchronize()
     assert sha.sha_get_device_status() == sha.SHA_OK
     return out
@@ -65,6 +65,31 @@ def test_clustered_matches_oracle(sha, case):
             check_against_oracle(w, q, k, v, idx, out, expected)
 
 
+# (workload, cluster, units per cluster, whole units per block): clusters
+# that hold whole units besides the ones they split, and a ragged last cluster
+MIXED = [
+    (W("m_mha", B=8, H_q=32, H_kv=32, N_kv=512, d=128, top_k=24, dtype="fp16", seed=421),
+     2, 3, 1),
+    (W("m_mha_ragged", B=5, H_q=16, H_kv=16, N_kv=900, d=128, top_k=7, dtype="bf16", seed=422),
+     3, 8, 2),
+    (W("m_gqa8", B=4, H_q=64, H_kv=8, N_kv=1000, d=128, top_k=5, dtype="bf16", seed=423),
+     2, 5, 2),
+    (W("m_gqa2_d64", B=6, H_q=8, H_kv=4, N_kv=700, d=64, top_k=3, dtype="fp16", seed=424),
+     4, 7, 1),
+    (W("m_all_whole", B=6, H_q=8, H_kv=8, N_kv=300, d=128, top_k=4, dtype="fp16", seed=425),
+     2, 4, 2),
+]
+
+
+@pytest.mark.parametrize("case", MIXED, ids=lambda c: c[0].name)
+def test_mixed_clustered_matches_oracle(sha, case):
+    w, c, upc, whole = case
+    q, k, v, idx = _on_gpu(w)
+    for _ in range(2):                      # repeated calls reuse the cluster barriers
+        out = _clustered(sha, w, q, k, v, idx, c, upc, whole)
+        check_against_oracle(w, q, k, v, idx, out)
+
+
 def test_clustered_repeat_bit_identical(sha):
     w = CASES[0][0]
     q, k, v, idx = _on_gpu(w)
@@ -97,12 +122,18 @@ def test_clustered_argument_checks(sha):
     w = W("c_args", B=1, H_q=8, H_kv=8, N_kv=300, d=128, top_k=2, dtype="fp16", seed=409)
     q, k, v, idx = _on_gpu(w)
     out = workloads.make_out(w, "cuda")
-    for c, upc, status in ((1, 1, sha.SHA_ERR_INVALID_ARG), (9, 1, sha.SHA_ERR_INVALID_ARG),
-                           (4, 1, sha.SHA_ERR_INVALID_ARG),      # 3 tiles: at most 3 pieces
-                           (2, 0, sha.SHA_ERR_INVALID_ARG)):
+    for c, upc, whole, status in ((1, 1, 0, sha.SHA_ERR_INVALID_ARG),
+                                  (9, 1, 0, sha.SHA_ERR_INVALID_ARG),
+                                  (4, 1, 0, sha.SHA_ERR_INVALID_ARG),   # 3 tiles: at most 3 pieces
+                                  (2, 0, 0, sha.SHA_ERR_INVALID_ARG),
+                                  (2, 3, 2, sha.SHA_ERR_INVALID_ARG),   # 4 whole units > 3
+                                  (2, 1, -1, sha.SHA_ERR_INVALID_ARG)):
         with pytest.raises(sha.ShaError) as e:
-            sha.sha_decode_clustered(q, k, v, idx, w.scale, out, c, upc)
+            sha.sha_decode_clustered(q, k, v, idx, w.scale, out, c, upc, whole)
         assert e.value.status == status
+    # clusters of 4 whose units all go whole need no piece per tile
+    sha.sha_decode_clustered(q, k, v, idx, w.scale, out, 4, 4, 1)
+    check_against_oracle(w, q, k, v, idx, out)
     # the multi-head FMA kernel's calls (d = 64, G = 1) and G > 8 are not served
     w64 = w.with_(d=64)
     q6, k6, v6, i6 = _on_gpu(w64)
@@ -135,7 +166,8 @@ def test_capacity_and_planner_choice(sha):
     torch.cuda.synchronize()
     assert sha.sha_get_device_status() == sha.SHA_OK
     check_against_oracle(w, q, k, v, idx, out)
-    forced = _clustered(sha, w, q, k, v, idx, plan["cluster"], plan["units_per_cluster"])
+    forced = _clustered(sha, w, q, k, v, idx, plan["cluster"], plan["units_per_cluster"],
+                        plan["whole_per_block"])
     assert np.array_equal(out_bits(out), out_bits(forced))
 
 

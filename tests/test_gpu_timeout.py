@@ -32,7 +32,7 @@ def libs():
         getattr(hooks, name).argtypes = args
         getattr(hooks, name).restype = i
     hooks.sha_decode_clustered.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, ctypes.c_float, vp,
-                                           i, i, i, vp]
+                                           i, i, i, i, vp]
     hooks.sha_decode_clustered.restype = i
     hooks.sha_get_device_status.argtypes = [vp]
     hooks.sha_get_device_status.restype = i
@@ -54,7 +54,7 @@ def _call(hooks, w, q, k, v, idx, out, cluster=0):
     a = (q.data_ptr(), k.data_ptr(), v.data_ptr(), idx.data_ptr(), w.B, w.H_q, w.H_kv, w.N_kv,
          w.d, w.top_k, w.scale, out.data_ptr())
     if cluster:
-        return hooks.sha_decode_clustered(*a, 0 if w.dtype == "fp16" else 1, cluster, 1, s)
+        return hooks.sha_decode_clustered(*a, 0 if w.dtype == "fp16" else 1, cluster, 1, 0, s)
     fn = hooks.sha_decode if w.dtype == "fp16" else hooks.sha_decode_bf16
     return fn(*a, s)
 

@@ -73,6 +73,9 @@ CLUSTERED = {
     "b1_n8192_k8": ((1, 32, 32, 8192, 128, 8), 8),      # 11.4 us; even cut 14.6
     "b8_n1920_k8": ((8, 32, 32, 1920, 128, 8), 2),      # 14.4 us; pieces 17.8
     "llama31_70b_gqa_16k": ((8, 64, 8, 16384, 128, 5), 3),   # 51.3 us; even cut 56.5
+    # a few units per block: clusters of 2, each block one whole unit and half of
+    # a shared one (6 tiles), against two whole units on some blocks (8 tiles)
+    "b8_n512_k24": ((8, 32, 32, 512, 128, 24), 2),
     # whole units win: short units with no idle SMs to gain
     "b8_n512_k8": ((8, 32, 32, 512, 128, 8), 0),        # 7.4 us; clusters of 2 7.8
     # more units than clusters fit at once: the planner's other cuts
@@ -92,8 +95,13 @@ def test_clustered_cut_of_measured_shapes(name):
     assert p["cluster"] == cluster, p
     if cluster:
         units = args[0] * args[5]
-        assert p["units_per_cluster"] == 1 and p["blocks"] == units * cluster
+        upc = p["units_per_cluster"]
+        assert p["blocks"] == -(-units // upc) * cluster
         assert p["workspace_bytes"] == 0 and p["pieces"] == 0
+        if name == "b8_n512_k24":
+            assert (upc, p["whole_per_block"]) == (3, 1)
+        else:
+            assert (upc, p["whole_per_block"]) == (1, 0)
     else:
         # without the clustered cut the plan is sha_decode_plan's
         q = sha.sha_decode_plan(*args, num_sms=148)
@@ -127,8 +135,12 @@ def test_clustered_plan_invariants(G, d):
                 if not c:
                     continue
                 units = B * k
-                # a cluster per unit, in one wave, each block at least one tile
+                upc, whole = p["units_per_cluster"], p["whole_per_block"]
+                clusters = -(-units // upc)
+                # one wave of clusters, each splitting at least one unit into
+                # pieces of at least one tile
                 assert 2 <= c <= 8 and c <= p["tiles_per_head"]
-                assert units <= B200_CLUSTERS[c] and p["blocks"] == units * c
+                assert clusters <= B200_CLUSTERS[c] and p["blocks"] == clusters * c
+                assert 0 <= c * whole < upc
                 assert G <= 8 and not (G == 1 and d == 64)
                 assert p["workspace_bytes"] == 0
