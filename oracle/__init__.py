@@ -53,6 +53,11 @@ def _load():
         lib.sha_oracle_decode_varlen.argtypes = [
             u16p, u16p, u16p, i32p, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int, f64p]
+        lib.sha_oracle_decode_tokens.restype = ctypes.c_longlong
+        lib.sha_oracle_decode_tokens.argtypes = [
+            u16p, u16p, u16p, i32p, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
+            f64p]
         lib.sha_oracle_decode_paged.restype = ctypes.c_longlong
         lib.sha_oracle_decode_paged.argtypes = [
             u16p, u16p, u16p, i32p, i32p, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -199,6 +204,30 @@ def sha_decode_varlen(q, k, v, batch_head_index, seqlens, scale, dtype, out=None
         _ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16),
         _ptr(idx, ctypes.c_int32), _ptr(lens, ctypes.c_int32), B, H_q, H_kv, N_max, d, top_k,
         float(scale), _dtype_code(dtype), _ptr(out, ctypes.c_double))
+    if bad < 0:
+        raise ValueError("inconsistent sizes")
+    return out, int(bad)
+
+
+def sha_decode_tokens(q, k, v, batch_head_index, tokens, scale, dtype, out=None):
+    """Head x token sparsity: unit (b, slot k) attends only to the keys listed in
+    tokens[b, k, :] (int32 [B, top_k, n_sel], positions in [0, N_kv) of its head).
+    Units with a position out of range are skipped and counted with bad head
+    ids.  Same other conventions as sha_decode.  Returns (out, count)."""
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, H_kv, N_kv, d = kb.shape
+    qb = qb.reshape(B, -1, d)
+    H_q = qb.shape[1]
+    idx = np.ascontiguousarray(np.asarray(batch_head_index, dtype=np.int32).reshape(B, -1))
+    top_k = idx.shape[1]
+    tok = np.ascontiguousarray(np.asarray(tokens, dtype=np.int32).reshape(B, top_k, -1))
+    n_sel = tok.shape[2]
+    if out is None:
+        out = np.full((B, H_q, d), np.nan, dtype=np.float64)
+    bad = _load().sha_oracle_decode_tokens(
+        _ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16),
+        _ptr(idx, ctypes.c_int32), _ptr(tok, ctypes.c_int32), B, H_q, H_kv, N_kv, d, top_k,
+        n_sel, float(scale), _dtype_code(dtype), _ptr(out, ctypes.c_double))
     if bad < 0:
         raise ValueError("inconsistent sizes")
     return out, int(bad)

@@ -325,6 +325,69 @@ long long sha_oracle_decode_varlen(const uint16_t *Q, const uint16_t *K,
 }
 
 /*
+ * Head x token sparsity.  The pages name it only as future work: combining
+ * head sparsity with token sparsity "may give multiplicative speedups"
+ * (papernotes.org summary, "局限与展望"); they give no method.  The plainest
+ * reading: each selected (batch row, head) unit attends to a given subset of
+ * its own head's keys,
+ *     tokens : [B, top_k, n_sel], key positions in [0, N_kv) of the head
+ *              selected by slot k of row b,
+ * and the unit's output is the attention equation restricted to those keys:
+ *     s_i = scale * <q, K[t_i]>,  O = sum_i exp(s_i - M) V[t_i] / sum_i exp(s_i - M),
+ * M = max_i s_i, i < n_sel.  A position listed twice counts twice (the subset
+ * is a list).  A unit with a position outside [0, N_kv) is skipped (nothing
+ * written) and counted with the out-of-range head ids.  Returns the count,
+ * or -1 for inconsistent sizes.
+ */
+long long sha_oracle_decode_tokens(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
+                                   const int32_t *batch_head_index, const int32_t *tokens,
+                                   int B, int H_q, int H_kv, int N_kv, int d, int top_k,
+                                   int n_sel, double scale, int dtype, double *out)
+{
+    if (B < 0 || H_kv <= 0 || H_q <= 0 || H_q % H_kv != 0 || N_kv <= 0 || d <= 0 ||
+        top_k < 0 || n_sel <= 0)
+        return -1;
+    int G = H_q / H_kv;
+    long long bad = 0;
+    long long units = (long long)B * top_k;
+#pragma omp parallel for schedule(dynamic, 1) reduction(+ : bad)
+    for (long long u = 0; u < units; ++u) {
+        long long b = u / top_k;
+        int h = batch_head_index[u];
+        const int32_t *t = tokens + (size_t)u * n_sel;
+        int ok = h >= 0 && h < H_kv;
+        for (int i = 0; ok && i < n_sel; ++i) ok = t[i] >= 0 && t[i] < N_kv;
+        if (!ok) {
+            bad += 1;
+            continue;
+        }
+        const uint16_t *K_bh = K + ((size_t)b * H_kv + h) * (size_t)N_kv * d;
+        const uint16_t *V_bh = V + ((size_t)b * H_kv + h) * (size_t)N_kv * d;
+        double *sc = (double *)malloc(sizeof(double) * (size_t)n_sel);
+        for (int j = 0; j < G; ++j) {
+            size_t row = ((size_t)b * H_q + (size_t)h * G + j) * (size_t)d;
+            double M = -INFINITY;
+            for (int i = 0; i < n_sel; ++i) {
+                sc[i] = score(Q + row, K_bh + (size_t)t[i] * d, d, scale, dtype);
+                if (sc[i] > M) M = sc[i];
+            }
+            double L = 0.0;
+            double *o = out + row;
+            for (int c = 0; c < d; ++c) o[c] = 0.0;
+            for (int i = 0; i < n_sel; ++i) {
+                double p = exp(sc[i] - M);
+                L += p;
+                const uint16_t *v_row = V_bh + (size_t)t[i] * d;
+                for (int c = 0; c < d; ++c) o[c] += p * widen(v_row[c], dtype);
+            }
+            for (int c = 0; c < d; ++c) o[c] /= L;
+        }
+        free(sc);
+    }
+    return bad;
+}
+
+/*
  * Selective head decode over a paged KV cache (the serving layout in which a
  * sequence's keys live in fixed-size pages of a shared pool):
  *   K, V        : [num_pages, H_kv, page_size, d]

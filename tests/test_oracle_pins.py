@@ -393,3 +393,96 @@ def test_selective_mlp_column_subset_is_the_same_sum():
     cols = [1, 7, 15]
     sub = oracle.selective_mlp(x, W1t, W2t[:, cols].contiguous(), S, "fp16")
     np.testing.assert_array_equal(sub, full[:, cols])
+
+
+# ---------------------------------------------------------------- head x token sparsity
+
+def _token_case(seed, B=3, H_q=8, H_kv=4, N_kv=40, d=16, top_k=2, n_sel=9, dtype="fp16"):
+    w = workloads.Workload("tok", B=B, H_q=H_q, H_kv=H_kv, N_kv=N_kv, d=d, top_k=top_k,
+                           dtype=dtype, seed=seed)
+    q, k, v = workloads.make_qkv(w)
+    idx = workloads.make_index(w).numpy()
+    rng = np.random.default_rng(seed)
+    tok = rng.integers(0, N_kv, size=(B, top_k, n_sel)).astype(np.int32)
+    return w, q, k, v, idx, tok
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_tokens_equal_the_unit_oracle_on_a_gathered_cache(dtype):
+    # restricting a unit to its listed keys is the ordinary per-unit attention
+    # over a cache that holds exactly those keys, in that order
+    w, q, k, v, idx, tok = _token_case(11, dtype=dtype)
+    got, bad = oracle.sha_decode_tokens(q, k, v, idx, tok, w.scale, dtype)
+    assert bad == 0
+    G = w.G
+    units = [(b, s) for b in range(w.B) for s in range(w.top_k)]
+    qu = torch.stack([q[b, idx[b, s] * G:(idx[b, s] + 1) * G] for b, s in units])
+    ku = torch.stack([k[b, idx[b, s]][torch.from_numpy(tok[b, s]).long()] for b, s in units])
+    vu = torch.stack([v[b, idx[b, s]][torch.from_numpy(tok[b, s]).long()] for b, s in units])
+    ref = oracle.sha_units(qu, ku, vu, w.scale, dtype)
+    for i, (b, s) in enumerate(units):
+        h = idx[b, s]
+        assert np.abs(got[b, h * G:(h + 1) * G] - ref[i]).max() < 1e-12
+
+
+def test_tokens_brute_force_numpy():
+    w, q, k, v, idx, tok = _token_case(12, B=2, H_q=2, H_kv=2, N_kv=13, d=8, top_k=1, n_sel=5)
+    got, _ = oracle.sha_decode_tokens(q, k, v, idx, tok, w.scale, w.dtype)
+    for b in range(w.B):
+        h = idx[b, 0]
+        qd = q[b, h].double().numpy()
+        K = k[b, h].double().numpy()[tok[b, 0]]
+        V = v[b, h].double().numpy()[tok[b, 0]]
+        s = w.scale * K @ qd
+        p = np.exp(s - s.max())
+        want = p @ V / p.sum()
+        assert np.abs(got[b, h] - want).max() < 1e-12
+
+
+def test_all_positions_in_order_is_the_full_decode():
+    w, q, k, v, idx, _ = _token_case(13, N_kv=23)
+    tok = np.broadcast_to(np.arange(w.N_kv, dtype=np.int32), (w.B, w.top_k, w.N_kv)).copy()
+    got, bad = oracle.sha_decode_tokens(q, k, v, idx, tok, w.scale, w.dtype)
+    full, _ = oracle.sha_decode(q, k, v, idx, w.scale, w.dtype)
+    assert bad == 0
+    written = ~np.isnan(full)
+    assert np.array_equal(np.isnan(got), np.isnan(full))
+    assert np.abs(got[written] - full[written]).max() < 1e-12
+
+
+def test_token_order_and_duplication_invariance():
+    w, q, k, v, idx, tok = _token_case(14, n_sel=6)
+    base, _ = oracle.sha_decode_tokens(q, k, v, idx, tok, w.scale, w.dtype)
+    rng = np.random.default_rng(5)
+    perm = np.stack([np.stack([rng.permutation(t) for t in row]) for row in tok])
+    shuffled, _ = oracle.sha_decode_tokens(q, k, v, idx, perm, w.scale, w.dtype)
+    doubled, _ = oracle.sha_decode_tokens(q, k, v, idx, np.repeat(tok, 2, axis=2), w.scale,
+                                          w.dtype)
+    m = ~np.isnan(base)
+    assert np.abs(shuffled[m] - base[m]).max() < 1e-12
+    assert np.abs(doubled[m] - base[m]).max() < 1e-12
+
+
+def test_single_token_returns_its_value_row():
+    w, q, k, v, idx, tok = _token_case(15, n_sel=1)
+    got, _ = oracle.sha_decode_tokens(q, k, v, idx, tok, w.scale, w.dtype)
+    for b in range(w.B):
+        for s in range(w.top_k):
+            h = idx[b, s]
+            want = v[b, h, tok[b, s, 0]].double().numpy()
+            for j in range(w.G):
+                assert np.array_equal(got[b, h * w.G + j], want)
+
+
+def test_units_with_out_of_range_tokens_are_skipped_and_counted():
+    w, q, k, v, idx, tok = _token_case(16)
+    tok[0, 1, 3] = w.N_kv
+    tok[2, 0, 0] = -1
+    got, bad = oracle.sha_decode_tokens(q, k, v, idx, tok, w.scale, w.dtype)
+    assert bad == 2
+    G = w.G
+    for b, s in ((0, 1), (2, 0)):
+        h = idx[b, s]
+        assert np.isnan(got[b, h * G:(h + 1) * G]).all()
+    h = idx[0, 0]
+    assert not np.isnan(got[0, h * G:(h + 1) * G]).any()
