@@ -258,6 +258,27 @@ def sha_decode_strided(q, k, v, batch_head_index, scale, out, seqlens=None, stre
     return out
 
 
+_lib.sha_decode_tokens.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
+                                   ctypes.c_float, _vp, _i, _vp]
+_lib.sha_decode_tokens.restype = _i
+
+
+def sha_decode_tokens(q, k, v, batch_head_index, tokens, scale, out, stream=None):
+    """Head x token sparsity: unit (b, slot k) attends only to the keys listed in
+    tokens[b, k, :] (int32 [B, top_k, n_sel] on the device, positions in
+    [0, N_kv) of the selected head's cache)."""
+    args, s = _decode_args(q, k, v, batch_head_index, scale, out, stream)
+    B, top_k = batch_head_index.shape
+    if (tokens.dim() != 3 or tokens.shape[0] != B or tokens.shape[1] != top_k
+            or tokens.dtype != torch.int32 or not tokens.is_contiguous()
+            or tokens.device != k.device):
+        raise ValueError("tokens must be a contiguous int32 [B, top_k, n_sel] tensor on k's device")
+    with torch.cuda.device(k.device):
+        _check(_lib.sha_decode_tokens(*args[:4], tokens.data_ptr(), *args[4:10],
+                                      tokens.shape[2], *args[10:], _dtype_code(k.dtype), s))
+    return out
+
+
 def _dtype_code(dtype):
     if dtype == torch.float16:
         return SHA_FP16

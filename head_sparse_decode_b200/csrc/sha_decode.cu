@@ -609,6 +609,18 @@ sha_status_t launch_look(const sha::DecodeParams &prm, sha_dtype_t dtype, bool f
                 : launch_one<T, D, kLayout, false>(prm, dtype, fma, dev, s, kv);
 }
 
+// Head x token sparsity: the grouped kernel's gathering build.
+template <typename T>
+sha_status_t launch_tokens(const sha::DecodeParams &prm, sha_dtype_t dtype, int d, bool look,
+                           int dev, cudaStream_t s)
+{
+    if (d == 128)
+        return look ? launch_gqa<T, 128, sha::kLayoutTokens, true>(prm, dtype, dev, s, nullptr)
+                    : launch_gqa<T, 128, sha::kLayoutTokens, false>(prm, dtype, dev, s, nullptr);
+    return look ? launch_gqa<T, 64, sha::kLayoutTokens, true>(prm, dtype, dev, s, nullptr)
+                : launch_gqa<T, 64, sha::kLayoutTokens, false>(prm, dtype, dev, s, nullptr);
+}
+
 // The clustered cut: the grouped kernel only, no scout.
 template <typename T>
 sha_status_t launch_cluster(const sha::DecodeParams &prm, sha_dtype_t dtype, int d, int dev,
@@ -711,6 +723,8 @@ struct KvLayout {
     int page_size = 0, max_pages = 0, num_pages = 0;
     bool strided = false;                   // K, V with the strides below (elements)
     KvStrides k_strides{}, v_strides{};
+    const int32_t *tokens = nullptr;        // head x token sparsity: [B, top_k, n_sel] (device)
+    int n_sel = 0;
 };
 
 // N_kv is the padded length (per-row lengths) or max_pages * page_size (paged).
@@ -738,6 +752,7 @@ sha_status_t decode_impl(const void *q, const void *k, const void *v, const int3
         return SHA_ERR_MISALIGNED;
     if (workspace && !aligned(workspace, 256)) return SHA_ERR_MISALIGNED;
     if (seqlens && !aligned(seqlens, 4)) return SHA_ERR_MISALIGNED;
+    if (lay.tokens && !aligned(lay.tokens, 4)) return SHA_ERR_MISALIGNED;
     if (lay.block_table && !aligned(lay.block_table, 4)) return SHA_ERR_MISALIGNED;
     const int G = H_q / H_kv;
 
@@ -747,19 +762,24 @@ sha_status_t decode_impl(const void *q, const void *k, const void *v, const int3
     if (st != SHA_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const ClusterCaps *caps =
-        cluster_caps(dev, d, !seqlens && !lay.strided && !lay.block_table);
+        cluster_caps(dev, d, !seqlens && !lay.strided && !lay.block_table && !lay.tokens);
     Plan pl;
     if (force.cluster) {
         st = forced_cluster_plan(B, H_q, H_kv, N_kv, d, top_k, force.cluster,
                                  force.units_per_cluster, force.whole_per_block, pl);
         if (st != SHA_OK) return st;
+    } else if (lay.tokens) {
+        // the call streams n_sel keys per unit: plan it as a cache that long
+        pl = make_plan(B, H_q, H_kv, lay.n_sel, d, top_k, num_splits, info->num_sms, false,
+                       nullptr);
     } else {
         pl = seqlens ? make_varlen_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits, info->num_sms)
                      : make_plan(B, H_q, H_kv, N_kv, d, top_k, num_splits, info->num_sms, false,
                                  caps);
     }
     const size_t need = pl.workspace_bytes();
-    const bool fma = fma_path(G, d, seqlens != nullptr);   // paged calls carry lengths too
+    // paged calls carry lengths too; gathered keys take the grouped kernel
+    const bool fma = !lay.tokens && fma_path(G, d, seqlens != nullptr);
     const bool look = pl.sched.cluster < 2 && lookahead_pays(pl, G, fma, seqlens != nullptr);
 
     if (library_workspace && need > 0) {
@@ -810,6 +830,8 @@ sha_status_t decode_impl(const void *q, const void *k, const void *v, const int3
     prm.tok_dim = 0;
     prm.head_dim = 1;
     prm.batch_dim = 2;
+    prm.tokens = lay.tokens;
+    prm.n_sel = lay.n_sel;
     if (lay.strided) {
         StridedMaps kv;
         int vt, vh, vb;
@@ -823,6 +845,9 @@ sha_status_t decode_impl(const void *q, const void *k, const void *v, const int3
             return launch_decode<sha::kLayoutStridedVarlen>(prm, dtype, d, fma, look, dev, s, &kv);
         return launch_decode<sha::kLayoutStrided>(prm, dtype, d, fma, look, dev, s, &kv);
     }
+    if (lay.tokens)
+        return dtype == SHA_FP16 ? launch_tokens<__half>(prm, dtype, d, look, dev, s)
+                                 : launch_tokens<__nv_bfloat16>(prm, dtype, d, look, dev, s);
     if (pl.sched.cluster >= 2)
         return dtype == SHA_FP16 ? launch_cluster<__half>(prm, dtype, d, dev, s)
                                  : launch_cluster<__nv_bfloat16>(prm, dtype, d, dev, s);
@@ -931,6 +956,20 @@ sha_status_t sha_decode_strided(const void *q, const void *k, const void *v,
         if (k_strides[i] % 8 || v_strides[i] % 8) return SHA_ERR_MISALIGNED;
         if (k_strides[i] >= (1ll << 39) || v_strides[i] >= (1ll << 39)) return SHA_ERR_INVALID_ARG;
     }
+    return decode_impl(q, k, v, batch_head_index, B, H_q, H_kv, N_kv, d, top_k, scale, out,
+                       dtype, nullptr, 0, 0, stream, true, lay);
+}
+
+sha_status_t sha_decode_tokens(const void *q, const void *k, const void *v,
+                               const int32_t *batch_head_index, const int32_t *tokens, int B,
+                               int H_q, int H_kv, int N_kv, int d, int top_k, int n_sel,
+                               float scale, void *out, sha_dtype_t dtype, void *stream)
+{
+    if (n_sel < 1) return SHA_ERR_INVALID_ARG;
+    if (B > 0 && top_k > 0 && !tokens) return SHA_ERR_INVALID_ARG;
+    KvLayout lay;
+    lay.tokens = tokens;
+    lay.n_sel = n_sel;
     return decode_impl(q, k, v, batch_head_index, B, H_q, H_kv, N_kv, d, top_k, scale, out,
                        dtype, nullptr, 0, 0, stream, true, lay);
 }

@@ -231,6 +231,40 @@ __device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32
         : "memory");
 }
 
+// ---- 16-byte asynchronous copies (not through the TMA unit) ---------------------
+
+// Copy 16 bytes global -> shared, bypassing L1; dst and src 16-byte aligned.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, uint64_t policy)
+{
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(
+                     smem_addr(dst)),
+                 "l"(src), "l"(policy)
+                 : "memory");
+}
+
+// The same into the shared address `dst`, reading only src_bytes (16 or 0)
+// of src and filling the rest of the 16 bytes with zeros.
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void *src,
+                                                 uint32_t src_bytes, uint64_t policy)
+{
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst),
+                 "l"(src), "r"(src_bytes), "l"(policy)
+                 : "memory");
+}
+
+// Arrive on `bar` (as one of its expected arrivals) once every cp.async this
+// thread has issued so far has landed.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // Orders this thread's generic-proxy shared-memory writes before later
 // async-proxy (bulk copy / TMA) accesses of the same bytes.
 __device__ __forceinline__ void fence_proxy_async_shared()

@@ -171,7 +171,8 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(&full[s], 1);
+            // a gathered tile is filled by every producer lane's copies
+            mbar_init(&full[s], kLayout == kLayoutTokens ? 32 : 1);
             mbar_init(&empty[s], C::kConsumerWarps);
         }
         mbar_init(part_bar, 1);
@@ -212,7 +213,7 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
         walk.S = S;
         walk.t = S.begin(blockIdx.x);
         walk.t_end = S.begin(blockIdx.x + 1);
-        walk.n_keys = p.N_kv;
+        walk.n_keys = kLayout == kLayoutTokens ? p.n_sel : p.N_kv;
     }
 
     // ------------------------------------------------------------ scout
@@ -229,7 +230,7 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
     if (warp == C::kConsumerWarps) {
         // A paged cache needs several page ids per tile: the whole warp gathers
         // them (one page box per lane).  Otherwise one lane drives the pipeline.
-        constexpr bool kWarpProducer = kLayout == kLayoutPaged;
+        constexpr bool kWarpProducer = kLayout == kLayoutPaged || kLayout == kLayoutTokens;
         if (!kWarpProducer && lane != 0) {
             if constexpr (kCluster) cluster_sync_unaligned();
             return;
@@ -293,6 +294,38 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
                                         &tm_v, bx * 64, off, pplane, &full[stage], policy);
                         }
                     }
+                } else if constexpr (kLayout == kLayoutTokens) {
+                    // the unit's listed keys: each lane copies whole K and V rows
+                    // with 16-byte cp.async into the swizzled tile (rows past the
+                    // list are zero-filled and masked by the consumers), and
+                    // arrives on the stage once its copies have landed
+                    const int n0 = j * C::kTile;
+                    const int rows = min(C::kTile, seg.n_keys - n0);
+                    const int32_t *tk = p.tokens + (size_t)seg.unit * p.n_sel + n0;
+                    const T *kb = static_cast<const T *>(p.k) + (size_t)plane * p.N_kv * D;
+                    const T *vb = static_cast<const T *>(p.v) + (size_t)plane * p.N_kv * D;
+                    const uint32_t kt = smem_addr(k_ring + stage * C::kTileBytes);
+                    const uint32_t vt = smem_addr(v_ring + stage * C::kTileBytes);
+                    for (int r = lane; r < C::kTile; r += 32) {
+                        int t = 0;
+                        uint32_t src_bytes = 0;
+                        if (r < rows) {
+                            t = tk[r];
+                            if ((unsigned)t >= (unsigned)p.N_kv) {
+                                atomicOr(&g_sha_status, kStatusBadIndex);
+                                t = 0;                  // stay inside the head's cache
+                            }
+                            src_bytes = 16;
+                        }
+                        const T *krow = kb + (size_t)t * D;
+                        const T *vrow = vb + (size_t)t * D;
+#pragma unroll
+                        for (int c = 0; c < D / 8; ++c) {
+                            cp_async16_zfill(swizzled<D>(kt, r, c), krow + c * 8, src_bytes, policy);
+                            cp_async16_zfill(swizzled<D>(vt, r, c), vrow + c * 8, src_bytes, policy);
+                        }
+                    }
+                    cp_async_arrive_noinc(&full[stage]);
                 } else if constexpr (layout_strided(kLayout)) {
                     // boxes of a 4-D map whose outer dimensions follow the caller's strides
                     int c[3];
@@ -320,6 +353,7 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
                 if (++stage == C::kStages) { stage = 0; phase ^= 1; }
             }
         }
+        if constexpr (kLayout == kLayoutTokens) cp_async_wait_all();
         if (lane == 0)
             for (int s = 0; s < C::kStages; ++s)
                 if (used & (1u << s)) mbar_wait_drain(&full[s], (last_parity >> s) & 1u);

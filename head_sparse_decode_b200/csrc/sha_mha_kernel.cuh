@@ -64,6 +64,10 @@ struct DecodeParams {
     // three outer dimensions are the token, head and batch dimensions in the
     // order of increasing stride; these give each one's position (0..2)
     int tok_dim, head_dim, batch_dim;
+    // head x token sparsity: unit u attends only to the keys tokens[u * n_sel ..
+    // u * n_sel + n_sel) of its head (positions in [0, N_kv))
+    const int32_t *tokens;
+    int n_sel;
 };
 
 // How K/V of a unit are found: one padded [N_kv] block per (b, h) with every
@@ -78,7 +82,10 @@ enum : int {
     kLayoutStridedVarlen = 4,
     // the padded layout of kLayoutFixed under the clustered cut (grouped kernel
     // only): thread-block clusters, split units merged in distributed shared memory
-    kLayoutCluster = 5
+    kLayoutCluster = 5,
+    // the padded layout, each unit restricted to a listed subset of its keys,
+    // gathered row by row (grouped kernel only)
+    kLayoutTokens = 6
 };
 
 // Layouts whose rows have their own lengths (planned on the device) and that

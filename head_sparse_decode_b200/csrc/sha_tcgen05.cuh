@@ -2,7 +2,7 @@
 // tensor-memory (TMEM) allocation, shared-memory matrix descriptors for
 // 128-byte-swizzled K-major operands, the kind::f16 MMA with an fp32
 // accumulator in TMEM, commit-to-mbarrier, TMEM -> register loads, and the
-// copies that fill the operands (TMA tiled loads, 16-byte cp.async).
+// TMA tiled loads that fill the operands (16-byte cp.async: sha_device.cuh).
 //
 // Operand layout used throughout: a K-major tile of R rows x 64 elements
 // (128 bytes per row) is one "K atom"; 8-row groups of an atom are 1024
@@ -175,30 +175,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(policy)
         : "memory");
-}
-
-// ---- 16-byte asynchronous copies (not through the TMA unit) ---------------------
-
-// Copy 16 bytes global -> shared, bypassing L1; dst and src 16-byte aligned.
-__device__ __forceinline__ void cp_async16(void *dst, const void *src, uint64_t policy)
-{
-    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(
-                     smem_addr(dst)),
-                 "l"(src), "l"(policy)
-                 : "memory");
-}
-
-// Arrive on `bar` (as one of its expected arrivals) once every cp.async this
-// thread has issued so far has landed.
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)
-{
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar))
-                 : "memory");
-}
-
-__device__ __forceinline__ void cp_async_wait_all()
-{
-    asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 }  // namespace sha

@@ -194,6 +194,31 @@ sha_status_t sha_decode_paged(const void *q, const void *k_pages, const void *v_
                               float scale, void *out, sha_dtype_t dtype, void *stream);
 
 /*
+ * sha_decode_tokens -- head x token sparsity.  Polar Sparsity names the
+ * combination of head sparsity with token sparsity as future work
+ * (papernotes.org summary, "局限与展望"); this entry point is its plainest
+ * form: each selected (row b, slot k) unit attends only to a caller-given
+ * list of its head's keys,
+ *     out[b, h*G + j, :] = softmax over i of (scale * q K[t_i]^T) V[t_i],
+ *     t_i = tokens[b, k, i],  i < n_sel,  h = batch_head_index[b, k],
+ * a listed position counting once per listing.
+ *   tokens : device pointer, int32 [B, top_k, n_sel], positions in [0, N_kv);
+ *            any order, repeats allowed
+ *   n_sel  : keys per unit, >= 1 (it need not be <= N_kv)
+ *   k, v   : [B, H_kv, N_kv, d] as for sha_decode; dtype SHA_FP16 or SHA_BF16.
+ * A position outside [0, N_kv) is bad input: the SHA_ERR_BAD_INDEX flag is
+ * raised, no memory outside the head's cache is read, and that unit's output
+ * is unspecified.  The listed K and V rows are gathered with 16-byte copies
+ * (each key row is read once per listing) and run on the grouped kernel for
+ * every G (d = 64 or 128).  Uses the library-owned per-device workspace, like
+ * sha_decode.
+ */
+sha_status_t sha_decode_tokens(const void *q, const void *k, const void *v,
+                               const int32_t *batch_head_index, const int32_t *tokens, int B,
+                               int H_q, int H_kv, int N_kv, int d, int top_k, int n_sel,
+                               float scale, void *out, sha_dtype_t dtype, void *stream);
+
+/*
  * sha_decode_workspace_size -- bytes of workspace sha_decode_ex needs for
  * these sizes and num_splits (0 = automatic) on the current device.  Host
  * only; reads the device's SM count.  Returns 0 for sizes sha_decode_ex

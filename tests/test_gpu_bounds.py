@@ -189,3 +189,22 @@ def test_strided_writes_only_its_rows(sha, G, d):
     _ok(sha)
     _check_out_padding(w, buf)
     check_against_oracle(w, q, k, v, idx, out)
+
+
+@pytest.mark.parametrize("G,d,n_sel", [(1, 128, 300), (8, 128, 129), (3, 64, 77)])
+def test_tokens_write_only_their_rows(sha, G, d, n_sel):
+    w = W("b_tokens", B=4, H_q=4 * G, H_kv=4, N_kv=500, d=d, top_k=3,
+          dtype="fp16" if G == 1 else "bf16", seed=740 + G)
+    q, k, v, idx = _inputs(w)
+    tok = workloads.make_tokens(w, n_sel).cuda()
+    buf, out = _guarded_out(w)
+    sha.sha_decode_tokens(q, k, v, idx, tok, w.scale, out)
+    _ok(sha)
+    _check_out_padding(w, buf)
+    import oracle
+    from parity import TOLERANCE, active_mask
+    want, _ = oracle.sha_decode_tokens(q.cpu(), k.cpu(), v.cpu(), idx.cpu().numpy(),
+                                       tok.cpu().numpy(), w.scale, w.dtype)
+    mask = active_mask(idx.cpu().numpy(), w.B, w.H_kv, w.G)
+    got = out.cpu().double().numpy()
+    assert np.abs(got[mask] - want[mask]).max() <= TOLERANCE[w.dtype]

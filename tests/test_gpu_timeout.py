@@ -66,7 +66,7 @@ def _status(hooks):
 CASES = [
     # more units than SMs: even cut, units split between blocks, merged
     # through the library workspace's slots and arrival counters
-    (W("timeout_gqa_kernel", B=32, H_q=16, H_kv=16, N_kv=1000, d=128, top_k=5, dtype="fp16",
+    (W("timeout_gqa_kernel", B=32, H_q=16, H_kv=16, N_kv=4000, d=128, top_k=5, dtype="fp16",
        seed=601), 0),
     (W("timeout_fma_kernel", B=32, H_q=16, H_kv=16, N_kv=1000, d=64, top_k=5, dtype="bf16",
        seed=602), 0),

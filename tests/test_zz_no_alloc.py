@@ -59,10 +59,11 @@ def _check_twice(sha, shapes):
 
 @pytest.mark.parametrize("dtype,d", [("fp16", 128), ("bf16", 64)])
 def test_noalloc_matches_the_allocating_entry_point_twice(sha, dtype, d):
-    # more units than SMs: the even tile cut, units split between neighbours
-    first = workloads.Workload("noalloc_a", B=32, H_q=16, H_kv=16, N_kv=1000, d=d, top_k=5,
+    # more units than SMs, over 32 tiles per block: the even tile cut, units
+    # split between neighbouring blocks
+    first = workloads.Workload("noalloc_a", B=32, H_q=16, H_kv=16, N_kv=4000, d=d, top_k=5,
                                dtype=dtype, seed=51)
-    second = first.with_(name="noalloc_b", B=24, N_kv=777, top_k=7, seed=52)
+    second = first.with_(name="noalloc_b", B=24, N_kv=3777, top_k=7, seed=52)
     _check_twice(sha, [first, second])
 
 

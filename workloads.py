@@ -129,6 +129,22 @@ def make_index(w: Workload):
     return torch.stack(rows).to(torch.int32).contiguous()
 
 
+def make_tokens(w: Workload, n_sel, seed_offset=13):
+    """int32 [B, top_k, n_sel] key positions for head x token sparsity: for every
+    unit a uniform random subset of [0, N_kv) without repetition when n_sel <=
+    N_kv (else every position once and the rest drawn again), sorted, from a
+    CPU generator seeded with seed + seed_offset."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed + seed_offset)
+    units = w.B * w.top_k
+    if n_sel <= w.N_kv:
+        keys = torch.rand((units, w.N_kv), generator=g).argsort(dim=1)[:, :n_sel]
+    else:
+        extra = torch.randint(0, w.N_kv, (units, n_sel - w.N_kv), generator=g)
+        keys = torch.cat([torch.arange(w.N_kv).expand(units, -1), extra], dim=1)
+    return keys.sort(dim=1).values.to(torch.int32).reshape(w.B, w.top_k, n_sel).contiguous()
+
+
 def make_qkv(w: Workload, device="cpu"):
     """Q [B, H_q, d], K and V [B, H_kv, N_kv, d], N(0,1) rounded to the workload dtype."""
     dt = TORCH_DTYPE[w.dtype]
