@@ -459,6 +459,7 @@ def run_ours(args, rank, world, local):
         extras["other_configs"] = other_configs(sha, w, dev, stream, peak, rank)
         extras["other_configs"].append(varlen_config(sha, dev, stream, peak, rank))
         extras["other_configs"].append(paged_config(sha, dev, stream, peak, rank))
+        extras["other_configs"].append(tokens_config(sha, dev, stream, peak, rank))
         extras["other_configs"].extend(strided_configs(sha, dev, stream, peak, rank))
         mlp = run_mlp(argparse.Namespace(batch=None), dev)
         extras["selective_mlp"] = {"config": mlp["config"], "cublas_dense_us": mlp["cublas_dense_us"],
@@ -609,6 +610,35 @@ def varlen_config(sha, dev, stream, peak, rank):
            "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
            "steps_per_s": round(steps / t, 1), "bytes_per_step": nbytes}
     del q, k, v
+    torch.cuda.empty_cache()
+    return res
+
+
+def tokens_config(sha, dev, stream, peak, rank, keep=4):
+    """OPT-66B shape with head x token sparsity: every selected head attends to a
+    seeded random quarter of its keys (sha_decode_tokens)."""
+    w = workloads.CONFIGS["opt66b"].with_(seed=1700 + 100 * rank)
+    q, k, v = workloads.make_qkv(w, device=dev)
+    idx = workloads.make_index(w).to(dev)
+    n_sel = w.N_kv // keep
+    tok = workloads.make_tokens(w, n_sel).to(dev)
+    out = workloads.make_out(w, dev)
+    # algorithmic bytes: the listed K+V rows, Q/O rows, the index and the lists
+    nbytes = (w.units * 2 * n_sel * w.d * 2 + 2 * w.units * w.G * w.d * 2 + 4 * w.units
+              + 4 * w.units * n_sel)
+
+    def call():
+        sha.sha_decode_tokens(q, k, v, idx, tok, w.scale, out)
+    for _ in range(20):
+        call()
+    steps = 500
+    t = timed_graphs(call, steps, dev, stream)
+    gbs = nbytes * steps / t / 1e9
+    res = {"workload": "opt66b_tokens_quarter", "keys_per_head": n_sel,
+           "us_per_step": round(t / steps * 1e6, 2), "gbs": round(gbs, 1),
+           "frac": round(gbs / peak, 4), "steps_per_s": round(steps / t, 1),
+           "bytes_per_step": nbytes}
+    del q, k, v, tok
     torch.cuda.empty_cache()
     return res
 

@@ -295,10 +295,11 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
                         }
                     }
                 } else if constexpr (kLayout == kLayoutTokens) {
-                    // the unit's listed keys: each lane copies whole K and V rows
-                    // with 16-byte cp.async into the swizzled tile (rows past the
-                    // list are zero-filled and masked by the consumers), and
-                    // arrives on the stage once its copies have landed
+                    // the unit's listed keys, gathered into the swizzled tile with
+                    // 16-byte cp.async: 8 lanes copy the 128 bytes of one row's box,
+                    // so an instruction moves 4 whole lines of 4 rows; rows past the
+                    // list are zero-filled (and masked by the consumers).  Each
+                    // lane arrives on the stage once its copies have landed.
                     const int n0 = j * C::kTile;
                     const int rows = min(C::kTile, seg.n_keys - n0);
                     const int32_t *tk = p.tokens + (size_t)seg.unit * p.n_sel + n0;
@@ -306,23 +307,36 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
                     const T *vb = static_cast<const T *>(p.v) + (size_t)plane * p.N_kv * D;
                     const uint32_t kt = smem_addr(k_ring + stage * C::kTileBytes);
                     const uint32_t vt = smem_addr(v_ring + stage * C::kTileBytes);
-                    for (int r = lane; r < C::kTile; r += 32) {
-                        int t = 0;
-                        uint32_t src_bytes = 0;
-                        if (r < rows) {
-                            t = tk[r];
-                            if ((unsigned)t >= (unsigned)p.N_kv) {
-                                atomicOr(&g_sha_status, kStatusBadIndex);
-                                t = 0;                  // stay inside the head's cache
-                            }
-                            src_bytes = 16;
-                        }
-                        const T *krow = kb + (size_t)t * D;
-                        const T *vrow = vb + (size_t)t * D;
+                    // the tile's positions, lane l holding rows l, l+32, ...
+                    int ids[C::kTile / 32];
 #pragma unroll
-                        for (int c = 0; c < D / 8; ++c) {
-                            cp_async16_zfill(swizzled<D>(kt, r, c), krow + c * 8, src_bytes, policy);
-                            cp_async16_zfill(swizzled<D>(vt, r, c), vrow + c * 8, src_bytes, policy);
+                    for (int i = 0; i < C::kTile / 32; ++i) {
+                        const int r = i * 32 + lane;
+                        int t = r < rows ? tk[r] : 0;
+                        if ((unsigned)t >= (unsigned)p.N_kv) {
+                            atomicOr(&g_sha_status, kStatusBadIndex);
+                            t = 0;                      // stay inside the head's cache
+                        }
+                        ids[i] = t;
+                    }
+                    const int sub = lane >> 3, ch = lane & 7;
+#pragma unroll
+                    for (int i = 0; i < C::kTile / 32; ++i) {
+#pragma unroll 2
+                        for (int r1 = 0; r1 < 32; r1 += 4) {
+                            const int r = i * 32 + r1 + sub;
+                            const int t = __shfl_sync(0xffffffffu, ids[i], r1 + sub);
+                            const uint32_t src_bytes = r < rows ? 16u : 0u;
+                            const T *krow = kb + (size_t)t * D;
+                            const T *vrow = vb + (size_t)t * D;
+#pragma unroll
+                            for (int bx = 0; bx < C::kBoxes; ++bx) {
+                                const int c = bx * 8 + ch;
+                                cp_async16_zfill(swizzled<D>(kt, r, c), krow + c * 8, src_bytes,
+                                                 policy);
+                                cp_async16_zfill(swizzled<D>(vt, r, c), vrow + c * 8, src_bytes,
+                                                 policy);
+                            }
                         }
                     }
                     cp_async_arrive_noinc(&full[stage]);
