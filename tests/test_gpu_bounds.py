@@ -208,3 +208,33 @@ def test_tokens_write_only_their_rows(sha, G, d, n_sel):
     mask = active_mask(idx.cpu().numpy(), w.B, w.H_kv, w.G)
     got = out.cpu().double().numpy()
     assert np.abs(got[mask] - want[mask]).max() <= TOLERANCE[w.dtype]
+
+
+@pytest.mark.parametrize("B,d,D,density", [(8, 9216, 36864, 0.1), (5, 768, 5000, 0.37),
+                                           (1, 12288, 4096, 0.5), (24, 512, 2048, 0.3)])
+def test_selective_mlp_writes_only_y_and_its_workspace(sha, B, d, D, density):
+    w = workloads.MlpWorkload("b_mlp", B=B, d=d, D=D, density=density, dtype="fp16",
+                              seed=750 + B)
+    dev = torch.device("cuda")
+    x, W1t, W2t, active = workloads.make_mlp(w, device=dev)
+    S, n_S = sha.sha_mlp_union(active)
+    n = B * d
+    ybuf = torch.empty(PAD + n + PAD, dtype=torch.float16, device=dev)
+    ybuf.view(torch.int16).fill_(np.int16(np.uint16(workloads.SENTINEL["fp16"])))
+    y = ybuf[PAD:PAD + n].view(B, d)
+    nbytes = sha.sha_selective_mlp_workspace_size(B, d, D)
+    nbytes = (nbytes + 255) // 256 * 256
+    wbuf, ws = _guarded_workspace(nbytes)
+    sha.sha_selective_mlp(x, W1t, W2t, S, n_S, y, workspace=ws)
+    _ok(sha)
+    bits = ybuf.view(torch.int16).cpu().numpy().view(np.uint16)
+    s = np.uint16(workloads.SENTINEL["fp16"])
+    assert (bits[:PAD] == s).all() and (bits[PAD + n:] == s).all(), "written outside y"
+    _check_ws_padding(wbuf, nbytes)
+    import oracle
+    from parity import mlp_excess
+    Sh = S[:int(n_S.item())].cpu().numpy()
+    cols = np.sort(np.random.default_rng(D).choice(d, min(d, 128), replace=False))
+    want = oracle.selective_mlp(x.cpu(), W1t.cpu(), W2t[:, cols].cpu().contiguous(), Sh, "fp16")
+    excess, err = mlp_excess(y[:, cols].cpu().double().numpy(), want, "fp16")
+    assert excess <= 0, err

@@ -149,3 +149,38 @@ def test_repeat_calls_are_bit_identical(sha, case):
     torch.cuda.synchronize()
     for y in ys[1:]:
         assert torch.equal(y.view(torch.int16), ys[0].view(torch.int16))
+
+
+@pytest.mark.parametrize("B,d,D,density,dtype,act", [
+    (8, 9216, 36864, 0.1, "fp16", "relu"),      # OPT-66B MLP, 10 % union
+    (8, 9216, 36864, 0.3, "bf16", "identity"),  # 30 %, no activation
+    (3, 9216, 36864, 0.02, "bf16", "relu"),     # fewer neuron groups than SMs
+    (1, 12288, 4096, 0.5, "fp16", "relu"),      # 12 column blocks of 1024
+    (7, 768, 5000, 0.37, "bf16", "relu"),       # one unit per group (d = one stage)
+    (8, 2560, 777, 1.0, "fp16", "identity"),    # union not a multiple of 16 or 128
+    (6, 9216, 36864, 1.0, "fp16", "relu"),      # every neuron
+])
+def test_small_batch_shapes_sampled(sha, B, d, D, density, dtype, act):
+    """Batches up to 8 over sparse to dense unions, a hidden size whose column
+    blocks outnumber the SMs, d of one stage, unions that are not a multiple of
+    the tile sizes, both activations.  Sampled output columns against the oracle,
+    and a repeated call gives the same bits."""
+    w = M("sk", B=B, d=d, D=D, density=density, dtype=dtype, seed=5200 + B + D % 97)
+    dev = torch.device("cuda")
+    x, W1t, W2t, active = workloads.make_mlp(w, device=dev)
+    S, n_S = sha.sha_mlp_union(active)
+    y = sha.sha_selective_mlp(x, W1t, W2t, S, n_S, activation=act)
+    torch.cuda.synchronize()
+    assert sha.sha_get_device_status() == sha.SHA_OK
+    n = int(n_S.item())
+    Sh = S[:n].cpu().numpy()
+    assert np.array_equal(Sh, oracle.mlp_union(active.cpu().numpy()))
+    cols = np.sort(np.random.default_rng(D).choice(d, min(d, 192), replace=False))
+    want = oracle.selective_mlp(x.cpu(), W1t.cpu(), W2t[:, cols].cpu().contiguous(), Sh,
+                                w.dtype, act=act)
+    excess, err = mlp_excess(y[:, cols].cpu().double().numpy(), want, w.dtype)
+    assert excess <= 0, err
+    # a second call gives the same bits (partial sums added in a fixed order)
+    y2 = sha.sha_selective_mlp(x, W1t, W2t, S, n_S, activation=act)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
