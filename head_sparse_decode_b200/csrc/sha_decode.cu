@@ -147,10 +147,12 @@ double stream_ns(long long max_tiles, long long active, double tile_bytes)
 
 // Multi-head calls (G = 1) with d = 128 and one length for every row run on
 // the grouped kernel's tensor-core path, one query row of the 16 an MMA
-// covers.  Under the power cap that a sustained decode load holds the GPU at,
-// it is 3-6 % faster than the FMA kernel (fewer instructions per byte).  The
-// FMA kernel keeps d = 64 and per-row lengths (paged caches included), where
-// it is faster.
+// covers.  On the OPT-66B step both kernels read exactly the algorithmic
+// bytes; the tensor-core path executes 2.25x fewer instructions and keeps the
+// issue slots half as busy.  Timed under the power cap that a sustained decode
+// load holds the GPU at it has measured 0-3.5 % faster, in bursts at full
+// clock 1-3 % slower.  The FMA kernel keeps d = 64 and per-row lengths (paged
+// caches included), where it is faster.
 #ifndef SHA_MHA_TENSOR_CORES
 #define SHA_MHA_TENSOR_CORES 1
 #endif
