@@ -557,9 +557,9 @@ sha_status_t launch_gqa(const sha::DecodeParams &prm, sha_dtype_t dtype, int dev
     st = kv_tensor_map(&tm_v, prm.v, dtype, D, rows, planes, box_rows);
     if (st != SHA_OK) return st;
     cudaError_t e = launch_kernel_cluster(
-        sha::sha_gqa_decode_kernel<T, D, kLayout, kLook>, prm.sched.num_ctas, C::threads(kLook),
-        C::kSmemBytes, stream, kLayout == sha::kLayoutCluster ? prm.sched.cluster : 0, prm, tm_k,
-        tm_v);
+        sha::sha_gqa_decode_kernel<T, D, kLayout, kLook>, prm.sched.num_ctas,
+        C::block_threads(kLook, kLayout == sha::kLayoutTokens), C::kSmemBytes, stream,
+        kLayout == sha::kLayoutCluster ? prm.sched.cluster : 0, prm, tm_k, tm_v);
     if (e != cudaSuccess) return launch_error(e);
     return SHA_OK;
 }
@@ -613,14 +613,12 @@ sha_status_t launch_look(const sha::DecodeParams &prm, sha_dtype_t dtype, bool f
 
 // Head x token sparsity: the grouped kernel's gathering build.
 template <typename T>
-sha_status_t launch_tokens(const sha::DecodeParams &prm, sha_dtype_t dtype, int d, bool look,
-                           int dev, cudaStream_t s)
+sha_status_t launch_tokens(const sha::DecodeParams &prm, sha_dtype_t dtype, int d, int dev,
+                           cudaStream_t s)
 {
-    if (d == 128)
-        return look ? launch_gqa<T, 128, sha::kLayoutTokens, true>(prm, dtype, dev, s, nullptr)
-                    : launch_gqa<T, 128, sha::kLayoutTokens, false>(prm, dtype, dev, s, nullptr);
-    return look ? launch_gqa<T, 64, sha::kLayoutTokens, true>(prm, dtype, dev, s, nullptr)
-                : launch_gqa<T, 64, sha::kLayoutTokens, false>(prm, dtype, dev, s, nullptr);
+    // the gathered build: extra gather warps, no scout
+    return d == 128 ? launch_gqa<T, 128, sha::kLayoutTokens, false>(prm, dtype, dev, s, nullptr)
+                    : launch_gqa<T, 64, sha::kLayoutTokens, false>(prm, dtype, dev, s, nullptr);
 }
 
 // The clustered cut: the grouped kernel only, no scout.
@@ -848,8 +846,8 @@ sha_status_t decode_impl(const void *q, const void *k, const void *v, const int3
         return launch_decode<sha::kLayoutStrided>(prm, dtype, d, fma, look, dev, s, &kv);
     }
     if (lay.tokens)
-        return dtype == SHA_FP16 ? launch_tokens<__half>(prm, dtype, d, look, dev, s)
-                                 : launch_tokens<__nv_bfloat16>(prm, dtype, d, look, dev, s);
+        return dtype == SHA_FP16 ? launch_tokens<__half>(prm, dtype, d, dev, s)
+                                 : launch_tokens<__nv_bfloat16>(prm, dtype, d, dev, s);
     if (pl.sched.cluster >= 2)
         return dtype == SHA_FP16 ? launch_cluster<__half>(prm, dtype, d, dev, s)
                                  : launch_cluster<__nv_bfloat16>(prm, dtype, d, dev, s);

@@ -53,6 +53,9 @@ namespace sha {
 #ifndef SHA_GQA_STAGES
 #define SHA_GQA_STAGES 3
 #endif
+#ifndef SHA_GQA_GATHER_WARPS
+#define SHA_GQA_GATHER_WARPS 4
+#endif
 
 template <int D>
 struct GqaConfig {
@@ -61,6 +64,15 @@ struct GqaConfig {
     static constexpr int kThreads = kConsumers + 32;   // + one producer warp
     // ... and a scout warp in the builds that finish a block's last unit on chip
     static constexpr int threads(bool look) { return kThreads + (look ? 32 : 0); }
+    // A gathered layout (listed key positions) is copied by kGatherWarps
+    // warps, each owning whole 32-row blocks of a tile: one warp's 16-byte
+    // copies in flight reach only about 2.6 TB/s, four about 6 TB/s.  That
+    // build has no scout warp (the register file holds 8 warps at this size).
+    static constexpr int kGatherWarps = SHA_GQA_GATHER_WARPS;
+    static constexpr int block_threads(bool look, bool gather)
+    {
+        return gather ? kThreads + 32 * (kGatherWarps - 1) : threads(look);
+    }
     static constexpr int kTile = SHA_GQA_TILE_KEYS;    // keys per tile (one pipeline stage)
     static constexpr int kSlices = kTile / 64;         // 64-key slices per tile
     static constexpr int kKeysPerWarp = 64 / kConsumerWarps;      // 16 per slice: one m16n8k16 k-step
@@ -102,6 +114,7 @@ struct GqaConfig {
     static constexpr int kSmemBytes = kAlignPad + kOwnerOffset + kOwnerGroups * 2;
     static_assert(2 * (threads(true) / 32) + 8 <= 32, "plan scratch fits");
     static_assert(kKeysPerWarp == 16, "one k-step of 16 keys per warp and slice");
+    static_assert((kTile / 32) % kGatherWarps == 0, "whole 32-row blocks per gather warp");
     static_assert(kTile % 64 == 0 && kTile <= 256, "whole 64-key slices, TMA box <= 256 rows");
     static_assert(kBoxBytes % 1024 == 0, "boxes stay 1 KiB aligned");
     static_assert(kConsumerWarps * kStateFloats >= 3 * kMaxMergeParts * kRows,
@@ -136,7 +149,7 @@ __device__ __forceinline__ uint32_t swizzled(uint32_t tile, int key, int chunk)
 }
 
 template <typename T, int D, int kLayout, bool kLook>
-__global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
+__global__ void __launch_bounds__(GqaConfig<D>::block_threads(kLook, kLayout == kLayoutTokens), 1)
     sha_gqa_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v)
 {
@@ -171,8 +184,8 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
-            // a gathered tile is filled by every producer lane's copies
-            mbar_init(&full[s], kLayout == kLayoutTokens ? 32 : 1);
+            // a gathered tile is filled by every gather lane's copies
+            mbar_init(&full[s], kLayout == kLayoutTokens ? 32 * C::kGatherWarps : 1);
             mbar_init(&empty[s], C::kConsumerWarps);
         }
         mbar_init(part_bar, 1);
@@ -227,7 +240,13 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
     }
 
     // ------------------------------------------------------------ producer
-    if (warp == C::kConsumerWarps) {
+    // gw: this warp's share of a gathered tile (0 for the producer warp; the
+    // token layout's further gather warps follow the scout)
+    static_assert(!(kLook && kLayout == kLayoutTokens), "the gathered build has no scout");
+    int gw = warp == C::kConsumerWarps ? 0 : -1;
+    if constexpr (kLayout == kLayoutTokens)
+        if (warp > C::kConsumerWarps) gw = warp - C::kConsumerWarps;
+    if (gw >= 0) {
         // A paged cache needs several page ids per tile: the whole warp gathers
         // them (one page box per lane).  Otherwise one lane drives the pipeline.
         constexpr bool kWarpProducer = kLayout == kLayoutPaged || kLayout == kLayoutTokens;
@@ -298,8 +317,10 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
                     // the unit's listed keys, gathered into the swizzled tile with
                     // 16-byte cp.async: 8 lanes copy the 128 bytes of one row's box,
                     // so an instruction moves 4 whole lines of 4 rows; rows past the
-                    // list are zero-filled (and masked by the consumers).  Each
-                    // lane arrives on the stage once its copies have landed.
+                    // list are zero-filled (and masked by the consumers).  Gather
+                    // warp gw takes the tile's 32-row blocks gw, gw + kGatherWarps,
+                    // ..., and each lane arrives on the stage once its copies have
+                    // landed.
                     const int n0 = j * C::kTile;
                     const int rows = min(C::kTile, seg.n_keys - n0);
                     const int32_t *tk = p.tokens + (size_t)seg.unit * p.n_sel + n0;
@@ -307,12 +328,13 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
                     const T *vb = static_cast<const T *>(p.v) + (size_t)plane * p.N_kv * D;
                     const uint32_t kt = smem_addr(k_ring + stage * C::kTileBytes);
                     const uint32_t vt = smem_addr(v_ring + stage * C::kTileBytes);
-                    // the tile's positions, lane l holding rows l, l+32, ...
+                    // the positions of this warp's row blocks, lane l holding rows
+                    // i*32 + l
                     int ids[C::kTile / 32];
 #pragma unroll
                     for (int i = 0; i < C::kTile / 32; ++i) {
                         const int r = i * 32 + lane;
-                        int t = r < rows ? tk[r] : 0;
+                        int t = (i % C::kGatherWarps == gw && r < rows) ? tk[r] : 0;
                         if ((unsigned)t >= (unsigned)p.N_kv) {
                             atomicOr(&g_sha_status, kStatusBadIndex);
                             t = 0;                      // stay inside the head's cache
@@ -322,6 +344,7 @@ __global__ void __launch_bounds__(GqaConfig<D>::threads(kLook), 1)
                     const int sub = lane >> 3, ch = lane & 7;
 #pragma unroll
                     for (int i = 0; i < C::kTile / 32; ++i) {
+                        if (i % C::kGatherWarps != gw) continue;
 #pragma unroll 2
                         for (int r1 = 0; r1 < 32; r1 += 4) {
                             const int r = i * 32 + r1 + sub;
