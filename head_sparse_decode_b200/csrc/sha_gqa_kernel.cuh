@@ -261,9 +261,25 @@ __global__ void __launch_bounds__(GqaConfig<D>::block_threads(kLook, kLayout == 
         bool ok = true;
         Walk wk = walk;
         Seg seg;
+        // gathered layout: the raw positions of this warp's row blocks of the
+        // next tile (lane l holding rows i*32 + l), loaded while the current
+        // tile's copies go out; a unit's first tile is loaded beside its head id
+        int pos_next[C::kTile / 32];
+        auto load_pos = [&](long long unit, int tile) {
+            const int n0 = tile * C::kTile;
+            const int rows = min(C::kTile, p.n_sel - n0);
+            const int32_t *tk = p.tokens + (size_t)unit * p.n_sel + n0;
+#pragma unroll
+            for (int i = 0; i < C::kTile / 32; ++i) {
+                const int r = i * 32 + lane;
+                pos_next[i] = (i % C::kGatherWarps == gw && r < rows) ? tk[r] : 0;
+            }
+        };
+        (void)load_pos;
         while (ok && wk.next(seg)) {
             const int b = (int)(seg.unit / p.top_k);
             const int h = p.idx[seg.unit];
+            if constexpr (kLayout == kLayoutTokens) load_pos(seg.unit, seg.first_tile);
             if ((unsigned)h >= (unsigned)p.H_kv) continue;
             const int plane = b * p.H_kv + h;
             for (int j = seg.first_tile; j < seg.first_tile + seg.num_tiles; ++j) {
@@ -323,24 +339,22 @@ __global__ void __launch_bounds__(GqaConfig<D>::block_threads(kLook, kLayout == 
                     // landed.
                     const int n0 = j * C::kTile;
                     const int rows = min(C::kTile, seg.n_keys - n0);
-                    const int32_t *tk = p.tokens + (size_t)seg.unit * p.n_sel + n0;
                     const T *kb = static_cast<const T *>(p.k) + (size_t)plane * p.N_kv * D;
                     const T *vb = static_cast<const T *>(p.v) + (size_t)plane * p.N_kv * D;
                     const uint32_t kt = smem_addr(k_ring + stage * C::kTileBytes);
                     const uint32_t vt = smem_addr(v_ring + stage * C::kTileBytes);
-                    // the positions of this warp's row blocks, lane l holding rows
-                    // i*32 + l
+                    // this tile's positions (loaded a tile ahead), checked
                     int ids[C::kTile / 32];
 #pragma unroll
                     for (int i = 0; i < C::kTile / 32; ++i) {
-                        const int r = i * 32 + lane;
-                        int t = (i % C::kGatherWarps == gw && r < rows) ? tk[r] : 0;
+                        int t = pos_next[i];
                         if ((unsigned)t >= (unsigned)p.N_kv) {
                             atomicOr(&g_sha_status, kStatusBadIndex);
                             t = 0;                      // stay inside the head's cache
                         }
                         ids[i] = t;
                     }
+                    if (j + 1 < seg.first_tile + seg.num_tiles) load_pos(seg.unit, j + 1);
                     const int sub = lane >> 3, ch = lane & 7;
 #pragma unroll
                     for (int i = 0; i < C::kTile / 32; ++i) {
