@@ -62,11 +62,13 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--config", default="opt66b", choices=sorted(workloads.CONFIGS))
     p.add_argument("--layout", default="head_major",
-                   choices=["head_major", "token_major", "varlen", "paged16"],
+                   choices=["head_major", "token_major", "varlen", "paged16", "tokens4"],
                    help="K/V cache of the timed step: [B, H_kv, N_kv, d] (sha_decode), "
                         "[B, N_kv, H_kv, d] (sha_decode_strided), per-row lengths uniform in "
-                        "[1, N_kv] (sha_decode_varlen) or 16-key pages in random pool order "
-                        "(sha_decode_paged); all but head_major imply --no-extras")
+                        "[1, N_kv] (sha_decode_varlen), 16-key pages in random pool order "
+                        "(sha_decode_paged), or each selected head attending to a seeded "
+                        "random quarter of its keys (sha_decode_tokens); all but head_major "
+                        "imply --no-extras")
     p.add_argument("--sustained-s", type=float, default=1.5,
                    help="seconds of graph-replayed steps in the sustained leg (0 skips it)")
     p.add_argument("--batch", type=int, default=None,
@@ -328,7 +330,8 @@ def aggregate(bytes_per_step, steps, elapsed_s, world, device="cuda"):
 KV_LAYOUTS = {"head_major": "[B, H_kv, N_kv, d]",
               "token_major": "[B, N_kv, H_kv, d] (strided views)",
               "varlen": "[B, H_kv, N_kv, d], per-row lengths uniform in [1, N_kv]",
-              "paged16": "pool [pages, H_kv, 16, d] + block table, random page order"}
+              "paged16": "pool [pages, H_kv, 16, d] + block table, random page order",
+              "tokens4": "[B, H_kv, N_kv, d], a listed quarter of each selected head's keys"}
 
 
 def paged_cache(k, v, w, page_size, dev):
@@ -405,6 +408,16 @@ def run_ours(args, rank, world, local):
 
         def step():
             sha.sha_decode_varlen(q, k, v, idx, lens_d, w.scale, out)
+    elif args.layout == "tokens4":
+        # each selected head attends to a seeded random quarter of its keys
+        args.no_extras = True
+        n_sel = w.N_kv // 4
+        tok = workloads.make_tokens(w, n_sel).to(dev)
+        bytes_step = (w.units * 2 * n_sel * w.d * 2 + 2 * w.units * w.G * w.d * 2
+                      + 4 * w.units + 4 * w.units * n_sel)
+
+        def step():
+            sha.sha_decode_tokens(q, k, v, idx, tok, w.scale, out)
     elif args.layout == "paged16":
         # the cache in 16-key pages scattered over a pool in random order
         args.no_extras = True
@@ -475,8 +488,8 @@ def run_ours(args, rank, world, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": w.dtype, "data": "synthetic N(0,1), seeded",
         "config": {**w.describe(), "parallelism": f"replicas x{world} (batch sharded by rank)",
-                   "accumulation": "fp32", "l2": "no flush: active K/V per step "
-                   f"{w.units * 2 * w.N_kv * w.d * 2 / 1e9:.2f} GB > 126 MB L2",
+                   "accumulation": "fp32", "l2": "no flush: bytes moved per step "
+                   f"{bytes_step / 1e9:.2f} GB > 126 MB L2",
                    "blocks": plan["blocks"], "tile_keys": plan["tile_keys"],
                    "cluster": plan["cluster"],
                    "kv_layout": KV_LAYOUTS[args.layout],

@@ -150,8 +150,9 @@ double stream_ns(long long max_tiles, long long active, double tile_bytes)
 // covers.  On the OPT-66B step both kernels read exactly the algorithmic
 // bytes; the tensor-core path executes 2.25x fewer instructions and keeps the
 // issue slots half as busy.  Timed under the power cap that a sustained decode
-// load holds the GPU at it has measured 0-3.5 % faster, in bursts at full
-// clock 1-3 % slower.  The FMA kernel keeps d = 64 and per-row lengths (paged
+// load holds the GPU at, the two have come out within 0.2 % of each other on
+// some boxes and 3.5 % apart in the tensor-core path's favour on others; in
+// bursts at full clock the FMA kernel is 1-3 % faster.  The FMA kernel keeps d = 64 and per-row lengths (paged
 // caches included), where it is faster.
 #ifndef SHA_MHA_TENSOR_CORES
 #define SHA_MHA_TENSOR_CORES 1
