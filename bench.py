@@ -265,23 +265,46 @@ def capture_graph(fn, n, dev):
     return g
 
 
-def timed_graphs(fn, steps, dev, stream, chunk=100):
+def timed_graphs(fn, steps, dev, stream, chunk=100, per_step=None):
     """Exactly `steps` calls of fn, launched by replaying CUDA graphs of up to
     `chunk` calls (the pages measure decode throughput under CUDA graphs), timed
-    with events on `stream`.  Returns seconds."""
+    with events on `stream`.  Returns seconds.  per_step: a list that receives
+    the mean seconds per call of each full graph replay (events between the
+    replays, inside the same timed region)."""
     chunk = max(1, min(chunk, steps))
     g_main = capture_graph(fn, chunk, dev)
     rem = steps % chunk
     g_rem = capture_graph(fn, rem, dev) if rem else None
     g_main.replay()                       # first replay uploads the graph
     torch.cuda.synchronize(dev)
+    n_main = steps // chunk
+    marks = ([torch.cuda.Event(enable_timing=True) for _ in range(n_main + 1)]
+             if per_step is not None else None)
 
     def run():
-        for _ in range(steps // chunk):
+        for i in range(n_main):
+            if marks is not None:
+                marks[i].record(stream)
             g_main.replay()
+        if marks is not None:
+            marks[n_main].record(stream)
         if g_rem is not None:
             g_rem.replay()
-    return timed(run, 1, stream)
+    t = timed(run, 1, stream)
+    if marks is not None:
+        per_step.extend(marks[i].elapsed_time(marks[i + 1]) / 1e3 / chunk for i in range(n_main))
+    return t
+
+
+def step_distribution(per_step, chunk):
+    """p10 / median / p90 of the per-call time over the graph replays (us)."""
+    if not per_step:
+        return None
+    xs = sorted(per_step)
+    pick = lambda q: xs[min(len(xs) - 1, int(q * (len(xs) - 1) + 0.5))] * 1e6
+    return {"p10_us": round(pick(0.1), 3), "median_us": round(pick(0.5), 3),
+            "p90_us": round(pick(0.9), 3), "graph_replays": len(xs),
+            "calls_per_replay": chunk}
 
 
 def sync_all(world, local):
@@ -448,7 +471,8 @@ def run_ours(args, rank, world, local):
         step()
     sync_all(world, local)
     t0 = time.time()
-    elapsed = timed_graphs(step, args.steps, dev, stream)
+    per_step = []
+    elapsed = timed_graphs(step, args.steps, dev, stream, per_step=per_step)
     t1 = time.time()
     sync_all(world, local)
     clocks = sampler.stop(t0, t1)
@@ -495,6 +519,8 @@ def run_ours(args, rank, world, local):
                    "kv_layout": KV_LAYOUTS[args.layout],
                    "launch": "CUDA graph replay, 100 steps per graph"},
         "steps_per_s": round(args.steps / t_max, 2),
+        # the per-call time of each 100-call graph replay of the timed region
+        "step_time": step_distribution(per_step, min(100, args.steps)),
         "tokens_per_s": round(world * w.B * args.steps / t_max, 1),
         "hbm_frac_of_measured": round(achieved / peak, 4),
         "copy_probe_gbs": round(copy_gbs, 1),
