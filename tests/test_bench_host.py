@@ -39,3 +39,15 @@ def test_source_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
     target.write_text(text.replace("constexpr int kMaxBlocks = 4096;",
                                    "constexpr int kMaxBlocks = 4095;", 1))
     assert _hash_of_tree(monkeypatch, str(tmp_path)) != base
+
+
+def test_step_distribution_percentiles():
+    # 41 graph replays with per-call times 100..140 us: p10/median/p90 by rank
+    per_step = [1e-6 * x for x in range(140, 99, -1)]
+    d = bench.step_distribution(per_step, 100)
+    assert d == {"p10_us": 104.0, "median_us": 120.0, "p90_us": 136.0, "graph_replays": 41,
+                 "calls_per_replay": 100}
+    assert bench.step_distribution([], 100) is None
+    one = bench.step_distribution([2.5e-4], 7)
+    assert one["p10_us"] == one["median_us"] == one["p90_us"] == 250.0
+    assert one["calls_per_replay"] == 7
