@@ -34,6 +34,9 @@ def libs():
     hooks.sha_decode_clustered.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, ctypes.c_float, vp,
                                            i, i, i, i, vp]
     hooks.sha_decode_clustered.restype = i
+    hooks.sha_decode_tokens.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, ctypes.c_float,
+                                        vp, i, vp]
+    hooks.sha_decode_tokens.restype = i
     hooks.sha_get_device_status.argtypes = [vp]
     hooks.sha_get_device_status.restype = i
     hooks.sha_test_set_wait_limit.argtypes = [ctypes.c_ulonglong]
@@ -112,3 +115,43 @@ def test_wait_gives_up_reports_and_recovers(libs, case):
     torch.cuda.synchronize()
     assert sha.sha_get_device_status() == sha.SHA_OK
     check_against_oracle(w, q, k, v, idx, out)
+
+
+def test_gathered_wait_gives_up_reports_and_recovers(libs):
+    """The head x token gather: four gather warps, each with its own bounded
+    waits, arriving on the same stages."""
+    sha, hooks = libs
+    w = W("timeout_tokens", B=16, H_q=32, H_kv=32, N_kv=3000, d=128, top_k=6, dtype="fp16",
+          seed=605)
+    q, k, v, idx = _inputs(w)
+    tok = workloads.make_tokens(w, 700).cuda()
+    s = torch.cuda.current_stream().cuda_stream
+
+    def call(out):
+        return hooks.sha_decode_tokens(q.data_ptr(), k.data_ptr(), v.data_ptr(), idx.data_ptr(),
+                                       tok.data_ptr(), w.B, w.H_q, w.H_kv, w.N_kv, w.d, w.top_k,
+                                       tok.shape[2], w.scale, out.data_ptr(), 0, s)
+
+    assert hooks.sha_get_device_status(None) == sha.SHA_OK
+    assert hooks.sha_test_set_wait_limit(1) == sha.SHA_OK
+    out = workloads.make_out(w, "cuda")
+    assert call(out) == sha.SHA_OK
+    torch.cuda.synchronize()
+    assert _status(hooks) == sha.SHA_ERR_TIMEOUT
+    from parity import TOLERANCE, active_mask
+    mask = active_mask(idx.cpu().numpy(), w.B, w.H_kv, w.G)
+    bits = out_bits(out).reshape(w.B, w.H_q, w.d)
+    assert (bits[~mask] == workloads.SENTINEL[w.dtype]).all()
+
+    assert hooks.sha_test_set_wait_limit(LIMIT_NS) == sha.SHA_OK
+    import numpy as np
+    import oracle
+    want, _ = oracle.sha_decode_tokens(q.cpu(), k.cpu(), v.cpu(), idx.cpu().numpy(),
+                                       tok.cpu().numpy(), w.scale, w.dtype)
+    for _ in range(2):
+        out = workloads.make_out(w, "cuda")
+        assert call(out) == sha.SHA_OK
+        torch.cuda.synchronize()
+        assert _status(hooks) == sha.SHA_OK
+        got = out.cpu().double().numpy()
+        assert np.abs(got[mask] - want[mask]).max() <= TOLERANCE[w.dtype]
