@@ -152,8 +152,8 @@ double stream_ns(long long max_tiles, long long active, double tile_bytes)
 // issue slots half as busy.  Timed under the power cap that a sustained decode
 // load holds the GPU at, the two have come out within 0.2 % of each other on
 // some boxes and 3.5 % apart in the tensor-core path's favour on others; in
-// bursts at full clock the FMA kernel is 1-3 % faster.  The FMA kernel keeps d = 64 and per-row lengths (paged
-// caches included), where it is faster.
+// bursts at full clock the FMA kernel is 1-3 % faster.  The FMA kernel keeps
+// d = 64 and per-row lengths (paged caches included), where it is faster.
 #ifndef SHA_MHA_TENSOR_CORES
 #define SHA_MHA_TENSOR_CORES 1
 #endif

@@ -240,8 +240,8 @@ __global__ void __launch_bounds__(GqaConfig<D>::block_threads(kLook, kLayout == 
     }
 
     // ------------------------------------------------------------ producer
-    // gw: this warp's share of a gathered tile (0 for the producer warp; the
-    // token layout's further gather warps follow the scout)
+    // gw: this warp's share of a gathered tile (0 for the producer warp; in the
+    // token layout's build, which has no scout, gather warps 1.. follow it)
     static_assert(!(kLook && kLayout == kLayoutTokens), "the gathered build has no scout");
     int gw = warp == C::kConsumerWarps ? 0 : -1;
     if constexpr (kLayout == kLayoutTokens)
