@@ -874,16 +874,22 @@ def run_mlp(args, dev=None):
         uws = torch.empty(sha._lib.sha_mlp_union_workspace_size(w.D), dtype=torch.uint8,
                           device=dev)
 
-        def layer():
+        def union():
             sha.sha_mlp_union(active, S, n_S, uws)
+
+        def layer():
+            union()
             sha.sha_selective_mlp(x, W1t, W2t, S, n_S, y, workspace=ws)
         for _ in range(10):
             layer()
         steps = 200
         t = timed_graphs(layer, steps, dev, stream, chunk=50)
         us = t / steps * 1e6
+        # the union's own time, replayed alone the same way
+        t_union = timed_graphs(union, steps, dev, stream, chunk=50)
         nbytes = w.algorithmic_bytes()
         points.append({"density": dens, "n_union": w.n_union(), "us_per_layer": round(us, 2),
+                       "union_us": round(t_union / steps * 1e6, 2),
                        "gbs": round(nbytes / (us * 1e-6) / 1e9, 1),
                        "frac": round(nbytes / (us * 1e-6) / 1e9 / peak, 4),
                        "bytes_per_layer": nbytes})
