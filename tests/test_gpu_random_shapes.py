@@ -1,7 +1,8 @@
 """Seeded random shapes against the float64 oracle: decode (G = 1..16, d = 64 /
-128, ragged key counts, top_k from 0 to H_kv, automatic and forced splits) and
-the Selective GEMM (batch 1..64 on both GEMM paths, ragged neuron counts,
-unions from almost empty to full, both activations)."""
+128, ragged key counts, top_k from 0 to H_kv, automatic and forced splits), head
+x token sparsity (random list lengths, repeats past the cache), and the
+Selective GEMM (batch 1..64 on both GEMM paths, ragged neuron counts, unions from
+almost empty to full, both activations)."""
 import numpy as np
 import pytest
 import torch
@@ -123,3 +124,45 @@ def test_random_selective_mlp_shape(sha, w, act):
     want = oracle.selective_mlp(x, W1t, W2t, want_S, w.dtype, act=act)
     excess, err = mlp_excess(y.cpu().double().numpy(), want, w.dtype)
     assert excess <= 0, err
+
+
+def _token_cases(n, seed):
+    """Head x token sparsity: random G, d, cache lengths and list lengths
+    (single keys, ragged last tiles, lists longer than the cache with
+    repeats), so every gather warp meets full, partial and empty row blocks."""
+    rng = np.random.default_rng(seed)
+    cases = []
+    for i in range(n):
+        G = int(rng.choice([1, 1, 2, 4, 8]))
+        H_kv = int(rng.integers(1, 13))
+        d = int(rng.choice([64, 128]))
+        N_kv = int(rng.integers(1, 2501))
+        top_k = int(rng.integers(1, H_kv + 1))
+        B = int(rng.integers(1, 17))
+        n_sel = int(rng.choice([1, int(rng.integers(1, 300)), int(rng.integers(1, 2 * N_kv + 2)),
+                                int(rng.integers(100, 1200))]))
+        dtype = str(rng.choice(["fp16", "bf16"]))
+        cases.append((W(f"tok{i}_B{B}_G{G}_Hkv{H_kv}_N{N_kv}_d{d}_k{top_k}_s{n_sel}_{dtype}", B=B,
+                        H_q=G * H_kv, H_kv=H_kv, N_kv=N_kv, d=d, top_k=top_k, dtype=dtype,
+                        seed=9800 + i), n_sel))
+    return cases
+
+
+@pytest.mark.parametrize("w,n_sel", _token_cases(16, 4321), ids=lambda c: getattr(c, "name", str(c)))
+def test_random_token_shape(sha, w, n_sel):
+    from parity import TOLERANCE, active_mask, out_bits
+    q, k, v = workloads.make_qkv(w)
+    idx = workloads.make_index(w)
+    tok = workloads.make_tokens(w, n_sel)
+    dev = torch.device("cuda")
+    out = workloads.make_out(w, dev)
+    sha.sha_decode_tokens(q.to(dev), k.to(dev), v.to(dev), idx.to(dev), tok.to(dev), w.scale, out)
+    torch.cuda.synchronize()
+    assert sha.sha_get_device_status() == sha.SHA_OK
+    want, _ = oracle.sha_decode_tokens(q, k, v, idx.numpy(), tok.numpy(), w.scale, w.dtype)
+    mask = active_mask(idx.numpy(), w.B, w.H_kv, w.G)
+    bits = out_bits(out).reshape(w.B, w.H_q, w.d)
+    assert (bits[~mask] == np.uint16(workloads.SENTINEL[w.dtype])).all()
+    if mask.any():
+        got = out.cpu().double().numpy()
+        assert np.abs(got[mask] - want[mask]).max() <= TOLERANCE[w.dtype]
