@@ -462,6 +462,21 @@ def sha_mlp_union(active, S=None, n_S=None, workspace=None, stream=None):
     return S, n_S
 
 
+_lib.sha_selective_mlp_plan.argtypes = [_i, _i, _i, _i, ctypes.POINTER(ctypes.c_int64)]
+_lib.sha_selective_mlp_plan.restype = _i
+
+
+def sha_selective_mlp_plan(B, d, D, num_sms=148):
+    """Host-side plan of a Selective GEMM layer: dict with batch_pad, tc_up,
+    tc_down, h_rows, down_splits, down_blocks, down_cols and workspace_bytes.
+    Raises ShaError for sizes the library rejects."""
+    plan = (ctypes.c_int64 * 8)()
+    _check(_lib.sha_selective_mlp_plan(B, d, D, num_sms, plan))
+    return {"batch_pad": plan[0], "tc_up": bool(plan[1]), "tc_down": bool(plan[2]),
+            "h_rows": plan[3], "down_splits": plan[4], "down_blocks": plan[5],
+            "down_cols": plan[6], "workspace_bytes": plan[7]}
+
+
 def sha_selective_mlp_workspace_size(B, d, D, device=None):
     with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
         return int(_lib.sha_selective_mlp_workspace_size(B, d, D))
@@ -519,6 +534,7 @@ __all__ = [
     "sha_decode", "sha_decode_bf16", "sha_decode_ex", "sha_decode_workspace_size",
     "sha_get_device_status", "sha_status_string", "sha_decode_plan", "sha_select_heads",
     "decode_from_scores", "sha_decode_varlen", "sha_decode_paged", "sha_mlp_union",
-    "sha_selective_mlp", "sha_selective_mlp_workspace_size", "sha_copy_bandwidth_probe", "decode",
+    "sha_selective_mlp", "sha_selective_mlp_workspace_size", "sha_selective_mlp_plan",
+    "sha_copy_bandwidth_probe", "decode",
     "alloc_workspace", "ShaError", "LIBRARY_PATH", "sha_decode_noalloc",
 ]

@@ -1550,6 +1550,7 @@ struct MlpPlan {
     bool tc_up;            // up-projection on tcgen05 (batches above 8)
     bool tc;               // down-projection on tcgen05 as well
     int down_splits, down_blocks;
+    int down_wc;           // output columns per warp-level down-projection item
     size_t up_bytes, h_bytes, down_bytes;
     size_t total() const { return up_bytes + h_bytes + down_bytes; }
 };
@@ -1589,6 +1590,7 @@ MlpPlan mlp_plan(int B, int d, int D, int sms)
     }
     pl.h_bytes = round_up((size_t)pl.h_rows * pl.bp * 2, 256);
     const int wc = stage_width(d, kmax);
+    pl.down_wc = wc;
     const int wchunks = d / wc;
     pl.down_splits = sms / wchunks > 0 ? sms / wchunks : 1;
     const int items = wchunks * pl.down_splits;
@@ -1776,6 +1778,22 @@ size_t sha_selective_mlp_workspace_size(int B, int d, int D)
     const int sms = device_sms(&dev);
     if (sms == 0) return 0;
     return mlp_plan(B, d, D, sms).total();
+}
+
+sha_status_t sha_selective_mlp_plan(int B, int d, int D, int num_sms, int64_t plan[8])
+{
+    if (!plan || B < 1 || D < 1 || d < 1 || num_sms < 1) return SHA_ERR_INVALID_ARG;
+    if (B > kMlpMaxBatch || d % 256 != 0) return SHA_ERR_UNSUPPORTED;
+    const MlpPlan pl = mlp_plan(B, d, D, num_sms);
+    plan[0] = pl.bp;
+    plan[1] = pl.tc_up ? 1 : 0;
+    plan[2] = pl.tc ? 1 : 0;
+    plan[3] = pl.h_rows;
+    plan[4] = pl.down_splits;
+    plan[5] = pl.down_blocks;
+    plan[6] = pl.down_wc;
+    plan[7] = (int64_t)pl.total();
+    return SHA_OK;
 }
 
 sha_status_t sha_selective_mlp(const void *x, const void *W1t, const void *W2t,

@@ -346,6 +346,26 @@ sha_status_t sha_mlp_union(const uint8_t *active, int B, int D, int32_t *S, int3
 size_t sha_selective_mlp_workspace_size(int B, int d, int D);
 
 /*
+ * sha_selective_mlp_plan -- how sha_selective_mlp runs a layer of these sizes
+ * on a device with num_sms SMs (host only, no CUDA call).  Writes
+ *   plan[0] = batch rows the MMA tiles are padded to   (8, 16, 32 or 64)
+ *   plan[1] = 1 if the up-projection runs on tcgen05, 0 on warp-level MMAs
+ *   plan[2] = 1 if the down-projection runs on tcgen05 as well
+ *   plan[3] = rows of the neuron-major activation buffer (D rounded up to 128)
+ *   plan[4] = neuron ranges per column chunk of the warp-level down-projection
+ *   plan[5] = thread blocks of the warp-level down-projection
+ *   plan[6] = output columns per warp-level down-projection item
+ *   plan[7] = workspace bytes (what sha_selective_mlp_workspace_size returns on
+ *             such a device)
+ * plan[4..6] describe the warp-level down-projection, which runs when
+ * plan[2] = 0.  The union size is only known on the device, so nothing here
+ * depends on it.  Returns SHA_ERR_INVALID_ARG (B, d, D or num_sms below 1, or
+ * plan NULL) or SHA_ERR_UNSUPPORTED (B > 64, d not a multiple of 256) as
+ * sha_selective_mlp would, SHA_OK otherwise.
+ */
+sha_status_t sha_selective_mlp_plan(int B, int d, int D, int num_sms, int64_t plan[8]);
+
+/*
  * sha_selective_mlp -- y [B, d] = sigma(x W1t[S]^T) W2t[S] over the first *n_S
  * ids of S (device memory; typically written by sha_mlp_union on the same
  * stream, so no host synchronisation is needed).
