@@ -155,3 +155,20 @@ def test_selective_mlp_host_checks(lib):
         ctypes.c_void_p] * 3 + [ctypes.c_size_t, ctypes.c_void_p]
     assert lib.sha_mlp_union(P, 0, 100, P, P, P, 1 << 20, None) == 1
     assert lib.sha_mlp_union(P, 2, 100, P, P, P, 1, None) == 7     # workspace too small
+
+
+def test_tokens_host_checks(lib):
+    P = 0x1000
+    lib.sha_decode_tokens.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 7 + [
+        ctypes.c_float, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
+
+    def call(tokens=P, B=2, d=128, top_k=2, n_sel=16, ptr=P):
+        # (B, H_q, H_kv, N_kv, d, top_k, n_sel)
+        return lib.sha_decode_tokens(ptr, ptr, ptr, ptr, tokens, B, 4, 4, 64, d, top_k, n_sel,
+                                     0.1, ptr, 0, None)
+    assert call(n_sel=0) == 1                        # no keys listed
+    assert call(tokens=None) == 1                    # no list
+    assert call(d=96) == 2                           # unsupported head dim
+    assert call(top_k=5) == 1                        # top_k above H_kv
+    assert call(ptr=0x1008) == 3                     # misaligned cache
+    assert call(tokens=None, B=0) == 0               # empty problem: nothing to read
