@@ -172,3 +172,22 @@ def test_tokens_host_checks(lib):
     assert call(top_k=5) == 1                        # top_k above H_kv
     assert call(ptr=0x1008) == 3                     # misaligned cache
     assert call(tokens=None, B=0) == 0               # empty problem: nothing to read
+
+
+def test_noalloc_host_checks(lib):
+    import head_sparse_decode_b200 as h
+    P = 0x1000
+    lib.sha_decode_noalloc.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 6 + [
+        ctypes.c_float, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
+
+    def call(H_q=4, H_kv=4, B=2, top_k=2, dtype=0, splits=0, ptr=P):
+        return lib.sha_decode_noalloc(ptr, ptr, ptr, ptr, B, H_q, H_kv, 64, 128, top_k, 0.1,
+                                      ptr, dtype, splits, None)
+    assert call(H_q=8, H_kv=4) == 2                  # grouped queries: not this entry point
+    assert call(dtype=7) == 2
+    assert call(splits=-1) == 1
+    assert call(ptr=0) == 1
+    assert call(ptr=0x1008) == 3
+    assert call(B=0, ptr=0) == 0                     # empty problem: nothing enqueued
+    # the binding reads the array's size from the library as built
+    assert lib.sha_noalloc_scratch_bytes() == h.NOALLOC_SCRATCH_BYTES == 512 * 1024
