@@ -191,3 +191,16 @@ def test_noalloc_host_checks(lib):
     assert call(B=0, ptr=0) == 0                     # empty problem: nothing enqueued
     # the binding reads the array's size from the library as built
     assert lib.sha_noalloc_scratch_bytes() == h.NOALLOC_SCRATCH_BYTES == 512 * 1024
+
+
+def test_clustered_host_checks(lib):
+    P = 0x1000
+    lib.sha_decode_clustered.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 6 + [
+        ctypes.c_float, ctypes.c_void_p] + [ctypes.c_int] * 4 + [ctypes.c_void_p]
+
+    def call(cluster=2, d=128):
+        return lib.sha_decode_clustered(P, P, P, P, 2, 4, 4, 64, d, 2, 0.1, P, 0, cluster, 2, 0,
+                                        None)
+    assert call(cluster=1) == 1                      # a cluster holds at least two blocks
+    assert call(cluster=0) == 1
+    assert call(d=96) == 2
